@@ -1,0 +1,20 @@
+"""B200-native forward + backward of the nanochat decoder behind a C ABI.
+
+`libnanochat_b200.so` (built from csrc/ by `build.py`) holds every kernel;
+this package is its thin Python binding.  `Model` adds PyTorch-owned device
+memory and streams on top.
+"""
+from ._binding import (NC_BF16, NC_EALIGN, NC_ECUDA, NC_EINVAL, NC_ENOMEM,  # noqa: F401
+                       NC_ENONFINITE, NC_ERANGE, NC_ESHAPE, NC_ETIMEOUT, NC_EUNSUPPORTED, NC_F32,
+                       NC_OK, LIB_PATH, NcError, load_library, nc_destroy, nc_fwd, nc_fwd_bwd,
+                       nc_get_dims, nc_init, nc_param_layout, nc_strerror, nc_sync_status,
+                       nc_workspace_bytes, nc_gemm, nc_attention_fwd, nc_attention_bwd,
+                       NC_EPI_STORE, NC_EPI_STORE_F32, NC_EPI_ADD, NC_EPI_RELU2, NC_EPI_DRELU2,
+                       NC_EPI_SOFTCAP)
+
+
+def __getattr__(name):
+    if name == "Model":
+        from .model import Model
+        return Model
+    raise AttributeError(name)

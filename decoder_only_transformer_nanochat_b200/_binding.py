@@ -1,0 +1,155 @@
+"""ctypes binding of libnanochat_b200.so, one Python function per C entry point.
+
+Argument marshalling only: every step of the decoder computation runs in the
+library's CUDA kernels.  Device buffers are passed as integer addresses and the
+stream as an integer cudaStream_t.  If the shared library has not been built
+the first call raises, naming the build step; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnanochat_b200.so")
+
+NC_OK = 0
+NC_EINVAL = 1
+NC_ESHAPE = 2
+NC_ENOMEM = 3
+NC_EUNSUPPORTED = 4
+NC_ECUDA = 5
+NC_ERANGE = 6
+NC_ENONFINITE = 7
+NC_ETIMEOUT = 8
+NC_EALIGN = 9
+
+NC_F32 = 0
+NC_BF16 = 1
+
+
+class NcError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {nc_strerror(code)} (status {code})")
+
+
+class nc_dims(ctypes.Structure):
+    _fields_ = [("depth", ctypes.c_int), ("width", ctypes.c_int), ("n_head", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("hidden", ctypes.c_int), ("vocab", ctypes.c_int),
+                ("seq", ctypes.c_int), ("dtype", ctypes.c_int), ("n_params", ctypes.c_int64)]
+
+
+class nc_param(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("offset", ctypes.c_int64),
+                ("rows", ctypes.c_int), ("cols", ctypes.c_int)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGS = {
+    "nc_init": (_I, [_I, _I, _I, _I, ctypes.POINTER(_P)]),
+    "nc_get_dims": (_I, [_P, ctypes.POINTER(nc_dims)]),
+    "nc_param_layout": (_I, [_P, _I, ctypes.POINTER(nc_param)]),
+    "nc_workspace_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_fwd_bwd": (_I, [_P, _P, _P, _P, _I, _I, _P, ctypes.c_size_t, _P, _P, _P, _P]),
+    "nc_fwd": (_I, [_P, _P, _P, _I, _I, _P, ctypes.c_size_t, _P, _P]),
+    "nc_sync_status": (_I, [_P, _P, _I]),
+    "nc_strerror": (ctypes.c_char_p, [_I]),
+    "nc_destroy": (None, [_P]),
+    "nc_gemm": (_I, [_P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _I,
+                     _I, _I, _I, _P]),
+    "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "nc_attention_bwd": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+}
+
+NC_EPI_STORE = 0
+NC_EPI_STORE_F32 = 1
+NC_EPI_ADD = 2
+NC_EPI_RELU2 = 3
+NC_EPI_DRELU2 = 4
+NC_EPI_SOFTCAP = 5
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library once; raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"{path} is missing: build it with "
+                      "`python -m decoder_only_transformer_nanochat_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def nc_init(depth: int, vocab: int, seq: int, dtype: int):
+    """Returns (status, handle)."""
+    h = _P()
+    rc = load_library().nc_init(depth, vocab, seq, dtype, ctypes.byref(h))
+    return rc, h.value
+
+
+def nc_get_dims(handle):
+    d = nc_dims()
+    rc = load_library().nc_get_dims(handle, ctypes.byref(d))
+    return rc, {f: getattr(d, f) for f, _ in nc_dims._fields_}
+
+
+def nc_param_layout(handle, index: int):
+    p = nc_param()
+    rc = load_library().nc_param_layout(handle, index, ctypes.byref(p))
+    return rc, (p.name.decode(), p.offset, p.rows, p.cols)
+
+
+def nc_workspace_bytes(handle, B: int, T: int):
+    n = ctypes.c_size_t()
+    rc = load_library().nc_workspace_bytes(handle, B, T, ctypes.byref(n))
+    return rc, n.value
+
+
+def nc_fwd_bwd(handle, weights, tokens, targets, B, T, workspace, ws_bytes, loss, token_loss,
+               grads, stream):
+    return load_library().nc_fwd_bwd(handle, weights, tokens, targets, B, T, workspace, ws_bytes,
+                                     loss, token_loss, grads, stream)
+
+
+def nc_fwd(handle, weights, tokens, B, T, workspace, ws_bytes, logits, stream):
+    return load_library().nc_fwd(handle, weights, tokens, B, T, workspace, ws_bytes, logits, stream)
+
+
+def nc_sync_status(handle, stream, timeout_ms: int) -> int:
+    return load_library().nc_sync_status(handle, stream, timeout_ms)
+
+
+def nc_strerror(code: int) -> str:
+    try:
+        return load_library().nc_strerror(code).decode()
+    except OSError:
+        return f"status {code}"
+
+
+def nc_destroy(handle) -> None:
+    if handle:
+        load_library().nc_destroy(handle)
+
+
+def nc_gemm(A, lda, a_mn, B, ldb, b_mn, D, ldd, M, N, K, dtype, epilogue, engine, stream) -> int:
+    return load_library().nc_gemm(A, lda, a_mn, B, ldb, b_mn, D, ldd, M, N, K, dtype, epilogue,
+                                  engine, stream)
+
+
+def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream) -> int:
+    return load_library().nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream)
+
+
+def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream) -> int:
+    return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine,
+                                           stream)

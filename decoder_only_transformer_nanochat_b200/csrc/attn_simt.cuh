@@ -1,0 +1,262 @@
+// Causal multi-query attention on CUDA cores with fp32 arithmetic: the
+// exact-fp32 path of the fp32 model.  One shared key/value head serves all H
+// query heads (energyai.berlin page, "Multi-Query Attention (MQA)"); scores
+// are q.k / sqrt(128) with keys j <= i.
+//
+// Layout: qkv rows [M, ld] = [q (H*128) | k (128) | v (128)], M = B*T;
+// O [M, H*128]; lse and D [B, H, T] fp32.
+//
+// Each query (or key) row is owned by 8 threads; thread `sub` owns dims
+// sub + 8*c, c < 16, and dot products are finished with 3 shuffles.
+#pragma once
+
+#include "common.cuh"
+
+namespace nc {
+
+constexpr int kSimtRows = 16;   // rows per block (16 rows * 8 threads = 128 threads)
+constexpr int kSimtKeys = 32;   // keys / queries per shared-memory tile
+
+__device__ __forceinline__ float sub8_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  return v;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) attn_fwd_simt_kernel(const T *__restrict__ qkv, int ld,
+                                                            T *__restrict__ O,
+                                                            float *__restrict__ lse, int T_len,
+                                                            int H) {
+  __shared__ float Ks[kSimtKeys][kHeadDim + 1];
+  __shared__ float Vs[kSimtKeys][kHeadDim + 1];
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int r = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const int i = blockIdx.x * kSimtRows + r;  // query position
+  const int C = H * kHeadDim;
+  const size_t row0 = (size_t)b * T_len;
+  const float scale = rsqrtf((float)kHeadDim);
+  float q[16], acc[16];
+  const bool valid = i < T_len;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    q[c] = valid ? to_f(qkv[(row0 + i) * ld + h * kHeadDim + sub + 8 * c]) * scale : 0.f;
+    acc[c] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int last = min(T_len - 1, blockIdx.x * kSimtRows + kSimtRows - 1);
+  for (int j0 = 0; j0 <= last; j0 += kSimtKeys) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
+      const int jj = e / kHeadDim, c = e % kHeadDim;
+      const int j = j0 + jj;
+      const bool ok = j < T_len;
+      Ks[jj][c] = ok ? to_f(qkv[(row0 + j) * ld + C + c]) : 0.f;
+      Vs[jj][c] = ok ? to_f(qkv[(row0 + j) * ld + C + kHeadDim + c]) : 0.f;
+    }
+    __syncthreads();
+    float s[kSimtKeys];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int jj = 0; jj < kSimtKeys; ++jj) {
+      float d = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) d = fmaf(q[c], Ks[jj][sub + 8 * c], d);
+      d = sub8_sum(d);
+      s[jj] = (j0 + jj <= i) ? d : -INFINITY;
+      tmax = fmaxf(tmax, s[jj]);
+    }
+    if (tmax == -INFINITY) continue;  // every key of this tile is in the future
+    const float mnew = fmaxf(m, tmax);
+    const float corr = expf(m - mnew);
+    l *= corr;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc[c] *= corr;
+#pragma unroll
+    for (int jj = 0; jj < kSimtKeys; ++jj) {
+      const float pj = expf(s[jj] - mnew);
+      l += pj;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[c] = fmaf(pj, Vs[jj][sub + 8 * c], acc[c]);
+    }
+    m = mnew;
+  }
+  if (!valid) return;
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    O[(row0 + i) * C + h * kHeadDim + sub + 8 * c] = from_f<T>(acc[c] * inv);
+  if (sub == 0) lse[((size_t)b * H + h) * T_len + i] = m + logf(l);
+}
+
+// dq_i = sum_j ds_ij k_j / sqrt(d),  ds_ij = p_ij (dO_i . v_j - D_i),
+// p_ij = exp(q_i.k_j/sqrt(d) - lse_i).  Written into the q part of dqkv.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
+    const T *__restrict__ qkv, int ld, const T *__restrict__ dO, const float *__restrict__ lse,
+    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H) {
+  __shared__ float Ks[kSimtKeys][kHeadDim + 1];
+  __shared__ float Vs[kSimtKeys][kHeadDim + 1];
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int r = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const int i = blockIdx.x * kSimtRows + r;
+  const int C = H * kHeadDim;
+  const size_t row0 = (size_t)b * T_len;
+  const float scale = rsqrtf((float)kHeadDim);
+  const bool valid = i < T_len;
+  float q[16], g[16], dq[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    q[c] = valid ? to_f(qkv[(row0 + i) * ld + h * kHeadDim + sub + 8 * c]) * scale : 0.f;
+    g[c] = valid ? to_f(dO[(row0 + i) * C + h * kHeadDim + sub + 8 * c]) : 0.f;
+    dq[c] = 0.f;
+  }
+  const size_t li = ((size_t)b * H + h) * T_len + (valid ? i : 0);
+  const float L = lse[li], Di = Dr[li];
+  const int last = min(T_len - 1, blockIdx.x * kSimtRows + kSimtRows - 1);
+  for (int j0 = 0; j0 <= last; j0 += kSimtKeys) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
+      const int jj = e / kHeadDim, c = e % kHeadDim;
+      const int j = j0 + jj;
+      const bool ok = j < T_len;
+      Ks[jj][c] = ok ? to_f(qkv[(row0 + j) * ld + C + c]) : 0.f;
+      Vs[jj][c] = ok ? to_f(qkv[(row0 + j) * ld + C + kHeadDim + c]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = 0; jj < kSimtKeys; ++jj) {
+      float s = 0.f, dp = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        s = fmaf(q[c], Ks[jj][sub + 8 * c], s);
+        dp = fmaf(g[c], Vs[jj][sub + 8 * c], dp);
+      }
+      s = sub8_sum(s);
+      dp = sub8_sum(dp);
+      const float p = (j0 + jj <= i) ? expf(s - L) : 0.f;
+      const float ds = p * (dp - Di) * scale;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) dq[c] = fmaf(ds, Ks[jj][sub + 8 * c], dq[c]);
+    }
+  }
+  if (!valid) return;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) dqkv[(row0 + i) * ld + h * kHeadDim + sub + 8 * c] = from_f<T>(dq[c]);
+}
+
+// dv_j = sum_h sum_{i>=j} p_ij dO_i ;  dk_j = sum_h sum_{i>=j} ds_ij q_i / sqrt(d)
+// (the shared head's gradients sum over every query head).  Written into the
+// k and v parts of dqkv.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
+    const T *__restrict__ qkv, int ld, const T *__restrict__ dO, const float *__restrict__ lse,
+    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H) {
+  __shared__ float Qs[kSimtKeys][kHeadDim + 1];
+  __shared__ float Gs[kSimtKeys][kHeadDim + 1];
+  __shared__ float Ls[kSimtKeys], Ds[kSimtKeys];
+  const int b = blockIdx.z;
+  const int r = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const int j = blockIdx.x * kSimtRows + r;  // key position
+  const int C = H * kHeadDim;
+  const size_t row0 = (size_t)b * T_len;
+  const float scale = rsqrtf((float)kHeadDim);
+  const bool valid = j < T_len;
+  float k[16], v[16], dk[16], dv[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    k[c] = valid ? to_f(qkv[(row0 + j) * ld + C + sub + 8 * c]) : 0.f;
+    v[c] = valid ? to_f(qkv[(row0 + j) * ld + C + kHeadDim + sub + 8 * c]) : 0.f;
+    dk[c] = 0.f;
+    dv[c] = 0.f;
+  }
+  const int first = blockIdx.x * kSimtRows;  // earliest query that sees a key of this block
+  for (int h = 0; h < H; ++h) {
+    for (int i0 = (first / kSimtKeys) * kSimtKeys; i0 < T_len; i0 += kSimtKeys) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
+        const int ii = e / kHeadDim, c = e % kHeadDim;
+        const int i = i0 + ii;
+        const bool ok = i < T_len;
+        Qs[ii][c] = ok ? to_f(qkv[(row0 + i) * ld + h * kHeadDim + c]) : 0.f;
+        Gs[ii][c] = ok ? to_f(dO[(row0 + i) * C + h * kHeadDim + c]) : 0.f;
+      }
+      if (threadIdx.x < kSimtKeys) {
+        const int i = i0 + threadIdx.x;
+        const bool ok = i < T_len;
+        Ls[threadIdx.x] = ok ? lse[((size_t)b * H + h) * T_len + i] : 0.f;
+        Ds[threadIdx.x] = ok ? Dr[((size_t)b * H + h) * T_len + i] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int ii = 0; ii < kSimtKeys; ++ii) {
+        const int i = i0 + ii;
+        float s = 0.f, dp = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          s = fmaf(Qs[ii][sub + 8 * c], k[c], s);
+          dp = fmaf(Gs[ii][sub + 8 * c], v[c], dp);
+        }
+        s = sub8_sum(s) * scale;
+        dp = sub8_sum(dp);
+        const bool live = valid && i < T_len && i >= j;
+        const float p = live ? expf(s - Ls[ii]) : 0.f;
+        const float ds = p * (dp - Ds[ii]) * scale;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          dv[c] = fmaf(p, Gs[ii][sub + 8 * c], dv[c]);
+          dk[c] = fmaf(ds, Qs[ii][sub + 8 * c], dk[c]);
+        }
+      }
+    }
+  }
+  if (!valid) return;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    dqkv[(row0 + j) * ld + C + sub + 8 * c] = from_f<T>(dk[c]);
+    dqkv[(row0 + j) * ld + C + kHeadDim + sub + 8 * c] = from_f<T>(dv[c]);
+  }
+}
+
+template <typename T>
+inline cudaError_t launch_attn_simt_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len,
+                                        int H, cudaStream_t st) {
+  dim3 grid((T_len + kSimtRows - 1) / kSimtRows, H, B);
+  attn_fwd_simt_kernel<T><<<grid, 128, 0, st>>>(qkv, ld, O, lse, T_len, H);
+  return cudaGetLastError();
+}
+
+template <typename T>
+inline cudaError_t launch_attn_simt_bwd(const T *qkv, int ld, const T *dO, const float *lse,
+                                        const float *Dr, T *dqkv, int B, int T_len, int H,
+                                        cudaStream_t st) {
+  dim3 g1((T_len + kSimtRows - 1) / kSimtRows, H, B);
+  attn_bwd_dq_simt_kernel<T><<<g1, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H);
+  dim3 g2((T_len + kSimtRows - 1) / kSimtRows, 1, B);
+  attn_bwd_dkdv_simt_kernel<T><<<g2, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H);
+  return cudaGetLastError();
+}
+
+}  // namespace nc
+
+namespace nc {
+
+template <typename T>
+inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H,
+                                   int num_sms, int engine, cudaStream_t st) {
+  (void)num_sms;
+  (void)engine;
+  return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
+}
+
+template <typename T>
+inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *dO, const float *lse,
+                                   const float *Dr, T *dqkv, int B, int T_len, int H, int num_sms,
+                                   int engine, cudaStream_t st) {
+  (void)num_sms;
+  (void)engine;
+  return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);
+}
+
+}  // namespace nc

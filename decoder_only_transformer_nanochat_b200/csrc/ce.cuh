@@ -1,0 +1,167 @@
+// Softcap + log-sum-exp + token cross-entropy, forward and backward fused, in
+// place over the unembedding output z [M, ldz]:
+//   s = 15 tanh(z / 15)             ("ten modern departures": logit softcap 15,
+//                                     computed in fp32)
+//   loss_i = logsumexp(s_i) - s_i[target_i]
+//   dz = (softmax(s_i) - onehot(target_i)) (1 - (s/15)^2) / M   written over z
+// No fp32 copy of the logits is ever materialised: each row is read once and
+// written once.
+#pragma once
+
+#include "common.cuh"
+
+namespace nc {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// tanh in the precision of the storage type: the hardware approximation
+// (relative error ~2^-11) for bf16 logits, whose storage rounding (2^-9) is
+// larger; the accurate library routine for fp32.
+template <typename T> __device__ __forceinline__ float softcap_tanh(float x);
+template <> __device__ __forceinline__ float softcap_tanh<bf16>(float x) { return tanh_fast(x); }
+template <> __device__ __forceinline__ float softcap_tanh<float>(float x) { return tanhf(x); }
+template <typename T> __device__ __forceinline__ float exp_t(float x);
+template <> __device__ __forceinline__ float exp_t<bf16>(float x) { return ex2_fast(x * kLog2e); }
+template <> __device__ __forceinline__ float exp_t<float>(float x) { return expf(x); }
+
+// ---------------------------------------------------------------------------
+// Register-resident version for bf16 rows of V = 512 threads * 8 * NVEC
+// values (65,536 for NVEC = 16).  tanh(z/15) is kept per element as fp16
+// (|t| <= 1, 11-bit mantissa: finer than the bf16 logit it came from).
+template <int NVEC>
+__global__ void __launch_bounds__(512, 1) ce_fused_bf16_kernel(
+    bf16 *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
+    float *__restrict__ token_loss, int M, int V, float inv_M, int *status) {
+  __shared__ float red[32];
+  __shared__ float s_target;
+  const int row = blockIdx.x;
+  if (row >= M) return;
+  bf16 *zr = z + (size_t)row * ldz;
+  int tgt = targets[row];
+  if (tgt < 0 || tgt >= V) {
+    if (threadIdx.x == 0) set_status(status, kStatusRange);
+    tgt = tgt < 0 ? 0 : V - 1;
+  }
+  __half2 t[NVEC][4];
+  float tmax = -1.f;
+#pragma unroll
+  for (int k = 0; k < NVEC; ++k) {
+    const int v = threadIdx.x + k * 512;
+    uint4 u = *reinterpret_cast<const uint4 *>(zr + v * 8);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __bfloat1622float2(h[j]);
+      const float a = tanh_fast(f.x * (1.f / kSoftcap)), b = tanh_fast(f.y * (1.f / kSoftcap));
+      t[k][j] = __floats2half2_rn(a, b);
+      const float2 r = __half22float2(t[k][j]);
+      tmax = fmaxf(tmax, fmaxf(r.x, r.y));
+      const int e = v * 8 + 2 * j;
+      if (e == tgt) s_target = kSoftcap * r.x;
+      if (e + 1 == tgt) s_target = kSoftcap * r.y;
+    }
+  }
+  const float smax = kSoftcap * block_max(tmax, red);
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < NVEC; ++k)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 r = __half22float2(t[k][j]);
+      sum += ex2_fast((kSoftcap * r.x - smax) * kLog2e) + ex2_fast((kSoftcap * r.y - smax) * kLog2e);
+    }
+  sum = block_sum(sum, red);  // contains __syncthreads: s_target is visible after it
+  const float lse = smax + __logf(sum);
+  if (threadIdx.x == 0) token_loss[row] = lse - s_target;
+#pragma unroll
+  for (int k = 0; k < NVEC; ++k) {
+    const int v = threadIdx.x + k * 512;
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 r = __half22float2(t[k][j]);
+      const int e = v * 8 + 2 * j;
+      float pa = ex2_fast((kSoftcap * r.x - lse) * kLog2e) - (e == tgt ? 1.f : 0.f);
+      float pb = ex2_fast((kSoftcap * r.y - lse) * kLog2e) - (e + 1 == tgt ? 1.f : 0.f);
+      h[j] = __floats2bfloat162_rn(pa * (1.f - r.x * r.x) * inv_M, pb * (1.f - r.y * r.y) * inv_M);
+    }
+    *reinterpret_cast<uint4 *>(zr + v * 8) = u;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// General version, any V and either dtype: two sweeps over the row (the
+// second is served by L2), online max/sum in the first.
+template <typename T>
+__global__ void __launch_bounds__(256) ce_fused_generic_kernel(
+    T *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
+    float *__restrict__ token_loss, int M, int V, float inv_M, int *status) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  if (row >= M) return;
+  T *zr = z + (size_t)row * ldz;
+  int tgt = targets[row];
+  if (tgt < 0 || tgt >= V) {
+    if (threadIdx.x == 0) set_status(status, kStatusRange);
+    tgt = tgt < 0 ? 0 : V - 1;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float s = kSoftcap * softcap_tanh<T>(to_f(zr[v]) * (1.f / kSoftcap));
+    if (s > m) {
+      l = l * exp_t<T>(m - s) + 1.f;
+      m = s;
+    } else {
+      l += exp_t<T>(s - m);
+    }
+  }
+  const float gm = block_max(m, red);
+  const float part = (m == -INFINITY) ? 0.f : l * exp_t<T>(m - gm);
+  const float s_t = kSoftcap * softcap_tanh<T>(to_f(zr[tgt]) * (1.f / kSoftcap));
+  const float tot = block_sum(part, red);  // syncs: every read of zr[tgt] precedes the writes
+  const float lse = gm + logf(tot);
+  if (threadIdx.x == 0) token_loss[row] = lse - s_t;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float tt = softcap_tanh<T>(to_f(zr[v]) * (1.f / kSoftcap));
+    const float p = exp_t<T>(kSoftcap * tt - lse) - (v == tgt ? 1.f : 0.f);
+    zr[v] = from_f<T>(p * (1.f - tt * tt) * inv_M);
+  }
+}
+
+// loss = mean of the per-token losses; flags a non-finite result.
+__global__ void __launch_bounds__(1024) loss_mean_kernel(const float *__restrict__ token_loss,
+                                                         int M, float *__restrict__ loss,
+                                                         int *status) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) s += (double)token_loss[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x == 0) {
+      const float r = (float)(s / (double)M);
+      *loss = r;
+      if (!isfinite(r)) set_status(status, kStatusNonFinite);
+    }
+  }
+}
+
+}  // namespace nc

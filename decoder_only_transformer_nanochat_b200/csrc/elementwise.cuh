@@ -1,0 +1,309 @@
+// Bandwidth-bound kernels of the decoder step: embedding gather + RMSNorm,
+// RMSNorm, RoPE + QK-norm, their backward passes and the embedding
+// scatter-add.  One warp owns one row; a row of C values is held in registers
+// (8 contiguous values per 16-byte access, C/8 accesses spread over the lanes)
+// so each row is read once and written once.
+//
+// Parameterless RMSNorm y = x / sqrt(mean(x^2) + eps) ("A Llama-class
+// transformer with ten modern departures": bare F.rms_norm after the
+// embedding, before attention, before the MLP and before the head).
+// Backward: dx = r (dy - y mean(dy y)), r = 1/sqrt(mean(x^2) + eps).
+#pragma once
+
+#include "common.cuh"
+
+namespace nc {
+
+// NV = 16-byte accesses per lane: a row of C values needs NV = ceil(C / 256).
+// Rows up to C = 32 lanes * 16 * 8 = 4096 are supported.
+constexpr int kMaxVecPerLane = 16;
+
+#define NC_DISPATCH_NV(C, KERNEL_CALL)                 \
+  do {                                                 \
+    const int nv_ = ((C) / 8 + 31) / 32;               \
+    switch (nv_) {                                     \
+      case 1: { constexpr int NV = 1; KERNEL_CALL; } break; \
+      case 2: { constexpr int NV = 2; KERNEL_CALL; } break; \
+      case 3: { constexpr int NV = 3; KERNEL_CALL; } break; \
+      case 4: { constexpr int NV = 4; KERNEL_CALL; } break; \
+      case 5: { constexpr int NV = 5; KERNEL_CALL; } break; \
+      case 6: { constexpr int NV = 6; KERNEL_CALL; } break; \
+      case 7: { constexpr int NV = 7; KERNEL_CALL; } break; \
+      case 8: { constexpr int NV = 8; KERNEL_CALL; } break; \
+      default: { constexpr int NV = 16; KERNEL_CALL; } break; \
+    }                                                  \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// x = rmsnorm(wte[tok]); r0 = 1/rms.  Token ids outside [0, V) are flagged
+// and clamped so the gather stays in bounds.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) embed_norm_kernel(
+    const int32_t *__restrict__ tokens, const T *__restrict__ wte, T *__restrict__ x,
+    float *__restrict__ r_out, int M, int C, int V, int *status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  int tok = tokens[row];
+  if (tok < 0 || tok >= V) {
+    if (lane == 0) set_status(status, kStatusRange);
+    tok = tok < 0 ? 0 : V - 1;
+  }
+  const int nv = C >> 3;
+  const T *src = wte + (size_t)tok * C;
+  float v[NV][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+      Vec8<T>::load(src + c * 8, v[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss += v[i][j] * v[i][j];
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)C + kEps);
+  T *dst = x + (size_t)row * C;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[i][j] *= r;
+      Vec8<T>::store(dst + c * 8, v[i]);
+    }
+  }
+  if (lane == 0) r_out[row] = r;
+}
+
+// y = rmsnorm(x) row-wise; r = 1/rms saved for the backward pass.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ x, T *__restrict__ y,
+                                                      float *__restrict__ r_out, int M, int C) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const int nv = C >> 3;
+  const T *src = x + (size_t)row * C;
+  float v[NV][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+      Vec8<T>::load(src + c * 8, v[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss += v[i][j] * v[i][j];
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)C + kEps);
+  T *dst = y + (size_t)row * C;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[i][j] *= r;
+      Vec8<T>::store(dst + c * 8, v[i]);
+    }
+  }
+  if (lane == 0) r_out[row] = r;
+}
+
+// RMSNorm backward with the residual-stream accumulation:
+//   g = r (dy - y mean(dy y));  dx = g (+ dx_old if accumulate)
+// dy is fp32 (a GEMM output), y the saved normalised value, dx kept in fp32
+// and also written in T as the next GEMM's operand.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
+    const float *__restrict__ dy, const T *__restrict__ y, const float *__restrict__ r,
+    float *__restrict__ dx, T *__restrict__ dx_t, int M, int C, int accumulate) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const int nv = C >> 3;
+  const size_t base = (size_t)row * C;
+  float g[NV][8], yy[NV][8];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+      Vec8<float>::load(dy + base + c * 8, g[i]);
+      Vec8<T>::load(y + base + c * 8, yy[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dot += g[i][j] * yy[i][j];
+    }
+  }
+  dot = warp_sum(dot) / (float)C;
+  const float rr = r[row];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+      float old[8];
+      if (accumulate) Vec8<float>::load(dx + base + c * 8, old);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        g[i][j] = rr * (g[i][j] - yy[i][j] * dot);
+        if (accumulate) g[i][j] += old[j];
+      }
+      Vec8<float>::store(dx + base + c * 8, g[i]);
+      Vec8<T>::store(dx_t + base + c * 8, g[i]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RoPE then QK-norm, in place on the q heads and the shared k head of the
+// fused qkv rows [M, ld] = [q (H*128) | k (128) | v (128)].
+// RoPE ("ten modern departures": theta 10,000) on half-split pairs (i, i+64):
+//   y_i = x_i cos - x_{i+64} sin,  y_{i+64} = x_i sin + x_{i+64} cos,
+// angle = pos * theta^(-i/64), pos = token index within its row of T.
+// QK-norm after RoPE: per-head parameterless RMSNorm over the 128 dims.
+// One warp per (token, head); lane l owns dims {2l, 2l+1} and {64+2l, 65+2l}.
+template <typename T> struct Pair2;
+template <> struct Pair2<bf16> {
+  static __device__ __forceinline__ float2 load(const bf16 *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+  }
+  static __device__ __forceinline__ void store(bf16 *p, float2 v) {
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
+  }
+};
+template <> struct Pair2<float> {
+  static __device__ __forceinline__ float2 load(const float *p) {
+    return *reinterpret_cast<const float2 *>(p);
+  }
+  static __device__ __forceinline__ void store(float *p, float2 v) {
+    *reinterpret_cast<float2 *>(p) = v;
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) rope_qknorm_kernel(
+    T *__restrict__ qkv, int ld, float *__restrict__ rq, float *__restrict__ rk,
+    const float *__restrict__ cos_t, const float *__restrict__ sin_t, int M, int T_len, int H) {
+  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= M * (H + 1)) return;
+  const int tok = item / (H + 1), h = item % (H + 1);
+  const int pos = tok % T_len;
+  T *p = qkv + (size_t)tok * ld + h * kHeadDim;
+  const int i0 = 2 * lane;
+  float2 a = Pair2<T>::load(p + i0), b = Pair2<T>::load(p + 64 + i0);
+  const float2 c = *reinterpret_cast<const float2 *>(cos_t + pos * 64 + i0);
+  const float2 s = *reinterpret_cast<const float2 *>(sin_t + pos * 64 + i0);
+  float2 y1 = make_float2(a.x * c.x - b.x * s.x, a.y * c.y - b.y * s.y);
+  float2 y2 = make_float2(a.x * s.x + b.x * c.x, a.y * s.y + b.y * c.y);
+  float ss = y1.x * y1.x + y1.y * y1.y + y2.x * y2.x + y2.y * y2.y;
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)kHeadDim + kEps);
+  Pair2<T>::store(p + i0, make_float2(y1.x * r, y1.y * r));
+  Pair2<T>::store(p + 64 + i0, make_float2(y2.x * r, y2.y * r));
+  if (lane == 0) {
+    if (h < H) rq[(size_t)tok * H + h] = r;
+    else rk[tok] = r;
+  }
+}
+
+// Backward of QK-norm then RoPE, in place on the q and k parts of dqkv:
+//   g = r (dy - y mean(dy y)) with y the saved normalised q/k,
+//   dx_i = g_i cos + g_{i+64} sin,  dx_{i+64} = -g_i sin + g_{i+64} cos.
+template <typename T>
+__global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
+    T *__restrict__ dqkv, const T *__restrict__ qkv, int ld, const float *__restrict__ rq,
+    const float *__restrict__ rk, const float *__restrict__ cos_t,
+    const float *__restrict__ sin_t, int M, int T_len, int H) {
+  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= M * (H + 1)) return;
+  const int tok = item / (H + 1), h = item % (H + 1);
+  const int pos = tok % T_len;
+  const size_t off = (size_t)tok * ld + h * kHeadDim;
+  const int i0 = 2 * lane;
+  float2 da = Pair2<T>::load(dqkv + off + i0), db = Pair2<T>::load(dqkv + off + 64 + i0);
+  float2 ya = Pair2<T>::load(qkv + off + i0), yb = Pair2<T>::load(qkv + off + 64 + i0);
+  float dot = da.x * ya.x + da.y * ya.y + db.x * yb.x + db.y * yb.y;
+  dot = warp_sum(dot) / (float)kHeadDim;
+  const float r = h < H ? rq[(size_t)tok * H + h] : rk[tok];
+  float2 ga = make_float2(r * (da.x - ya.x * dot), r * (da.y - ya.y * dot));
+  float2 gb = make_float2(r * (db.x - yb.x * dot), r * (db.y - yb.y * dot));
+  const float2 c = *reinterpret_cast<const float2 *>(cos_t + pos * 64 + i0);
+  const float2 s = *reinterpret_cast<const float2 *>(sin_t + pos * 64 + i0);
+  Pair2<T>::store(dqkv + off + i0, make_float2(ga.x * c.x + gb.x * s.x, ga.y * c.y + gb.y * s.y));
+  Pair2<T>::store(dqkv + off + 64 + i0,
+                  make_float2(-ga.x * s.x + gb.x * c.x, -ga.y * s.y + gb.y * c.y));
+}
+
+// ---------------------------------------------------------------------------
+// Embedding backward: through the norm after the embedding, then summed into
+// the rows of dwte that the tokens select (repeated tokens add up).
+//   y = wte[tok] r0;  g = r0 (dx - y mean(dx y));  dwte[tok] += g
+// dwte must be zeroed beforehand.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) embed_bwd_kernel(
+    const float *__restrict__ dx, const int32_t *__restrict__ tokens, const T *__restrict__ wte,
+    const float *__restrict__ r0, float *__restrict__ dwte, int M, int C, int V) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  int tok = tokens[row];
+  tok = tok < 0 ? 0 : (tok >= V ? V - 1 : tok);
+  const int nv = C >> 3;
+  const float r = r0[row];
+  const size_t base = (size_t)row * C;
+  float g[NV][8], yy[NV][8];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+      Vec8<float>::load(dx + base + c * 8, g[i]);
+      Vec8<T>::load(wte + (size_t)tok * C + c * 8, yy[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        yy[i][j] *= r;
+        dot += g[i][j] * yy[i][j];
+      }
+    }
+  }
+  dot = warp_sum(dot) / (float)C;
+  float *dst = dwte + (size_t)tok * C;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (lane + 32 * i);
+    if (c < nv) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) atomicAdd(dst + c * 8 + j, r * (g[i][j] - yy[i][j] * dot));
+    }
+  }
+}
+
+// D[b,h,t] = sum_c dO[t,h,c] O[t,h,c]  (the softmax-backward row term).
+template <typename T>
+__global__ void __launch_bounds__(256) attn_rowdot_kernel(const T *__restrict__ dO,
+                                                          const T *__restrict__ O,
+                                                          float *__restrict__ D, int M,
+                                                          int T_len, int H) {
+  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= M * H) return;
+  const int tok = item / H, h = item % H;
+  const size_t off = (size_t)tok * H * kHeadDim + h * kHeadDim + lane * 4;
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; j += 2) {
+    float2 a = Pair2<T>::load(dO + off + j), b = Pair2<T>::load(O + off + j);
+    s += a.x * b.x + a.y * b.y;
+  }
+  s = warp_sum(s);
+  if (lane == 0) {
+    const int bb = tok / T_len, t = tok % T_len;
+    D[((size_t)bb * H + h) * T_len + t] = s;
+  }
+}
+
+}  // namespace nc

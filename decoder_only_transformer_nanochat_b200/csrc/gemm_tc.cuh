@@ -1,0 +1,509 @@
+// bf16 GEMM on the 5th-generation tensor cores (sm_100a):
+//   TMA (128-byte swizzle) -> 4-stage shared-memory ring -> tcgen05.mma
+//   (cta_group::1, M=128, N=256, K=16, fp32 accumulate in TMEM) -> tcgen05.ld
+//   -> fused epilogue -> global.
+// Persistent: one CTA per SM walks a static list of (tile, k-split) units.
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues MMAs (one
+// elected lane), warps 2..5 drain the accumulator (each warp reads the 32
+// TMEM lanes its warp index selects).  Two TMEM accumulators (2 x 256 fp32
+// columns) let the epilogue of one tile overlap the main loop of the next.
+//
+// Operand layouts (see gemm_common.cuh): a K-major operand is loaded as one
+// box of [64 k x rows] (128 bytes of k per row, 8-row swizzle atoms of 1 KB);
+// an MN-major operand as boxes of [64 mn x 64 k] (128 bytes of mn per k-row),
+// stacked 8 KB apart along mn.  The shared-memory descriptors encode both
+// canonical forms.
+//
+// Every wait is bounded: after kWaitNs without progress a CTA raises its
+// abort flag, records kStatusTimeout in the status word, drains what it has
+// in flight (again bounded), frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "gemm_common.cuh"
+
+namespace nc {
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;      // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr uint64_t kWaitNs = 4000000000ull;         // 4 s without progress = abort
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct Unit {
+  int m_blk, n_blk, kb0, kb1;
+};
+
+struct Params {
+  int M, N, K;
+  int n_m, n_n;        // tile counts
+  int splits, kblocks;  // k-splits per tile, k-blocks of BK in K
+  int units;
+  int a_mn, b_mn;
+  void *D;
+  int64_t ldd;
+  int epi;
+  int atomic_out;       // split-K: reduce fp32 output with red.global.add
+  int *status;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false if this CTA is aborting (flag set here or elsewhere).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          int *status) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        *abort_flag = 1;
+        set_status(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// tcgen05 shared-memory matrix descriptor: start >>4 in [0,14), leading byte
+// offset >>4 in [16,30), stride byte offset >>4 in [32,46), fixed 0b001 in
+// [46,49), 128-byte swizzle (2) in [61,64).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFF) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, major
+// of each operand, N>>3 and M>>4.
+__host__ __device__ constexpr uint32_t make_idesc(int a_mn, int b_mn, int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ Unit unit_of(const Params &p, int u) {
+  // tiles grouped 16 m-blocks at a time so CTAs in flight share B tiles in L2
+  const int tile = u / p.splits, split = u % p.splits;
+  const int G = 16;
+  const int per_group = G * p.n_n;
+  const int g = tile / per_group;
+  const int first_m = g * G;
+  const int gsize = min(p.n_m - first_m, G);
+  const int r = tile % per_group;
+  Unit x;
+  x.m_blk = first_m + r % gsize;
+  x.n_blk = r / gsize;
+  const int per = (p.kblocks + p.splits - 1) / p.splits;
+  x.kb0 = split * per;
+  x.kb1 = min(p.kblocks, x.kb0 + per);
+  return x;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// Epilogue of 32 consecutive columns [n, n+32) of row m.
+__device__ __forceinline__ void epilogue_chunk(const Params &p, int m, int n, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.epi == EPI_STORE_F32) {
+    float *d = reinterpret_cast<float *>(p.D) + (size_t)m * p.ldd + n;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = n + 4 * q;
+      if (c + 4 <= p.N) {
+        if (p.atomic_out) red_add_v4(d + 4 * q, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        else *reinterpret_cast<float4 *>(d + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (c + j < p.N) {
+            if (p.atomic_out) atomicAdd(d + 4 * q + j, v[4 * q + j]);
+            else d[4 * q + j] = v[4 * q + j];
+          }
+      }
+    }
+    return;
+  }
+  bf16 *d = reinterpret_cast<bf16 *>(p.D) + (size_t)m * p.ldd + n;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = n + 8 * q;
+    float o[8], old[8];
+    const bool full = c + 8 <= p.N;
+    if (p.epi == EPI_ADD || p.epi == EPI_DRELU2) {
+      if (full) Vec8<bf16>::load(d + 8 * q, old);
+      else
+        for (int j = 0; j < 8; ++j) old[j] = (c + j < p.N) ? __bfloat162float(d[8 * q + j]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float a = v[8 * q + j];
+      switch (p.epi) {
+        case EPI_ADD: o[j] = old[j] + a; break;
+        case EPI_RELU2: { const float t = fmaxf(a, 0.f); o[j] = t * t; } break;
+        case EPI_DRELU2: o[j] = a * 2.f * sqrtf(old[j]); break;
+        case EPI_SOFTCAP: o[j] = softcap_fast(a); break;
+        default: o[j] = a; break;
+      }
+    }
+    if (full) Vec8<bf16>::store(d + 8 * q, o);
+    else
+      for (int j = 0; j < 8; ++j)
+        if (c + j < p.N) d[8 * q + j] = __float2bfloat16_rn(o[j]);
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * STAGES + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const Unit x = unit_of(p, u);
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          mbar_expect_tx(full_bar(stage), STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_2d(sa, &map_a, k0, x.m_blk * BM, full_bar(stage));
+          } else {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d(sa + i * 8192, &map_a, x.m_blk * BM + 64 * i, k0, full_bar(stage));
+          }
+          if (!p.b_mn) {
+            tma_load_2d(sb, &map_b, k0, x.n_blk * BN, full_bar(stage));
+          } else {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, &map_b, x.n_blk * BN + 64 * i, k0, full_bar(stage));
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // make sure no copy of ours is still landing before the CTA can exit:
+      // wait (bounded) on the last min(issued, STAGES) stages we filled
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(full_bar(stage), phase) && globaltimer() - t0 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc = make_idesc(p.a_mn, p.b_mn, BM, BN);
+      // descriptor offsets: K-major -> SBO 1 KB (8-row atoms), k step 32 B;
+      // MN-major -> LBO 8 KB (64-wide mn atoms), SBO 1 KB (8 k-rows), k step 2 KB
+      const uint32_t a_lbo = p.a_mn ? 8192 : 16, a_sbo = 1024, a_kstep = p.a_mn ? 2048 : 32;
+      const uint32_t b_lbo = p.b_mn ? 8192 : 16, b_sbo = 1024, b_kstep = p.b_mn ? 2048 : 32;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const Unit x = unit_of(p, u);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc(sa + kk * a_kstep, a_lbo, a_sbo);
+            const uint64_t bd = smem_desc(sb + kk * b_kstep, b_lbo, b_sbo);
+            tc_mma(d_tmem, ad, bd, idesc, (kb > x.kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // every MMA this thread issued has completed once the drain barrier flips
+      tc_commit(drain_bar);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 ----------------
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+      const Unit x = unit_of(p, u);
+      // every lane waits; the vote re-converges the warp for the .sync.aligned loads
+      const bool ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int m = x.m_blk * BM + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n = x.n_blk * BN + c * 32;
+        if (n >= p.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        if (m < p.M) epilogue_chunk(p, m, n, r);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------- host side -------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn &encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  return fn;
+}
+
+// 2D bf16 map over a row-major [rows, cols] matrix with row stride ld
+// elements; box = box_cols (innermost, 64 = 128 bytes) x box_rows.
+inline bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                     int box_cols, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split K over several units when the tile count would leave SMs idle:
+// choose the split count that best fills whole waves, with a small cost per
+// extra split (each split adds one fp32 reduction pass over the tile).
+inline int choose_splits(int tiles, int kblocks, int num_sms) {
+  if (tiles >= 2 * num_sms) return 1;
+  int best = 1;
+  double best_score = -1.0;
+  for (int s = 1; s <= 16; ++s) {
+    if (s > 1 && kblocks / s < 8) break;
+    const int units = tiles * s;
+    const int waves = (units + num_sms - 1) / num_sms;
+    const double eff = (double)units / (double)(waves * num_sms);
+    const double score = eff - 0.015 * (s - 1);
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = s;
+    }
+  }
+  return best;
+}
+
+}  // namespace tc
+
+inline cudaError_t tc_init() {
+  if (!tc::encode_fn()) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    tc::encode_fn() = reinterpret_cast<tc::EncodeTiledFn>(fn);
+  }
+  return cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              tc::SMEM_BYTES);
+}
+
+template <typename T>
+inline bool tc_gemm_supported(const GemmProblem &p) {
+  if (sizeof(T) != 2) return false;
+  if (p.M < 1 || p.N < 1 || p.K < 1) return false;
+  if ((p.lda % 8) || (p.ldb % 8)) return false;
+  if (((uintptr_t)p.A & 15) || ((uintptr_t)p.B & 15) || ((uintptr_t)p.D & 15)) return false;
+  if (p.epi == EPI_STORE_F32 ? (p.ldd % 4) : (p.ldd % 8)) return false;
+  return tc::encode_fn() != nullptr;
+}
+
+inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status, cudaStream_t st) {
+  using namespace tc;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (!g.a_mn) ok = make_map(&ma, g.A, g.M, g.K, g.lda, 64, BM);
+  else ok = make_map(&ma, g.A, g.K, g.M, g.lda, 64, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  if (!g.b_mn) ok = make_map(&mb, g.B, g.N, g.K, g.ldb, 64, BN);
+  else ok = make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  Params p;
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.n_m = (g.M + BM - 1) / BM;
+  p.n_n = (g.N + BN - 1) / BN;
+  p.kblocks = (g.K + BK - 1) / BK;
+  const int tiles = p.n_m * p.n_n;
+  p.splits = g.epi == EPI_STORE_F32 ? choose_splits(tiles, p.kblocks, num_sms) : 1;
+  {
+    // every split must own at least one k-block
+    const int per = (p.kblocks + p.splits - 1) / p.splits;
+    p.splits = (p.kblocks + per - 1) / per;
+  }
+  p.units = tiles * p.splits;
+  p.a_mn = g.a_mn; p.b_mn = g.b_mn;
+  p.D = g.D; p.ldd = g.ldd; p.epi = g.epi;
+  p.atomic_out = p.splits > 1;
+  p.status = status;
+  if (p.atomic_out) {
+    // fp32 partial sums are added into a zeroed output
+    cudaError_t e = cudaMemset2DAsync(g.D, (size_t)g.ldd * 4, 0, (size_t)g.N * 4, (size_t)g.M, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int grid = p.units < num_sms ? p.units : num_sms;
+  gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nc

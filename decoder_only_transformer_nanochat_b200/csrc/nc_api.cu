@@ -1,0 +1,538 @@
+// C ABI of the nanochat decoder step: argument checks, workspace carving and
+// the forward / backward launch sequence on the caller's stream.
+//
+// Model ("Nanochat: full-stack LLM training in 8,000 lines for $72", sections
+// "One dial controls everything" and "A Llama-class transformer with ten
+// modern departures"; energyai.berlin page, "Multi-Query Attention"):
+//   x = norm(wte[tok])
+//   per block l: xn = norm(x); [q|k|v] = xn [Wq;Wk;Wv]^T; q,k = norm(rope(q,k));
+//                O = causal attention; x += O Wo^T;
+//                xn2 = norm(x); a = relu(xn2 W1^T)^2; x += a W2^T
+//   xf = norm(x); z = xf Wout^T; s = 15 tanh(z/15); loss = mean CE(s, target)
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <chrono>
+#include <thread>
+#include <vector>
+
+#include "../../include/nanochat_b200.h"
+#include "../../include/nanochat_b200_ops.h"
+#include "attn_simt.cuh"
+#include "ce.cuh"
+#include "elementwise.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+
+using namespace nc;
+
+struct nc_model {
+  int depth, C, H, F, V, seq, dtype;
+  int64_t n_params;
+  int device;
+  int num_sms;
+  float *rope_cos;  // [seq, 64] fp32
+  float *rope_sin;
+  int *status;      // device status word
+  std::vector<nc_param> params;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+template <typename T>
+struct Work {
+  std::vector<T *> xn, qkv, O, xn2, a;
+  std::vector<float *> r1, rq, rk, lse, r2;
+  T *x, *xf, *z, *dxb, *dO, *dqkv;
+  float *r0, *rf, *tok_loss, *dx, *dy32, *Drow;
+  int64_t ldz;
+};
+
+// Lay the workspace out (base == nullptr only measures it).
+template <typename T>
+size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
+  const size_t M = (size_t)B * T_len;
+  const int C = m->C, H = m->H, F = m->F, L = m->depth;
+  const int64_t ldqkv = C + 2 * kHeadDim;
+  const int64_t ldz = ((int64_t)m->V + 63) / 64 * 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char * {
+    char *p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  const size_t es = sizeof(T);
+  if (w) {
+    w->xn.resize(L); w->qkv.resize(L); w->O.resize(L); w->xn2.resize(L); w->a.resize(L);
+    w->r1.resize(L); w->rq.resize(L); w->rk.resize(L); w->lse.resize(L); w->r2.resize(L);
+  }
+  for (int l = 0; l < L; ++l) {
+    T *xn = (T *)take(M * C * es);
+    float *r1 = (float *)take(M * 4);
+    T *qkv = (T *)take(M * ldqkv * es);
+    float *rq = (float *)take(M * H * 4);
+    float *rk = (float *)take(M * 4);
+    T *O = (T *)take(M * C * es);
+    float *lse = (float *)take(M * H * 4);
+    T *xn2 = (T *)take(M * C * es);
+    float *r2 = (float *)take(M * 4);
+    T *a = (T *)take(M * F * es);
+    if (w) {
+      w->xn[l] = xn; w->r1[l] = r1; w->qkv[l] = qkv; w->rq[l] = rq; w->rk[l] = rk;
+      w->O[l] = O; w->lse[l] = lse; w->xn2[l] = xn2; w->r2[l] = r2; w->a[l] = a;
+    }
+  }
+  T *x = (T *)take(M * C * es);
+  float *r0 = (float *)take(M * 4);
+  T *xf = (T *)take(M * C * es);
+  float *rf = (float *)take(M * 4);
+  T *z = (T *)take(M * ldz * es);
+  float *tok_loss = (float *)take(M * 4);
+  float *dx = (float *)take(M * C * 4);
+  T *dxb = (T *)take(M * C * es);
+  float *dy32 = (float *)take(M * C * 4);
+  T *dO = (T *)take(M * C * es);
+  T *dqkv = (T *)take(M * ldqkv * es);
+  float *Drow = (float *)take(M * H * 4);
+  if (w) {
+    w->x = x; w->r0 = r0; w->xf = xf; w->rf = rf; w->z = z; w->ldz = ldz;
+    w->tok_loss = tok_loss; w->dx = dx; w->dxb = dxb; w->dy32 = dy32; w->dO = dO;
+    w->dqkv = dqkv; w->Drow = Drow;
+  }
+  return off;
+}
+
+// Weight pointers of the flat buffer, layout order of nc_param_layout.
+template <typename T>
+struct Weights {
+  const T *wte, *lm_head;
+  std::vector<const T *> wqkv, wo, w1, w2;  // wq, wk, wv are contiguous: [C+256, C]
+};
+
+template <typename T>
+Weights<T> weight_ptrs(const nc_model *m, const void *weights) {
+  const T *base = (const T *)weights;
+  Weights<T> w;
+  w.wte = base + m->params[0].offset;
+  w.lm_head = base + m->params.back().offset;
+  for (int l = 0; l < m->depth; ++l) {
+    w.wqkv.push_back(base + m->params[1 + 6 * l].offset);
+    w.wo.push_back(base + m->params[1 + 6 * l + 3].offset);
+    w.w1.push_back(base + m->params[1 + 6 * l + 4].offset);
+    w.w2.push_back(base + m->params[1 + 6 * l + 5].offset);
+  }
+  return w;
+}
+
+#define NC_CHECK_LAUNCH()                              \
+  do {                                                 \
+    cudaError_t e_ = cudaGetLastError();               \
+    if (e_ != cudaSuccess) {                           \
+      fprintf(stderr, "nanochat_b200: %s at %s:%d\n",  \
+              cudaGetErrorString(e_), __FILE__, __LINE__); \
+      return NC_ECUDA;                                 \
+    }                                                  \
+  } while (0)
+
+template <typename T>
+int gemm(const nc_model *m, const GemmProblem &p, cudaStream_t st) {
+  if (p.M <= 0 || p.N <= 0) return NC_OK;
+  cudaError_t e;
+  if (tc_gemm_supported<T>(p)) e = launch_gemm_tc(p, m->num_sms, m->status, st);
+  else e = launch_gemm_simt<T>(p, st);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nanochat_b200: gemm launch: %s\n", cudaGetErrorString(e));
+    return NC_ECUDA;
+  }
+  return NC_OK;
+}
+
+inline GemmProblem gp(int M, int N, int K, const void *A, int64_t lda, int a_mn, const void *B,
+                      int64_t ldb, int b_mn, void *D, int64_t ldd, int epi) {
+  GemmProblem p;
+  p.M = M; p.N = N; p.K = K; p.A = A; p.lda = lda; p.a_mn = a_mn; p.B = B; p.ldb = ldb;
+  p.b_mn = b_mn; p.D = D; p.ldd = ldd; p.epi = epi;
+  return p;
+}
+
+inline unsigned rows_grid(size_t rows, int rows_per_block) {
+  return (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+}
+
+#define NC_TRY(x)              \
+  do {                         \
+    int rc_ = (x);             \
+    if (rc_ != NC_OK) return rc_; \
+  } while (0)
+
+// Forward through the blocks and the final norm; leaves xf, rf in the workspace.
+template <typename T>
+int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B, int T_len,
+                 Work<T> &w, cudaStream_t st) {
+  const int M = B * T_len, C = m->C, H = m->H, F = m->F;
+  const int ldqkv = C + 2 * kHeadDim;
+  NC_DISPATCH_NV(C, (embed_norm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                        tokens, W.wte, w.x, w.r0, M, C, m->V, m->status)));
+  NC_CHECK_LAUNCH();
+  for (int l = 0; l < m->depth; ++l) {
+    NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xn[l],
+                                                                               w.r1[l], M, C)));
+    NC_CHECK_LAUNCH();
+    NC_TRY(gemm<T>(m, gp(M, ldqkv, C, w.xn[l], C, 0, W.wqkv[l], C, 0, w.qkv[l], ldqkv, EPI_STORE), st));
+    rope_qknorm_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+        w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H);
+    NC_CHECK_LAUNCH();
+    if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0, st) !=
+        cudaSuccess)
+      return NC_ECUDA;
+    NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, w.x, C, EPI_ADD), st));
+    NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xn2[l],
+                                                                               w.r2[l], M, C)));
+    NC_CHECK_LAUNCH();
+    NC_TRY(gemm<T>(m, gp(M, F, C, w.xn2[l], C, 0, W.w1[l], C, 0, w.a[l], F, EPI_RELU2), st));
+    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w2[l], F, 0, w.x, C, EPI_ADD), st));
+  }
+  NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xf, w.rf, M, C)));
+  NC_CHECK_LAUNCH();
+  return NC_OK;
+}
+
+template <typename T>
+int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const int32_t *targets,
+                 int B, int T_len, void *workspace, float *loss, float *token_loss, float *grads,
+                 cudaStream_t st) {
+  Work<T> w;
+  carve<T>(m, B, T_len, (char *)workspace, &w);
+  const Weights<T> W = weight_ptrs<T>(m, weights);
+  const int M = B * T_len, C = m->C, H = m->H, F = m->F, V = m->V;
+  const int ldqkv = C + 2 * kHeadDim;
+  NC_TRY(forward_body<T>(m, W, tokens, B, T_len, w, st));
+
+  // head: z = xf Wout^T, then softcap + CE forward and backward in place
+  NC_TRY(gemm<T>(m, gp(M, V, C, w.xf, C, 0, W.lm_head, C, 0, w.z, w.ldz, EPI_STORE), st));
+  float *tl = token_loss ? token_loss : w.tok_loss;
+  const float inv_M = 1.f / (float)M;
+  if (sizeof(T) == 2 && V == 65536) {
+    ce_fused_bf16_kernel<16><<<M, 512, 0, st>>>((bf16 *)w.z, w.ldz, targets, tl, M, V, inv_M,
+                                                m->status);
+  } else {
+    ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(w.z, w.ldz, targets, tl, M, V, inv_M, m->status);
+  }
+  NC_CHECK_LAUNCH();
+  loss_mean_kernel<<<1, 1024, 0, st>>>(tl, M, loss, m->status);
+  NC_CHECK_LAUNCH();
+
+  // gradient pointers (fp32, same layout as the weights)
+  auto G = [&](int idx) { return grads + m->params[idx].offset; };
+  const int last = (int)m->params.size() - 1;
+  // dWout = dz^T xf ;  dxf = dz Wout
+  NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, EPI_STORE_F32), st));
+  NC_TRY(gemm<T>(m, gp(M, C, V, w.z, w.ldz, 0, W.lm_head, C, 1, w.dy32, C, EPI_STORE_F32), st));
+  NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                        w.dy32, w.xf, w.rf, w.dx, w.dxb, M, C, 0)));
+  NC_CHECK_LAUNCH();
+
+  for (int l = m->depth - 1; l >= 0; --l) {
+    const int pi = 1 + 6 * l;
+    // MLP: x += a W2^T, a = relu(h)^2, h = xn2 W1^T
+    NC_TRY(gemm<T>(m, gp(C, F, M, w.dxb, C, 1, w.a[l], F, 1, G(pi + 5), F, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, F, C, w.dxb, C, 0, W.w2[l], F, 1, w.a[l], F, EPI_DRELU2), st));
+    NC_TRY(gemm<T>(m, gp(F, C, M, w.a[l], F, 1, w.xn2[l], C, 1, G(pi + 4), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w1[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
+    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                          w.dy32, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1)));
+    NC_CHECK_LAUNCH();
+    // attention: x += O Wo^T
+    NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
+    attn_rowdot_kernel<T><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>(w.dO, w.O[l], w.Drow, M,
+                                                                         T_len, H);
+    NC_CHECK_LAUNCH();
+    if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
+                           m->num_sms, 0, st) != cudaSuccess)
+      return NC_ECUDA;
+    rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+        w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H);
+    NC_CHECK_LAUNCH();
+    // [q|k|v] = xn [Wq;Wk;Wv]^T
+    NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
+    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                          w.dy32, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1)));
+    NC_CHECK_LAUNCH();
+  }
+  // embedding: through the first norm, summed into the selected rows
+  if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
+  NC_DISPATCH_NV(C, (embed_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                        w.dx, tokens, W.wte, w.r0, G(0), M, C, V)));
+  NC_CHECK_LAUNCH();
+  return NC_OK;
+}
+
+template <typename T>
+int fwd_impl(nc_model *m, const void *weights, const int32_t *tokens, int B, int T_len,
+             void *workspace, void *logits, cudaStream_t st) {
+  Work<T> w;
+  carve<T>(m, B, T_len, (char *)workspace, &w);
+  const Weights<T> W = weight_ptrs<T>(m, weights);
+  const int M = B * T_len;
+  NC_TRY(forward_body<T>(m, W, tokens, B, T_len, w, st));
+  return gemm<T>(m, gp(M, m->V, m->C, w.xf, m->C, 0, W.lm_head, m->C, 0, logits, m->V, EPI_SOFTCAP), st);
+}
+
+int check_step_args(const nc_model *m, const void *weights, const int32_t *tokens, int B, int T,
+                    void *workspace, size_t ws_bytes) {
+  if (!m || !weights || !tokens || !workspace) return NC_EINVAL;
+  if (B < 1 || T < 1 || T > m->seq) return NC_ESHAPE;
+  if ((int64_t)B * T > (int64_t)1 << 30) return NC_ESHAPE;
+  size_t need = 0;
+  need = m->dtype == NC_F32 ? carve<float>(m, B, T, nullptr, nullptr)
+                            : carve<bf16>(m, B, T, nullptr, nullptr);
+  if (ws_bytes < need) return NC_ENOMEM;
+  if (((uintptr_t)weights & 15) || ((uintptr_t)workspace & (kAlign - 1)) || ((uintptr_t)tokens & 3))
+    return NC_EALIGN;
+  return NC_OK;
+}
+
+
+int op_device_sms(int *num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
+  if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
+  if (tc_init() != cudaSuccess) return NC_ECUDA;
+  return NC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
+  if (!out) return NC_EINVAL;
+  *out = nullptr;
+  if (depth < 1 || vocab < 2 || seq < 1) return NC_EINVAL;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  const int C = kHeadDim * ((64 * depth + kHeadDim - 1) / kHeadDim);
+  if (C > 32 * kMaxVecPerLane * 8) return NC_EINVAL;  // widest row the row kernels hold
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return NC_ECUDA;
+  if (prop.major != 10) return NC_EUNSUPPORTED;
+
+  nc_model *m = new nc_model();
+  m->depth = depth; m->C = C; m->H = C / kHeadDim; m->F = 4 * C; m->V = vocab; m->seq = seq;
+  m->dtype = dtype; m->device = dev; m->num_sms = prop.multiProcessorCount;
+  int64_t off = 0;
+  auto add = [&](const char *name, int rows, int cols) {
+    nc_param p;
+    memset(&p, 0, sizeof(p));
+    snprintf(p.name, sizeof(p.name), "%s", name);
+    p.offset = off; p.rows = rows; p.cols = cols;
+    off += (int64_t)rows * cols;
+    m->params.push_back(p);
+  };
+  add("wte", vocab, C);
+  char nm[24];
+  for (int l = 0; l < depth; ++l) {
+    snprintf(nm, sizeof(nm), "h%d.wq", l); add(nm, C, C);
+    snprintf(nm, sizeof(nm), "h%d.wk", l); add(nm, kHeadDim, C);
+    snprintf(nm, sizeof(nm), "h%d.wv", l); add(nm, kHeadDim, C);
+    snprintf(nm, sizeof(nm), "h%d.wo", l); add(nm, C, C);
+    snprintf(nm, sizeof(nm), "h%d.w1", l); add(nm, 4 * C, C);
+    snprintf(nm, sizeof(nm), "h%d.w2", l); add(nm, C, 4 * C);
+  }
+  add("lm_head", vocab, C);
+  m->n_params = off;
+
+  // RoPE table: angle = pos * 10000^(-i/64), built in float64, rounded once.
+  std::vector<float> hc((size_t)seq * 64), hs((size_t)seq * 64);
+  for (int p = 0; p < seq; ++p)
+    for (int i = 0; i < 64; ++i) {
+      const double ang = (double)p * pow(10000.0, -(double)i / 64.0);
+      hc[(size_t)p * 64 + i] = (float)cos(ang);
+      hs[(size_t)p * 64 + i] = (float)sin(ang);
+    }
+  bool ok = cudaMalloc(&m->rope_cos, hc.size() * 4) == cudaSuccess &&
+            cudaMalloc(&m->rope_sin, hs.size() * 4) == cudaSuccess &&
+            cudaMalloc(&m->status, 256) == cudaSuccess &&
+            cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemset(m->status, 0, 256) == cudaSuccess;
+  if (!ok || tc_init() != cudaSuccess) {
+    nc_destroy(m);
+    return NC_ECUDA;
+  }
+  *out = m;
+  return NC_OK;
+}
+
+int nc_get_dims(const nc_model *m, nc_dims *out) {
+  if (!m || !out) return NC_EINVAL;
+  out->depth = m->depth; out->width = m->C; out->n_head = m->H; out->head_dim = kHeadDim;
+  out->hidden = m->F; out->vocab = m->V; out->seq = m->seq; out->dtype = m->dtype;
+  out->n_params = m->n_params;
+  return NC_OK;
+}
+
+int nc_param_layout(const nc_model *m, int index, nc_param *out) {
+  if (!m || !out || index < 0 || index >= (int)m->params.size()) return NC_EINVAL;
+  *out = m->params[index];
+  return NC_OK;
+}
+
+int nc_workspace_bytes(const nc_model *m, int B, int T, size_t *out) {
+  if (!m || !out) return NC_EINVAL;
+  if (B < 1 || T < 1 || T > m->seq) return NC_ESHAPE;
+  *out = m->dtype == NC_F32 ? carve<float>(m, B, T, nullptr, nullptr)
+                            : carve<bf16>(m, B, T, nullptr, nullptr);
+  return NC_OK;
+}
+
+int nc_fwd_bwd(nc_model *m, const void *weights, const int32_t *tokens, const int32_t *targets,
+               int B, int T, void *workspace, size_t ws_bytes, float *loss, float *token_loss,
+               float *grads, void *stream) {
+  int rc = check_step_args(m, weights, tokens, B, T, workspace, ws_bytes);
+  if (rc != NC_OK) return rc;
+  if (!targets || !loss || !grads) return NC_EINVAL;
+  if (((uintptr_t)grads & 15) || ((uintptr_t)targets & 3) || ((uintptr_t)loss & 3)) return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->dtype == NC_F32)
+    return fwd_bwd_impl<float>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, st);
+  return fwd_bwd_impl<bf16>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, st);
+}
+
+int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B, int T, void *workspace,
+           size_t ws_bytes, void *logits, void *stream) {
+  int rc = check_step_args(m, weights, tokens, B, T, workspace, ws_bytes);
+  if (rc != NC_OK) return rc;
+  if (!logits) return NC_EINVAL;
+  if ((uintptr_t)logits & 15) return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->dtype == NC_F32) return fwd_impl<float>(m, weights, tokens, B, T, workspace, logits, st);
+  return fwd_impl<bf16>(m, weights, tokens, B, T, workspace, logits, st);
+}
+
+int nc_sync_status(nc_model *m, void *stream, int timeout_ms) {
+  if (!m) return NC_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaEvent_t ev;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return NC_ECUDA;
+  if (cudaEventRecord(ev, st) != cudaSuccess) {
+    cudaEventDestroy(ev);
+    return NC_ECUDA;
+  }
+  const auto t0 = std::chrono::steady_clock::now();
+  cudaError_t q;
+  while ((q = cudaEventQuery(ev)) == cudaErrorNotReady) {
+    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                        std::chrono::steady_clock::now() - t0).count();
+    if (ms >= timeout_ms) {
+      cudaEventDestroy(ev);
+      return NC_ETIMEOUT;
+    }
+    std::this_thread::sleep_for(std::chrono::microseconds(100));
+  }
+  cudaEventDestroy(ev);
+  if (q != cudaSuccess) return NC_ECUDA;
+  int word = 0;
+  if (cudaMemcpyAsync(&word, m->status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(m->status, 0, sizeof(int), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return NC_ECUDA;
+  if (word & kStatusRange) return NC_ERANGE;
+  if (word & kStatusNonFinite) return NC_ENONFINITE;
+  if (word & kStatusTimeout) return NC_ETIMEOUT;
+  return NC_OK;
+}
+
+const char *nc_strerror(int code) {
+  switch (code) {
+    case NC_OK: return "ok";
+    case NC_EINVAL: return "invalid argument";
+    case NC_ESHAPE: return "invalid shape (B < 1, T < 1 or T > seq)";
+    case NC_ENOMEM: return "workspace too small";
+    case NC_EUNSUPPORTED: return "unsupported device or dtype (needs sm_100)";
+    case NC_ECUDA: return "CUDA runtime error";
+    case NC_ERANGE: return "token or target id outside [0, vocab)";
+    case NC_ENONFINITE: return "non-finite loss";
+    case NC_ETIMEOUT: return "timed out";
+    case NC_EALIGN: return "misaligned device pointer";
+    default: return "unknown status";
+  }
+}
+
+void nc_destroy(nc_model *m) {
+  if (!m) return;
+  if (m->rope_cos) cudaFree(m->rope_cos);
+  if (m->rope_sin) cudaFree(m->rope_sin);
+  if (m->status) cudaFree(m->status);
+  delete m;
+}
+
+
+int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, int b_mn, void *D,
+            int64_t ldd, int M, int N, int K, int dtype, int epilogue, int engine, void *stream) {
+  if (!A || !B || !D) return NC_EINVAL;
+  if (M < 1 || N < 1 || K < 1) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (epilogue < NC_EPI_STORE || epilogue > NC_EPI_SOFTCAP || (a_mn | b_mn) & ~1) return NC_EINVAL;
+  int num_sms = 0;
+  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  const GemmProblem p = gp(M, N, K, A, lda, a_mn, B, ldb, b_mn, D, ldd, epilogue);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dtype == NC_BF16) {
+    if (engine == 0 && tc_gemm_supported<bf16>(p)) e = launch_gemm_tc(p, num_sms, nullptr, st);
+    else e = launch_gemm_simt<bf16>(p, st);
+  } else {
+    e = launch_gemm_simt<float>(p, st);
+  }
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
+                     int dtype, int engine, void *stream) {
+  if (!qkv || !O || !lse) return NC_EINVAL;
+  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
+  int num_sms = 0;
+  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dtype == NC_BF16)
+    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, num_sms, engine, st);
+  else if (dtype == NC_F32)
+    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, num_sms, engine, st);
+  else
+    return NC_EUNSUPPORTED;
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
+                     float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                     void *stream) {
+  if (!qkv || !O || !dO || !lse || !Drow || !dqkv) return NC_EINVAL;
+  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
+  int num_sms = 0;
+  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int M = B * T;
+  cudaError_t e;
+  if (dtype == NC_BF16) {
+    attn_rowdot_kernel<bf16><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const bf16 *)dO, (const bf16 *)O, Drow, M, T, H);
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms, engine, st);
+  } else if (dtype == NC_F32) {
+    attn_rowdot_kernel<float><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const float *)dO, (const float *)O, Drow, M, T, H);
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H, num_sms, engine, st);
+  } else {
+    return NC_EUNSUPPORTED;
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+}  // extern "C"

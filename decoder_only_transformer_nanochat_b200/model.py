@@ -1,0 +1,81 @@
+"""Convenience wrapper over the C ABI that uses PyTorch only for device memory
+and the current CUDA stream.  Every computation is done by the CUDA library."""
+from __future__ import annotations
+
+import torch
+
+from . import _binding as B
+
+
+class Model:
+    """One nanochat decoder of the given depth (one dial: width = depth*64,
+    heads = width/128) on the current CUDA device."""
+
+    def __init__(self, depth: int, vocab: int = 65536, seq: int = 2048, dtype: str = "bf16"):
+        self.dtype_code = B.NC_BF16 if dtype == "bf16" else B.NC_F32
+        self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        rc, self.handle = B.nc_init(depth, vocab, seq, self.dtype_code)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_init")
+        rc, self.dims = B.nc_get_dims(self.handle)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_get_dims")
+        self.layout = []
+        for i in range(2 + 6 * depth):
+            rc, p = B.nc_param_layout(self.handle, i)
+            if rc != B.NC_OK:
+                raise B.NcError(rc, "nc_param_layout")
+            self.layout.append(p)
+        self.n_params = self.dims["n_params"]
+        self._ws = None
+        self._ws_key = None
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            B.nc_destroy(h)
+            self.handle = None
+
+    def workspace(self, Bsz: int, T: int) -> torch.Tensor:
+        rc, n = B.nc_workspace_bytes(self.handle, Bsz, T)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_workspace_bytes")
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = None
+            self._ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+        return self._ws
+
+    @staticmethod
+    def _stream():
+        return torch.cuda.current_stream().cuda_stream
+
+    def fwd_bwd(self, weights: torch.Tensor, tokens: torch.Tensor, targets: torch.Tensor,
+                grads: torch.Tensor | None = None, loss: torch.Tensor | None = None,
+                token_loss: torch.Tensor | None = None):
+        Bsz, T = tokens.shape
+        ws = self.workspace(Bsz, T)
+        if grads is None:
+            grads = torch.empty(self.n_params, dtype=torch.float32, device="cuda")
+        if loss is None:
+            loss = torch.empty(1, dtype=torch.float32, device="cuda")
+        rc = B.nc_fwd_bwd(self.handle, weights.data_ptr(), tokens.data_ptr(), targets.data_ptr(),
+                          Bsz, T, ws.data_ptr(), ws.numel(), loss.data_ptr(),
+                          token_loss.data_ptr() if token_loss is not None else None,
+                          grads.data_ptr(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_fwd_bwd")
+        return loss, grads
+
+    def fwd(self, weights: torch.Tensor, tokens: torch.Tensor, logits: torch.Tensor | None = None):
+        Bsz, T = tokens.shape
+        ws = self.workspace(Bsz, T)
+        if logits is None:
+            logits = torch.empty(Bsz, T, self.dims["vocab"], dtype=self.torch_dtype, device="cuda")
+        rc = B.nc_fwd(self.handle, weights.data_ptr(), tokens.data_ptr(), Bsz, T, ws.data_ptr(),
+                      ws.numel(), logits.data_ptr(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_fwd")
+        return logits
+
+    def sync_status(self, timeout_ms: int = 60000) -> int:
+        return B.nc_sync_status(self.handle, self._stream(), timeout_ms)

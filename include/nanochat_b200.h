@@ -1,0 +1,145 @@
+/*
+ * nanochat_b200.h -- C ABI of one training step (forward + backward) of the
+ * nanochat depth-parameterised GPT decoder on an NVIDIA B200 (sm_100a).
+ *
+ * The model is the one the nanochat pages describe:
+ *   - one dial: width C = depth*64 (snapped up to a multiple of 128), C/128
+ *     query heads of dim 128, depth blocks ("Nanochat: full-stack LLM training
+ *     in 8,000 lines for $72", section "One dial controls everything"; "nanochat
+ *     - full-stack ChatGPT in ~8k lines", section "2. Pretrain");
+ *   - parameterless RMSNorm after the embedding, before attention, before the
+ *     MLP and before the head; RoPE with theta 10,000; QK-norm after RoPE;
+ *     causal softmax attention; relu^2 MLP at 4x width; logit softcap
+ *     15*tanh(z/15) in fp32; untied embedding / unembedding (first page,
+ *     section "A Llama-class transformer with ten modern departures");
+ *   - one key/value head shared by all query heads (energyai.berlin page,
+ *     section "Multi-Query Attention (MQA)");
+ *   - the loss is the mean over all B*T positions of the token cross-entropy.
+ *
+ * Conventions
+ *   - All pointers named "device" are CUDA device pointers on the current
+ *     device; the caller owns every buffer passed in (weights, tokens,
+ *     targets, workspace, loss, gradients, logits).  The library owns only its
+ *     handle, a RoPE cos/sin table and a small device status word.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every compute call only enqueues work on that stream: it never
+ *     synchronises the host and never allocates device memory.
+ *   - Weight layout: one flat buffer in the model dtype (fp32 or bf16), each
+ *     matrix [out, in] row-major (y = x W^T), in this order:
+ *       wte[V,C]; per layer l: wq[C,C], wk[128,C], wv[128,C], wo[C,C],
+ *       w1[4C,C], w2[C,4C]; lm_head[V,C].
+ *     nc_param_layout() returns each tensor's name, element offset and shape.
+ *   - Gradients are fp32 in the same layout and are overwritten by each call.
+ *   - Errors: every function returns an nc_status.  Argument errors are
+ *     detected on the host before anything is enqueued.  Problems that only
+ *     the device can see (a token id outside [0, vocab), a non-finite loss, a
+ *     kernel wait that ran out of time) set the device status word, which
+ *     nc_sync_status() reads and clears.
+ */
+#ifndef NANOCHAT_B200_H
+#define NANOCHAT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NC_OK = 0,
+  NC_EINVAL = 1,        /* null pointer, depth < 1, vocab < 2, seq < 1, bad index */
+  NC_ESHAPE = 2,        /* B < 1, T < 1 or T > seq */
+  NC_ENOMEM = 3,        /* workspace smaller than nc_workspace_bytes() */
+  NC_EUNSUPPORTED = 4,  /* current device is not sm_100, or unknown dtype */
+  NC_ECUDA = 5,         /* a CUDA runtime call failed (launch, memcpy, event) */
+  NC_ERANGE = 6,        /* device: a token or target id outside [0, vocab) */
+  NC_ENONFINITE = 7,    /* device: the loss came out NaN or infinite */
+  NC_ETIMEOUT = 8,      /* nc_sync_status ran out of time, or a kernel wait expired */
+  NC_EALIGN = 9         /* a device pointer is not 16-byte aligned */
+} nc_status;
+
+/* Compute dtype, mirroring the pages' single COMPUTE_DTYPE switch
+ * (aimarketly.com copy of the nanochat README, "Precision / dtype"):
+ * NC_F32 stores and computes everything in fp32; NC_BF16 stores weights,
+ * activations and logits in bf16 and accumulates every reduction in fp32. */
+typedef enum { NC_F32 = 0, NC_BF16 = 1 } nc_dtype;
+
+typedef struct nc_model nc_model;
+
+typedef struct {
+  int depth;      /* number of blocks L */
+  int width;      /* C */
+  int n_head;     /* query heads H = C / 128 */
+  int head_dim;   /* 128 */
+  int hidden;     /* MLP hidden width F = 4C */
+  int vocab;      /* V */
+  int seq;        /* longest T accepted */
+  int dtype;      /* nc_dtype */
+  int64_t n_params;
+} nc_dims;
+
+typedef struct {
+  char name[24];    /* "wte", "h<l>.wq", ..., "lm_head" */
+  int64_t offset;   /* element offset in the flat weight / gradient buffer */
+  int rows, cols;
+} nc_param;
+
+/* Create a model handle for the current CUDA device.  depth >= 1 sets every
+ * shape (one dial); vocab >= 2; seq >= 1 is the longest sequence T accepted.
+ * Builds the RoPE table (theta 10,000) for positions [0, seq) on the host in
+ * float64, rounds it to fp32 once and uploads it.  Returns NC_EUNSUPPORTED on
+ * a device that is not compute capability 10.x.  *out receives the handle. */
+int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out);
+
+/* Shapes of the model. */
+int nc_get_dims(const nc_model *m, nc_dims *out);
+
+/* Name, offset and shape of weight tensor `index`, 0 <= index < 2 + 6*depth,
+ * in storage order. */
+int nc_param_layout(const nc_model *m, int index, nc_param *out);
+
+/* Bytes of device workspace that nc_fwd_bwd / nc_fwd need for B rows of T
+ * tokens.  The workspace holds every saved activation and scratch tensor. */
+int nc_workspace_bytes(const nc_model *m, int B, int T, size_t *out);
+
+/* One training step: loss and the gradient of the loss with respect to every
+ * weight.
+ *   weights    device, n_params elements of the model dtype, layout above
+ *   tokens     device int32 [B,T], ids in [0, vocab)
+ *   targets    device int32 [B,T], ids in [0, vocab)
+ *   workspace  device, ws_bytes >= nc_workspace_bytes(B, T), 256-byte aligned
+ *   loss       device fp32 [1]: mean over B*T positions of
+ *              logsumexp(s_i) - s_i[target_i], s = 15 tanh(z/15)
+ *   token_loss device fp32 [B,T] per-position losses, or NULL
+ *   grads      device fp32 [n_params], overwritten
+ * Out-of-range ids are clamped for addressing and flagged NC_ERANGE. */
+int nc_fwd_bwd(nc_model *m, const void *weights, const int32_t *tokens,
+               const int32_t *targets, int B, int T, void *workspace,
+               size_t ws_bytes, float *loss, float *token_loss, float *grads,
+               void *stream);
+
+/* Forward only: softcapped logits s = 15 tanh(z/15) of every position.
+ *   logits  device [B,T,vocab] in the model dtype (row-major, vocab fastest)
+ * Other arguments as nc_fwd_bwd. */
+int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B,
+           int T, void *workspace, size_t ws_bytes, void *logits, void *stream);
+
+/* Wait at most timeout_ms for the work enqueued so far on `stream` to finish
+ * (polling, never blocking longer), then read and clear the device status
+ * word.  Returns NC_ETIMEOUT if the stream is still busy, else the first
+ * device-side error recorded (NC_ERANGE, NC_ENONFINITE, NC_ETIMEOUT) or NC_OK. */
+int nc_sync_status(nc_model *m, void *stream, int timeout_ms);
+
+/* Static string for a status code. */
+const char *nc_strerror(int code);
+
+/* Free the handle and the memory it owns.  The caller must make sure no work
+ * that uses it is still running. */
+void nc_destroy(nc_model *m);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NANOCHAT_B200_H */

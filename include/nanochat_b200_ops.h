@@ -1,0 +1,73 @@
+/*
+ * nanochat_b200_ops.h -- op-level entry points of libnanochat_b200.so: the
+ * dense contractions and the attention of the decoder step, exposed on their
+ * own so each kernel can be checked and timed in isolation.  nc_fwd_bwd
+ * (nanochat_b200.h) runs the same kernels.
+ *
+ * Same conventions as nanochat_b200.h: device pointers owned by the caller,
+ * work enqueued on `stream` (a cudaStream_t as void*), no host sync, no
+ * device allocation, nc_status return codes.
+ */
+#ifndef NANOCHAT_B200_OPS_H
+#define NANOCHAT_B200_OPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "nanochat_b200.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues fused into the GEMM (the element-wise steps that follow each
+ * projection of the block, "A Llama-class transformer with ten modern
+ * departures"):
+ *   NC_EPI_STORE      D = acc                (D in dtype)
+ *   NC_EPI_STORE_F32  D = acc                (D fp32)
+ *   NC_EPI_ADD        D = D + acc            (residual add; D in dtype)
+ *   NC_EPI_RELU2      D = relu(acc)^2        (relu^2 MLP activation)
+ *   NC_EPI_DRELU2     D = acc * 2 sqrt(D)    (its backward: D holds relu(h)^2)
+ *   NC_EPI_SOFTCAP    D = 15 tanh(acc / 15)  (logit softcap) */
+enum {
+  NC_EPI_STORE = 0,
+  NC_EPI_STORE_F32 = 1,
+  NC_EPI_ADD = 2,
+  NC_EPI_RELU2 = 3,
+  NC_EPI_DRELU2 = 4,
+  NC_EPI_SOFTCAP = 5
+};
+
+/* D[m,n] = epilogue(sum_k A(m,k) B(n,k)), fp32 accumulation.
+ *   A(m,k) = A[m*lda + k] if a_mn == 0 (K-major) else A[k*lda + m] (MN-major)
+ *   B(n,k) = B[n*ldb + k] if b_mn == 0 else B[k*ldb + n]
+ *   D[m,n] = D[m*ldd + n]
+ * dtype (nc_dtype) is the type of A, B and of D unless NC_EPI_STORE_F32.
+ * engine: 0 = the path nc_fwd_bwd takes (tcgen05 tensor cores for bf16
+ * operands whose strides are multiples of 8 elements and pointers 16-byte
+ * aligned, CUDA cores otherwise), 1 = force the CUDA-core kernel.
+ * M, N, K >= 1. */
+int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, int b_mn, void *D,
+            int64_t ldd, int M, int N, int K, int dtype, int epilogue, int engine, void *stream);
+
+/* Causal multi-query attention forward (energyai.berlin page, "Multi-Query
+ * Attention (MQA)": one key/value head shared by the H query heads).
+ *   qkv  device [B*T, ld] rows [q (H*128) | k (128) | v (128)], ld >= 128*(H+2)
+ *   O    device [B*T, H*128]: O_h = softmax(q_h k^T / sqrt(128) + causal) v
+ *   lse  device fp32 [B, H, T]: log-sum-exp of each score row
+ * engine: 0 = the path nc_fwd_bwd takes, 1 = force the CUDA-core kernel. */
+int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
+                     int dtype, int engine, void *stream);
+
+/* Its backward.  dO [B*T, H*128] and O as above, lse from the forward.
+ *   Drow  device fp32 [B, H, T] scratch, receives rowsum(dO * O)
+ *   dqkv  device [B*T, ld]: dq per head; dk, dv summed over the query heads */
+int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
+                     float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                     void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NANOCHAT_B200_OPS_H */

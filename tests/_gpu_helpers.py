@@ -1,0 +1,80 @@
+"""Shared pieces of the GPU parity tests: run the CUDA step through the C ABI
+on seeded inputs and compare it with the fp64 oracle on the same inputs."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+
+# tolerances of the two precisions
+F32_LOSS_REL = 1e-5          # |dloss| / |loss|
+F32_GRAD_MAXABS = 1e-4       # per tensor: max|dg| <= 1e-4 * max|g|
+BF16_LOSS_ABS = 1e-2         # |dloss|
+BF16_GRAD_COS = 0.999        # per tensor cosine similarity
+
+
+def to_device(flat: np.ndarray, dtype: str):
+    import torch
+    if dtype == "f32":
+        return torch.from_numpy(flat).cuda()
+    return torch.from_numpy(flat.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def make_case(depth, V, B, T, dtype, seed, dist, std_override=None):
+    lay = oracle.param_layout(depth, V)
+    flat, W = synth.make_weights(lay, seed, dtype, std_override=std_override)
+    tok, tgt = synth.token_rows(seed, B, T, V, dist)
+    return lay, flat, W, tok, tgt
+
+
+def gpu_step(model, flat, tok, tgt, dtype):
+    import torch
+    w = to_device(flat, dtype)
+    t = torch.from_numpy(tok).cuda()
+    g = torch.from_numpy(tgt).cuda()
+    tl = torch.empty(tok.shape, dtype=torch.float32, device="cuda")
+    loss, grads = model.fwd_bwd(w, t, g, token_loss=tl)
+    rc = model.sync_status(120000)
+    torch.cuda.synchronize()
+    return rc, float(loss.item()), tl.cpu().numpy().astype(np.float64), grads.cpu().numpy().astype(np.float64)
+
+
+def split_grads(grads_flat, lay):
+    out, off = {}, 0
+    for name, r, c in lay:
+        out[name] = grads_flat[off:off + r * c].reshape(r, c)
+        off += r * c
+    return out
+
+
+def cosine(a, b):
+    na, nb = np.linalg.norm(a), np.linalg.norm(b)
+    if na == 0 and nb == 0:
+        return 1.0
+    return float(np.sum(a * b) / (na * nb))
+
+
+def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_ref=None):
+    """Assert the precision's tolerances; return a per-tensor report."""
+    g_gpu = split_grads(g_gpu_flat, lay)
+    report = {}
+    if dtype == "f32":
+        assert abs(loss_gpu - loss_ref) <= F32_LOSS_REL * abs(loss_ref), (loss_gpu, loss_ref)
+        for name, _, _ in lay:
+            ref = g_ref[name]
+            err = np.max(np.abs(g_gpu[name] - ref))
+            scale = np.max(np.abs(ref))
+            report[name] = err / scale if scale > 0 else err
+            assert err <= F32_GRAD_MAXABS * scale, (name, err, scale)
+        if tl_gpu is not None:
+            np.testing.assert_allclose(tl_gpu, tl_ref, rtol=1e-5, atol=1e-5)
+    else:
+        assert abs(loss_gpu - loss_ref) <= BF16_LOSS_ABS, (loss_gpu, loss_ref)
+        for name, _, _ in lay:
+            c = cosine(g_gpu[name], g_ref[name])
+            report[name] = c
+            assert c >= BF16_GRAD_COS, (name, c)
+        if tl_gpu is not None:
+            assert np.max(np.abs(tl_gpu - tl_ref)) <= 0.05
+    return report

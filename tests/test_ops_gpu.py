@@ -1,0 +1,205 @@
+"""Kernel-level parity through the op entry points (nanochat_b200_ops.h):
+the GEMM with every operand layout and fused epilogue, and causal MQA
+attention forward / backward, each against a float64 CPU reference computed
+from the same (bf16-rounded) inputs."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nc():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from decoder_only_transformer_nanochat_b200 import build
+    build.build()
+    import decoder_only_transformer_nanochat_b200 as m
+    return m
+
+
+def _bf16(x):
+    return synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(x.astype(np.float32)))
+
+
+def _dev(x, dtype):
+    import torch
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(np.ascontiguousarray(x, dtype=np.float32))
+        return torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+def _stored(logical, mn, pad):
+    """Storage of a logical [rows, K] operand: K-major rows (ld = K + pad) or
+    MN-major [K, rows] (ld = rows + pad)."""
+    rows, K = logical.shape
+    if not mn:
+        s = np.zeros((rows, K + pad))
+        s[:, :K] = logical
+        return s, K + pad
+    s = np.zeros((K, rows + pad))
+    s[:, :rows] = logical.T
+    return s, rows + pad
+
+
+EPIS = ["STORE", "STORE_F32", "ADD", "RELU2", "DRELU2", "SOFTCAP"]
+
+GEMM_CASES = [
+    # M, N, K, a_mn, b_mn, pad
+    (256, 512, 128, 0, 0, 0),
+    (300, 520, 200, 0, 0, 8),      # ragged M, N, K (zero-filled tails)
+    (384, 1280, 1280, 0, 1, 0),    # input-gradient layout
+    (1280, 768, 640, 1, 1, 0),     # weight-gradient layout
+    (200, 264, 72, 1, 1, 8),       # ragged weight-gradient layout
+    (130, 300, 96, 1, 0, 8),
+    (256, 256, 8192, 1, 1, 0),     # few tiles, long K: split-K path for fp32 output
+]
+
+
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,pad", GEMM_CASES)
+@pytest.mark.parametrize("epi", EPIS)
+@pytest.mark.parametrize("engine", [0, 1])
+def test_gemm_bf16(nc, M, N, K, a_mn, b_mn, pad, epi, engine):
+    import torch
+    if engine == 1 and K > 2048 and epi != "STORE_F32":
+        pytest.skip("covered by the tensor-core engine")
+    seed = M * 7 + N * 3 + K + a_mn * 11 + b_mn * 13
+    A = _bf16(synth.normal(seed, 1, M * K).reshape(M, K))
+    B = _bf16(synth.normal(seed, 2, N * K).reshape(N, K))
+    As, lda = _stored(A, a_mn, pad)
+    Bs, ldb = _stored(B, b_mn, pad)
+    A_dev = _dev(As / math.sqrt(K), "bf16")
+    A_used = _bf16(As / math.sqrt(K))
+    A_log = A_used[:, :K] if not a_mn else A_used[:, :M].T
+    acc = A_log @ B.T
+    ldd = N + pad
+    code = getattr(nc, "NC_EPI_" + epi)
+    if epi == "STORE_F32":
+        D = torch.zeros(M, ldd, dtype=torch.float32, device="cuda")
+        ref = acc
+    else:
+        D0 = _bf16(synth.normal(seed, 3, M * ldd).reshape(M, ldd))
+        if epi == "DRELU2":
+            D0 = _bf16(np.maximum(D0, 0) ** 2)
+        D = _dev(D0, "bf16")
+        old = D0[:, :N]
+        ref = {"STORE": lambda: acc, "ADD": lambda: old + acc,
+               "RELU2": lambda: np.maximum(acc, 0) ** 2,
+               "DRELU2": lambda: acc * 2 * np.sqrt(old),
+               "SOFTCAP": lambda: 15 * np.tanh(acc / 15)}[epi]()
+    B_dev = _dev(Bs, "bf16")
+    rc = nc.nc_gemm(A_dev.data_ptr(), lda, a_mn, B_dev.data_ptr(), ldb, b_mn, D.data_ptr(), ldd,
+                    M, N, K, nc.NC_BF16, code, engine, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    got = D.float().cpu().numpy().astype(np.float64)
+    scale = np.abs(ref).max()
+    if epi == "STORE_F32":
+        np.testing.assert_allclose(got[:, :N], ref, rtol=0, atol=2e-5 * scale)
+    else:
+        # one bf16 rounding of the output (plus the input rounding of D)
+        err = np.abs(got[:, :N] - ref)
+        assert np.all(err <= 2 ** -8 * np.abs(ref) + 2e-3 * scale), float(err.max())
+    if pad and epi != "STORE_F32":
+        np.testing.assert_array_equal(got[:, N:], D0[:, N:])  # nothing written past N
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 70, 33), (64, 257, 300)])
+def test_gemm_f32(nc, M, N, K):
+    import torch
+    A = synth.normal(M + N, 1, M * K).reshape(M, K).astype(np.float32).astype(np.float64)
+    B = synth.normal(M + N, 2, N * K).reshape(N, K).astype(np.float32).astype(np.float64)
+    for a_mn in (0, 1):
+        for b_mn in (0, 1):
+            As, lda = _stored(A, a_mn, 0)
+            Bs, ldb = _stored(B, b_mn, 0)
+            D = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+            Ad, Bd = _dev(As, "f32"), _dev(Bs, "f32")
+            rc = nc.nc_gemm(Ad.data_ptr(), lda, a_mn, Bd.data_ptr(), ldb, b_mn, D.data_ptr(), N,
+                            M, N, K, nc.NC_F32, nc.NC_EPI_STORE, 0,
+                            torch.cuda.current_stream().cuda_stream)
+            assert rc == 0
+            got = D.cpu().numpy().astype(np.float64)
+            ref = A @ B.T
+            np.testing.assert_allclose(got, ref, rtol=0, atol=1e-5 * np.abs(ref).max())
+
+
+def _attn_inputs(B, T, H, seed, dtype):
+    """q, k normalised per head (as after QK-norm), v plain."""
+    ld = 128 * (H + 2)
+    q = synth.normal(seed, 1, B * T * H * 128).reshape(B, T, H, 128)
+    k = synth.normal(seed, 2, B * T * 128).reshape(B, T, 128)
+    v = synth.normal(seed, 3, B * T * 128).reshape(B, T, 128)
+    q, _ = oracle.rmsnorm(q)
+    k, _ = oracle.rmsnorm(k)
+    qkv = np.concatenate([q.reshape(B * T, H * 128), k.reshape(B * T, 128), v.reshape(B * T, 128)], 1)
+    if dtype == "bf16":
+        qkv = _bf16(qkv)
+    else:
+        qkv = qkv.astype(np.float32).astype(np.float64)
+    q = qkv[:, :H * 128].reshape(B, T, H, 128)
+    k = qkv[:, H * 128:H * 128 + 128].reshape(B, T, 128)
+    v = qkv[:, H * 128 + 128:].reshape(B, T, 128)
+    return qkv, ld, q, k, v
+
+
+ATTN_CASES = [(1, 1, 1), (2, 9, 2), (1, 130, 3), (2, 256, 2), (1, 515, 10)]
+
+
+@pytest.mark.parametrize("B,T,H", ATTN_CASES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("engine", [0, 1])
+def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
+    import torch
+    code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
+    qkv, ld, q, k, v = _attn_inputs(B, T, H, 100 + T + H, dtype)
+    st = torch.cuda.current_stream().cuda_stream
+    qkv_d = _dev(qkv, dtype)
+    O = torch.zeros(B * T, H * 128, dtype=qkv_d.dtype, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    assert nc.nc_attention_fwd(qkv_d.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, code,
+                               engine, st) == 0
+    O_ref = np.empty((B, T, H, 128))
+    lse_ref = np.empty((B, H, T))
+    for b in range(B):
+        O_ref[b], lse_ref[b] = oracle.attention(q[b], k[b], v[b])
+    got_O = O.float().cpu().numpy().reshape(B, T, H, 128)
+    got_lse = lse.cpu().numpy()
+    tolO = 1e-5 if dtype == "f32" else 1.5e-2
+    np.testing.assert_allclose(got_O, O_ref, rtol=0, atol=tolO * np.abs(O_ref).max())
+    np.testing.assert_allclose(got_lse, lse_ref, rtol=0, atol=1e-5 if dtype == "f32" else 2e-3)
+    # backward with a random upstream gradient, using the kernel's own O
+    dO = synth.normal(7 + T, 4, B * T * H * 128).reshape(B * T, H * 128)
+    dO = _bf16(dO) if dtype == "bf16" else dO.astype(np.float32).astype(np.float64)
+    dO_d = _dev(dO, dtype)
+    Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    dqkv = torch.zeros(B * T, ld, dtype=qkv_d.dtype, device="cuda")
+    assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
+                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine, st) == 0
+    got = dqkv.float().cpu().numpy().astype(np.float64)
+    dq_ref = np.empty((B, T, H, 128))
+    dk_ref = np.empty((B, T, 128))
+    dv_ref = np.empty((B, T, 128))
+    for b in range(B):
+        dq_ref[b], dk_ref[b], dv_ref[b] = oracle.attention_bwd(dO.reshape(B, T, H, 128)[b], q[b], k[b], v[b])
+    parts = [(got[:, :H * 128], dq_ref.reshape(B * T, -1)), (got[:, H * 128:H * 128 + 128], dk_ref.reshape(B * T, -1)),
+             (got[:, H * 128 + 128:], dv_ref.reshape(B * T, -1))]
+    for g, r in parts:
+        scale = np.abs(r).max()
+        if T == 1 and r is not parts[2][1]:
+            # one key: the softmax is constant, dq and dk vanish
+            assert np.max(np.abs(g)) <= 1e-6
+            continue
+        if dtype == "f32":
+            np.testing.assert_allclose(g, r, rtol=0, atol=1e-4 * scale)
+        else:
+            cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
+            assert cos > 0.9995, cos
+            assert np.max(np.abs(g - r)) <= 3e-2 * scale
