@@ -45,6 +45,11 @@ class nc_param(ctypes.Structure):
                 ("rows", ctypes.c_int), ("cols", ctypes.c_int)]
 
 
+class nc_kernel_stat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -59,6 +64,8 @@ _SIGS = {
     "nc_sync_status": (_I, [_P, _P, _I]),
     "nc_strerror": (ctypes.c_char_p, [_I]),
     "nc_destroy": (None, [_P]),
+    "nc_profile": (_I, [_P, _I]),
+    "nc_profile_read": (_I, [_P, ctypes.POINTER(nc_kernel_stat), _I, ctypes.POINTER(_I)]),
     "nc_gemm": (_I, [_P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _I,
                      _I, _I, _I, _P]),
     "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -153,3 +160,17 @@ def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream) -> int:
 def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream) -> int:
     return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine,
                                            stream)
+
+
+def nc_profile(handle, enable: int) -> int:
+    return load_library().nc_profile(handle, enable)
+
+
+def nc_profile_read(handle, max_classes: int = 32):
+    """Returns (status, [ {name, launches, ms, flops, bytes}, ... ])."""
+    arr = (nc_kernel_stat * max_classes)()
+    n = _I()
+    rc = load_library().nc_profile_read(handle, arr, max_classes, ctypes.byref(n))
+    out = [dict(name=arr[i].name.decode(), launches=arr[i].launches, ms=arr[i].ms,
+                flops=arr[i].flops, bytes=arr[i].bytes) for i in range(n.value)]
+    return rc, out

@@ -10,6 +10,7 @@
 // sub + 8*c, c < 16, and dot products are finished with 3 shuffles.
 #pragma once
 
+#include "attn_mma.cuh"
 #include "common.cuh"
 
 namespace nc {
@@ -246,7 +247,8 @@ template <typename T>
 inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H,
                                    int num_sms, int engine, cudaStream_t st) {
   (void)num_sms;
-  (void)engine;
+  if (sizeof(T) == 2 && engine == 0 && fa::supported(qkv, ld, O))
+    return fa::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, st);
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
 }
 
@@ -255,7 +257,9 @@ inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *dO, const floa
                                    const float *Dr, T *dqkv, int B, int T_len, int H, int num_sms,
                                    int engine, cudaStream_t st) {
   (void)num_sms;
-  (void)engine;
+  if (sizeof(T) == 2 && engine == 0 && fa::supported(qkv, ld, dO) && fa::supported(dqkv, ld, dqkv))
+    return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len,
+                          H, st);
   return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);
 }
 

@@ -27,6 +27,15 @@
 
 using namespace nc;
 
+// kernel classes of the per-launch accounting
+enum KernelClass {
+  K_GEMM_TC, K_GEMM_SIMT, K_ATTN_FWD, K_ATTN_BWD, K_EMBED, K_RMSNORM, K_ROPE_QKNORM, K_CE,
+  K_LOSS_MEAN, K_RMSNORM_BWD, K_ROWDOT, K_ROPE_QKNORM_BWD, K_EMBED_BWD, K_NUM_CLASSES
+};
+static const char *kClassName[K_NUM_CLASSES] = {
+    "gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd", "embed_norm", "rmsnorm", "rope_qknorm",
+    "ce_fused", "loss_mean", "rmsnorm_bwd", "attn_rowdot", "rope_qknorm_bwd", "embed_bwd"};
+
 struct nc_model {
   int depth, C, H, F, V, seq, dtype;
   int64_t n_params;
@@ -36,6 +45,14 @@ struct nc_model {
   float *rope_sin;
   int *status;      // device status word
   std::vector<nc_param> params;
+  // accounting (see nc_profile)
+  bool prof = false;
+  std::vector<cudaEvent_t> events;
+  size_t events_used = 0;
+  std::vector<std::pair<int, size_t>> records;  // (class, index of the start event)
+  int64_t launches[K_NUM_CLASSES] = {};
+  double flops[K_NUM_CLASSES] = {};
+  double bytes[K_NUM_CLASSES] = {};
 };
 
 namespace {
@@ -138,16 +155,50 @@ Weights<T> weight_ptrs(const nc_model *m, const void *weights) {
     }                                                  \
   } while (0)
 
+// Start event of one launch when profiling is on; -1 otherwise.
+long prof_begin(nc_model *m, cudaStream_t st) {
+  if (!m->prof) return -1;
+  while (m->events.size() < m->events_used + 2) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    m->events.push_back(e);
+  }
+  const size_t i = m->events_used;
+  if (cudaEventRecord(m->events[i], st) != cudaSuccess) return -1;
+  m->events_used += 2;
+  return (long)i;
+}
+
+void prof_end(nc_model *m, cudaStream_t st, long ev, int cls, double flops, double bytes) {
+  m->launches[cls] += 1;
+  m->flops[cls] += flops;
+  m->bytes[cls] += bytes;
+  if (ev >= 0 && cudaEventRecord(m->events[ev + 1], st) == cudaSuccess)
+    m->records.push_back({cls, (size_t)ev});
+}
+
+// Launch one kernel with its accounting: class, algorithmic flops and bytes.
+#define NC_RUN(cls, fl, by, LAUNCH)                                  \
+  do {                                                               \
+    const long ev_ = prof_begin(m, st);                              \
+    LAUNCH;                                                          \
+    NC_CHECK_LAUNCH();                                               \
+    prof_end(m, st, ev_, (cls), (double)(fl), (double)(by));         \
+  } while (0)
+
 template <typename T>
-int gemm(const nc_model *m, const GemmProblem &p, cudaStream_t st) {
+int gemm(nc_model *m, const GemmProblem &p, cudaStream_t st) {
   if (p.M <= 0 || p.N <= 0) return NC_OK;
   cudaError_t e;
-  if (tc_gemm_supported<T>(p)) e = launch_gemm_tc(p, m->num_sms, m->status, st);
+  const bool tcp = tc_gemm_supported<T>(p);
+  const long ev = prof_begin(m, st);
+  if (tcp) e = launch_gemm_tc(p, m->num_sms, m->status, st);
   else e = launch_gemm_simt<T>(p, st);
   if (e != cudaSuccess) {
     fprintf(stderr, "nanochat_b200: gemm launch: %s\n", cudaGetErrorString(e));
     return NC_ECUDA;
   }
+  prof_end(m, st, ev, tcp ? K_GEMM_TC : K_GEMM_SIMT, 2.0 * p.M * (double)p.N * p.K, 0.0);
   return NC_OK;
 }
 
@@ -175,29 +226,32 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
                  Work<T> &w, cudaStream_t st) {
   const int M = B * T_len, C = m->C, H = m->H, F = m->F;
   const int ldqkv = C + 2 * kHeadDim;
-  NC_DISPATCH_NV(C, (embed_norm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                        tokens, W.wte, w.x, w.r0, M, C, m->V, m->status)));
-  NC_CHECK_LAUNCH();
+  const double es = sizeof(T);
+  const double attn_flops = 2.0 * B * H * (double)kHeadDim * T_len * (T_len + 1.0);
+  NC_RUN(K_EMBED, 0, M * (8.0 + 2.0 * C * es),
+         NC_DISPATCH_NV(C, (embed_norm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                               tokens, W.wte, w.x, w.r0, M, C, m->V, m->status))));
   for (int l = 0; l < m->depth; ++l) {
-    NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xn[l],
-                                                                               w.r1[l], M, C)));
-    NC_CHECK_LAUNCH();
+    NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
+           NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                 w.x, w.xn[l], w.r1[l], M, C))));
     NC_TRY(gemm<T>(m, gp(M, ldqkv, C, w.xn[l], C, 0, W.wqkv[l], C, 0, w.qkv[l], ldqkv, EPI_STORE), st));
-    rope_qknorm_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
-        w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H);
-    NC_CHECK_LAUNCH();
-    if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0, st) !=
-        cudaSuccess)
-      return NC_ECUDA;
+    NC_RUN(K_ROPE_QKNORM, 0, M * (2.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
+           (rope_qknorm_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+               w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
+    NC_RUN(K_ATTN_FWD, attn_flops, 0,
+           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0,
+                                  st) != cudaSuccess) return NC_ECUDA);
     NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, w.x, C, EPI_ADD), st));
-    NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xn2[l],
-                                                                               w.r2[l], M, C)));
-    NC_CHECK_LAUNCH();
+    NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
+           NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                 w.x, w.xn2[l], w.r2[l], M, C))));
     NC_TRY(gemm<T>(m, gp(M, F, C, w.xn2[l], C, 0, W.w1[l], C, 0, w.a[l], F, EPI_RELU2), st));
     NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w2[l], F, 0, w.x, C, EPI_ADD), st));
   }
-  NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(w.x, w.xf, w.rf, M, C)));
-  NC_CHECK_LAUNCH();
+  NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
+         NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                               w.x, w.xf, w.rf, M, C))));
   return NC_OK;
 }
 
@@ -210,6 +264,8 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   const Weights<T> W = weight_ptrs<T>(m, weights);
   const int M = B * T_len, C = m->C, H = m->H, F = m->F, V = m->V;
   const int ldqkv = C + 2 * kHeadDim;
+  const double es = sizeof(T);
+  const double attn_bwd_flops = 4.0 * B * H * (double)kHeadDim * T_len * (T_len + 1.0);
   NC_TRY(forward_body<T>(m, W, tokens, B, T_len, w, st));
 
   // head: z = xf Wout^T, then softcap + CE forward and backward in place
@@ -217,24 +273,26 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   float *tl = token_loss ? token_loss : w.tok_loss;
   const float inv_M = 1.f / (float)M;
   if (sizeof(T) == 2 && V == 65536) {
-    ce_fused_bf16_kernel<16><<<M, 512, 0, st>>>((bf16 *)w.z, w.ldz, targets, tl, M, V, inv_M,
-                                                m->status);
+    NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
+           (ce_fused_bf16_kernel<16><<<M, 512, 0, st>>>((bf16 *)w.z, w.ldz, targets, tl, M, V,
+                                                        inv_M, m->status)));
   } else {
-    ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(w.z, w.ldz, targets, tl, M, V, inv_M, m->status);
+    NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
+           (ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(w.z, w.ldz, targets, tl, M, V, inv_M,
+                                                          m->status)));
   }
-  NC_CHECK_LAUNCH();
-  loss_mean_kernel<<<1, 1024, 0, st>>>(tl, M, loss, m->status);
-  NC_CHECK_LAUNCH();
+  NC_RUN(K_LOSS_MEAN, 0, M * 4.0, (loss_mean_kernel<<<1, 1024, 0, st>>>(tl, M, loss, m->status)));
 
   // gradient pointers (fp32, same layout as the weights)
   auto G = [&](int idx) { return grads + m->params[idx].offset; };
   const int last = (int)m->params.size() - 1;
+  const double nbwd = M * (12.0 * C + 2.0 * C * es + 4.0);  // dy, dx_old, dx in fp32; y, dx_t in T
   // dWout = dz^T xf ;  dxf = dz Wout
   NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, EPI_STORE_F32), st));
   NC_TRY(gemm<T>(m, gp(M, C, V, w.z, w.ldz, 0, W.lm_head, C, 1, w.dy32, C, EPI_STORE_F32), st));
-  NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                        w.dy32, w.xf, w.rf, w.dx, w.dxb, M, C, 0)));
-  NC_CHECK_LAUNCH();
+  NC_RUN(K_RMSNORM_BWD, 0, nbwd - M * 4.0 * C,
+         NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                               w.dy32, w.xf, w.rf, w.dx, w.dxb, M, C, 0))));
 
   for (int l = m->depth - 1; l >= 0; --l) {
     const int pi = 1 + 6 * l;
@@ -243,33 +301,33 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     NC_TRY(gemm<T>(m, gp(M, F, C, w.dxb, C, 0, W.w2[l], F, 1, w.a[l], F, EPI_DRELU2), st));
     NC_TRY(gemm<T>(m, gp(F, C, M, w.a[l], F, 1, w.xn2[l], C, 1, G(pi + 4), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w1[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
-    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                          w.dy32, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1)));
-    NC_CHECK_LAUNCH();
+    NC_RUN(K_RMSNORM_BWD, 0, nbwd,
+           NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                 w.dy32, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1))));
     // attention: x += O Wo^T
     NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
-    attn_rowdot_kernel<T><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>(w.dO, w.O[l], w.Drow, M,
-                                                                         T_len, H);
-    NC_CHECK_LAUNCH();
-    if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
-                           m->num_sms, 0, st) != cudaSuccess)
-      return NC_ECUDA;
-    rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
-        w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H);
-    NC_CHECK_LAUNCH();
+    NC_RUN(K_ROWDOT, 0, M * (2.0 * C * es + 4.0 * H),
+           (attn_rowdot_kernel<T><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>(w.dO, w.O[l], w.Drow,
+                                                                                M, T_len, H)));
+    NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
+           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
+                                  m->num_sms, 0, st) != cudaSuccess) return NC_ECUDA);
+    NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
+           (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+               w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     // [q|k|v] = xn [Wq;Wk;Wv]^T
     NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
-    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                          w.dy32, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1)));
-    NC_CHECK_LAUNCH();
+    NC_RUN(K_RMSNORM_BWD, 0, nbwd,
+           NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                 w.dy32, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
   }
   // embedding: through the first norm, summed into the selected rows
   if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
-  NC_DISPATCH_NV(C, (embed_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                        w.dx, tokens, W.wte, w.r0, G(0), M, C, V)));
-  NC_CHECK_LAUNCH();
+  NC_RUN(K_EMBED_BWD, 0, M * (8.0 * C + C * es + 8.0),
+         NC_DISPATCH_NV(C, (embed_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                               w.dx, tokens, W.wte, w.r0, G(0), M, C, V))));
   return NC_OK;
 }
 
@@ -303,7 +361,7 @@ int op_device_sms(int *num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
   if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
-  if (tc_init() != cudaSuccess) return NC_ECUDA;
+  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess) return NC_ECUDA;
   return NC_OK;
 }
 
@@ -363,7 +421,7 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
-  if (!ok || tc_init() != cudaSuccess) {
+  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess) {
     nc_destroy(m);
     return NC_ECUDA;
   }
@@ -450,6 +508,44 @@ int nc_sync_status(nc_model *m, void *stream, int timeout_ms) {
   return NC_OK;
 }
 
+int nc_profile(nc_model *m, int enable) {
+  if (!m) return NC_EINVAL;
+  m->prof = enable != 0;
+  return NC_OK;
+}
+
+int nc_profile_read(nc_model *m, nc_kernel_stat *out, int max, int *count) {
+  if (!m || (!out && max > 0) || !count) return NC_EINVAL;
+  double ms[K_NUM_CLASSES] = {};
+  int rc = NC_OK;
+  if (!m->records.empty()) {
+    if (cudaEventSynchronize(m->events[m->records.back().second + 1]) != cudaSuccess) rc = NC_ECUDA;
+    for (const auto &r : m->records) {
+      float t = 0.f;
+      if (rc == NC_OK && cudaEventElapsedTime(&t, m->events[r.second], m->events[r.second + 1]) == cudaSuccess)
+        ms[r.first] += t;
+    }
+  }
+  int n = 0;
+  for (int c = 0; c < K_NUM_CLASSES; ++c) {
+    if (!m->launches[c]) continue;
+    if (n < max) {
+      memset(&out[n], 0, sizeof(nc_kernel_stat));
+      snprintf(out[n].name, sizeof(out[n].name), "%s", kClassName[c]);
+      out[n].launches = m->launches[c];
+      out[n].ms = ms[c];
+      out[n].flops = m->flops[c];
+      out[n].bytes = m->bytes[c];
+    }
+    ++n;
+  }
+  *count = n < max ? n : max;
+  m->records.clear();
+  m->events_used = 0;
+  for (int c = 0; c < K_NUM_CLASSES; ++c) { m->launches[c] = 0; m->flops[c] = 0; m->bytes[c] = 0; }
+  return rc;
+}
+
 const char *nc_strerror(int code) {
   switch (code) {
     case NC_OK: return "ok";
@@ -468,6 +564,7 @@ const char *nc_strerror(int code) {
 
 void nc_destroy(nc_model *m) {
   if (!m) return;
+  for (cudaEvent_t e : m->events) cudaEventDestroy(e);
   if (m->rope_cos) cudaFree(m->rope_cos);
   if (m->rope_sin) cudaFree(m->rope_sin);
   if (m->status) cudaFree(m->status);

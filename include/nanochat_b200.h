@@ -131,6 +131,27 @@ int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B,
  * device-side error recorded (NC_ERANGE, NC_ENONFINITE, NC_ETIMEOUT) or NC_OK. */
 int nc_sync_status(nc_model *m, void *stream, int timeout_ms);
 
+/* Per-kernel accounting of the work enqueued through one handle, for
+ * measurement.  Launch counts and algorithmic work (flops: 2 per multiply-add
+ * of the mathematical definition, causal attention counted over j <= i only;
+ * bytes: the tensors a kernel must read and write once) are always summed.
+ * With profiling on, every launch is also bracketed by two CUDA events on
+ * the caller's stream and the device time between them is summed. */
+typedef struct {
+  char name[24];      /* kernel class: "gemm_tc", "gemm_simt", "attn_fwd", ... */
+  int64_t launches;
+  double ms;          /* summed device time; 0 unless profiling was on */
+  double flops;
+  double bytes;
+} nc_kernel_stat;
+
+/* Turn event timing of every launch on (enable != 0) or off. */
+int nc_profile(nc_model *m, int enable);
+
+/* Wait for the recorded events, write up to `max` per-class sums into `out`
+ * (classes with no launch are skipped), set *count, and reset the sums. */
+int nc_profile_read(nc_model *m, nc_kernel_stat *out, int max, int *count);
+
 /* Static string for a status code. */
 const char *nc_strerror(int code);
 
