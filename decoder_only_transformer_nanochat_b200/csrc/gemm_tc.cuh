@@ -34,7 +34,10 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;      // 48 KB
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t kWaitNs = 4000000000ull;         // 4 s without progress = abort
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// bf16 outputs leave through a 128 x 128 staging tile (two 64-column boxes of
+// 128 rows x 128 B, 128-byte swizzle) written by TMA bulk stores
+constexpr int STAGING_BYTES = 2 * BM * 128;          // 32 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 struct Unit {
   int m_blk, n_blk, kb0, kb1;
@@ -107,6 +110,36 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "%3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// barrier among the 128 epilogue threads only
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// the same barrier with an AND vote, so every epilogue thread takes the same branch
+__device__ __forceinline__ bool epi_vote_all(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -238,14 +271,48 @@ __device__ __forceinline__ void epilogue_chunk(const Params &p, int m, int n, co
   }
 }
 
+// relu(h) = sqrt(relu(h)^2): the hardware approximation (relative error near
+// 2^-23, exact 0 at 0) is far below the bf16 rounding of the result, and
+// avoids the IEEE square root's slow path in the epilogue's inner loop.
+__device__ __forceinline__ float sqrt_fast(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// bf16 epilogue of 32 columns (chunk c of the 128-column half) of staging row r:
+// 16-byte unit u of the row sits at (u ^ (r & 7)) within its 128-byte box row.
+__device__ __forceinline__ void epilogue_stage(int epi, uint8_t *staging, int r, int c, const uint32_t (&acc)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int unit = c * 4 + q;  // 0..15 over the 128 columns
+    uint8_t *ptr = staging + (unit >> 3) * (BM * 128) + r * 128 + (((unit & 7) ^ (r & 7)) << 4);
+    float old[8], o[8];
+    if (epi == EPI_ADD || epi == EPI_DRELU2) Vec8<bf16>::load(reinterpret_cast<const bf16 *>(ptr), old);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float a = __uint_as_float(acc[8 * q + j]);
+      switch (epi) {
+        case EPI_ADD: o[j] = old[j] + a; break;
+        case EPI_RELU2: { const float t = fmaxf(a, 0.f); o[j] = t * t; } break;
+        case EPI_DRELU2: o[j] = a * 2.f * sqrt_fast(old[j]); break;
+        case EPI_SOFTCAP: o[j] = softcap_fast(a); break;
+        default: o[j] = a; break;
+      }
+    }
+    Vec8<bf16>::store(reinterpret_cast<bf16 *>(ptr), o);
+  }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                   const Params p) {
+                   const __grid_constant__ CUtensorMap map_d, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+  uint8_t *staging = smem + STAGES * STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(staging + STAGING_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, aux
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 6);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -253,6 +320,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * STAGES + 2 + a); };
   const uint32_t drain_bar = smem_u32(bars + 2 * STAGES + 4);
+  const uint32_t aux_bar = smem_u32(bars + 2 * STAGES + 5);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -264,6 +332,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty_bar(a), 128);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(aux_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
@@ -364,28 +433,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue warps 2..5 ----------------
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int r = quarter * 32 + lane;  // tile row owned by this thread
+    const bool leader = warp == 2 && lane == 0;  // issues the epilogue's TMA copies
+    const bool f32_out = p.epi == EPI_STORE_F32;
+    const bool aux = p.epi == EPI_ADD || p.epi == EPI_DRELU2;
+    const uint32_t st_addr = smem_u32(staging);
     int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+    uint32_t acc_phase = 0, aux_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit x = unit_of(p, u);
-      // every lane waits; the vote re-converges the warp for the .sync.aligned loads
-      const bool ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      // every lane waits; the vote over all epilogue threads keeps their
+      // branches (and named barriers) uniform and re-converges each warp
+      ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      __syncwarp();
+      if (!ok) break;
       tc_fence_after();
-      const int m = x.m_blk * BM + quarter * 32 + lane;
+      const int m0 = x.m_blk * BM;
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if (f32_out) {
+        const int m = m0 + r;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n = x.n_blk * BN + c * 32;
-        if (n >= p.N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        if (m < p.M) epilogue_chunk(p, m, n, r);
+        for (int c = 0; c < BN / 32; ++c) {
+          const int n = x.n_blk * BN + c * 32;
+          if (n >= p.N) break;  // warp-uniform
+          uint32_t rr[32];
+          tmem_ld32(t_row + c * 32, rr);
+          if (m < p.M) epilogue_chunk(p, m, n, rr);
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+      } else {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          // half 0 always starts inside N; half 1 runs only if half 0 did not reach N
+          const int n_half = x.n_blk * BN + half * 128;
+          const bool box1 = n_half + 64 < p.N;
+          if (leader) {
+            bulk_wait_read0();  // the previous stores have finished reading the staging tile
+            if (aux) {
+              mbar_expect_tx(aux_bar, box1 ? 2 * BM * 128 : BM * 128);
+              tma_load_2d(st_addr, &map_d, n_half, m0, aux_bar);
+              if (box1) tma_load_2d(st_addr + BM * 128, &map_d, n_half + 64, m0, aux_bar);
+            }
+          }
+          if (aux) {
+            ok = epi_vote_all(mbar_wait(aux_bar, aux_phase, abort_flag, p.status));
+            aux_phase ^= 1;
+            if (!ok) break;
+          } else {
+            epi_bar();
+          }
+          __syncwarp();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(t_row + half * 128 + c * 32, rr);
+            epilogue_stage(p.epi, staging, r, c, rr);
+          }
+          if (half == 1 || n_half + 128 >= p.N) {
+            // accumulator fully read: hand TMEM back to the MMA warp
+            tc_fence_before();
+            mbar_arrive(tempty_bar(acc));
+          }
+          fence_proxy_async();
+          epi_bar();
+          if (leader) {
+            tma_store_2d(&map_d, st_addr, n_half, m0);
+            if (box1) tma_store_2d(&map_d, st_addr + BM * 128, n_half + 64, m0);
+            bulk_commit();
+          }
+          if (n_half + 128 >= p.N) break;
+        }
+        if (!ok) break;
       }
-      tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (leader) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -479,6 +603,8 @@ inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status
   if (!g.b_mn) ok = make_map(&mb, g.B, g.N, g.K, g.ldb, 64, BN);
   else ok = make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 64);
   if (!ok) return cudaErrorInvalidValue;
+  CUtensorMap md = ma;  // fp32 outputs are written directly; the map is unused
+  if (g.epi != EPI_STORE_F32 && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
   Params p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.n_m = (g.M + BM - 1) / BM;
@@ -502,7 +628,7 @@ inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status
     if (e != cudaSuccess) return e;
   }
   const int grid = p.units < num_sms ? p.units : num_sms;
-  gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, p);
+  gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, md, p);
   return cudaGetLastError();
 }
 

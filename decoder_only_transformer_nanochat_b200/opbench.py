@@ -1,0 +1,105 @@
+"""Time one kernel of the decoder step in isolation, at the shapes of one
+training step of the d20 workload (M = 16 x 2048 tokens, C = 1280, F = 5120,
+V = 65536, H = 10), through the op-level C entry points.  Used for per-kernel
+timing and for small, single-kernel ncu captures.
+
+    python -m decoder_only_transformer_nanochat_b200.opbench --op w1_fwd --iters 5
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+M, C, F, V, H = 16 * 2048, 1280, 5120, 65536, 10
+B, T = 16, 2048
+
+# name: (M, N, K, a_mn, b_mn, epilogue)
+GEMMS = {
+    "qkv_fwd": (M, C + 256, C, 0, 0, "STORE"),
+    "o_fwd": (M, C, C, 0, 0, "ADD"),
+    "w1_fwd": (M, F, C, 0, 0, "RELU2"),
+    "w2_fwd": (M, C, F, 0, 0, "ADD"),
+    "head_fwd": (M, V, C, 0, 0, "STORE"),
+    "w2_dgrad": (M, F, C, 0, 1, "DRELU2"),
+    "w1_dgrad": (M, C, F, 0, 1, "STORE_F32"),
+    "w1_wgrad": (F, C, M, 1, 1, "STORE_F32"),
+    "w2_wgrad": (C, F, M, 1, 1, "STORE_F32"),
+    "o_wgrad": (C, C, M, 1, 1, "STORE_F32"),
+    "head_dgrad": (M, C, V, 0, 1, "STORE_F32"),
+    "head_wgrad": (V, C, M, 1, 1, "STORE_F32"),
+}
+
+
+def main():
+    import torch
+
+    import decoder_only_transformer_nanochat_b200 as nc
+    from decoder_only_transformer_nanochat_b200 import build
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", required=True, choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm"])
+    ap.add_argument("--shape", default=None, help="for --op gemm: M,N,K,a_mn,b_mn,EPILOGUE")
+    ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--engine", type=int, default=0)
+    args = ap.parse_args()
+    build.build()
+    g = torch.Generator(device="cuda").manual_seed(0)
+    st = torch.cuda.current_stream().cuda_stream
+    if args.op == "gemm":
+        f = args.shape.split(",")
+        GEMMS["gemm"] = (int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4]), f[5])
+    if args.op in GEMMS:
+        m, n, k, a_mn, b_mn, epi = GEMMS[args.op]
+        A = (torch.randn(m * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+        Bm = (torch.randn(n * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+        out_f32 = epi == "STORE_F32"
+        D = torch.rand(m * n, device="cuda", generator=g, dtype=torch.float32)
+        if not out_f32:
+            D = D.to(torch.bfloat16)
+        lda = m if a_mn else k
+        ldb = n if b_mn else k
+        code = getattr(nc, "NC_EPI_" + epi)
+
+        def run():
+            rc = nc.nc_gemm(A.data_ptr(), lda, a_mn, Bm.data_ptr(), ldb, b_mn, D.data_ptr(), n, m, n, k,
+                            nc.NC_BF16, code, args.engine, st)
+            assert rc == 0, rc
+        flops = 2.0 * m * n * k
+    else:
+        ld = 128 * (H + 2)
+        qkv = (torch.randn(B * T * ld, device="cuda", generator=g) * 0.09).to(torch.bfloat16)
+        O = torch.empty(B * T * H * 128, device="cuda", dtype=torch.bfloat16)
+        lse = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
+        rc = nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16,
+                                 args.engine, st)
+        assert rc == 0
+        dO = (torch.randn(B * T * H * 128, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+        Dr = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
+        dqkv = torch.empty(B * T * ld, device="cuda", dtype=torch.bfloat16)
+        causal = 2.0 * B * H * 128 * T * (T + 1.0)
+        if args.op == "attn_fwd":
+            def run():
+                assert nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H,
+                                           nc.NC_BF16, args.engine, st) == 0
+            flops = causal
+        else:
+            def run():
+                assert nc.nc_attention_bwd(qkv.data_ptr(), ld, O.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                                           Dr.data_ptr(), dqkv.data_ptr(), B, T, H, nc.NC_BF16, args.engine,
+                                           st) == 0
+            flops = 2.0 * causal
+    run()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.iters)]
+    for i in range(args.iters):
+        ev[2 * i].record()
+        run()
+        ev[2 * i + 1].record()
+    torch.cuda.synchronize()
+    ms = sorted(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.iters))
+    med = ms[len(ms) // 2]
+    print(json.dumps({"op": args.op, "shape": args.shape, "median_ms": med, "min_ms": ms[0],
+                      "tflops": flops / (med / 1000) / 1e12}))
+
+
+if __name__ == "__main__":
+    main()

@@ -14,6 +14,7 @@ natural-language token frequencies), with targets = tokens shifted by one.
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass
 
 import numpy as np
@@ -60,20 +61,41 @@ def uniform01(seed: int, tag: int, n: int) -> np.ndarray:
     return (z >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
 
 
+_WCHUNK = 1 << 20
+
+
+def _normal_pairs(seed, tag, lo, hi):
+    """Normals 2*lo .. 2*hi-1 of the stream (Box-Muller on uniform pairs lo..hi-1)."""
+    z = splitmix64(seed, tag, 2 * (hi - lo), offset=2 * lo)
+    u = (z >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
+    u1 = 1.0 - u[0::2]  # (0, 1]
+    u2 = u[1::2]
+    r = np.sqrt(-2.0 * np.log(u1))
+    t = 2.0 * math.pi * u2
+    out = np.empty(2 * (hi - lo))
+    out[0::2] = r * np.cos(t)
+    out[1::2] = r * np.sin(t)
+    return out
+
+
 def normal(seed: int, tag: int, n: int) -> np.ndarray:
-    """n standard normals by Box-Muller, two per pair of uniforms."""
+    """n standard normals by Box-Muller, two per pair of uniforms.  Chunks are
+    independent (counter-based stream), so they are filled by a thread pool;
+    the values do not depend on the split."""
     m = (n + 1) // 2
     out = np.empty(2 * m, dtype=np.float64)
-    for lo in range(0, m, _CHUNK):
-        hi = min(m, lo + _CHUNK)
-        z = splitmix64(seed, tag, 2 * (hi - lo), offset=2 * lo)
-        u = (z >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
-        u1 = 1.0 - u[0::2]  # (0, 1]
-        u2 = u[1::2]
-        r = np.sqrt(-2.0 * np.log(u1))
-        t = 2.0 * math.pi * u2
-        out[2 * lo:2 * hi:2] = r * np.cos(t)
-        out[2 * lo + 1:2 * hi:2] = r * np.sin(t)
+    spans = [(lo, min(m, lo + _CHUNK)) for lo in range(0, m, _CHUNK)]
+
+    def fill(sp):
+        out[2 * sp[0]:2 * sp[1]] = _normal_pairs(seed, tag, sp[0], sp[1])
+
+    if len(spans) <= 1:
+        for sp in spans:
+            fill(sp)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(len(spans), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, spans))
     return out[:n]
 
 
@@ -125,30 +147,46 @@ def init_std(name: str, rows: int, cols: int) -> float:
     return 1.0 / math.sqrt(cols)
 
 
-def make_weights(layout, seed: int, dtype: str, std_override: dict | None = None):
+def make_weights(layout, seed: int, dtype: str, std_override: dict | None = None, want_f64: bool = True):
     """Draw every tensor of `layout` (a list of (name, rows, cols)).
 
     Returns (flat, f64) where `flat` is the storage a device buffer receives
     (float32, or uint16 bf16 bits) in layout order, and `f64` maps each name to
-    the float64 value of exactly what was stored.
+    the float64 value of exactly what was stored (empty if not want_f64).
+    Work is split into independent (tensor, chunk) jobs run by a thread pool;
+    every element is computed the same way whatever the split.
     """
+    from concurrent.futures import ThreadPoolExecutor
     std_override = std_override or {}
     total = sum(r * c for _, r, c in layout)
     flat = np.empty(total, dtype=np.float32 if dtype == "f32" else np.uint16)
-    f64 = {}
+    f64 = {name: np.empty((rows, cols)) for name, rows, cols in layout} if want_f64 else {}
+    jobs = []
     off = 0
     for i, (name, rows, cols) in enumerate(layout):
         n = rows * cols
-        std = std_override.get(name, init_std(name, rows, cols))
-        w32 = (normal(seed, TAG_WEIGHTS + i, n) * std).astype(np.float32)
+        m = (n + 1) // 2
+        for lo in range(0, m, _WCHUNK):
+            jobs.append((i, name, off, n, lo, min(m, lo + _WCHUNK), std_override.get(name, init_std(name, rows, cols))))
+        off += n
+
+    def run(job):
+        i, name, base, n, lo, hi, std = job
+        tmp = _normal_pairs(seed, TAG_WEIGHTS + i, lo, hi)
+        a, b = 2 * lo, min(n, 2 * hi)
+        w32 = (tmp[:b - a] * std).astype(np.float32)
         if dtype == "f32":
-            flat[off:off + n] = w32
-            f64[name] = w32.astype(np.float64).reshape(rows, cols)
+            flat[base + a:base + b] = w32
+            if want_f64:
+                f64[name].reshape(-1)[a:b] = w32
         else:
             bits = f32_to_bf16_bits(w32)
-            flat[off:off + n] = bits
-            f64[name] = bf16_bits_to_f64(bits).reshape(rows, cols)
-        off += n
+            flat[base + a:base + b] = bits
+            if want_f64:
+                f64[name].reshape(-1)[a:b] = bf16_bits_to_f64(bits)
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(run, jobs))
     return flat, f64
 
 
