@@ -11,6 +11,7 @@
 #pragma once
 
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 
 namespace nc {
@@ -243,11 +244,14 @@ inline cudaError_t launch_attn_simt_bwd(const T *qkv, int ld, const T *dO, const
 
 namespace nc {
 
+// engine 0: tensor-core kernels (tcgen05 forward), 1: CUDA cores, 2: warp-level MMA
 template <typename T>
 inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H,
-                                   int num_sms, int engine, cudaStream_t st) {
+                                   int num_sms, int engine, int *status, cudaStream_t st) {
   (void)num_sms;
-  if (sizeof(T) == 2 && engine == 0 && fa::supported(qkv, ld, O))
+  if (sizeof(T) == 2 && engine == 0 && fatc::supported(qkv, ld, O))
+    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, status, st);
+  if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, O))
     return fa::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, st);
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
 }
@@ -257,7 +261,8 @@ inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *dO, const floa
                                    const float *Dr, T *dqkv, int B, int T_len, int H, int num_sms,
                                    int engine, cudaStream_t st) {
   (void)num_sms;
-  if (sizeof(T) == 2 && engine == 0 && fa::supported(qkv, ld, dO) && fa::supported(dqkv, ld, dqkv))
+  if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, dO) &&
+      fa::supported(dqkv, ld, dqkv))
     return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len,
                           H, st);
   return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);

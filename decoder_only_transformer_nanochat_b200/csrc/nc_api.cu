@@ -241,7 +241,7 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
                w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     NC_RUN(K_ATTN_FWD, attn_flops, 0,
            if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0,
-                                  st) != cudaSuccess) return NC_ECUDA);
+                                  m->status, st) != cudaSuccess) return NC_ECUDA);
     NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, w.x, C, EPI_ADD), st));
     NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
            NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
@@ -361,7 +361,7 @@ int op_device_sms(int *num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
   if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
-  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess) return NC_ECUDA;
+  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess) return NC_ECUDA;
   return NC_OK;
 }
 
@@ -421,7 +421,7 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
-  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess) {
+  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess) {
     nc_destroy(m);
     return NC_ECUDA;
   }
@@ -601,9 +601,9 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == NC_BF16)
-    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, num_sms, engine, st);
+    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, num_sms, engine, nullptr, st);
   else if (dtype == NC_F32)
-    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, num_sms, engine, st);
+    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, num_sms, engine, nullptr, st);
   else
     return NC_EUNSUPPORTED;
   return e == cudaSuccess ? NC_OK : NC_ECUDA;

@@ -55,7 +55,8 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
  *   qkv  device [B*T, ld] rows [q (H*128) | k (128) | v (128)], ld >= 128*(H+2)
  *   O    device [B*T, H*128]: O_h = softmax(q_h k^T / sqrt(128) + causal) v
  *   lse  device fp32 [B, H, T]: log-sum-exp of each score row
- * engine: 0 = the path nc_fwd_bwd takes, 1 = force the CUDA-core kernel. */
+ * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores), 1 = the
+ * CUDA-core kernel, 2 = the warp-level MMA kernels (bf16; else as 1). */
 int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
                      int dtype, int engine, void *stream);
 

@@ -155,7 +155,7 @@ ATTN_CASES = [(1, 1, 1), (2, 9, 2), (1, 130, 3), (2, 256, 2), (1, 515, 10)]
 
 @pytest.mark.parametrize("B,T,H", ATTN_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 2])
 def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
     import torch
     code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
