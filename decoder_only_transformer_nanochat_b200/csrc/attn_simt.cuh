@@ -259,8 +259,11 @@ inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B
 template <typename T>
 inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *dO, const float *lse,
                                    const float *Dr, T *dqkv, int B, int T_len, int H, int num_sms,
-                                   int engine, cudaStream_t st) {
+                                   int engine, int *status, cudaStream_t st) {
   (void)num_sms;
+  if (sizeof(T) == 2 && engine == 0 && fatc::supported_bwd(qkv, ld, dO, dqkv))
+    return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len, H,
+                            status, st);
   if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, dO) &&
       fa::supported(dqkv, ld, dqkv))
     return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len,

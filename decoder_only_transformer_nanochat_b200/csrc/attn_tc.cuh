@@ -295,6 +295,476 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Backward.  With P = exp(S - lse) recomputed from the saved log-sum-exp and
+// D = rowsum(dO * O):  dS = P (dO V^T - D),  dQ = dS K / sqrt(d),
+// dK = dS^T Q / sqrt(d) and dV = P^T dO, the last two summed over every query
+// head that shares the key/value head.
+
+// ---------------- dQ: CTA = 128 queries of one (b, h), keys in tiles of 64 ----------------
+constexpr int kBK = 64;
+constexpr int kDqStages = 3;
+constexpr int kKVTile64 = kBK * kD * 2;   // 16 KB
+constexpr int kDsTile = kQ * kBK * 2;     // 16 KB: [128 q x 64 keys] bf16
+constexpr int kDqSmem = 1024 + 2 * kTileBytes + kDqStages * 2 * kKVTile64 + 2 * kDsTile + 256;
+
+struct BwdParams {
+  int T, H, n_tiles, ld;
+  const float *lse;   // [B, H, T]
+  const float *Drow;  // [B, H, T]
+  int *status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128
+                          const __grid_constant__ CUtensorMap map_kv,   // qkv, box 64 x 64
+                          const __grid_constant__ CUtensorMap map_do,   // dO [B][T][C], box 64 x 128
+                          const __grid_constant__ CUtensorMap map_dq,   // dqkv, box 64 x 128
+                          const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem, *sG = sQ + kTileBytes;
+  uint8_t *sKV = sG + kTileBytes;  // stage s: K at s*32K, V at s*32K + 16K
+  uint8_t *sDS = sKV + kDqStages * 2 * kKVTile64;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sDS + 2 * kDsTile);
+  // q_full, kv_full[3], kv_empty[3], s_full[2], s_empty[2], ds_full[2], ds_empty[2], fin, drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint32_t q_full = smem_u32(bars);
+  auto kv_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto kv_empty = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
+  auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
+  auto ds_full = [&](int s) { return smem_u32(bars + 11 + s); };
+  auto ds_empty = [&](int s) { return smem_u32(bars + 13 + s); };
+  const uint32_t fin = smem_u32(bars + 15), drain = smem_u32(bars + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = gridDim.x / p.n_tiles;
+  const int qt = p.n_tiles - 1 - (int)blockIdx.x / BH;
+  const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
+  const int q0 = qt * kQ;
+  const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK;
+  const int C = p.H * kD;
+  // TMEM columns: S[2] at 0, 64; dP[2] at 128, 192; dQ at 256
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kDqStages; ++s) { mbar_init(kv_full(s), 1); mbar_init(kv_empty(s), 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full(s), 1); mbar_init(s_empty(s), 128);
+      mbar_init(ds_full(s), 128); mbar_init(ds_empty(s), 1);
+    }
+    mbar_init(fin, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(q_full, 2 * kTileBytes);
+      for (int i = 0; i < 2; ++i) {
+        tma_load_3d(smem_u32(sQ) + i * 16384, &map_q, h * kD + 64 * i, q0, b, q_full);
+        tma_load_3d(smem_u32(sG) + i * 16384, &map_do, h * kD + 64 * i, q0, b, q_full);
+      }
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % kDqStages;
+        if (!mbar_wait(kv_empty(st), ((j / kDqStages) & 1) ^ 1, abort_flag, p.status)) break;
+        const uint32_t k_dst = smem_u32(sKV) + st * 2 * kKVTile64, v_dst = k_dst + kKVTile64;
+        mbar_expect_tx(kv_full(st), 2 * kKVTile64);
+        for (int i = 0; i < 2; ++i) {
+          tma_load_3d(k_dst + i * 8192, &map_kv, C + 64 * i, j * kBK, b, kv_full(st));
+          tma_load_3d(v_dst + i * 8192, &map_kv, C + kD + 64 * i, j * kBK, b, kv_full(st));
+        }
+        ++issued;
+      }
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
+      for (int j = max(0, issued - kDqStages); j < issued; ++j) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(kv_full(j % kDqStages), (j / kDqStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc(0, 0, kQ, kBK);   // Q K^T, dO V^T
+      const uint32_t idesc_q = make_idesc(0, 1, kQ, kD);    // dS K (K as MN-major B)
+      const uint32_t aQ = smem_u32(sQ), aG = smem_u32(sG);
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      auto issue_sdp = [&](int j) -> bool {
+        const int st = j % kDqStages, bb = j & 1;
+        if (!mbar_wait(kv_full(st), (j / kDqStages) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(s_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t bK = smem_u32(sKV) + st * 2 * kKVTile64, bV = bK + kKVTile64;
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+          const uint32_t oa = (s >> 2) * 16384 + (s & 3) * 32, ob = (s >> 2) * 8192 + (s & 3) * 32;
+          tc_mma(tmem + bb * kBK, smem_desc(aQ + oa, 16, 1024), smem_desc(bK + ob, 16, 1024), idesc_s, s > 0);
+          tc_mma(tmem + 128 + bb * kBK, smem_desc(aG + oa, 16, 1024), smem_desc(bV + ob, 16, 1024), idesc_s,
+                 s > 0);
+        }
+        tc_commit(s_full(bb));
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      if (ok && n_kv > 1) ok = issue_sdp(1);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int bb = j & 1, st = j % kDqStages;
+        if (!mbar_wait(ds_full(bb), (j >> 1) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t aS = smem_u32(sDS) + bb * kDsTile, bK = smem_u32(sKV) + st * 2 * kKVTile64;
+#pragma unroll
+        for (int s = 0; s < kBK / 16; ++s)
+          tc_mma(tmem + 256, smem_desc(aS + s * 32, 16, 1024), smem_desc(bK + s * 2048, 8192, 1024), idesc_q,
+                 (j > 0 || s > 0) ? 1u : 0u);
+        tc_commit(ds_empty(bb));
+        tc_commit(kv_empty(st));
+        if (j + 2 < n_kv && !issue_sdp(j + 2)) break;
+      }
+      tc_commit(fin);
+      tc_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int row = q0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sc = rsqrtf((float)kD) * kLog2e;
+    const int rr_ = min(row, p.T - 1);
+    const float L = p.lse[((int64_t)b * p.H + h) * p.T + rr_] * kLog2e;
+    const float Dv = p.Drow[((int64_t)b * p.H + h) * p.T + rr_];
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int bb = j & 1;
+      ok = mbar_wait(s_full(bb), (j >> 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const int kv0 = j * kBK;
+      const bool need_mask = kv0 + kBK > q0 || kv0 + kBK > p.T;
+      uint32_t packed[kBK / 2];
+#pragma unroll
+      for (int c = 0; c < kBK / 32; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(lane_base + bb * kBK + c * 32, sv);
+        tmem_ld32(lane_base + 128 + bb * kBK + c * 32, dv);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float d2[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            float pr = ex2(__uint_as_float(sv[i + t]) * sc - L);
+            const int key = kv0 + c * 32 + i + t;
+            if (need_mask && (key > row || key >= p.T)) pr = 0.f;
+            d2[t] = pr * (__uint_as_float(dv[i + t]) - Dv);
+          }
+          packed[(c * 32 + i) / 2] = pack2(d2[0], d2[1]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_empty(bb));
+      ok = mbar_wait(ds_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      uint8_t *dst = sDS + bb * kDsTile;
+#pragma unroll
+      for (int u = 0; u < kBK / 8; ++u)
+        *reinterpret_cast<uint4 *>(dst + r * 128 + ((u ^ (r & 7)) << 4)) =
+            make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(ds_full(bb));
+    }
+    if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float scale = rsqrtf((float)kD);
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_base + 256 + c * 32, rr);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack2(__uint_as_float(rr[8 * u + 0]) * scale, __uint_as_float(rr[8 * u + 1]) * scale);
+          w.y = pack2(__uint_as_float(rr[8 * u + 2]) * scale, __uint_as_float(rr[8 * u + 3]) * scale);
+          w.z = pack2(__uint_as_float(rr[8 * u + 4]) * scale, __uint_as_float(rr[8 * u + 5]) * scale);
+          w.w = pack2(__uint_as_float(rr[8 * u + 6]) * scale, __uint_as_float(rr[8 * u + 7]) * scale);
+          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, c * 4 + u)) = w;  // Q is no longer read
+        }
+      }
+    }
+    fence_proxy_async();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && warp == 2 && lane == 0) {
+      for (int i = 0; i < 2; ++i) tma_store_3d(&map_dq, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
+      bulk_commit();
+      bulk_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------- dK, dV: CTA = 128 keys of row b; loop over heads x 64-query tiles ----------------
+constexpr int kBQ2 = 64;
+constexpr int kKvStages = 3;
+constexpr int kQTile64 = kBQ2 * kD * 2;          // 16 KB
+constexpr int kQStage = 2 * kQTile64 + 1024;     // Q, dO, then L[64], D[64]; keeps 1 KB alignment
+constexpr int kPTile = kQ * kBQ2 * 2;            // [128 keys x 64 q] bf16, 16 KB
+constexpr int kKvSmemTc = 1024 + 2 * kTileBytes + kKvStages * kQStage + 2 * kPTile + 256;
+static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0 && kPTile % 1024 == 0,
+              "128-byte-swizzled TMA tiles need 1 KB-aligned shared-memory addresses");
+static_assert(kKvSmemTc <= 232448 && kDqSmem <= 232448 && kSmem <= 232448, "shared memory per CTA");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap map_k,    // qkv, box 64 x 128
+                            const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 64
+                            const __grid_constant__ CUtensorMap map_do,   // dO, box 64 x 64
+                            const __grid_constant__ CUtensorMap map_out,  // dqkv, box 64 x 128
+                            const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sK = smem, *sV = sK + kTileBytes;
+  uint8_t *sQS = sV + kTileBytes;                 // stage s at s*kQStage: Q, dO, L, D
+  uint8_t *sP = sQS + kKvStages * kQStage;        // P^T then dS^T (16 KB each)
+  uint8_t *sDS = sP + kPTile;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sDS + kPTile);
+  // kv_full, q_full[3], q_empty[3], s_full[2], s_empty[2], pds_full, pds_empty, fin, drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint32_t kv_full = smem_u32(bars);
+  auto q_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto q_empty = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
+  auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
+  const uint32_t pds_full = smem_u32(bars + 11), pds_empty = smem_u32(bars + 12);
+  const uint32_t fin = smem_u32(bars + 13), drain = smem_u32(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Bn = gridDim.x / p.n_tiles;
+  const int kt = (int)blockIdx.x / Bn;  // key tile 0 has the most work: launched first
+  const int b = (int)blockIdx.x % Bn;
+  const int k0 = kt * kQ;
+  const int C = p.H * kD;
+  const int first = k0 / kBQ2;
+  const int n_q = (p.T + kBQ2 - 1) / kBQ2 - first;
+  const int n_it = n_q * p.H;
+  // TMEM columns: S^T[2] at 0, 64; dP^T[2] at 128, 192; dV at 256; dK at 384
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < kKvStages; ++s) { mbar_init(q_full(s), 32); mbar_init(q_empty(s), 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(s_full(s), 1); mbar_init(s_empty(s), 128); }
+    mbar_init(pds_full, 128);
+    mbar_init(pds_empty, 1);
+    mbar_init(fin, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- producer warp: TMA for tiles, plain loads for lse and D ----------------
+    if (lane == 0) {
+      mbar_expect_tx(kv_full, 2 * kTileBytes);
+      for (int i = 0; i < 2; ++i) {
+        tma_load_3d(smem_u32(sK) + i * 16384, &map_k, C + 64 * i, k0, b, kv_full);
+        tma_load_3d(smem_u32(sV) + i * 16384, &map_k, C + kD + 64 * i, k0, b, kv_full);
+      }
+    }
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int st = it % kKvStages;
+      const bool okw = mbar_wait(q_empty(st), ((it / kKvStages) & 1) ^ 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      const int hh = it / n_q, qq0 = (first + it % n_q) * kBQ2;
+      uint8_t *stage = sQS + st * kQStage;
+      float *Ls = reinterpret_cast<float *>(stage + 2 * kQTile64), *Ds = Ls + kBQ2;
+      for (int i = lane; i < kBQ2; i += 32) {
+        const int q = min(qq0 + i, p.T - 1);
+        Ls[i] = p.lse[((int64_t)b * p.H + hh) * p.T + q] * kLog2e;
+        Ds[i] = p.Drow[((int64_t)b * p.H + hh) * p.T + q];
+      }
+      if (lane == 0) {
+        mbar_expect_tx(q_full(st), 2 * kQTile64);
+        const uint32_t dst = smem_u32(stage);
+        for (int i = 0; i < 2; ++i) {
+          tma_load_3d(dst + i * 8192, &map_q, hh * kD + 64 * i, qq0, b, q_full(st));
+          tma_load_3d(dst + kQTile64 + i * 8192, &map_do, hh * kD + 64 * i, qq0, b, q_full(st));
+        }
+      } else {
+        mbar_arrive(q_full(st));
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(kv_full, 0) && globaltimer() - t0 < kWaitNs) {}
+      for (int it = max(0, issued - kKvStages); it < issued; ++it) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(q_full(it % kKvStages), (it / kKvStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc(0, 0, kQ, kBQ2);  // K Q^T, V dO^T
+      const uint32_t idesc_g = make_idesc(0, 1, kQ, kD);    // P^T dO, dS^T Q
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
+      auto issue_s = [&](int it) -> bool {
+        const int st = it % kKvStages, bb = it & 1;
+        if (!mbar_wait(q_full(st), (it / kKvStages) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(s_empty(bb), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t bQ = smem_u32(sQS + st * kQStage), bG = bQ + kQTile64;
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+          const uint32_t oa = (s >> 2) * 16384 + (s & 3) * 32, ob = (s >> 2) * 8192 + (s & 3) * 32;
+          tc_mma(tmem + bb * kBQ2, smem_desc(aK + oa, 16, 1024), smem_desc(bQ + ob, 16, 1024), idesc_s, s > 0);
+          tc_mma(tmem + 128 + bb * kBQ2, smem_desc(aV + oa, 16, 1024), smem_desc(bG + ob, 16, 1024), idesc_s,
+                 s > 0);
+        }
+        tc_commit(s_full(bb));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && n_it > 1) ok = issue_s(1);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int st = it % kKvStages;
+        if (!mbar_wait(pds_full, it & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t bQ = smem_u32(sQS + st * kQStage), bG = bQ + kQTile64;
+        const uint32_t aP = smem_u32(sP), aS = smem_u32(sDS);
+#pragma unroll
+        for (int s = 0; s < kBQ2 / 16; ++s) {
+          const uint32_t acc = (it > 0 || s > 0) ? 1u : 0u;
+          tc_mma(tmem + 256, smem_desc(aP + s * 32, 16, 1024), smem_desc(bG + s * 2048, 8192, 1024), idesc_g, acc);
+          tc_mma(tmem + 384, smem_desc(aS + s * 32, 16, 1024), smem_desc(bQ + s * 2048, 8192, 1024), idesc_g, acc);
+        }
+        tc_commit(pds_empty);
+        tc_commit(q_empty(st));
+        if (it + 2 < n_it && !issue_s(it + 2)) break;
+      }
+      tc_commit(fin);
+      tc_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ---------------- softmax-backward warps: thread = key row ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sc = rsqrtf((float)kD) * kLog2e;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int bb = it & 1, st = it % kKvStages;
+      const int qq0 = (first + it % n_q) * kBQ2;
+      ok = mbar_wait(s_full(bb), (it >> 1) & 1, abort_flag, p.status) &&
+           mbar_wait(q_full(st), (it / kKvStages) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const float *Ls = reinterpret_cast<const float *>(sQS + st * kQStage + 2 * kQTile64), *Ds = Ls + kBQ2;
+      const bool need_mask = qq0 < k0 + kQ || qq0 + kBQ2 > p.T;
+      uint32_t pp[kBQ2 / 2], dd[kBQ2 / 2];
+#pragma unroll
+      for (int c = 0; c < kBQ2 / 32; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(lane_base + bb * kBQ2 + c * 32, sv);
+        tmem_ld32(lane_base + 128 + bb * kBQ2 + c * 32, dv);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int qi = c * 32 + i + t;
+            float v = ex2(__uint_as_float(sv[i + t]) * sc - Ls[qi]);
+            if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T)) v = 0.f;
+            pr[t] = v;
+            ds[t] = v * (__uint_as_float(dv[i + t]) - Ds[qi]);
+          }
+          pp[(c * 32 + i) / 2] = pack2(pr[0], pr[1]);
+          dd[(c * 32 + i) / 2] = pack2(ds[0], ds[1]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_empty(bb));
+      ok = mbar_wait(pds_empty, (it & 1) ^ 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+#pragma unroll
+      for (int u = 0; u < kBQ2 / 8; ++u) {
+        const int off = r * 128 + ((u ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4 *>(sP + off) = make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
+        *reinterpret_cast<uint4 *>(sDS + off) = make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(pds_full);
+    }
+    if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float scale = rsqrtf((float)kD);
+#pragma unroll 1
+      for (int g = 0; g < 2; ++g) {  // g = 0: dK (scaled) into the K tile, g = 1: dV into the V tile
+        uint8_t *dst = g == 0 ? sK : sV;
+        const float f = g == 0 ? scale : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(lane_base + (g == 0 ? 384 : 256) + c * 32, rr);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack2(__uint_as_float(rr[8 * u + 0]) * f, __uint_as_float(rr[8 * u + 1]) * f);
+            w.y = pack2(__uint_as_float(rr[8 * u + 2]) * f, __uint_as_float(rr[8 * u + 3]) * f);
+            w.z = pack2(__uint_as_float(rr[8 * u + 4]) * f, __uint_as_float(rr[8 * u + 5]) * f);
+            w.w = pack2(__uint_as_float(rr[8 * u + 6]) * f, __uint_as_float(rr[8 * u + 7]) * f);
+            *reinterpret_cast<uint4 *>(dst + tile_unit(r, c * 4 + u)) = w;
+          }
+        }
+      }
+    }
+    fence_proxy_async();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && warp == 2 && lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        tma_store_3d(&map_out, smem_u32(sK) + i * 16384, C + 64 * i, k0, b);
+        tma_store_3d(&map_out, smem_u32(sV) + i * 16384, C + kD + 64 * i, k0, b);
+      }
+      bulk_commit();
+      bulk_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------- host side -------------------------------
 
 // 3-D bf16 map over [B][T][cols] with row stride ld elements.
@@ -309,7 +779,12 @@ inline bool make_map3(CUtensorMap *map, const void *base, int B, int T, int cols
 }
 
 inline cudaError_t init() {
-  return cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemTc);
+  return e;
 }
 
 inline bool supported(const void *qkv, int64_t ld, const void *O) {
@@ -331,6 +806,39 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.status = status;
   attn_fwd_tc_kernel<<<B * H * p.n_qt, kThreads, kSmem, st>>>(mqk, mv, mo, p);
   return cudaGetLastError();
+}
+
+}  // namespace fatc
+}  // namespace nc
+
+namespace nc {
+namespace fatc {
+
+inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *dO, const float *lse, const float *Drow,
+                              bf16 *dqkv, int B, int T, int H, int *status, cudaStream_t st) {
+  CUtensorMap mq128, mkv64, mdo128, mdo64, mout;
+  const int C = H * kD;
+  if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mkv64, qkv, B, T, (int)ld, ld, 64) ||
+      !make_map3(&mdo128, dO, B, T, C, C, 128) || !make_map3(&mdo64, dO, B, T, C, C, 64) ||
+      !make_map3(&mout, dqkv, B, T, (int)ld, ld, 128))
+    return cudaErrorInvalidValue;
+  BwdParams p;
+  p.T = T;
+  p.H = H;
+  p.ld = (int)ld;
+  p.lse = lse;
+  p.Drow = Drow;
+  p.status = status;
+  p.n_tiles = (T + kQ - 1) / kQ;
+  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kThreads, kDqSmem, st>>>(mq128, mkv64, mdo128, mout, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kThreads, kKvSmemTc, st>>>(mq128, mkv64, mdo64, mout, p);
+  return cudaGetLastError();
+}
+
+inline bool supported_bwd(const void *qkv, int64_t ld, const void *dO, const void *dqkv) {
+  return supported(qkv, ld, dO) && ((uintptr_t)dqkv & 15) == 0;
 }
 
 }  // namespace fatc

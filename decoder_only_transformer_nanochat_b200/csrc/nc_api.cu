@@ -312,7 +312,7 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
                                                                                 M, T_len, H)));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
            if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
-                                  m->num_sms, 0, st) != cudaSuccess) return NC_ECUDA);
+                                  m->num_sms, 0, m->status, st) != cudaSuccess) return NC_ECUDA);
     NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
            (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
                w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
@@ -621,10 +621,10 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
   cudaError_t e;
   if (dtype == NC_BF16) {
     attn_rowdot_kernel<bf16><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const bf16 *)dO, (const bf16 *)O, Drow, M, T, H);
-    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms, engine, st);
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   } else if (dtype == NC_F32) {
     attn_rowdot_kernel<float><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const float *)dO, (const float *)O, Drow, M, T, H);
-    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H, num_sms, engine, st);
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   } else {
     return NC_EUNSUPPORTED;
   }
