@@ -193,12 +193,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float s[kKV];
+      {
+        uint32_t rr[kKV / 32][32];
 #pragma unroll
-      for (int c = 0; c < kKV / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + st * kKV + c * 32, rr);
+        for (int c = 0; c < kKV / 32; ++c) tmem_ld32_nw(lane_base + st * kKV + c * 32, rr[c]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]) * sc;
+        for (int c = 0; c < kKV / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[c][i]) * sc;
       }
       tc_fence_before();
       mbar_arrive(s_empty(st));
@@ -308,6 +311,12 @@ constexpr int kKVTile64 = kBK * kD * 2;   // 16 KB
 constexpr int kDsTile = kQ * kBK * 2;     // 16 KB: [128 q x 64 keys] bf16
 constexpr int kDqSmem = 1024 + 2 * kTileBytes + kDqStages * 2 * kKVTile64 + 2 * kDsTile + 256;
 
+// backward kernels: warp 0 TMA, warp 1 MMA, warps 2..9 element-wise; the
+// element-wise warps w and w+4 share TMEM lane quarter (w & 3) and split the
+// tile's columns between them (warpgroup g = (w - 2) / 4 takes half g)
+constexpr int kBwdThreads = 320;
+constexpr int kSoft = 256;
+
 struct BwdParams {
   int T, H, n_tiles, ld;
   const float *lse;   // [B, H, T]
@@ -315,7 +324,7 @@ struct BwdParams {
   int *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128
                           const __grid_constant__ CUtensorMap map_kv,   // qkv, box 64 x 64
                           const __grid_constant__ CUtensorMap map_do,   // dO [B][T][C], box 64 x 128
@@ -351,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < kDqStages; ++s) { mbar_init(kv_full(s), 1); mbar_init(kv_empty(s), 1); }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full(s), 1); mbar_init(s_empty(s), 128);
-      mbar_init(ds_full(s), 128); mbar_init(ds_empty(s), 1);
+      mbar_init(s_full(s), 1); mbar_init(s_empty(s), kSoft);
+      mbar_init(ds_full(s), kSoft); mbar_init(ds_empty(s), 1);
     }
     mbar_init(fin, 1);
     mbar_init(drain, 1);
@@ -434,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
     }
   } else {
-    const int quarter = warp & 3;
+    // ---------------- element-wise warps: thread = query row, half g of the keys ----------------
+    const int quarter = warp & 3, g = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int row = q0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -442,42 +452,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rr_ = min(row, p.T - 1);
     const float L = p.lse[((int64_t)b * p.H + h) * p.T + rr_] * kLog2e;
     const float Dv = p.Drow[((int64_t)b * p.H + h) * p.T + rr_];
+    const int c0 = g * 32;  // this thread's 32 keys of the 64-key tile
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int bb = j & 1;
       ok = mbar_wait(s_full(bb), (j >> 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const int kv0 = j * kBK;
-      const bool need_mask = kv0 + kBK > q0 || kv0 + kBK > p.T;
-      uint32_t packed[kBK / 2];
-#pragma unroll
-      for (int c = 0; c < kBK / 32; ++c) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + bb * kBK + c * 32, sv);
-        tmem_ld32(lane_base + 128 + bb * kBK + c * 32, dv);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float d2[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            float pr = ex2(__uint_as_float(sv[i + t]) * sc - L);
-            const int key = kv0 + c * 32 + i + t;
-            if (need_mask && (key > row || key >= p.T)) pr = 0.f;
-            d2[t] = pr * (__uint_as_float(dv[i + t]) - Dv);
-          }
-          packed[(c * 32 + i) / 2] = pack2(d2[0], d2[1]);
-        }
-      }
+      uint32_t sv[32], dv[32];
+      tmem_ld32_nw(lane_base + bb * kBK + c0, sv);
+      tmem_ld32_nw(lane_base + 128 + bb * kBK + c0, dv);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty(bb));
+      const int kv0 = j * kBK + c0;
+      const bool need_mask = kv0 + 32 > q0 || kv0 + 32 > p.T;
+      uint32_t packed[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float d2[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          float pr = ex2(__uint_as_float(sv[i + t]) * sc - L);
+          const int key = kv0 + i + t;
+          if (need_mask && (key > row || key >= p.T)) pr = 0.f;
+          d2[t] = pr * (__uint_as_float(dv[i + t]) - Dv);
+        }
+        packed[i / 2] = pack2(d2[0], d2[1]);
+      }
       ok = mbar_wait(ds_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       uint8_t *dst = sDS + bb * kDsTile;
 #pragma unroll
-      for (int u = 0; u < kBK / 8; ++u)
-        *reinterpret_cast<uint4 *>(dst + r * 128 + ((u ^ (r & 7)) << 4)) =
+      for (int u = 0; u < 4; ++u) {
+        const int uu = 4 * g + u;
+        *reinterpret_cast<uint4 *>(dst + r * 128 + ((uu ^ (r & 7)) << 4)) =
             make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+      }
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(ds_full(bb));
@@ -488,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float scale = rsqrtf((float)kD);
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 2 * g; c < 2 * g + 2; ++c) {  // 64 of the 128 dQ columns
         uint32_t rr[32];
         tmem_ld32(lane_base + 256 + c * 32, rr);
 #pragma unroll
@@ -503,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     fence_proxy_async();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok && warp == 2 && lane == 0) {
       for (int i = 0; i < 2; ++i) tma_store_3d(&map_dq, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
       bulk_commit();
@@ -530,7 +541,7 @@ static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0 && kPTile % 1024 == 
               "128-byte-swizzled TMA tiles need 1 KB-aligned shared-memory addresses");
 static_assert(kKvSmemTc <= 232448 && kDqSmem <= 232448 && kSmem <= 232448, "shared memory per CTA");
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap map_k,    // qkv, box 64 x 128
                             const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 64
                             const __grid_constant__ CUtensorMap map_do,   // dO, box 64 x 64
@@ -566,9 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMEM columns: S^T[2] at 0, 64; dP^T[2] at 128, 192; dV at 256; dK at 384
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < kKvStages; ++s) { mbar_init(q_full(s), 32); mbar_init(q_empty(s), 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(s_full(s), 1); mbar_init(s_empty(s), 128); }
-    mbar_init(pds_full, 128);
+    for (int s = 0; s < kKvStages; ++s) { mbar_init(q_full(s), 33); mbar_init(q_empty(s), 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(s_full(s), 1); mbar_init(s_empty(s), kSoft); }
+    mbar_init(pds_full, kSoft);
     mbar_init(pds_empty, 1);
     mbar_init(fin, 1);
     mbar_init(drain, 1);
@@ -597,12 +608,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, okw)) break;
       const int hh = it / n_q, qq0 = (first + it % n_q) * kBQ2;
       uint8_t *stage = sQS + st * kQStage;
-      float *Ls = reinterpret_cast<float *>(stage + 2 * kQTile64), *Ds = Ls + kBQ2;
+      // lse and D of the tile's queries: 4-byte asynchronous copies whose
+      // completion arrives on the stage's barrier, so this warp never blocks
+      const uint32_t ls_dst = smem_u32(stage + 2 * kQTile64), ds_dst = ls_dst + kBQ2 * 4;
       for (int i = lane; i < kBQ2; i += 32) {
         const int q = min(qq0 + i, p.T - 1);
-        Ls[i] = p.lse[((int64_t)b * p.H + hh) * p.T + q] * kLog2e;
-        Ds[i] = p.Drow[((int64_t)b * p.H + hh) * p.T + q];
+        const int64_t gi = ((int64_t)b * p.H + hh) * p.T + q;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ls_dst + 4 * i), "l"(p.lse + gi) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ds_dst + 4 * i), "l"(p.Drow + gi) : "memory");
       }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(q_full(st)) : "memory");
       if (lane == 0) {
         mbar_expect_tx(q_full(st), 2 * kQTile64);
         const uint32_t dst = smem_u32(stage);
@@ -610,11 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(dst + i * 8192, &map_q, hh * kD + 64 * i, qq0, b, q_full(st));
           tma_load_3d(dst + kQTile64 + i * 8192, &map_do, hh * kD + 64 * i, qq0, b, q_full(st));
         }
-      } else {
-        mbar_arrive(q_full(st));
       }
       ++issued;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       const uint64_t t0 = globaltimer();
       while (!mbar_try(kv_full, 0) && globaltimer() - t0 < kWaitNs) {}
@@ -669,50 +683,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
     }
   } else {
-    // ---------------- softmax-backward warps: thread = key row ----------------
-    const int quarter = warp & 3;
+    // ---------------- element-wise warps: thread = key row, half g of the queries ----------------
+    const int quarter = warp & 3, g = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = rsqrtf((float)kD) * kLog2e;
+    const int c0 = g * 32;  // this thread's 32 queries of the 64-query tile
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int bb = it & 1, st = it % kKvStages;
-      const int qq0 = (first + it % n_q) * kBQ2;
+      const int qq0 = (first + it % n_q) * kBQ2 + c0;
       ok = mbar_wait(s_full(bb), (it >> 1) & 1, abort_flag, p.status) &&
            mbar_wait(q_full(st), (it / kKvStages) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const float *Ls = reinterpret_cast<const float *>(sQS + st * kQStage + 2 * kQTile64), *Ds = Ls + kBQ2;
-      const bool need_mask = qq0 < k0 + kQ || qq0 + kBQ2 > p.T;
-      uint32_t pp[kBQ2 / 2], dd[kBQ2 / 2];
-#pragma unroll
-      for (int c = 0; c < kBQ2 / 32; ++c) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + bb * kBQ2 + c * 32, sv);
-        tmem_ld32(lane_base + 128 + bb * kBQ2 + c * 32, dv);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pr[2], ds[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int qi = c * 32 + i + t;
-            float v = ex2(__uint_as_float(sv[i + t]) * sc - Ls[qi]);
-            if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T)) v = 0.f;
-            pr[t] = v;
-            ds[t] = v * (__uint_as_float(dv[i + t]) - Ds[qi]);
-          }
-          pp[(c * 32 + i) / 2] = pack2(pr[0], pr[1]);
-          dd[(c * 32 + i) / 2] = pack2(ds[0], ds[1]);
-        }
-      }
+      uint32_t sv[32], dv[32];
+      tmem_ld32_nw(lane_base + bb * kBQ2 + c0, sv);
+      tmem_ld32_nw(lane_base + 128 + bb * kBQ2 + c0, dv);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty(bb));
+      const float4 *Ls4 = reinterpret_cast<const float4 *>(sQS + st * kQStage + 2 * kQTile64) + c0 / 4;
+      const float4 *Ds4 = Ls4 + kBQ2 / 4;
+      const bool need_mask = qq0 < key + 1 || qq0 + 32 > p.T;
+      uint32_t pp[16], dd[16];
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 l4 = Ls4[i4], d4 = Ds4[i4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float pr[4], ds[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int qi = 4 * i4 + t;
+          float v = ex2(__uint_as_float(sv[qi]) * sc - lv[t] * kLog2e);
+          if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T)) v = 0.f;
+          pr[t] = v;
+          ds[t] = v * (__uint_as_float(dv[qi]) - dvv[t]);
+        }
+        pp[2 * i4] = pack2(pr[0], pr[1]);
+        pp[2 * i4 + 1] = pack2(pr[2], pr[3]);
+        dd[2 * i4] = pack2(ds[0], ds[1]);
+        dd[2 * i4 + 1] = pack2(ds[2], ds[3]);
+      }
       ok = mbar_wait(pds_empty, (it & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
 #pragma unroll
-      for (int u = 0; u < kBQ2 / 8; ++u) {
-        const int off = r * 128 + ((u ^ (r & 7)) << 4);
+      for (int u = 0; u < 4; ++u) {
+        const int off = r * 128 + (((4 * g + u) ^ (r & 7)) << 4);
         *reinterpret_cast<uint4 *>(sP + off) = make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
         *reinterpret_cast<uint4 *>(sDS + off) = make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
       }
@@ -724,29 +742,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      const float scale = rsqrtf((float)kD);
+      // warpgroup 0 drains dK (scaled) into the K tile, warpgroup 1 dV into the V tile
+      uint8_t *dst = g == 0 ? sK : sV;
+      const float f = g == 0 ? rsqrtf((float)kD) : 1.f;
 #pragma unroll 1
-      for (int g = 0; g < 2; ++g) {  // g = 0: dK (scaled) into the K tile, g = 1: dV into the V tile
-        uint8_t *dst = g == 0 ? sK : sV;
-        const float f = g == 0 ? scale : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(lane_base + (g == 0 ? 384 : 256) + c * 32, rr);
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_base + (g == 0 ? 384 : 256) + c * 32, rr);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack2(__uint_as_float(rr[8 * u + 0]) * f, __uint_as_float(rr[8 * u + 1]) * f);
-            w.y = pack2(__uint_as_float(rr[8 * u + 2]) * f, __uint_as_float(rr[8 * u + 3]) * f);
-            w.z = pack2(__uint_as_float(rr[8 * u + 4]) * f, __uint_as_float(rr[8 * u + 5]) * f);
-            w.w = pack2(__uint_as_float(rr[8 * u + 6]) * f, __uint_as_float(rr[8 * u + 7]) * f);
-            *reinterpret_cast<uint4 *>(dst + tile_unit(r, c * 4 + u)) = w;
-          }
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack2(__uint_as_float(rr[8 * u + 0]) * f, __uint_as_float(rr[8 * u + 1]) * f);
+          w.y = pack2(__uint_as_float(rr[8 * u + 2]) * f, __uint_as_float(rr[8 * u + 3]) * f);
+          w.z = pack2(__uint_as_float(rr[8 * u + 4]) * f, __uint_as_float(rr[8 * u + 5]) * f);
+          w.w = pack2(__uint_as_float(rr[8 * u + 6]) * f, __uint_as_float(rr[8 * u + 7]) * f);
+          *reinterpret_cast<uint4 *>(dst + tile_unit(r, c * 4 + u)) = w;
         }
       }
     }
     fence_proxy_async();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok && warp == 2 && lane == 0) {
       for (int i = 0; i < 2; ++i) {
         tma_store_3d(&map_out, smem_u32(sK) + i * 16384, C + 64 * i, k0, b);
@@ -830,10 +845,10 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *dO, const
   p.Drow = Drow;
   p.status = status;
   p.n_tiles = (T + kQ - 1) / kQ;
-  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kThreads, kDqSmem, st>>>(mq128, mkv64, mdo128, mout, p);
+  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mkv64, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kThreads, kKvSmemTc, st>>>(mq128, mkv64, mdo64, mout, p);
+  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mkv64, mdo64, mout, p);
   return cudaGetLastError();
 }
 
