@@ -273,9 +273,10 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   float *tl = token_loss ? token_loss : w.tok_loss;
   const float inv_M = 1.f / (float)M;
   if (sizeof(T) == 2 && V == 65536) {
+    const int grid = M < m->num_sms ? M : m->num_sms;
     NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
-           (ce_fused_bf16_kernel<16><<<M, 512, 0, st>>>((bf16 *)w.z, w.ldz, targets, tl, M, V,
-                                                        inv_M, m->status)));
+           (ce_fused_bf16_persistent_kernel<8><<<grid, kCeThreads, V * 2, st>>>(
+               (bf16 *)w.z, w.ldz, targets, tl, M, V, inv_M, m->status)));
   } else {
     NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
            (ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(w.z, w.ldz, targets, tl, M, V, inv_M,
@@ -361,7 +362,9 @@ int op_device_sms(int *num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
   if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
-  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess) return NC_ECUDA;
+  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess ||
+      cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           65536 * 2) != cudaSuccess) return NC_ECUDA;
   return NC_OK;
 }
 
@@ -421,7 +424,9 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
-  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess) {
+  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess ||
+      cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           65536 * 2) != cudaSuccess) {
     nc_destroy(m);
     return NC_ECUDA;
   }
