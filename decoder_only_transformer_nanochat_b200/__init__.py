@@ -10,7 +10,8 @@ from ._binding import (NC_BF16, NC_EALIGN, NC_ECUDA, NC_EINVAL, NC_ENOMEM,  # no
                        nc_get_dims, nc_init, nc_param_layout, nc_strerror, nc_sync_status,
                        nc_workspace_bytes, nc_gemm, nc_attention_fwd, nc_attention_bwd,
                        NC_EPI_STORE, NC_EPI_STORE_F32, NC_EPI_ADD, NC_EPI_RELU2, NC_EPI_DRELU2,
-                       NC_EPI_SOFTCAP, nc_profile, nc_profile_read)
+                       NC_EPI_SOFTCAP, nc_profile, nc_profile_read,
+                       nc_attention_bwd_noalloc, NC_ATTN_BWD_NOALLOC_MAX_ROWS)
 
 
 def __getattr__(name):

@@ -64,6 +64,7 @@ _SIGS = {
     "nc_sync_status": (_I, [_P, _P, _I]),
     "nc_strerror": (ctypes.c_char_p, [_I]),
     "nc_destroy": (None, [_P]),
+    "nc_attention_bwd_noalloc": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "nc_profile": (_I, [_P, _I]),
     "nc_profile_read": (_I, [_P, ctypes.POINTER(nc_kernel_stat), _I, ctypes.POINTER(_I)]),
     "nc_gemm": (_I, [_P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _I,
@@ -174,3 +175,13 @@ def nc_profile_read(handle, max_classes: int = 32):
     out = [dict(name=arr[i].name.decode(), launches=arr[i].launches, ms=arr[i].ms,
                 flops=arr[i].flops, bytes=arr[i].bytes) for i in range(n.value)]
     return rc, out
+
+
+NC_ATTN_BWD_NOALLOC_MAX_ROWS = 1 << 20
+
+
+def nc_attention_bwd_noalloc(qkv, ld, O, dO, lse, dqkv, B, T, H, dtype, engine, stream) -> int:
+    """nc_attention_bwd without the Drow scratch argument: the library's fixed
+    device scratch is used instead, for callers that cannot allocate."""
+    return load_library().nc_attention_bwd_noalloc(qkv, ld, O, dO, lse, dqkv, B, T, H, dtype, engine,
+                                                   stream)

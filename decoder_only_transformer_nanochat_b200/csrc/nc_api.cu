@@ -14,6 +14,7 @@
 #include <string.h>
 
 #include <chrono>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -358,6 +359,26 @@ int check_step_args(const nc_model *m, const void *weights, const int32_t *token
 }
 
 
+// Fixed device scratch of nc_attention_bwd_noalloc (rowsum(dO * O)), and its
+// device address per device, looked up once with that device current.
+static __device__ __align__(256) float g_attn_bwd_rowdot[NC_ATTN_BWD_NOALLOC_MAX_ROWS];
+constexpr int kMaxDevices = 64;
+static float *g_attn_bwd_rowdot_addr[kMaxDevices] = {};
+static std::mutex g_attn_bwd_rowdot_mutex;
+
+int noalloc_scratch(float **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NC_ECUDA;
+  std::lock_guard<std::mutex> lock(g_attn_bwd_rowdot_mutex);
+  if (!g_attn_bwd_rowdot_addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_attn_bwd_rowdot) != cudaSuccess || !ptr) return NC_ECUDA;
+    g_attn_bwd_rowdot_addr[dev] = static_cast<float *>(ptr);
+  }
+  *out = g_attn_bwd_rowdot_addr[dev];
+  return NC_OK;
+}
+
 int op_device_sms(int *num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
@@ -549,6 +570,34 @@ int nc_profile_read(nc_model *m, nc_kernel_stat *out, int max, int *count) {
   m->events_used = 0;
   for (int c = 0; c < K_NUM_CLASSES; ++c) { m->launches[c] = 0; m->flops[c] = 0; m->bytes[c] = 0; }
   return rc;
+}
+
+int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,
+                             const float *lse, void *dqkv, int B, int T, int H, int dtype,
+                             int engine, void *stream) {
+  if (!qkv || !O || !dO || !lse || !dqkv) return NC_EINVAL;
+  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
+  if ((int64_t)B * H * T > NC_ATTN_BWD_NOALLOC_MAX_ROWS) return NC_ENOMEM;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  float *Drow = nullptr;
+  int rc = noalloc_scratch(&Drow);
+  if (rc != NC_OK) return rc;
+  int num_sms = 0;
+  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int M = B * T;
+  cudaError_t e;
+  if (dtype == NC_BF16) {
+    attn_rowdot_kernel<bf16><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const bf16 *)dO, (const bf16 *)O, Drow, M, T, H);
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms,
+                              engine, nullptr, st);
+  } else {
+    attn_rowdot_kernel<float><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const float *)dO, (const float *)O, Drow, M, T, H);
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H,
+                               num_sms, engine, nullptr, st);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 const char *nc_strerror(int code) {

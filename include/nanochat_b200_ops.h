@@ -67,6 +67,38 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
                      float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
                      void *stream);
 
+/* Largest B*H*T that nc_attention_bwd_noalloc accepts: the number of fp32
+ * entries of its fixed device scratch (4 MiB). */
+#define NC_ATTN_BWD_NOALLOC_MAX_ROWS (1 << 20)
+
+/* nc_attention_bwd for callers that cannot allocate device memory: the same
+ * computation and arguments minus Drow.  No passage of the nanochat pages
+ * corresponds to this entry point; it exists for the library's users.
+ *
+ * Who needs it: code that must not call cudaMalloc or any allocating routine
+ * -- for example a process whose device memory is handed out once at start-up
+ * by its own allocator and may not grow, or a latency-sensitive loop that
+ * cannot afford the device-wide synchronisation cudaMalloc/cudaFree imply --
+ * but still has to run the attention backward, which needs a B*H*T fp32
+ * scratch for rowsum(dO * O).
+ *
+ * What it does instead: the scratch is a file-scope device array of
+ * NC_ATTN_BWD_NOALLOC_MAX_ROWS floats inside the library, so every GPU that
+ * loads the library holds those 4 MiB until the process exits.  The first
+ * call on a device looks the array's device address up (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any
+ * stream capture.  The call itself allocates nothing.
+ *
+ * Limits and sharing: B*H*T > NC_ATTN_BWD_NOALLOC_MAX_ROWS returns NC_ENOMEM
+ * before anything is enqueued.  Every call on a device uses the same array and
+ * leaves its contents behind; each call overwrites every entry it reads, so no
+ * clearing is needed between calls, but two calls that overlap on the GPU
+ * (different streams, or different host threads) race on the array and give
+ * wrong results: serialise them. */
+int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,
+                             const float *lse, void *dqkv, int B, int T, int H, int dtype,
+                             int engine, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
