@@ -376,6 +376,287 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ===========================================================================
+// Two-CTA version (cta_group::2): a cluster of 2 CTAs on neighbouring SMs
+// computes a 256 x 256 tile.  CTA r owns rows [128r, 128r+128) of the tile
+// (its A slice and its half of the accumulator) and loads half of B
+// (tile columns [128r, 128r+128)); the leader (r = 0) issues every MMA, which
+// reads A and B from both CTAs' shared memory.  Per SM a k-block moves 32 KB
+// instead of 48 KB for the same flops, so six stages fit and L2 traffic for
+// the B operand halves.  Both CTAs' TMA loads complete on the leader's "full"
+// barrier; the leader's commits arrive on both CTAs' "empty" and "tmem full"
+// barriers; both CTAs' epilogue threads release the accumulator on the
+// leader's "tmem empty" barrier.
+constexpr int BN2 = 256, BH2 = 128;                  // tile N, B rows per CTA
+constexpr int STAGES2 = 6;
+constexpr int STAGE_BYTES2 = A_BYTES + BH2 * BK * 2;  // 32 KB
+constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + 256;
+static_assert(SMEM_BYTES2 <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// arrive on the barrier at the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
+      "r"(rank)
+      : "memory");
+}
+// shared::cluster address of the location at this offset in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// barrier `bar_cluster` (a shared::cluster address: the pair leader's barrier)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// commit of the pair's MMAs, arriving on the barrier at this offset in every CTA of `mask`
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ Unit unit_of2(const Params &p, int u) {
+  // p.n_m counts 256-row blocks here
+  return unit_of(p, u);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const __grid_constant__ CUtensorMap map_d, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *staging = smem + STAGES2 * STAGE_BYTES2;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(staging + STAGING_BYTES);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, aux
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES2 + 6);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES2 + s); };
+  auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * STAGES2 + a); };
+  auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * STAGES2 + 2 + a); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * STAGES2 + 4);
+  const uint32_t aux_bar = smem_u32(bars + 2 * STAGES2 + 5);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 256);  // both CTAs' epilogue threads
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(aux_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = cluster; u < p.units && ok; u += n_clusters) {
+        const Unit x = unit_of2(p, u);
+        const int m_row = x.m_blk * 256 + (int)rank * BM;
+        const int n_row = x.n_blk * BN2 + (int)rank * BH2;
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
+          const uint32_t sb = sa + A_BYTES;
+          if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES2);
+          const uint32_t fb = cluster_addr(full_bar(stage), 0);
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_2d_pair(sa, &map_a, k0, m_row, fb);
+          } else {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d_pair(sa + i * 8192, &map_a, m_row + 64 * i, k0, fb);
+          }
+          if (!p.b_mn) {
+            tma_load_2d_pair(sb, &map_b, k0, n_row, fb);
+          } else {
+#pragma unroll
+            for (int i = 0; i < BH2 / 64; ++i) tma_load_2d_pair(sb + i * 8192, &map_b, n_row + 64 * i, k0, fb);
+          }
+          ++issued;
+          if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+        }
+      }
+      // our copies complete on the leader's barriers; every one of them is
+      // consumed by an MMA before the leader's final commit, which the final
+      // cluster barrier orders before either CTA exits
+      (void)issued;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = make_idesc(p.a_mn, p.b_mn, 256, BN2);
+      const uint32_t a_lbo = p.a_mn ? 8192 : 16, a_kstep = p.a_mn ? 2048 : 32;
+      const uint32_t b_lbo = p.b_mn ? 8192 : 16, b_kstep = p.b_mn ? 2048 : 32;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = cluster; u < p.units && ok; u += n_clusters) {
+        const Unit x = unit_of2(p, u);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN2;
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_pair(d_tmem, smem_desc(sa + kk * a_kstep, a_lbo, 1024), smem_desc(sb + kk * b_kstep, b_lbo, 1024),
+                        idesc, (kb > x.kb0 || kk > 0) ? 1u : 0u);
+          tc_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull_bar(acc), 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      tc_commit_pair(drain_bar, 0x1);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const bool ep_leader = warp == 2 && lane == 0;
+    const bool f32_out = p.epi == EPI_STORE_F32;
+    const bool aux = p.epi == EPI_ADD || p.epi == EPI_DRELU2;
+    const uint32_t st_addr = smem_u32(staging);
+    int acc = 0;
+    uint32_t acc_phase = 0, aux_phase = 0;
+    bool ok = true;
+    auto release_tmem = [&](int a) {
+      tc_fence_before();
+      if (leader) mbar_arrive(tempty_bar(a));
+      else mbar_arrive_remote(tempty_bar(a), 0);
+    };
+    for (int u = cluster; u < p.units && ok; u += n_clusters) {
+      const Unit x = unit_of2(p, u);
+      ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      __syncwarp();
+      if (!ok) break;
+      tc_fence_after();
+      const int m0 = x.m_blk * 256 + (int)rank * BM;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN2;
+      if (f32_out) {
+        const int m = m0 + r;
+#pragma unroll 1
+        for (int c = 0; c < BN2 / 32; ++c) {
+          const int n = x.n_blk * BN2 + c * 32;
+          if (n >= p.N) break;  // warp-uniform
+          uint32_t rr[32];
+          tmem_ld32(t_row + c * 32, rr);
+          if (m < p.M) epilogue_chunk(p, m, n, rr);
+        }
+        release_tmem(acc);
+      } else {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const int n_half = x.n_blk * BN2 + half * 128;
+          const bool box1 = n_half + 64 < p.N;
+          if (ep_leader) {
+            bulk_wait_read0();
+            if (aux) {
+              mbar_expect_tx(aux_bar, box1 ? 2 * BM * 128 : BM * 128);
+              tma_load_2d(st_addr, &map_d, n_half, m0, aux_bar);
+              if (box1) tma_load_2d(st_addr + BM * 128, &map_d, n_half + 64, m0, aux_bar);
+            }
+          }
+          if (aux) {
+            ok = epi_vote_all(mbar_wait(aux_bar, aux_phase, abort_flag, p.status));
+            aux_phase ^= 1;
+            if (!ok) break;
+          } else {
+            epi_bar();
+          }
+          __syncwarp();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(t_row + half * 128 + c * 32, rr);
+            epilogue_stage(p.epi, staging, r, c, rr);
+          }
+          if (half == 1 || n_half + 128 >= p.N) release_tmem(acc);
+          fence_proxy_async();
+          epi_bar();
+          if (ep_leader) {
+            tma_store_2d(&map_d, st_addr, n_half, m0);
+            if (box1) tma_store_2d(&map_d, st_addr + BM * 128, n_half + 64, m0);
+            bulk_commit();
+          }
+          if (n_half + 128 >= p.N) break;
+        }
+        if (!ok) break;
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (ep_leader) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer can still signal or read it
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ------------------------------- host side -------------------------------
 
 // 2D bf16 map over a row-major [rows, cols] matrix with row stride ld
@@ -424,8 +705,11 @@ inline cudaError_t tc_init() {
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
     tc::encode_fn() = reinterpret_cast<tc::EncodeTiledFn>(fn);
   }
-  return cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              tc::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(tc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       tc::SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES2);
+  return e;
 }
 
 template <typename T>
@@ -438,7 +722,12 @@ inline bool tc_gemm_supported(const GemmProblem &p) {
   return tc::encode_fn() != nullptr;
 }
 
-inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status, cudaStream_t st) {
+inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *status, cudaStream_t st);
+
+// pair = 1: the two-CTA kernel (M >= 256), pair = 0: the one-CTA kernel
+inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status, cudaStream_t st,
+                                  int pair = 1) {
+  if (pair && g.M >= 256) return launch_gemm_tc2(g, num_sms, status, st);
   using namespace tc;
   CUtensorMap ma, mb;
   bool ok;
@@ -475,6 +764,59 @@ inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status
   const int grid = p.units < num_sms ? p.units : num_sms;
   gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, md, p);
   return cudaGetLastError();
+}
+
+}  // namespace nc
+
+namespace nc {
+
+inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *status, cudaStream_t st) {
+  using namespace tc;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (!g.a_mn) ok = make_map(&ma, g.A, g.M, g.K, g.lda, 64, BM);
+  else ok = make_map(&ma, g.A, g.K, g.M, g.lda, 64, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  if (!g.b_mn) ok = make_map(&mb, g.B, g.N, g.K, g.ldb, 64, BH2);
+  else ok = make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  CUtensorMap md = ma;
+  if (g.epi != EPI_STORE_F32 && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
+  Params p;
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.n_m = (g.M + 255) / 256;
+  p.n_n = (g.N + BN2 - 1) / BN2;
+  p.kblocks = (g.K + BK - 1) / BK;
+  const int n_clusters = num_sms / 2;
+  const int tiles = p.n_m * p.n_n;
+  p.splits = g.epi == EPI_STORE_F32 ? choose_splits(tiles, p.kblocks, n_clusters) : 1;
+  {
+    const int per = (p.kblocks + p.splits - 1) / p.splits;
+    p.splits = (p.kblocks + per - 1) / per;
+  }
+  p.units = tiles * p.splits;
+  p.a_mn = g.a_mn; p.b_mn = g.b_mn;
+  p.D = g.D; p.ldd = g.ldd; p.epi = g.epi;
+  p.atomic_out = p.splits > 1;
+  p.status = status;
+  if (p.atomic_out) {
+    cudaError_t e = cudaMemset2DAsync(g.D, (size_t)g.ldd * 4, 0, (size_t)g.N * 4, (size_t)g.M, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int clusters = p.units < n_clusters ? p.units : n_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES2;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, mb, md, p);
 }
 
 }  // namespace nc

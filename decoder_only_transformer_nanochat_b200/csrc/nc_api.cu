@@ -638,7 +638,8 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == NC_BF16) {
-    if (engine == 0 && tc_gemm_supported<bf16>(p)) e = launch_gemm_tc(p, num_sms, nullptr, st);
+    if ((engine == 0 || engine == 2) && tc_gemm_supported<bf16>(p))
+      e = launch_gemm_tc(p, num_sms, nullptr, st, engine == 0 ? 1 : 0);
     else e = launch_gemm_simt<bf16>(p, st);
   } else {
     e = launch_gemm_simt<float>(p, st);

@@ -45,7 +45,9 @@ enum {
  * dtype (nc_dtype) is the type of A, B and of D unless NC_EPI_STORE_F32.
  * engine: 0 = the path nc_fwd_bwd takes (tcgen05 tensor cores for bf16
  * operands whose strides are multiples of 8 elements and pointers 16-byte
- * aligned, CUDA cores otherwise), 1 = force the CUDA-core kernel.
+ * aligned -- pairs of CTAs on 256 x 256 tiles when M >= 256, one CTA per
+ * 128 x 256 tile otherwise -- CUDA cores for the rest), 1 = force the
+ * CUDA-core kernel, 2 = tcgen05 with one CTA per tile.
  * M, N, K >= 1. */
 int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, int b_mn, void *D,
             int64_t ldd, int M, int N, int K, int dtype, int epilogue, int engine, void *stream);

@@ -60,13 +60,16 @@ GEMM_CASES = [
     (200, 264, 72, 1, 1, 8),       # ragged weight-gradient layout
     (130, 300, 96, 1, 0, 8),
     (256, 256, 8192, 1, 1, 0),     # few tiles, long K: split-K path for fp32 output
+    (520, 392, 136, 0, 1, 8),      # M not a multiple of 256: the second CTA of a pair is partly empty
+    (1280, 5120, 256, 1, 1, 0),    # weight-gradient shape with a full second CTA
 ]
 
 
 @pytest.mark.parametrize("M,N,K,a_mn,b_mn,pad", GEMM_CASES)
 @pytest.mark.parametrize("epi", EPIS)
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 2])
 def test_gemm_bf16(nc, M, N, K, a_mn, b_mn, pad, epi, engine):
+    # engine 0: pairs of CTAs on 256 x 256 tiles when M >= 256; 2: one CTA per tile; 1: CUDA cores
     import torch
     if engine == 1 and K > 2048 and epi != "STORE_F32":
         pytest.skip("covered by the tensor-core engine")
