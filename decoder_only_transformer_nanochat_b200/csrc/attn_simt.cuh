@@ -11,6 +11,7 @@
 #pragma once
 
 #include "attn_mma.cuh"
+#include "elementwise.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 
@@ -256,18 +257,21 @@ inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
 }
 
+// D = rowsum(dO * O) is computed inside the tcgen05 dQ kernel; the other
+// engines get it from attn_rowdot_kernel first.  Drow is [B, H, T] scratch.
 template <typename T>
-inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *dO, const float *lse,
-                                   const float *Dr, T *dqkv, int B, int T_len, int H, int num_sms,
-                                   int engine, int *status, cudaStream_t st) {
+inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *O, const T *dO, const float *lse, float *Dr,
+                                   T *dqkv, int B, int T_len, int H, int num_sms, int engine, int *status,
+                                   cudaStream_t st) {
   (void)num_sms;
-  if (sizeof(T) == 2 && engine == 0 && fatc::supported_bwd(qkv, ld, dO, dqkv))
-    return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len, H,
-                            status, st);
+  if (sizeof(T) == 2 && engine == 0 && fatc::supported_bwd(qkv, ld, O, dO, dqkv))
+    return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B,
+                            T_len, H, status, st);
+  const int M = B * T_len;
+  attn_rowdot_kernel<T><<<(unsigned)(((size_t)M * H + 7) / 8), 256, 0, st>>>(dO, O, Dr, M, T_len, H);
   if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, dO) &&
       fa::supported(dqkv, ld, dqkv))
-    return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len,
-                          H, st);
+    return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len, H, st);
   return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);
 }
 

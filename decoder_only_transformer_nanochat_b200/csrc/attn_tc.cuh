@@ -309,7 +309,7 @@ constexpr int kBK = 64;
 constexpr int kDqStages = 3;
 constexpr int kKVTile64 = kBK * kD * 2;   // 16 KB
 constexpr int kDsTile = kQ * kBK * 2;     // 16 KB: [128 q x 64 keys] bf16
-constexpr int kDqSmem = 1024 + 2 * kTileBytes + kDqStages * 2 * kKVTile64 + 2 * kDsTile + 256;
+constexpr int kDqSmem = 1024 + 2 * kTileBytes + kDqStages * 2 * kKVTile64 + 2 * kDsTile + 256 + 1024;
 
 // backward kernels: warp 0 TMA, warp 1 MMA, warps 2..9 element-wise; the
 // element-wise warps w and w+4 share TMEM lane quarter (w & 3) and split the
@@ -320,7 +320,8 @@ constexpr int kSoft = 256;
 struct BwdParams {
   int T, H, n_tiles, ld;
   const float *lse;   // [B, H, T]
-  const float *Drow;  // [B, H, T]
+  float *Drow;        // [B, H, T]: rowsum(dO * O), written by the dQ kernel
+  const bf16 *O;      // [B*T, H*128]
   int *status;
 };
 
@@ -451,9 +452,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sc = rsqrtf((float)kD) * kLog2e;
     const int rr_ = min(row, p.T - 1);
     const float L = p.lse[((int64_t)b * p.H + h) * p.T + rr_] * kLog2e;
-    const float Dv = p.Drow[((int64_t)b * p.H + h) * p.T + rr_];
     const int c0 = g * 32;  // this thread's 32 keys of the 64-key tile
-    bool ok = true;
+    // D = rowsum(dO * O) for this row: dO from the shared tile, O from global;
+    // warpgroup g sums dims [64g, 64g + 64) and the halves meet in shared memory
+    float *sDpart = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [2][128]
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+    {
+      float part = 0.f;
+      if (row < p.T) {
+        const bf16 *orow = p.O + ((int64_t)b * p.T + row) * C + h * kD + 64 * g;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float o8[8], g8[8];
+          Vec8<bf16>::load(orow + 8 * u, o8);
+          Vec8<bf16>::load(reinterpret_cast<const bf16 *>(sG + g * 16384 + r * 128 + ((u ^ (r & 7)) << 4)), g8);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part += o8[i] * g8[i];
+        }
+      }
+      sDpart[g * kQ + r] = part;
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float Dv = sDpart[r] + sDpart[kQ + r];
+    if (g == 0 && row < p.T) p.Drow[((int64_t)b * p.H + h) * p.T + row] = Dv;
     for (int j = 0; j < n_kv; ++j) {
       const int bb = j & 1;
       ok = mbar_wait(s_full(bb), (j >> 1) & 1, abort_flag, p.status);
@@ -829,8 +850,8 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
 namespace nc {
 namespace fatc {
 
-inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *dO, const float *lse, const float *Drow,
-                              bf16 *dqkv, int B, int T, int H, int *status, cudaStream_t st) {
+inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const bf16 *dO, const float *lse,
+                              float *Drow, bf16 *dqkv, int B, int T, int H, int *status, cudaStream_t st) {
   CUtensorMap mq128, mkv64, mdo128, mdo64, mout;
   const int C = H * kD;
   if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mkv64, qkv, B, T, (int)ld, ld, 64) ||
@@ -843,6 +864,7 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *dO, const
   p.ld = (int)ld;
   p.lse = lse;
   p.Drow = Drow;
+  p.O = O;
   p.status = status;
   p.n_tiles = (T + kQ - 1) / kQ;
   attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mkv64, mdo128, mout, p);
@@ -852,8 +874,8 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *dO, const
   return cudaGetLastError();
 }
 
-inline bool supported_bwd(const void *qkv, int64_t ld, const void *dO, const void *dqkv) {
-  return supported(qkv, ld, dO) && ((uintptr_t)dqkv & 15) == 0;
+inline bool supported_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const void *dqkv) {
+  return supported(qkv, ld, dO) && ((uintptr_t)dqkv & 15) == 0 && ((uintptr_t)O & 15) == 0;
 }
 
 }  // namespace fatc

@@ -114,11 +114,11 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ x, T
 
 // RMSNorm backward with the residual-stream accumulation:
 //   g = r (dy - y mean(dy y));  dx = g (+ dx_old if accumulate)
-// dy is fp32 (a GEMM output), y the saved normalised value, dx kept in fp32
+// dy is a GEMM output in T, y the saved normalised value, dx kept in fp32
 // and also written in T as the next GEMM's operand.
 template <typename T, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
-    const float *__restrict__ dy, const T *__restrict__ y, const float *__restrict__ r,
+    const T *__restrict__ dy, const T *__restrict__ y, const float *__restrict__ r,
     float *__restrict__ dx, T *__restrict__ dx_t, int M, int C, int accumulate) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
   for (int i = 0; i < NV; ++i) {
     const int c = (lane + 32 * i);
     if (c < nv) {
-      Vec8<float>::load(dy + base + c * 8, g[i]);
+      Vec8<T>::load(dy + base + c * 8, g[i]);
       Vec8<T>::load(y + base + c * 8, yy[i]);
 #pragma unroll
       for (int j = 0; j < 8; ++j) dot += g[i][j] * yy[i][j];
@@ -182,30 +182,68 @@ template <> struct Pair2<float> {
   }
 };
 
+// One warp per token: the q heads and the k head of a token are H+1
+// contiguous 128-wide rows; each half-warp holds one head, 8 values per lane
+// (lane j of the half-warp: dims 8j..8j+7), so a warp covers two heads per
+// step with 16-byte accesses.  The RoPE partner of dim i < 64 is dim i + 64,
+// held by lane j + 8 of the same half-warp (one shuffle); the head's sum of
+// squares is a 16-lane reduction.
+template <typename T>
+__device__ __forceinline__ void rope_pair_tables(const float *cos_t, const float *sin_t, int pos, int j,
+                                                 float (&c)[8], float (&s)[8]) {
+  const int i0 = (j & 7) * 8;  // dims i0..i0+7 of the first half share their angles with i0+64..
+  const float4 *cp = reinterpret_cast<const float4 *>(cos_t + pos * 64 + i0);
+  const float4 *sp = reinterpret_cast<const float4 *>(sin_t + pos * 64 + i0);
+  const float4 c0 = cp[0], c1 = cp[1], s0 = sp[0], s1 = sp[1];
+  c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+  s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w; s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+}
+
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) rope_qknorm_kernel(
     T *__restrict__ qkv, int ld, float *__restrict__ rq, float *__restrict__ rk,
     const float *__restrict__ cos_t, const float *__restrict__ sin_t, int M, int T_len, int H) {
-  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int tok = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (item >= M * (H + 1)) return;
-  const int tok = item / (H + 1), h = item % (H + 1);
+  if (tok >= M) return;
   const int pos = tok % T_len;
-  T *p = qkv + (size_t)tok * ld + h * kHeadDim;
-  const int i0 = 2 * lane;
-  float2 a = Pair2<T>::load(p + i0), b = Pair2<T>::load(p + 64 + i0);
-  const float2 c = *reinterpret_cast<const float2 *>(cos_t + pos * 64 + i0);
-  const float2 s = *reinterpret_cast<const float2 *>(sin_t + pos * 64 + i0);
-  float2 y1 = make_float2(a.x * c.x - b.x * s.x, a.y * c.y - b.y * s.y);
-  float2 y2 = make_float2(a.x * s.x + b.x * c.x, a.y * s.y + b.y * c.y);
-  float ss = y1.x * y1.x + y1.y * y1.y + y2.x * y2.x + y2.y * y2.y;
-  ss = warp_sum(ss);
-  const float r = rsqrtf(ss / (float)kHeadDim + kEps);
-  Pair2<T>::store(p + i0, make_float2(y1.x * r, y1.y * r));
-  Pair2<T>::store(p + 64 + i0, make_float2(y2.x * r, y2.y * r));
-  if (lane == 0) {
-    if (h < H) rq[(size_t)tok * H + h] = r;
-    else rk[tok] = r;
+  const int hw = lane >> 4, j = lane & 15;
+  float c[8], s[8];
+  rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
+  T *row = qkv + (size_t)tok * ld;
+  for (int h0 = 0; h0 < H + 1; h0 += 2) {
+    const int h = h0 + hw;
+    const bool live = h < H + 1;  // uniform per half-warp
+    float x[8];
+    if (live) Vec8<T>::load(row + h * kHeadDim + j * 8, x);
+    else
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    float y[8], ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float partner = __shfl_xor_sync(0xffffffffu, x[i], 8);
+      // first half: y_i = x_i cos - x_{i+64} sin ; second half: y_{i+64} = x_i sin + x_{i+64} cos
+      y[i] = j < 8 ? x[i] * c[i] - partner * s[i] : partner * s[i] + x[i] * c[i];
+      ss += y[i] * y[i];
+    }
+    ss = half_warp_sum(ss);
+    const float r = rsqrtf(ss / (float)kHeadDim + kEps);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] *= r;
+    if (live) {
+      Vec8<T>::store(row + h * kHeadDim + j * 8, y);
+      if (j == 0) {
+        if (h < H) rq[(size_t)tok * H + h] = r;
+        else rk[tok] = r;
+      }
+    }
   }
 }
 
@@ -217,25 +255,42 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
     T *__restrict__ dqkv, const T *__restrict__ qkv, int ld, const float *__restrict__ rq,
     const float *__restrict__ rk, const float *__restrict__ cos_t,
     const float *__restrict__ sin_t, int M, int T_len, int H) {
-  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int tok = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (item >= M * (H + 1)) return;
-  const int tok = item / (H + 1), h = item % (H + 1);
+  if (tok >= M) return;
   const int pos = tok % T_len;
-  const size_t off = (size_t)tok * ld + h * kHeadDim;
-  const int i0 = 2 * lane;
-  float2 da = Pair2<T>::load(dqkv + off + i0), db = Pair2<T>::load(dqkv + off + 64 + i0);
-  float2 ya = Pair2<T>::load(qkv + off + i0), yb = Pair2<T>::load(qkv + off + 64 + i0);
-  float dot = da.x * ya.x + da.y * ya.y + db.x * yb.x + db.y * yb.y;
-  dot = warp_sum(dot) / (float)kHeadDim;
-  const float r = h < H ? rq[(size_t)tok * H + h] : rk[tok];
-  float2 ga = make_float2(r * (da.x - ya.x * dot), r * (da.y - ya.y * dot));
-  float2 gb = make_float2(r * (db.x - yb.x * dot), r * (db.y - yb.y * dot));
-  const float2 c = *reinterpret_cast<const float2 *>(cos_t + pos * 64 + i0);
-  const float2 s = *reinterpret_cast<const float2 *>(sin_t + pos * 64 + i0);
-  Pair2<T>::store(dqkv + off + i0, make_float2(ga.x * c.x + gb.x * s.x, ga.y * c.y + gb.y * s.y));
-  Pair2<T>::store(dqkv + off + 64 + i0,
-                  make_float2(-ga.x * s.x + gb.x * c.x, -ga.y * s.y + gb.y * c.y));
+  const int hw = lane >> 4, j = lane & 15;
+  float c[8], s[8];
+  rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
+  T *drow = dqkv + (size_t)tok * ld;
+  const T *yrow = qkv + (size_t)tok * ld;
+  for (int h0 = 0; h0 < H + 1; h0 += 2) {
+    const int h = h0 + hw;
+    const bool live = h < H + 1;
+    float dy[8], y[8];
+    if (live) {
+      Vec8<T>::load(drow + h * kHeadDim + j * 8, dy);
+      Vec8<T>::load(yrow + h * kHeadDim + j * 8, y);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { dy[i] = 0.f; y[i] = 0.f; }
+    }
+    const float r = live ? (h < H ? rq[(size_t)tok * H + h] : rk[tok]) : 0.f;
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dot += dy[i] * y[i];
+    dot = half_warp_sum(dot) / (float)kHeadDim;
+    float g[8], out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) g[i] = r * (dy[i] - y[i] * dot);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float partner = __shfl_xor_sync(0xffffffffu, g[i], 8);
+      // first half: g_i cos + g_{i+64} sin ; second half: -g_i sin + g_{i+64} cos
+      out[i] = j < 8 ? g[i] * c[i] + partner * s[i] : g[i] * c[i] - partner * s[i];
+    }
+    if (live) Vec8<T>::store(drow + h * kHeadDim + j * 8, out);
+  }
 }
 
 // ---------------------------------------------------------------------------

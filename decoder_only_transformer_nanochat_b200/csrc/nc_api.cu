@@ -65,8 +65,8 @@ template <typename T>
 struct Work {
   std::vector<T *> xn, qkv, O, xn2, a;
   std::vector<float *> r1, rq, rk, lse, r2;
-  T *x, *xf, *z, *dxb, *dO, *dqkv;
-  float *r0, *rf, *tok_loss, *dx, *dy32, *Drow;
+  T *x, *xf, *z, *dxb, *dO, *dqkv, *dy;
+  float *r0, *rf, *tok_loss, *dx, *Drow;
   int64_t ldz;
 };
 
@@ -112,13 +112,13 @@ size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
   float *tok_loss = (float *)take(M * 4);
   float *dx = (float *)take(M * C * 4);
   T *dxb = (T *)take(M * C * es);
-  float *dy32 = (float *)take(M * C * 4);
+  T *dy = (T *)take(M * C * es);
   T *dO = (T *)take(M * C * es);
   T *dqkv = (T *)take(M * ldqkv * es);
   float *Drow = (float *)take(M * H * 4);
   if (w) {
     w->x = x; w->r0 = r0; w->xf = xf; w->rf = rf; w->z = z; w->ldz = ldz;
-    w->tok_loss = tok_loss; w->dx = dx; w->dxb = dxb; w->dy32 = dy32; w->dO = dO;
+    w->tok_loss = tok_loss; w->dx = dx; w->dxb = dxb; w->dy = dy; w->dO = dO;
     w->dqkv = dqkv; w->Drow = Drow;
   }
   return off;
@@ -238,7 +238,7 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
                                  w.x, w.xn[l], w.r1[l], M, C))));
     NC_TRY(gemm<T>(m, gp(M, ldqkv, C, w.xn[l], C, 0, W.wqkv[l], C, 0, w.qkv[l], ldqkv, EPI_STORE), st));
     NC_RUN(K_ROPE_QKNORM, 0, M * (2.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
-           (rope_qknorm_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+           (rope_qknorm_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     NC_RUN(K_ATTN_FWD, attn_flops, 0,
            if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0,
@@ -288,13 +288,13 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   // gradient pointers (fp32, same layout as the weights)
   auto G = [&](int idx) { return grads + m->params[idx].offset; };
   const int last = (int)m->params.size() - 1;
-  const double nbwd = M * (12.0 * C + 2.0 * C * es + 4.0);  // dy, dx_old, dx in fp32; y, dx_t in T
+  const double nbwd = M * (8.0 * C + 3.0 * C * es + 4.0);  // dx_old, dx in fp32; dy, y, dx_t in T
   // dWout = dz^T xf ;  dxf = dz Wout
   NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, EPI_STORE_F32), st));
-  NC_TRY(gemm<T>(m, gp(M, C, V, w.z, w.ldz, 0, W.lm_head, C, 1, w.dy32, C, EPI_STORE_F32), st));
+  NC_TRY(gemm<T>(m, gp(M, C, V, w.z, w.ldz, 0, W.lm_head, C, 1, w.dy, C, EPI_STORE), st));
   NC_RUN(K_RMSNORM_BWD, 0, nbwd - M * 4.0 * C,
          NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                               w.dy32, w.xf, w.rf, w.dx, w.dxb, M, C, 0))));
+                               w.dy, w.xf, w.rf, w.dx, w.dxb, M, C, 0))));
 
   for (int l = m->depth - 1; l >= 0; --l) {
     const int pi = 1 + 6 * l;
@@ -302,28 +302,25 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     NC_TRY(gemm<T>(m, gp(C, F, M, w.dxb, C, 1, w.a[l], F, 1, G(pi + 5), F, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, F, C, w.dxb, C, 0, W.w2[l], F, 1, w.a[l], F, EPI_DRELU2), st));
     NC_TRY(gemm<T>(m, gp(F, C, M, w.a[l], F, 1, w.xn2[l], C, 1, G(pi + 4), C, EPI_STORE_F32), st));
-    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w1[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w1[l], C, 1, w.dy, C, EPI_STORE), st));
     NC_RUN(K_RMSNORM_BWD, 0, nbwd,
            NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                                 w.dy32, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1))));
+                                 w.dy, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1))));
     // attention: x += O Wo^T
     NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
-    NC_RUN(K_ROWDOT, 0, M * (2.0 * C * es + 4.0 * H),
-           (attn_rowdot_kernel<T><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>(w.dO, w.O[l], w.Drow,
-                                                                                M, T_len, H)));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
-           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
+           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
                                   m->num_sms, 0, m->status, st) != cudaSuccess) return NC_ECUDA);
     NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
-           (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M * (H + 1), 8), 256, 0, st>>>(
+           (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     // [q|k|v] = xn [Wq;Wk;Wv]^T
     NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, EPI_STORE_F32), st));
-    NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy32, C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy, C, EPI_STORE), st));
     NC_RUN(K_RMSNORM_BWD, 0, nbwd,
            NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                                 w.dy32, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
+                                 w.dy, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
   }
   // embedding: through the first norm, summed into the selected rows
   if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
@@ -587,14 +584,13 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
   cudaStream_t st = (cudaStream_t)stream;
   const int M = B * T;
   cudaError_t e;
+  (void)M;
   if (dtype == NC_BF16) {
-    attn_rowdot_kernel<bf16><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const bf16 *)dO, (const bf16 *)O, Drow, M, T, H);
-    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms,
-                              engine, nullptr, st);
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
+                              (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   } else {
-    attn_rowdot_kernel<float><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const float *)dO, (const float *)O, Drow, M, T, H);
-    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H,
-                               num_sms, engine, nullptr, st);
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
+                               (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
@@ -674,12 +670,13 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
   cudaStream_t st = (cudaStream_t)stream;
   const int M = B * T;
   cudaError_t e;
+  (void)M;
   if (dtype == NC_BF16) {
-    attn_rowdot_kernel<bf16><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const bf16 *)dO, (const bf16 *)O, Drow, M, T, H);
-    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)dO, lse, Drow, (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
+                              (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   } else if (dtype == NC_F32) {
-    attn_rowdot_kernel<float><<<rows_grid((size_t)M * H, 8), 256, 0, st>>>((const float *)dO, (const float *)O, Drow, M, T, H);
-    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)dO, lse, Drow, (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
+                               (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
   } else {
     return NC_EUNSUPPORTED;
   }
