@@ -30,10 +30,13 @@ using namespace tc;
 
 constexpr int kQ = 128, kKV = 128, kD = 128;
 constexpr int kThreads = 192;
+constexpr int kFwdThreads = 320;  // TMA warp, MMA warp, 8 softmax warps
 constexpr int kTileBytes = kQ * kD * 2;      // 32 KB: Q, K, V or P tile
 constexpr int kStageBytes = 2 * kTileBytes;  // K + V
-constexpr int kSmem = 1024 + kTileBytes /*Q*/ + 2 * kStageBytes + kTileBytes /*P*/ + 256;
-constexpr int kTmemCols = 512;               // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kSmem = 1024 + kTileBytes /*Q*/ + (kKStages + kVStages) * kTileBytes + 256 + 3072;
+constexpr int kTmemCols = 512;               // S0 [0,128), S1 [128,256), O [256,384), P [384,448)
+constexpr int kPCol = 384;                   // P as bf16 pairs: key k of row m at lane m, column kPCol + k/2
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
 
@@ -41,6 +44,47 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for x in [-126, 0] on the FMA pipe: x = n + f with n = round(x) (the
+// 1.5 * 2^23 shifter), f in [-1/2, 1/2], 2^f by a cubic whose coefficients
+// were fitted here to the relative error (max 1.0e-4, far below the bf16
+// rounding of a probability); n goes straight into the exponent bits.
+// Used for half of the softmax exponentials so the MUFU unit does not
+// bound the tile.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float p = fmaf(f, fmaf(f, fmaf(f, 0.05500858f, 0.24221037f), 0.69328290f), 1.f);
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// MMA with the A operand read from TMEM (K-major, bf16 pairs per column)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// AND over the 256 element-wise threads (named barrier 1), so that all of
+// them take the same branch and keep meeting at the same barriers
+__device__ __forceinline__ bool epi_vote_all256(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -60,7 +104,7 @@ struct FwdParams {
   int *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
                        const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
                        const __grid_constant__ CUtensorMap map_o,    // O [B][T][C], box 64 x 128
@@ -68,20 +112,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem;
-  uint8_t *sKV = sQ + kTileBytes;                 // stage s: K at s*64K, V at s*64K + 32K
-  uint8_t *sP = sKV + 2 * kStageBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sP + kTileBytes);
-  // bars: q_full, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
+  uint8_t *sK = sQ + kTileBytes;                  // K ring: kKStages tiles
+  uint8_t *sV = sK + kKStages * kTileBytes;       // V ring: kVStages tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kVStages * kTileBytes);
+  // bars: q_full, k_full[3], k_empty[3], s_full[2], s_empty[2], p_full, o_done, drain,
+  //       v_full[2], v_empty[2].  K and V have rings of their own: K_j is free as
+  //       soon as S_j is computed, so the loads of K_{j+2}, K_{j+3} overlap softmax j.
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t q_full = smem_u32(bars + 0);
-  auto kv_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto kv_empty = [&](int s) { return smem_u32(bars + 3 + s); };
-  auto s_full = [&](int s) { return smem_u32(bars + 5 + s); };
-  auto s_empty = [&](int s) { return smem_u32(bars + 7 + s); };
-  const uint32_t p_full = smem_u32(bars + 9);
-  const uint32_t o_done = smem_u32(bars + 10);
-  const uint32_t drain = smem_u32(bars + 11);
+  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto k_empty = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
+  auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
+  const uint32_t p_full = smem_u32(bars + 11);
+  const uint32_t o_done = smem_u32(bars + 12);
+  const uint32_t drain = smem_u32(bars + 13);
+  auto v_full = [&](int s) { return smem_u32(bars + 14 + s); };
+  auto v_empty = [&](int s) { return smem_u32(bars + 16 + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = gridDim.x / p.n_qt;
@@ -93,13 +141,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
-      mbar_init(s_full(s), 1);
-      mbar_init(s_empty(s), 128);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
     }
-    mbar_init(p_full, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(s_empty(s), 256);
+    }
+    mbar_init(p_full, 256);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -116,24 +168,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------- TMA producer ----------------
       mbar_expect_tx(q_full, kTileBytes);
       for (int i = 0; i < 2; ++i) tma_load_3d(smem_u32(sQ) + i * 16384, &map_qk, h * kD + 64 * i, q0, b, q_full);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      int issued_k = 0, issued_v = 0;
+      auto load_k = [&](int j) -> bool {
+        const int st = j % kKStages;
+        if (!mbar_wait(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
+        const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
+        mbar_expect_tx(k_full(st), kTileBytes);
+        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, j * kKV, b, k_full(st));
+        ++issued_k;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(kv_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-        const uint32_t k_dst = smem_u32(sKV) + st * kStageBytes, v_dst = k_dst + kTileBytes;
-        mbar_expect_tx(kv_full(st), kStageBytes);
-        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, j * kKV, b, kv_full(st));
+        if (!mbar_wait(v_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
+        mbar_expect_tx(v_full(st), kTileBytes);
         for (int hh = 0; hh < 2; ++hh)
           for (int a = 0; a < 2; ++a)
-            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, j * kKV + 64 * hh, b, kv_full(st));
-        ++issued;
+            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, j * kKV + 64 * hh, b, v_full(st));
+        ++issued_v;
+        return true;
+      };
+      // K runs two tiles ahead of V: K_{j+2} is requested before V_j
+      bool okp = load_k(0) && (n_kv < 2 || load_k(1));
+      for (int j = 0; j < n_kv && okp; ++j) {
+        if (j + 2 < n_kv && !load_k(j + 2)) break;
+        if (!load_v(j)) break;
       }
       // no copy of ours may still be landing when the CTA exits
       const uint64_t t0 = globaltimer();
       while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued - 2); j < issued; ++j) {
+      for (int j = max(0, issued_k - kKStages); j < issued_k; ++j) {
         const uint64_t t1 = globaltimer();
-        while (!mbar_try(kv_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(k_full(j % kKStages), (j / kKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+      for (int j = max(0, issued_v - 2); j < issued_v; ++j) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(v_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
     }
   } else if (warp == 1) {
@@ -141,14 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = make_idesc(0, 0, kQ, kKV);   // Q K^T: both K-major
       const uint32_t idesc_o = make_idesc(0, 1, kQ, kD);    // P V: V is MN-major
-      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(kv_full(st), (j >> 1) & 1, abort_flag, p.status)) return false;
+        const int st = j & 1, ks = j % kKStages;
+        if (!mbar_wait(k_full(ks), (j / kKStages) & 1, abort_flag, p.status)) return false;
         if (!mbar_wait(s_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t bK = smem_u32(sKV) + st * kStageBytes;
+        const uint32_t bK = smem_u32(sK) + ks * kTileBytes;
 #pragma unroll
         for (int s = 0; s < kD / 16; ++s) {
           const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
@@ -156,104 +227,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                  s > 0 ? 1u : 0u);
         }
         tc_commit(s_full(st));
+        tc_commit(k_empty(ks));
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int j = 0; j < n_kv && ok; ++j) {
         if (j + 1 < n_kv && !issue_s(j + 1)) break;
         if (!mbar_wait(p_full, j & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(v_full(j & 1), (j >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t bV = smem_u32(sKV) + (j & 1) * kStageBytes + kTileBytes;
+        const uint32_t bV = smem_u32(sV) + (j & 1) * kTileBytes;
 #pragma unroll
         for (int s = 0; s < kKV / 16; ++s) {
-          const uint32_t a_off = (s >> 2) * 16384 + (s & 3) * 32;    // P: K-major, k = keys
           const uint32_t b_off = (s >> 2) * 16384 + (s & 3) * 2048;  // V: MN-major, k rows
-          tc_mma(tmem + 2 * kKV, smem_desc(aP + a_off, 16, 1024), smem_desc(bV + b_off, 8192, 1024), idesc_o,
-                 (j > 0 || s > 0) ? 1u : 0u);
+          // P from TMEM: 16 keys = 8 columns of bf16 pairs
+          tc_mma_ts(tmem + 2 * kKV, tmem + kPCol + 8 * s, smem_desc(bV + b_off, 8192, 1024), idesc_o,
+                    (j > 0 || s > 0) ? 1u : 0u);
         }
         tc_commit(o_done);
-        tc_commit(kv_empty(j & 1));
+        tc_commit(v_empty(j & 1));
       }
       tc_commit(drain);
       const uint64_t t0 = globaltimer();
       while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
     }
   } else {
-    // ---------------- softmax warps 2..5: thread = query row ----------------
-    const int quarter = warp & 3;
+    // ---------------- softmax warps 2..9: thread = query row, key half g ----------------
+    // warps w and w + 4 share TMEM lane quarter (w & 3); warpgroup g = (w - 2) / 4
+    // takes keys [64g, 64g + 64) of each tile and the same half of O's columns
+    const int quarter = warp & 3, g = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int row = q0 + r;
+    const int c0 = 64 * g;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float *sMax = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [2 tiles][2 halves][128]
+    float *sSum = sMax + 2 * 2 * kQ;                                                   // [2 halves][128]
     const float sc = rsqrtf((float)kD) * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j & 1;
       ok = mbar_wait(s_full(st), (j >> 1) & 1, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      float s[kKV];
-      {
-        uint32_t rr[kKV / 32][32];
-#pragma unroll
-        for (int c = 0; c < kKV / 32; ++c) tmem_ld32_nw(lane_base + st * kKV + c * 32, rr[c]);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; }
+      float s[64];
+      if (ok) {
+        tc_fence_after();
+        uint32_t rr[2][32];
+        tmem_ld32_nw(lane_base + st * kKV + c0, rr[0]);
+        tmem_ld32_nw(lane_base + st * kKV + c0 + 32, rr[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kKV / 32; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[c][i]) * sc;
-      }
-      tc_fence_before();
-      mbar_arrive(s_empty(st));
-      const int kv0 = j * kKV;
-      if (kv0 + kKV > q0 || kv0 + kKV > p.T) {
+        tc_fence_before();
+        mbar_arrive(s_empty(st));
+      } else {
 #pragma unroll
-        for (int i = 0; i < kKV; ++i)
+        for (int i = 0; i < 64; ++i) s[i] = 0.f;
+      }
+      const int kv0 = j * kKV + c0;
+      if (kv0 + 64 > q0 || kv0 + 64 > p.T) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
           if (kv0 + i > row || kv0 + i >= p.T) s[i] = -INFINITY;
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < kKV; ++i) mx = fmaxf(mx, s[i]);
+      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      // the row max over both halves: exchange through shared memory (buffer j & 1)
+      sMax[(st * 2 + g) * kQ + r] = mx;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      mx = fmaxf(sMax[(st * 2) * kQ + r], sMax[(st * 2 + 1) * kQ + r]);
+      // every softmax warp learns whether any of them gave up; all take the same branch
+      ok = epi_vote_all256(ok);
+      if (!ok) break;
+      // the exponent base for this tile; it only moves when the max grows by > 2^8
+      const bool grow = j == 0 || mx > m_used + kRescaleLog2;
+      const float corr = (j > 0 && grow) ? ex2(m_used - mx) : 1.f;
+      if (grow) {
+        l *= corr;
+        m_used = mx;
+      }
+      // P_j in registers first: the exponentials overlap the previous P V
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float e0 = ex2(s[i] - m_used), e1 = ex2_poly(s[i + 1] - m_used);
+        sum += e0 + e1;
+        pk[i / 2] = pack2(e0, e1);
+      }
       // P_{j-1} V_{j-1} must be done before P_j overwrites P and before O is touched
       if (j > 0) {
         ok = mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, ok)) ok = false;
+        ok = epi_vote_all256(ok);
+        if (!ok) break;
         tc_fence_after();
-      }
-      const bool grow = mx > m_used + kRescaleLog2;
-      if (j == 0) {
-        m_used = mx;
-      } else if (__any_sync(0xffffffffu, grow)) {
-        const float corr = grow ? ex2(m_used - mx) : 1.f;
-        if (grow) {
-          l *= corr;
-          m_used = mx;
-        }
+        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(lane_base + 2 * kKV + c * 32, rr);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(lane_base + 2 * kKV + c0 + c * 32, rr);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * corr);
-          tmem_st32(lane_base + 2 * kKV + c * 32, rr);
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * corr);
+            tmem_st32(lane_base + 2 * kKV + c0 + c * 32, rr);
+          }
         }
       }
-      float sum = 0.f;
-#pragma unroll
-      for (int u = 0; u < kKV / 8; ++u) {
-        float e[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          e[i] = ex2(s[8 * u + i] - m_used);
-          sum += e[i];
-        }
-        uint4 w;
-        w.x = pack2(e[0], e[1]);
-        w.y = pack2(e[2], e[3]);
-        w.z = pack2(e[4], e[5]);
-        w.w = pack2(e[6], e[7]);
-        *reinterpret_cast<uint4 *>(sP + tile_unit(r, u)) = w;
-      }
+      tmem_st32(lane_base + kPCol + 32 * g, pk);  // keys [64g, 64g + 64) of this row
       l += sum;
       fence_proxy_async();
       tc_fence_before();
@@ -262,13 +345,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue: O / l, lse ----------------
     if (ok) ok = mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
+    sSum[g * kQ + r] = l;
+    ok = epi_vote_all256(ok);
+    const float lt = sSum[r] + sSum[kQ + r];
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lt;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t rr[32];
-        tmem_ld32(lane_base + 2 * kKV + c * 32, rr);
+        tmem_ld32(lane_base + 2 * kKV + c0 + c * 32, rr);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint4 w;
@@ -276,13 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = pack2(__uint_as_float(rr[8 * u + 2]) * inv, __uint_as_float(rr[8 * u + 3]) * inv);
           w.z = pack2(__uint_as_float(rr[8 * u + 4]) * inv, __uint_as_float(rr[8 * u + 5]) * inv);
           w.w = pack2(__uint_as_float(rr[8 * u + 6]) * inv, __uint_as_float(rr[8 * u + 7]) * inv);
-          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, c * 4 + u)) = w;  // Q is no longer read
+          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, 8 * g + c * 4 + u)) = w;  // Q is no longer read
         }
       }
-      if (row < p.T) p.lse[((int64_t)b * p.H + h) * p.T + row] = (m_used + __log2f(l)) * (1.f / kLog2e);
+      if (g == 0 && row < p.T) p.lse[((int64_t)b * p.H + h) * p.T + row] = (m_used + __log2f(lt)) * (1.f / kLog2e);
     }
     fence_proxy_async();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok && warp == 2 && lane == 0) {
       for (int i = 0; i < 2; ++i) tma_store_3d(&map_o, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
       bulk_commit();
@@ -840,7 +926,7 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.n_qt = (T + kQ - 1) / kQ;
   p.lse = lse;
   p.status = status;
-  attn_fwd_tc_kernel<<<B * H * p.n_qt, kThreads, kSmem, st>>>(mqk, mv, mo, p);
+  attn_fwd_tc_kernel<<<B * H * p.n_qt, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
   return cudaGetLastError();
 }
 
