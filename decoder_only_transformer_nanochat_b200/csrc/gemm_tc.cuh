@@ -57,17 +57,27 @@ struct Params {
 };
 
 __device__ __forceinline__ Unit unit_of(const Params &p, int u) {
-  // tiles grouped 16 m-blocks at a time so CTAs in flight share B tiles in L2
-  const int tile = u / p.splits, split = u % p.splits;
-  const int G = 16;
-  const int per_group = G * p.n_n;
-  const int g = tile / per_group;
-  const int first_m = g * G;
-  const int gsize = min(p.n_m - first_m, G);
-  const int r = tile % per_group;
+  // Units in flight at once should share operand panels in L2.  k-splits are
+  // the slowest index, so a wave works on one K slice of many tiles.  With
+  // few N tiles the N tiles of an M block are consecutive (its A panel is read
+  // once per wave); with many, tiles are grouped 16 M blocks at a time with M
+  // fastest (each B panel serves 16 M blocks).
+  const int tiles = p.n_m * p.n_n;
+  const int split = u / tiles, tile = u % tiles;
   Unit x;
-  x.m_blk = first_m + r % gsize;
-  x.n_blk = r / gsize;
+  if (p.n_n <= 16) {
+    x.m_blk = tile / p.n_n;
+    x.n_blk = tile % p.n_n;
+  } else {
+    const int G = 16;
+    const int per_group = G * p.n_n;
+    const int g = tile / per_group;
+    const int first_m = g * G;
+    const int gsize = min(p.n_m - first_m, G);
+    const int r = tile % per_group;
+    x.m_blk = first_m + r % gsize;
+    x.n_blk = r / gsize;
+  }
   const int per = (p.kblocks + p.splits - 1) / p.splits;
   x.kb0 = split * per;
   x.kb1 = min(p.kblocks, x.kb0 + per);
