@@ -390,12 +390,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 // dK = dS^T Q / sqrt(d) and dV = P^T dO, the last two summed over every query
 // head that shares the key/value head.
 
-// ---------------- dQ: CTA = 128 queries of one (b, h), keys in tiles of 64 ----------------
-constexpr int kBK = 64;
-constexpr int kDqStages = 3;
-constexpr int kKVTile64 = kBK * kD * 2;   // 16 KB
-constexpr int kDsTile = kQ * kBK * 2;     // 16 KB: [128 q x 64 keys] bf16
-constexpr int kDqSmem = 1024 + 2 * kTileBytes + kDqStages * 2 * kKVTile64 + 2 * kDsTile + 256 + 1024;
+// ---------------- dQ: CTA = 128 queries of one (b, h), keys in tiles of 128 ----------------
+// 128-key tiles keep every MMA at N = 128 (an M = 128, N = 64 MMA takes as
+// long as an N = 128 one), and halve the hand-offs per key.
+constexpr int kBK = 128;
+constexpr int kDqKStages = 3, kDqVStages = 2;  // K is read by S and dQ, V only by dP: separate rings
+constexpr int kDsCol = 384;                    // dS[2] as bf16 pairs: key k of row m at column 384 + 64 b + k/2
+constexpr int kDqSmem = 1024 + 2 * kTileBytes + (kDqKStages + kDqVStages) * kTileBytes + 256 + 1024;
 
 // backward kernels: warp 0 TMA, warp 1 MMA, warps 2..9 element-wise; the
 // element-wise warps w and w+4 share TMEM lane quarter (w & 3) and split the
@@ -412,28 +413,30 @@ struct BwdParams {
 };
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128
-                          const __grid_constant__ CUtensorMap map_kv,   // qkv, box 64 x 64
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128 (Q, K, V tiles)
                           const __grid_constant__ CUtensorMap map_do,   // dO [B][T][C], box 64 x 128
                           const __grid_constant__ CUtensorMap map_dq,   // dqkv, box 64 x 128
                           const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem, *sG = sQ + kTileBytes;
-  uint8_t *sKV = sG + kTileBytes;  // stage s: K at s*32K, V at s*32K + 16K
-  uint8_t *sDS = sKV + kDqStages * 2 * kKVTile64;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sDS + 2 * kDsTile);
-  // q_full, kv_full[3], kv_empty[3], s_full[2], s_empty[2], ds_full[2], ds_empty[2], fin, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+  uint8_t *sK = sG + kTileBytes;                 // K ring
+  uint8_t *sV = sK + kDqKStages * kTileBytes;    // V ring
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kDqVStages * kTileBytes);
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_empty, ds_full[2], ds_empty[2], fin, drain
+  constexpr int kB = 1 + 2 * kDqKStages + 2 * kDqVStages;
+  static_assert((kB + 8) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t q_full = smem_u32(bars);
-  auto kv_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto kv_empty = [&](int s) { return smem_u32(bars + 4 + s); };
-  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
-  auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
-  auto ds_full = [&](int s) { return smem_u32(bars + 11 + s); };
-  auto ds_empty = [&](int s) { return smem_u32(bars + 13 + s); };
-  const uint32_t fin = smem_u32(bars + 15), drain = smem_u32(bars + 16);
+  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto k_empty = [&](int s) { return smem_u32(bars + 1 + kDqKStages + s); };
+  auto v_full = [&](int s) { return smem_u32(bars + 1 + 2 * kDqKStages + s); };
+  auto v_empty = [&](int s) { return smem_u32(bars + 1 + 2 * kDqKStages + kDqVStages + s); };
+  const uint32_t s_full = smem_u32(bars + kB), s_empty = smem_u32(bars + kB + 1);
+  auto ds_full = [&](int s) { return smem_u32(bars + kB + 2 + s); };
+  auto ds_empty = [&](int s) { return smem_u32(bars + kB + 4 + s); };
+  const uint32_t fin = smem_u32(bars + kB + 6), drain = smem_u32(bars + kB + 7);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = gridDim.x / p.n_tiles;
@@ -442,14 +445,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int q0 = qt * kQ;
   const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK;
   const int C = p.H * kD;
-  // TMEM columns: S[2] at 0, 64; dP[2] at 128, 192; dQ at 256
+  // TMEM columns: S at 0, dP at 128 (one buffer, free again as soon as the
+  // element-wise warps have loaded it); dQ at 256; dS[2] (bf16 pairs) at 384, 448
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kDqStages; ++s) { mbar_init(kv_full(s), 1); mbar_init(kv_empty(s), 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full(s), 1); mbar_init(s_empty(s), kSoft);
-      mbar_init(ds_full(s), kSoft); mbar_init(ds_empty(s), 1);
-    }
+    for (int s = 0; s < kDqKStages; ++s) { mbar_init(k_full(s), 1); mbar_init(k_empty(s), 1); }
+    for (int s = 0; s < kDqVStages; ++s) { mbar_init(v_full(s), 1); mbar_init(v_empty(s), 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, kSoft);
+    for (int s = 0; s < 2; ++s) { mbar_init(ds_full(s), kSoft); mbar_init(ds_empty(s), 1); }
     mbar_init(fin, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -470,59 +474,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
-        const int st = j % kDqStages;
-        if (!mbar_wait(kv_empty(st), ((j / kDqStages) & 1) ^ 1, abort_flag, p.status)) break;
-        const uint32_t k_dst = smem_u32(sKV) + st * 2 * kKVTile64, v_dst = k_dst + kKVTile64;
-        mbar_expect_tx(kv_full(st), 2 * kKVTile64);
-        for (int i = 0; i < 2; ++i) {
-          tma_load_3d(k_dst + i * 8192, &map_kv, C + 64 * i, j * kBK, b, kv_full(st));
-          tma_load_3d(v_dst + i * 8192, &map_kv, C + kD + 64 * i, j * kBK, b, kv_full(st));
-        }
+        const int ks = j % kDqKStages, vs = j % kDqVStages;
+        if (!mbar_wait(k_empty(ks), ((j / kDqKStages) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_expect_tx(k_full(ks), kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, j * kBK, b, k_full(ks));
+        if (!mbar_wait(v_empty(vs), ((j / kDqVStages) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_expect_tx(v_full(vs), kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, j * kBK, b,
+                      v_full(vs));
         ++issued;
       }
+      // let the loads in flight land before the CTA can exit
       const uint64_t t0 = globaltimer();
       while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued - kDqStages); j < issued; ++j) {
+      for (int j = max(0, issued - kDqVStages); j < issued; ++j) {
         const uint64_t t1 = globaltimer();
-        while (!mbar_try(kv_full(j % kDqStages), (j / kDqStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(k_full(j % kDqKStages), (j / kDqKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(v_full(j % kDqVStages), (j / kDqVStages) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc(0, 0, kQ, kBK);   // Q K^T, dO V^T
-      const uint32_t idesc_q = make_idesc(0, 1, kQ, kD);    // dS K (K as MN-major B)
-      const uint32_t aQ = smem_u32(sQ), aG = smem_u32(sG);
+      const uint32_t idesc_q = make_idesc(0, 1, kQ, kD);    // dS K: dS from TMEM, K as MN-major B
+      // Descriptors are built once; (byte offset >> 4) added to one moves its
+      // start address (shared addresses stay below 2^18, so the 14-bit field
+      // cannot carry).  The issuing thread shares its scheduler with two
+      // element-wise warps, so every instruction it saves shortens the
+      // hand-offs that keep the tensor pipe fed.
+      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dGd = smem_desc(smem_u32(sG), 16, 1024);
+      const uint64_t dKs = smem_desc(smem_u32(sK), 16, 1024);      // K-major view of K stage 0
+      const uint64_t dKm = smem_desc(smem_u32(sK), 16384, 1024);   // MN-major view of K stage 0
+      const uint64_t dVs = smem_desc(smem_u32(sV), 16, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       auto issue_sdp = [&](int j) -> bool {
-        const int st = j % kDqStages, bb = j & 1;
-        if (!mbar_wait(kv_full(st), (j / kDqStages) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(s_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        const int ks = j % kDqKStages, vs = j % kDqVStages;
+        if (!mbar_wait(k_full(ks), (j / kDqKStages) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(v_full(vs), (j / kDqVStages) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t bK = smem_u32(sKV) + st * 2 * kKVTile64, bV = bK + kKVTile64;
+        const uint64_t k = dKs + (uint64_t)((ks * kTileBytes) >> 4), v = dVs + (uint64_t)((vs * kTileBytes) >> 4);
 #pragma unroll
         for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t oa = (s >> 2) * 16384 + (s & 3) * 32, ob = (s >> 2) * 8192 + (s & 3) * 32;
-          tc_mma(tmem + bb * kBK, smem_desc(aQ + oa, 16, 1024), smem_desc(bK + ob, 16, 1024), idesc_s, s > 0);
-          tc_mma(tmem + 128 + bb * kBK, smem_desc(aG + oa, 16, 1024), smem_desc(bV + ob, 16, 1024), idesc_s,
-                 s > 0);
+          const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+          tc_mma(tmem + 0, dQd + o, k + o, idesc_s, s > 0);
+          tc_mma(tmem + 128, dGd + o, v + o, idesc_s, s > 0);
         }
-        tc_commit(s_full(bb));
+        tc_commit(s_full);
+        tc_commit(v_empty(vs));  // V is read by dP only
         return true;
       };
+      // Fixed order S_{j+1}, then dQ += dS_j K_j: the scores of the next tile
+      // are on the tensor core while the element-wise warps turn S_j into dS_j.
       if (ok) ok = issue_sdp(0);
-      if (ok && n_kv > 1) ok = issue_sdp(1);
       for (int j = 0; j < n_kv && ok; ++j) {
-        const int bb = j & 1, st = j % kDqStages;
-        if (!mbar_wait(ds_full(bb), (j >> 1) & 1, abort_flag, p.status)) break;
+        if (j + 1 < n_kv && !(ok = issue_sdp(j + 1))) break;
+        const int bb = j & 1, ks = j % kDqKStages;
+        if (!(ok = mbar_wait(ds_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
         tc_fence_after();
-        const uint32_t aS = smem_u32(sDS) + bb * kDsTile, bK = smem_u32(sKV) + st * 2 * kKVTile64;
+        const uint64_t k = dKm + (uint64_t)((ks * kTileBytes) >> 4);
 #pragma unroll
         for (int s = 0; s < kBK / 16; ++s)
-          tc_mma(tmem + 256, smem_desc(aS + s * 32, 16, 1024), smem_desc(bK + s * 2048, 8192, 1024), idesc_q,
-                 (j > 0 || s > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 256, tmem + kDsCol + bb * 64 + 8 * s, k + ((s * 2048) >> 4), idesc_q,
+                    (j > 0 || s > 0) ? 1u : 0u);
         tc_commit(ds_empty(bb));
-        tc_commit(kv_empty(st));
-        if (j + 2 < n_kv && !issue_sdp(j + 2)) break;
+        tc_commit(k_empty(ks));
       }
       tc_commit(fin);
       tc_commit(drain);
@@ -538,7 +556,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sc = rsqrtf((float)kD) * kLog2e;
     const int rr_ = min(row, p.T - 1);
     const float L = p.lse[((int64_t)b * p.H + h) * p.T + rr_] * kLog2e;
-    const int c0 = g * 32;  // this thread's 32 keys of the 64-key tile
+    const int c0 = g * 64;  // this thread's 64 keys of the 128-key tile
     // D = rowsum(dO * O) for this row: dO from the shared tile, O from global;
     // warpgroup g sums dims [64g, 64g + 64) and the halves meet in shared memory
     float *sDpart = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [2][128]
@@ -563,20 +581,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (g == 0 && row < p.T) p.Drow[((int64_t)b * p.H + h) * p.T + row] = Dv;
     for (int j = 0; j < n_kv; ++j) {
       const int bb = j & 1;
-      ok = mbar_wait(s_full(bb), (j >> 1) & 1, abort_flag, p.status);
+      ok = mbar_wait(s_full, j & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[32], dv[32];
-      tmem_ld32_nw(lane_base + bb * kBK + c0, sv);
-      tmem_ld32_nw(lane_base + 128 + bb * kBK + c0, dv);
+      // all 64 S and dP values of this row half at once, so the buffer is
+      // free for the next tile's MMAs before any arithmetic here
+      uint32_t sv[64], dv[64];
+      tmem_ld32_nw(lane_base + c0, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32_nw(lane_base + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32_nw(lane_base + 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(dv));
+      tmem_ld32_nw(lane_base + 128 + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(s_empty(bb));
+      mbar_arrive(s_empty);
       const int kv0 = j * kBK + c0;
-      const bool need_mask = kv0 + 32 > q0 || kv0 + 32 > p.T;
-      uint32_t packed[16];
+      const bool need_mask = kv0 + 64 > q0 || kv0 + 64 > p.T;
+      uint32_t packed[32];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
+      for (int i = 0; i < 64; i += 2) {
         float d2[2];
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -587,16 +609,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         packed[i / 2] = pack2(d2[0], d2[1]);
       }
+      // dS_j into TMEM buffer bb once dQ += dS_{j-2} K_{j-2} has read it
       ok = mbar_wait(ds_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      uint8_t *dst = sDS + bb * kDsTile;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int uu = 4 * g + u;
-        *reinterpret_cast<uint4 *>(dst + r * 128 + ((uu ^ (r & 7)) << 4)) =
-            make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-      }
-      fence_proxy_async();
+      tmem_st32(lane_base + kDsCol + bb * 64 + 32 * g, packed);
       tc_fence_before();
       mbar_arrive(ds_full(bb));
     }
@@ -639,12 +655,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------- dK, dV: CTA = 128 keys of row b; loop over heads x 64-query tiles ----------------
 constexpr int kBQ2 = 64;
-constexpr int kKvStages = 3;
+constexpr int kKvStages = 4;
 constexpr int kQTile64 = kBQ2 * kD * 2;          // 16 KB
 constexpr int kQStage = 2 * kQTile64 + 1024;     // Q, dO, then L[64], D[64]; keeps 1 KB alignment
-constexpr int kPTile = kQ * kBQ2 * 2;            // [128 keys x 64 q] bf16, 16 KB
-constexpr int kKvSmemTc = 1024 + 2 * kTileBytes + kKvStages * kQStage + 2 * kPTile + 256;
-static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0 && kPTile % 1024 == 0,
+constexpr int kKvSmemTc = 1024 + 2 * kTileBytes + kKvStages * kQStage + 256;
+static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0,
               "128-byte-swizzled TMA tiles need 1 KB-aligned shared-memory addresses");
 static_assert(kKvSmemTc <= 232448 && kDqSmem <= 232448 && kSmem <= 232448, "shared memory per CTA");
 
@@ -658,19 +673,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sK = smem, *sV = sK + kTileBytes;
   uint8_t *sQS = sV + kTileBytes;                 // stage s at s*kQStage: Q, dO, L, D
-  uint8_t *sP = sQS + kKvStages * kQStage;        // P^T then dS^T (16 KB each)
-  uint8_t *sDS = sP + kPTile;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sDS + kPTile);
-  // kv_full, q_full[3], q_empty[3], s_full[2], s_empty[2], pds_full, pds_empty, fin, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sQS + kKvStages * kQStage);
+  // kv_full, q_full[S] (Q, dO tiles), ld_full[S] (L, D), q_empty[S], s_full, s_empty,
+  // pds_full[2], pds_empty[2], fin, drain
+  constexpr int kB = 1 + 3 * kKvStages;
+  static_assert((kB + 8) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t kv_full = smem_u32(bars);
   auto q_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto q_empty = [&](int s) { return smem_u32(bars + 4 + s); };
-  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
-  auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
-  const uint32_t pds_full = smem_u32(bars + 11), pds_empty = smem_u32(bars + 12);
-  const uint32_t fin = smem_u32(bars + 13), drain = smem_u32(bars + 14);
+  auto ld_full = [&](int s) { return smem_u32(bars + 1 + kKvStages + s); };
+  auto q_empty = [&](int s) { return smem_u32(bars + 1 + 2 * kKvStages + s); };
+  const uint32_t s_full = smem_u32(bars + kB), s_empty = smem_u32(bars + kB + 1);
+  auto pds_full = [&](int s) { return smem_u32(bars + kB + 2 + s); };
+  auto pds_empty = [&](int s) { return smem_u32(bars + kB + 4 + s); };
+  const uint32_t fin = smem_u32(bars + kB + 6), drain = smem_u32(bars + kB + 7);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Bn = gridDim.x / p.n_tiles;
@@ -681,13 +698,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int first = k0 / kBQ2;
   const int n_q = (p.T + kBQ2 - 1) / kBQ2 - first;
   const int n_it = n_q * p.H;
-  // TMEM columns: S^T[2] at 0, 64; dP^T[2] at 128, 192; dV at 256; dK at 384
+  // TMEM columns: S^T at 0, dP^T at 64 (one buffer, free again as soon as
+  // the element-wise warps have loaded it); P^T[b] at 128 + 64b and dS^T[b]
+  // at 160 + 64b as bf16 pairs (query q of the tile at column q/2), the
+  // A operands of the dV, dK MMAs; dV at 256; dK at 384.
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < kKvStages; ++s) { mbar_init(q_full(s), 33); mbar_init(q_empty(s), 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(s_full(s), 1); mbar_init(s_empty(s), kSoft); }
-    mbar_init(pds_full, kSoft);
-    mbar_init(pds_empty, 1);
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(ld_full(s), 32);
+      mbar_init(q_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, kSoft);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(pds_full(s), kSoft);
+      mbar_init(pds_empty(s), 1);
+    }
     mbar_init(fin, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -724,7 +751,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ls_dst + 4 * i), "l"(p.lse + gi) : "memory");
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ds_dst + 4 * i), "l"(p.Drow + gi) : "memory");
       }
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(q_full(st)) : "memory");
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(ld_full(st)) : "memory");
       if (lane == 0) {
         mbar_expect_tx(q_full(st), 2 * kQTile64);
         const uint32_t dst = smem_u32(stage);
@@ -742,47 +769,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int it = max(0, issued - kKvStages); it < issued; ++it) {
         const uint64_t t1 = globaltimer();
         while (!mbar_try(q_full(it % kKvStages), (it / kKvStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(ld_full(it % kKvStages), (it / kKvStages) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc(0, 0, kQ, kBQ2);  // K Q^T, V dO^T
-      const uint32_t idesc_g = make_idesc(0, 1, kQ, kD);    // P^T dO, dS^T Q
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+      const uint32_t idesc_g = make_idesc(0, 1, kQ, kD);    // P^T dO, dS^T Q: A from TMEM, B MN-major
+      // Descriptors built once; (byte offset >> 4) added moves the start
+      // address (no carry: shared addresses are below 2^18).
+      const uint64_t dKd = smem_desc(smem_u32(sK), 16, 1024), dVd = smem_desc(smem_u32(sV), 16, 1024);
+      const uint64_t dQs = smem_desc(smem_u32(sQS), 16, 1024);    // K-major view of stage 0
+      const uint64_t dQm = smem_desc(smem_u32(sQS), 8192, 1024);  // MN-major view of stage 0
       bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
-      auto issue_s = [&](int it) -> bool {
-        const int st = it % kKvStages, bb = it & 1;
-        if (!mbar_wait(q_full(st), (it / kKvStages) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(s_empty(bb), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % kKvStages;
+        if (!mbar_wait(q_full(st), (j / kKvStages) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t bQ = smem_u32(sQS + st * kQStage), bG = bQ + kQTile64;
+        const uint64_t q = dQs + (uint64_t)((st * kQStage) >> 4), g = q + (kQTile64 >> 4);
 #pragma unroll
         for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t oa = (s >> 2) * 16384 + (s & 3) * 32, ob = (s >> 2) * 8192 + (s & 3) * 32;
-          tc_mma(tmem + bb * kBQ2, smem_desc(aK + oa, 16, 1024), smem_desc(bQ + ob, 16, 1024), idesc_s, s > 0);
-          tc_mma(tmem + 128 + bb * kBQ2, smem_desc(aV + oa, 16, 1024), smem_desc(bG + ob, 16, 1024), idesc_s,
-                 s > 0);
+          const uint32_t oa = ((s >> 2) * 16384 + (s & 3) * 32) >> 4, ob = ((s >> 2) * 8192 + (s & 3) * 32) >> 4;
+          tc_mma(tmem + 0, dKd + oa, q + ob, idesc_s, s > 0);
+          tc_mma(tmem + 64, dVd + oa, g + ob, idesc_s, s > 0);
         }
-        tc_commit(s_full(bb));
+        tc_commit(s_full);
         return true;
       };
+      // Fixed order S^T_{j+1}, then dV += P^T_j dO_j, dK += dS^T_j Q_j: the
+      // next scores are on the tensor core while tile j is turned into P, dS.
       if (ok) ok = issue_s(0);
-      if (ok && n_it > 1) ok = issue_s(1);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int st = it % kKvStages;
-        if (!mbar_wait(pds_full, it & 1, abort_flag, p.status)) break;
+      for (int j = 0; j < n_it && ok; ++j) {
+        if (j + 1 < n_it && !(ok = issue_s(j + 1))) break;
+        const int st = j % kKvStages, bb = j & 1;
+        if (!(ok = mbar_wait(pds_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
         tc_fence_after();
-        const uint32_t bQ = smem_u32(sQS + st * kQStage), bG = bQ + kQTile64;
-        const uint32_t aP = smem_u32(sP), aS = smem_u32(sDS);
+        const uint64_t q = dQm + (uint64_t)((st * kQStage) >> 4), g = q + (kQTile64 >> 4);
 #pragma unroll
         for (int s = 0; s < kBQ2 / 16; ++s) {
-          const uint32_t acc = (it > 0 || s > 0) ? 1u : 0u;
-          tc_mma(tmem + 256, smem_desc(aP + s * 32, 16, 1024), smem_desc(bG + s * 2048, 8192, 1024), idesc_g, acc);
-          tc_mma(tmem + 384, smem_desc(aS + s * 32, 16, 1024), smem_desc(bQ + s * 2048, 8192, 1024), idesc_g, acc);
+          const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
+          const uint32_t a_col = 128 + bb * 64 + 8 * s;  // queries 16s .. 16s+15
+          tc_mma_ts(tmem + 256, tmem + a_col, g + ((s * 2048) >> 4), idesc_g, acc);
+          tc_mma_ts(tmem + 384, tmem + a_col + 32, q + ((s * 2048) >> 4), idesc_g, acc);
         }
-        tc_commit(pds_empty);
+        tc_commit(pds_empty(bb));
         tc_commit(q_empty(st));
-        if (it + 2 < n_it && !issue_s(it + 2)) break;
       }
       tc_commit(fin);
       tc_commit(drain);
@@ -801,16 +833,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < n_it; ++it) {
       const int bb = it & 1, st = it % kKvStages;
       const int qq0 = (first + it % n_q) * kBQ2 + c0;
-      ok = mbar_wait(s_full(bb), (it >> 1) & 1, abort_flag, p.status) &&
-           mbar_wait(q_full(st), (it / kKvStages) & 1, abort_flag, p.status);
+      ok = mbar_wait(s_full, it & 1, abort_flag, p.status) &&
+           mbar_wait(ld_full(st), (it / kKvStages) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[32], dv[32];
-      tmem_ld32_nw(lane_base + bb * kBQ2 + c0, sv);
-      tmem_ld32_nw(lane_base + 128 + bb * kBQ2 + c0, dv);
+      tmem_ld32_nw(lane_base + c0, sv);
+      tmem_ld32_nw(lane_base + 64 + c0, dv);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(s_empty(bb));
+      mbar_arrive(s_empty);  // the next tile's S^T, dP^T may overwrite them now
       const float4 *Ls4 = reinterpret_cast<const float4 *>(sQS + st * kQStage + 2 * kQTile64) + c0 / 4;
       const float4 *Ds4 = Ls4 + kBQ2 / 4;
       const bool need_mask = qq0 < key + 1 || qq0 + 32 > p.T;
@@ -833,17 +865,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dd[2 * i4] = pack2(ds[0], ds[1]);
         dd[2 * i4 + 1] = pack2(ds[2], ds[3]);
       }
-      ok = mbar_wait(pds_empty, (it & 1) ^ 1, abort_flag, p.status);
+      // P^T, dS^T into buffer bb once the MMAs of tile it - 2 have read it
+      ok = mbar_wait(pds_empty(bb), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int off = r * 128 + (((4 * g + u) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4 *>(sP + off) = make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-        *reinterpret_cast<uint4 *>(sDS + off) = make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-      }
-      fence_proxy_async();
+      tmem_st16_nw(lane_base + 128 + bb * 64 + 16 * g, pp);
+      tmem_st16_nw(lane_base + 160 + bb * 64 + 16 * g, dd);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(pds_full);
+      mbar_arrive(pds_full(bb));
     }
     if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
@@ -953,7 +982,7 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   p.O = O;
   p.status = status;
   p.n_tiles = (T + kQ - 1) / kQ;
-  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mkv64, mdo128, mout, p);
+  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mkv64, mdo64, mout, p);

@@ -53,6 +53,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase (try_wait may suspend the thread for a while
+// before it gives up, which stalls a loop that polls several barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait; false if this CTA is aborting (flag set here or elsewhere).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int *status) {
@@ -70,6 +83,29 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
+
+// Deadline of a loop that polls several barriers at once (an MMA warp that
+// issues whichever group of MMAs is ready first): reset() on every step of
+// progress; expired() turns true when this CTA is aborting or kWaitNs passed
+// without progress (it then raises the abort flag and the timeout status).
+struct PollDeadline {
+  uint64_t t0;
+  uint32_t n;
+  __device__ __forceinline__ void reset() {
+    t0 = globaltimer();
+    n = 0;
+  }
+  __device__ __forceinline__ bool expired(volatile int *abort_flag, int *status) {
+    if ((++n & 255) != 0) return false;
+    if (*abort_flag) return true;
+    if (globaltimer() - t0 > kWaitNs) {
+      *abort_flag = 1;
+      set_status(status, kStatusTimeout);
+      return true;
+    }
+    return false;
+  }
+};
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             uint32_t bar) {
@@ -197,6 +233,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+
+// TMEM store of 16 consecutive 32-bit columns of this thread's lane, without
+// the wait: call tmem_wait_st() before the columns are handed on.
+__device__ __forceinline__ void tmem_st16_nw(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
                                             uint32_t bar) {
