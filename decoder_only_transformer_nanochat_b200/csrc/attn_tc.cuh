@@ -653,20 +653,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-// ---------------- dK, dV: CTA = 128 keys of row b; loop over heads x 64-query tiles ----------------
-constexpr int kBQ2 = 64;
-constexpr int kKvStages = 4;
-constexpr int kQTile64 = kBQ2 * kD * 2;          // 16 KB
-constexpr int kQStage = 2 * kQTile64 + 1024;     // Q, dO, then L[64], D[64]; keeps 1 KB alignment
+// ---------------- dK, dV: CTA = 128 keys of row b; loop over heads x 128-query tiles ----------------
+// 128-query tiles keep every MMA at N = 128.  TMEM holds one 128-column
+// score buffer X that takes S^T and then dP^T of a tile in turn, P^T and dS^T
+// as bf16 A operands, and the dV, dK accumulators:
+//   X [0,128)   P^T [128,192)   dS^T [192,256)   dV [256,384)   dK [384,512)
+// Per tile the tensor core runs S^T = K Q^T, dP^T = V dO^T (once the
+// element-wise warps have loaded S^T), dV += P^T dO (once P^T is stored),
+// S^T of the next tile (once dP^T is loaded), dK += dS^T Q.
+constexpr int kBQ2 = 128;
+constexpr int kKvStages = 2;
+constexpr int kQStage = 2 * kTileBytes + 1024;   // Q, dO, then L[128], D[128]; keeps 1 KB alignment
 constexpr int kKvSmemTc = 1024 + 2 * kTileBytes + kKvStages * kQStage + 256;
+constexpr int kXCol = 0, kPtCol = 128, kDstCol = 192, kDvCol = 256, kDkCol = 384;
 static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0,
               "128-byte-swizzled TMA tiles need 1 KB-aligned shared-memory addresses");
 static_assert(kKvSmemTc <= 232448 && kDqSmem <= 232448 && kSmem <= 232448, "shared memory per CTA");
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap map_k,    // qkv, box 64 x 128
-                            const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 64
-                            const __grid_constant__ CUtensorMap map_do,   // dO, box 64 x 64
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap map_qkv,  // qkv, box 64 x 128 (K, V, Q)
+                            const __grid_constant__ CUtensorMap map_do,   // dO, box 64 x 128
                             const __grid_constant__ CUtensorMap map_out,  // dqkv, box 64 x 128
                             const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -674,20 +680,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *sK = smem, *sV = sK + kTileBytes;
   uint8_t *sQS = sV + kTileBytes;                 // stage s at s*kQStage: Q, dO, L, D
   uint64_t *bars = reinterpret_cast<uint64_t *>(sQS + kKvStages * kQStage);
-  // kv_full, q_full[S] (Q, dO tiles), ld_full[S] (L, D), q_empty[S], s_full, s_empty,
-  // pds_full[2], pds_empty[2], fin, drain
+  // kv_full, q_full[S] (Q, dO tiles), ld_full[S] (L, D), q_empty[S], then the hand-offs below
   constexpr int kB = 1 + 3 * kKvStages;
-  static_assert((kB + 8) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 8);
+  static_assert((kB + 10) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 10);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t kv_full = smem_u32(bars);
   auto q_full = [&](int s) { return smem_u32(bars + 1 + s); };
   auto ld_full = [&](int s) { return smem_u32(bars + 1 + kKvStages + s); };
   auto q_empty = [&](int s) { return smem_u32(bars + 1 + 2 * kKvStages + s); };
-  const uint32_t s_full = smem_u32(bars + kB), s_empty = smem_u32(bars + kB + 1);
-  auto pds_full = [&](int s) { return smem_u32(bars + kB + 2 + s); };
-  auto pds_empty = [&](int s) { return smem_u32(bars + kB + 4 + s); };
-  const uint32_t fin = smem_u32(bars + kB + 6), drain = smem_u32(bars + kB + 7);
+  const uint32_t s_full = smem_u32(bars + kB), dp_full = smem_u32(bars + kB + 1);      // MMA -> element-wise
+  const uint32_t s_taken = smem_u32(bars + kB + 2), dp_taken = smem_u32(bars + kB + 3);  // X loaded
+  const uint32_t p_full = smem_u32(bars + kB + 4), p_empty = smem_u32(bars + kB + 5);
+  const uint32_t ds_full = smem_u32(bars + kB + 6), ds_empty = smem_u32(bars + kB + 7);
+  const uint32_t fin = smem_u32(bars + kB + 8), drain = smem_u32(bars + kB + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Bn = gridDim.x / p.n_tiles;
@@ -698,10 +704,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int first = k0 / kBQ2;
   const int n_q = (p.T + kBQ2 - 1) / kBQ2 - first;
   const int n_it = n_q * p.H;
-  // TMEM columns: S^T at 0, dP^T at 64 (one buffer, free again as soon as
-  // the element-wise warps have loaded it); P^T[b] at 128 + 64b and dS^T[b]
-  // at 160 + 64b as bf16 pairs (query q of the tile at column q/2), the
-  // A operands of the dV, dK MMAs; dV at 256; dK at 384.
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < kKvStages; ++s) {
@@ -710,11 +712,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(q_empty(s), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_empty, kSoft);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(pds_full(s), kSoft);
-      mbar_init(pds_empty(s), 1);
-    }
+    mbar_init(dp_full, 1);
+    mbar_init(s_taken, kSoft);
+    mbar_init(dp_taken, kSoft);
+    mbar_init(p_full, kSoft);
+    mbar_init(p_empty, 1);
+    mbar_init(ds_full, kSoft);
+    mbar_init(ds_empty, 1);
     mbar_init(fin, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -731,8 +735,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       mbar_expect_tx(kv_full, 2 * kTileBytes);
       for (int i = 0; i < 2; ++i) {
-        tma_load_3d(smem_u32(sK) + i * 16384, &map_k, C + 64 * i, k0, b, kv_full);
-        tma_load_3d(smem_u32(sV) + i * 16384, &map_k, C + kD + 64 * i, k0, b, kv_full);
+        tma_load_3d(smem_u32(sK) + i * 16384, &map_qkv, C + 64 * i, k0, b, kv_full);
+        tma_load_3d(smem_u32(sV) + i * 16384, &map_qkv, C + kD + 64 * i, k0, b, kv_full);
       }
     }
     int issued = 0;
@@ -744,7 +748,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint8_t *stage = sQS + st * kQStage;
       // lse and D of the tile's queries: 4-byte asynchronous copies whose
       // completion arrives on the stage's barrier, so this warp never blocks
-      const uint32_t ls_dst = smem_u32(stage + 2 * kQTile64), ds_dst = ls_dst + kBQ2 * 4;
+      const uint32_t ls_dst = smem_u32(stage + 2 * kTileBytes), ds_dst = ls_dst + kBQ2 * 4;
       for (int i = lane; i < kBQ2; i += 32) {
         const int q = min(qq0 + i, p.T - 1);
         const int64_t gi = ((int64_t)b * p.H + hh) * p.T + q;
@@ -753,11 +757,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(ld_full(st)) : "memory");
       if (lane == 0) {
-        mbar_expect_tx(q_full(st), 2 * kQTile64);
+        mbar_expect_tx(q_full(st), 2 * kTileBytes);
         const uint32_t dst = smem_u32(stage);
         for (int i = 0; i < 2; ++i) {
-          tma_load_3d(dst + i * 8192, &map_q, hh * kD + 64 * i, qq0, b, q_full(st));
-          tma_load_3d(dst + kQTile64 + i * 8192, &map_do, hh * kD + 64 * i, qq0, b, q_full(st));
+          tma_load_3d(dst + i * 16384, &map_qkv, hh * kD + 64 * i, qq0, b, q_full(st));
+          tma_load_3d(dst + kTileBytes + i * 16384, &map_do, hh * kD + 64 * i, qq0, b, q_full(st));
         }
       }
       ++issued;
@@ -774,46 +778,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_s = make_idesc(0, 0, kQ, kBQ2);  // K Q^T, V dO^T
+      const uint32_t idesc_x = make_idesc(0, 0, kQ, kBQ2);  // K Q^T, V dO^T
       const uint32_t idesc_g = make_idesc(0, 1, kQ, kD);    // P^T dO, dS^T Q: A from TMEM, B MN-major
       // Descriptors built once; (byte offset >> 4) added moves the start
       // address (no carry: shared addresses are below 2^18).
       const uint64_t dKd = smem_desc(smem_u32(sK), 16, 1024), dVd = smem_desc(smem_u32(sV), 16, 1024);
-      const uint64_t dQs = smem_desc(smem_u32(sQS), 16, 1024);    // K-major view of stage 0
-      const uint64_t dQm = smem_desc(smem_u32(sQS), 8192, 1024);  // MN-major view of stage 0
+      const uint64_t dQs = smem_desc(smem_u32(sQS), 16, 1024);     // K-major view of stage 0
+      const uint64_t dQm = smem_desc(smem_u32(sQS), 16384, 1024);  // MN-major view of stage 0
+      constexpr uint32_t kGo = kTileBytes >> 4;                    // Q -> dO within a stage
       bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kKvStages;
-        if (!mbar_wait(q_full(st), (j / kKvStages) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint64_t q = dQs + (uint64_t)((st * kQStage) >> 4), g = q + (kQTile64 >> 4);
+      auto x_mma = [&](uint64_t a, uint64_t bq) {
 #pragma unroll
         for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t oa = ((s >> 2) * 16384 + (s & 3) * 32) >> 4, ob = ((s >> 2) * 8192 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + 0, dKd + oa, q + ob, idesc_s, s > 0);
-          tc_mma(tmem + 64, dVd + oa, g + ob, idesc_s, s > 0);
+          const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+          tc_mma(tmem + kXCol, a + o, bq + o, idesc_x, s > 0);
         }
-        tc_commit(s_full);
-        return true;
       };
-      // Fixed order S^T_{j+1}, then dV += P^T_j dO_j, dK += dS^T_j Q_j: the
-      // next scores are on the tensor core while tile j is turned into P, dS.
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_it && ok; ++j) {
-        if (j + 1 < n_it && !(ok = issue_s(j + 1))) break;
-        const int st = j % kKvStages, bb = j & 1;
-        if (!(ok = mbar_wait(pds_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        const uint64_t q = dQm + (uint64_t)((st * kQStage) >> 4), g = q + (kQTile64 >> 4);
+      auto g_mma = [&](uint32_t d_col, uint32_t a_col, uint64_t bq, bool first_tile) {
 #pragma unroll
-        for (int s = 0; s < kBQ2 / 16; ++s) {
-          const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
-          const uint32_t a_col = 128 + bb * 64 + 8 * s;  // queries 16s .. 16s+15
-          tc_mma_ts(tmem + 256, tmem + a_col, g + ((s * 2048) >> 4), idesc_g, acc);
-          tc_mma_ts(tmem + 384, tmem + a_col + 32, q + ((s * 2048) >> 4), idesc_g, acc);
+        for (int s = 0; s < kBQ2 / 16; ++s)
+          tc_mma_ts(tmem + d_col, tmem + a_col + 8 * s, bq + ((s * 2048) >> 4), idesc_g,
+                    (!first_tile || s > 0) ? 1u : 0u);
+      };
+      // S^T_0
+      if (ok) ok = mbar_wait(q_full(0), 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        x_mma(dKd, dQs);
+        tc_commit(s_full);
+      }
+      for (int j = 0; j < n_it && ok; ++j) {
+        const int st = j % kKvStages;
+        const uint64_t qs = dQs + (uint64_t)((st * kQStage) >> 4), qm = dQm + (uint64_t)((st * kQStage) >> 4);
+        const uint32_t par = j & 1;
+        // dP^T_j = V dO_j^T once S^T_j has left X
+        if (!(ok = mbar_wait(s_taken, par, abort_flag, p.status))) break;
+        tc_fence_after();
+        x_mma(dVd, qs + kGo);
+        tc_commit(dp_full);
+        // dV += P^T_j dO_j
+        if (!(ok = mbar_wait(p_full, par, abort_flag, p.status))) break;
+        tc_fence_after();
+        g_mma(kDvCol, kPtCol, qm + kGo, j == 0);
+        tc_commit(p_empty);
+        // S^T_{j+1} = K Q_{j+1}^T once dP^T_j has left X
+        if (j + 1 < n_it) {
+          const int st1 = (j + 1) % kKvStages;
+          if (!(ok = mbar_wait(dp_taken, par, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(q_full(st1), ((j + 1) / kKvStages) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          x_mma(dKd, dQs + (uint64_t)((st1 * kQStage) >> 4));
+          tc_commit(s_full);
         }
-        tc_commit(pds_empty(bb));
+        // dK += dS^T_j Q_j; the stage is free after this
+        if (!(ok = mbar_wait(ds_full, par, abort_flag, p.status))) break;
+        tc_fence_after();
+        g_mma(kDkCol, kDstCol, qm, j == 0);
+        tc_commit(ds_empty);
         tc_commit(q_empty(st));
       }
       tc_commit(fin);
@@ -828,51 +849,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int key = k0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = rsqrtf((float)kD) * kLog2e;
-    const int c0 = g * 32;  // this thread's 32 queries of the 64-query tile
+    const int c0 = g * 64;  // this thread's 64 queries of the 128-query tile
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int bb = it & 1, st = it % kKvStages;
+      const int st = it % kKvStages;
+      const uint32_t par = it & 1;
       const int qq0 = (first + it % n_q) * kBQ2 + c0;
-      ok = mbar_wait(s_full, it & 1, abort_flag, p.status) &&
+      ok = mbar_wait(s_full, par, abort_flag, p.status) &&
            mbar_wait(ld_full(st), (it / kKvStages) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[32], dv[32];
-      tmem_ld32_nw(lane_base + c0, sv);
-      tmem_ld32_nw(lane_base + 64 + c0, dv);
+      uint32_t xv[64];
+      tmem_ld32_nw(lane_base + kXCol + c0, *reinterpret_cast<uint32_t(*)[32]>(xv));
+      tmem_ld32_nw(lane_base + kXCol + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(xv + 32));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(s_empty);  // the next tile's S^T, dP^T may overwrite them now
-      const float4 *Ls4 = reinterpret_cast<const float4 *>(sQS + st * kQStage + 2 * kQTile64) + c0 / 4;
-      const float4 *Ds4 = Ls4 + kBQ2 / 4;
-      const bool need_mask = qq0 < key + 1 || qq0 + 32 > p.T;
-      uint32_t pp[16], dd[16];
+      mbar_arrive(s_taken);  // X may take dP^T now
+      const float *Ls = reinterpret_cast<const float *>(sQS + st * kQStage + 2 * kTileBytes) + c0;
+      const float *Ds = Ls + kBQ2;
+      const bool need_mask = qq0 < key + 1 || qq0 + 64 > p.T;
+      float pr[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int i4 = 0; i4 < 8; ++i4) {
-        const float4 l4 = Ls4[i4], d4 = Ds4[i4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pr[4], ds[4];
+      for (int i4 = 0; i4 < 16; ++i4) {
+        const float4 l4 = reinterpret_cast<const float4 *>(Ls)[i4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int qi = 4 * i4 + t;
-          float v = ex2(__uint_as_float(sv[qi]) * sc - lv[t] * kLog2e);
+          float v = ex2(__uint_as_float(xv[qi]) * sc - lv[t] * kLog2e);
           if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T)) v = 0.f;
-          pr[t] = v;
-          ds[t] = v * (__uint_as_float(dv[qi]) - dvv[t]);
+          pr[qi] = v;
         }
-        pp[2 * i4] = pack2(pr[0], pr[1]);
-        pp[2 * i4 + 1] = pack2(pr[2], pr[3]);
-        dd[2 * i4] = pack2(ds[0], ds[1]);
-        dd[2 * i4 + 1] = pack2(ds[2], ds[3]);
+        pk[2 * i4] = pack2(pr[4 * i4], pr[4 * i4 + 1]);
+        pk[2 * i4 + 1] = pack2(pr[4 * i4 + 2], pr[4 * i4 + 3]);
       }
-      // P^T, dS^T into buffer bb once the MMAs of tile it - 2 have read it
-      ok = mbar_wait(pds_empty(bb), ((it >> 1) & 1) ^ 1, abort_flag, p.status);
+      // P^T once dV += P^T_{it-1} dO has read the previous one
+      ok = mbar_wait(p_empty, par ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tmem_st16_nw(lane_base + 128 + bb * 64 + 16 * g, pp);
-      tmem_st16_nw(lane_base + 160 + bb * 64 + 16 * g, dd);
-      tmem_wait_st();
+      tmem_st32(lane_base + kPtCol + 32 * g, pk);
       tc_fence_before();
-      mbar_arrive(pds_full(bb));
+      mbar_arrive(p_full);
+      ok = mbar_wait(dp_full, par, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32_nw(lane_base + kXCol + c0, *reinterpret_cast<uint32_t(*)[32]>(xv));
+      tmem_ld32_nw(lane_base + kXCol + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(xv + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dp_taken);  // X may take the next S^T now
+#pragma unroll
+      for (int i4 = 0; i4 < 16; ++i4) {
+        const float4 d4 = reinterpret_cast<const float4 *>(Ds)[i4];
+        const float dd4[4] = {d4.x, d4.y, d4.z, d4.w};
+        float ds[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) ds[t] = pr[4 * i4 + t] * (__uint_as_float(xv[4 * i4 + t]) - dd4[t]);
+        pk[2 * i4] = pack2(ds[0], ds[1]);
+        pk[2 * i4 + 1] = pack2(ds[2], ds[3]);
+      }
+      ok = mbar_wait(ds_empty, par ^ 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tmem_st32(lane_base + kDstCol + 32 * g, pk);
+      tc_fence_before();
+      mbar_arrive(ds_full);
     }
     if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
@@ -884,7 +924,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(lane_base + (g == 0 ? 384 : 256) + c * 32, rr);
+        tmem_ld32(lane_base + (g == 0 ? kDkCol : kDvCol) + c * 32, rr);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint4 w;
@@ -967,10 +1007,9 @@ namespace fatc {
 
 inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const bf16 *dO, const float *lse,
                               float *Drow, bf16 *dqkv, int B, int T, int H, int *status, cudaStream_t st) {
-  CUtensorMap mq128, mkv64, mdo128, mdo64, mout;
+  CUtensorMap mq128, mdo128, mout;
   const int C = H * kD;
-  if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mkv64, qkv, B, T, (int)ld, ld, 64) ||
-      !make_map3(&mdo128, dO, B, T, C, C, 128) || !make_map3(&mdo64, dO, B, T, C, C, 64) ||
+  if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mdo128, dO, B, T, C, C, 128) ||
       !make_map3(&mout, dqkv, B, T, (int)ld, ld, 128))
     return cudaErrorInvalidValue;
   BwdParams p;
@@ -985,7 +1024,7 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mkv64, mdo64, mout, p);
+  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
   return cudaGetLastError();
 }
 
