@@ -212,19 +212,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = make_idesc(0, 0, kQ, kKV);   // Q K^T: both K-major
       const uint32_t idesc_o = make_idesc(0, 1, kQ, kD);    // P V: V is MN-major
-      const uint32_t aQ = smem_u32(sQ);
+      // Descriptors built once; (byte offset >> 4) added moves the start
+      // address (no carry: shared addresses are below 2^18).
+      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dKd = smem_desc(smem_u32(sK), 16, 1024);
+      const uint64_t dVd = smem_desc(smem_u32(sV), 8192, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       auto issue_s = [&](int j) -> bool {
         const int st = j & 1, ks = j % kKStages;
         if (!mbar_wait(k_full(ks), (j / kKStages) & 1, abort_flag, p.status)) return false;
         if (!mbar_wait(s_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t bK = smem_u32(sK) + ks * kTileBytes;
+        const uint64_t bK = dKd + (uint64_t)((ks * kTileBytes) >> 4);
 #pragma unroll
         for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-          tc_mma(tmem + st * kKV, smem_desc(aQ + off, 16, 1024), smem_desc(bK + off, 16, 1024), idesc_s,
-                 s > 0 ? 1u : 0u);
+          const uint32_t off = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+          tc_mma(tmem + st * kKV, dQd + off, bK + off, idesc_s, s > 0 ? 1u : 0u);
         }
         tc_commit(s_full(st));
         tc_commit(k_empty(ks));
@@ -236,13 +238,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(p_full, j & 1, abort_flag, p.status)) break;
         if (!mbar_wait(v_full(j & 1), (j >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t bV = smem_u32(sV) + (j & 1) * kTileBytes;
+        const uint64_t bV = dVd + (uint64_t)(((j & 1) * kTileBytes) >> 4);
 #pragma unroll
         for (int s = 0; s < kKV / 16; ++s) {
-          const uint32_t b_off = (s >> 2) * 16384 + (s & 3) * 2048;  // V: MN-major, k rows
+          const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;  // V: MN-major, k rows
           // P from TMEM: 16 keys = 8 columns of bf16 pairs
-          tc_mma_ts(tmem + 2 * kKV, tmem + kPCol + 8 * s, smem_desc(bV + b_off, 8192, 1024), idesc_o,
-                    (j > 0 || s > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 2 * kKV, tmem + kPCol + 8 * s, bV + b_off, idesc_o, (j > 0 || s > 0) ? 1u : 0u);
         }
         tc_commit(o_done);
         tc_commit(v_empty(j & 1));
