@@ -195,17 +195,26 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
     if (threadIdx.x == 0 && row + (int)gridDim.x < M)
       ce_fetch_row(buf, z + (size_t)(row + gridDim.x) * ldz, row_bytes, bar);
     const float smax2 = kSoftcap * kLog2e * block_max(tmax, red);
+    // e = exp(s - smax); t is replaced by w = e (1 - t^2), the row's gradient
+    // up to the factor 1 / (sum M), so the write-out needs no second
+    // exponential (two MUFU operations per logit instead of three).  w lies in
+    // [0, 1]; in fp16 it keeps 11 bits where it matters and flushes only
+    // entries far below the bf16 resolution of the row's largest ones.
     float sum = 0.f;
 #pragma unroll
     for (int k = 0; k < NVEC; ++k)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 r = __half22float2(t[k][j]);
-        sum += ex2_fast(kSoftcap * kLog2e * r.x - smax2) + ex2_fast(kSoftcap * kLog2e * r.y - smax2);
+        const float ea = ex2_fast(kSoftcap * kLog2e * r.x - smax2);
+        const float eb = ex2_fast(kSoftcap * kLog2e * r.y - smax2);
+        sum += ea + eb;
+        t[k][j] = __floats2half2_rn(ea * (1.f - r.x * r.x), eb * (1.f - r.y * r.y));
       }
     sum = block_sum(sum, red);  // contains __syncthreads: s_target is visible after it
     const float lse2 = smax2 + __log2f(sum);  // log-sum-exp in the log2 domain
     if (threadIdx.x == 0) token_loss[row] = lse2 * kLn2 - s_target;
+    const float scale = inv_M / sum;
     bf16 *zrow = z + (size_t)row * ldz;
 #pragma unroll
     for (int k = 0; k < NVEC; ++k) {
@@ -214,17 +223,15 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
       __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float2 r = __half22float2(t[k][j]);
-        const float pa = ex2_fast(kSoftcap * kLog2e * r.x - lse2);
-        const float pb = ex2_fast(kSoftcap * kLog2e * r.y - lse2);
-        h[j] = __floats2bfloat162_rn(pa * (1.f - r.x * r.x) * inv_M, pb * (1.f - r.y * r.y) * inv_M);
+        const float2 w = __half22float2(t[k][j]);
+        h[j] = __floats2bfloat162_rn(w.x * scale, w.y * scale);
       }
-      // the one-hot term of the target lives in exactly one thread's vector
+      // the one-hot term of the target lives in exactly one thread's vector;
+      // its p and 1 - t^2 come from the target's own softcapped logit
       if ((unsigned)(tgt - v * 8) < 8u) {
         const int j = (tgt - v * 8) >> 1;
-        const float2 r = __half22float2(t[k][j]);
-        const float rt = (tgt & 1) ? r.y : r.x;
-        const float pt = ex2_fast(kSoftcap * kLog2e * rt - lse2) - 1.f;
+        const float rt = s_target * (1.f / kSoftcap);
+        const float pt = ex2_fast(kLog2e * s_target - lse2) - 1.f;
         const bf16 val = __float2bfloat16_rn(pt * (1.f - rt * rt) * inv_M);
         if (tgt & 1) h[j].y = val;
         else h[j].x = val;

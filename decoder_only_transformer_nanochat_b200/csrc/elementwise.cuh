@@ -125,33 +125,40 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
   if (row >= M) return;
   const int nv = C >> 3;
   const size_t base = (size_t)row * C;
-  float g[NV][8], yy[NV][8];
+  // Pass 1: dot(dy, y) over the row, with the fp32 dx_old it will add to
+  // requested into L2 meanwhile.  Nothing is kept across the reduction, so
+  // the kernel runs at a register count that keeps many rows in flight.
   float dot = 0.f;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (lane + 32 * i);
     if (c < nv) {
-      Vec8<T>::load(dy + base + c * 8, g[i]);
-      Vec8<T>::load(y + base + c * 8, yy[i]);
+      float g[8], yy[8];
+      Vec8<T>::load(dy + base + c * 8, g);
+      Vec8<T>::load(y + base + c * 8, yy);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) dot += g[i][j] * yy[i][j];
+      for (int j = 0; j < 8; ++j) dot += g[j] * yy[j];
+      if (accumulate) asm volatile("prefetch.global.L2 [%0];" ::"l"(dx + base + c * 8));
     }
   }
   dot = warp_sum(dot) / (float)C;
   const float rr = r[row];
+  // Pass 2: dy and y again (now in L1 or L2), then dx and its copy in T.
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (lane + 32 * i);
     if (c < nv) {
-      float old[8];
+      float g[8], yy[8], old[8];
+      Vec8<T>::load(dy + base + c * 8, g);
+      Vec8<T>::load(y + base + c * 8, yy);
       if (accumulate) Vec8<float>::load(dx + base + c * 8, old);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        g[i][j] = rr * (g[i][j] - yy[i][j] * dot);
-        if (accumulate) g[i][j] += old[j];
+        g[j] = rr * (g[j] - yy[j] * dot);
+        if (accumulate) g[j] += old[j];
       }
-      Vec8<float>::store(dx + base + c * 8, g[i]);
-      Vec8<T>::store(dx_t + base + c * 8, g[i]);
+      Vec8<float>::store(dx + base + c * 8, g);
+      Vec8<T>::store(dx_t + base + c * 8, g);
     }
   }
 }
