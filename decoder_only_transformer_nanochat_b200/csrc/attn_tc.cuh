@@ -35,8 +35,8 @@ constexpr int kTileBytes = kQ * kD * 2;      // 32 KB: Q, K, V or P tile
 constexpr int kStageBytes = 2 * kTileBytes;  // K + V
 constexpr int kKStages = 3, kVStages = 2;
 constexpr int kSmem = 1024 + kTileBytes /*Q*/ + (kKStages + kVStages) * kTileBytes + 256 + 3072;
-constexpr int kTmemCols = 512;               // S0 [0,128), S1 [128,256), O [256,384), P [384,448)
-constexpr int kPCol = 384;                   // P as bf16 pairs: key k of row m at lane m, column kPCol + k/2
+constexpr int kTmemCols = 512;               // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
+constexpr int kPCol = 384;                   // P_j as bf16 pairs: key k of row m at lane m, column kPCol + 64 (j&1) + k/2
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
 
@@ -115,21 +115,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t *sK = sQ + kTileBytes;                  // K ring: kKStages tiles
   uint8_t *sV = sK + kKStages * kTileBytes;       // V ring: kVStages tiles
   uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kVStages * kTileBytes);
-  // bars: q_full, k_full[3], k_empty[3], s_full[2], s_empty[2], p_full, o_done, drain,
-  //       v_full[2], v_empty[2].  K and V have rings of their own: K_j is free as
-  //       soon as S_j is computed, so the loads of K_{j+2}, K_{j+3} overlap softmax j.
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+  // bars: q_full, k_full[3], k_empty[3], s_full[2], s_empty[2], p_full[2], drain,
+  //       v_full[2], v_empty[2], o_done[2].  K and V have rings of their own: K_j is
+  //       free as soon as S_j is computed, so the loads of K_{j+2}, K_{j+3} overlap
+  //       softmax j.  P has two TMEM buffers: P_{j+1} is written while P_j V_j runs.
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t q_full = smem_u32(bars + 0);
   auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
   auto k_empty = [&](int s) { return smem_u32(bars + 4 + s); };
   auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
   auto s_empty = [&](int s) { return smem_u32(bars + 9 + s); };
-  const uint32_t p_full = smem_u32(bars + 11);
-  const uint32_t o_done = smem_u32(bars + 12);
+  auto p_full = [&](int s) { return smem_u32(bars + 11 + s); };
   const uint32_t drain = smem_u32(bars + 13);
   auto v_full = [&](int s) { return smem_u32(bars + 14 + s); };
   auto v_empty = [&](int s) { return smem_u32(bars + 16 + s); };
+  auto o_done = [&](int s) { return smem_u32(bars + 18 + s); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = gridDim.x / p.n_qt;
@@ -150,9 +151,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(v_empty(s), 1);
       mbar_init(s_full(s), 1);
       mbar_init(s_empty(s), 256);
+      mbar_init(p_full(s), 256);
+      mbar_init(o_done(s), 1);
     }
-    mbar_init(p_full, 256);
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -235,17 +236,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok) ok = issue_s(0);
       for (int j = 0; j < n_kv && ok; ++j) {
         if (j + 1 < n_kv && !issue_s(j + 1)) break;
-        if (!mbar_wait(p_full, j & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag, p.status)) break;
         if (!mbar_wait(v_full(j & 1), (j >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint64_t bV = dVd + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+        const uint32_t a_p = tmem + kPCol + 64 * (j & 1);
 #pragma unroll
         for (int s = 0; s < kKV / 16; ++s) {
           const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;  // V: MN-major, k rows
           // P from TMEM: 16 keys = 8 columns of bf16 pairs
-          tc_mma_ts(tmem + 2 * kKV, tmem + kPCol + 8 * s, bV + b_off, idesc_o, (j > 0 || s > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 2 * kKV, a_p + 8 * s, bV + b_off, idesc_o, (j > 0 || s > 0) ? 1u : 0u);
         }
-        tc_commit(o_done);
+        tc_commit(o_done(j & 1));
         tc_commit(v_empty(j & 1));
       }
       tc_commit(drain);
@@ -315,18 +317,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float e0 = ex2(s[i] - m_used), e1 = ex2_poly(s[i + 1] - m_used);
+        // one exponential in four on the FMA pipe: measured fastest (half makes
+        // the loop issue-bound, none leaves it MUFU-bound)
+        const float e0 = ex2(s[i] - m_used);
+        const float e1 = (i & 2) ? ex2_poly(s[i + 1] - m_used) : ex2(s[i + 1] - m_used);
         sum += e0 + e1;
         pk[i / 2] = pack2(e0, e1);
       }
-      // P_{j-1} V_{j-1} must be done before P_j overwrites P and before O is touched
+      // P_j goes to buffer j & 1 once P_{j-2} V_{j-2} has read it; a rescale of
+      // O (rare: the base moves only when the max grows by more than 2^8) needs
+      // P_{j-1} V_{j-1} done as well
       if (j > 0) {
-        ok = mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status);
+        const bool rescale = __any_sync(0xffffffffu, grow);
+        if (rescale) ok = mbar_wait(o_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.status);
+        else if (j >= 2) ok = mbar_wait(o_done(j & 1), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, ok)) ok = false;
         ok = epi_vote_all256(ok);
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
+        if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {
             uint32_t rr[32];
@@ -337,14 +346,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      tmem_st32(lane_base + kPCol + 32 * g, pk);  // keys [64g, 64g + 64) of this row
+      tmem_st32(lane_base + kPCol + 64 * (j & 1) + 32 * g, pk);  // keys [64g, 64g + 64) of this row
       l += sum;
-      fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(j & 1));
     }
     // ---------------- epilogue: O / l, lse ----------------
-    if (ok) ok = mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, p.status);
+    if (ok) ok = mbar_wait(o_done((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
     sSum[g * kQ + r] = l;
     ok = epi_vote_all256(ok);
