@@ -306,19 +306,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0, aux_phase = 0;
     bool ok = true;
-    // The residual / relu^2 input tile of a unit is requested into L2 one unit
-    // ahead, so its TMA load in the epilogue does not wait on DRAM.
-    auto prefetch_aux = [&](int u2) {
-      if (!aux || !leader || u2 >= p.units) return;
-      const Unit x2 = unit_of(p, u2);
-      if (x2.m_blk * BM >= p.M) return;
-      for (int cc = 0; cc < BN; cc += 64)
-        if (x2.n_blk * BN + cc < p.N) tma_prefetch_2d(&map_d, x2.n_blk * BN + cc, x2.m_blk * BM);
-    };
-    prefetch_aux(blockIdx.x);
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit x = unit_of(p, u);
-      prefetch_aux(u + gridDim.x);
       // every lane waits; the vote over all epilogue threads keeps their
       // branches (and named barriers) uniform and re-converges each warp
       ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
@@ -605,20 +594,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (leader) mbar_arrive(tempty_bar(a));
       else mbar_arrive_remote(tempty_bar(a), 0);
     };
-    // The residual / relu^2 input tile of a unit is requested into L2 one unit
-    // ahead, so its TMA load in the epilogue does not wait on DRAM.
-    auto prefetch_aux = [&](int u2) {
-      if (!aux || !ep_leader || u2 >= p.units) return;
-      const Unit x2 = unit_of2(p, u2);
-      const int m2 = x2.m_blk * 256 + (int)rank * BM;
-      if (m2 >= p.M) return;
-      for (int cc = 0; cc < BN2; cc += 64)
-        if (x2.n_blk * BN2 + cc < p.N) tma_prefetch_2d(&map_d, x2.n_blk * BN2 + cc, m2);
-    };
-    prefetch_aux(cluster);
     for (int u = cluster; u < p.units && ok; u += n_clusters) {
       const Unit x = unit_of2(p, u);
-      prefetch_aux(u + n_clusters);
       ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
       __syncwarp();
       if (!ok) break;
