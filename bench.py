@@ -159,14 +159,25 @@ def dist_setup(gpus: int):
     return world, rank, local
 
 
-def reduce_max(x: float, world: int) -> float:
+def reduce_max(x: float, world: int, device: str = "cuda") -> float:
+    """Maximum of x over the ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Seed of rank `rank`'s token rows: every rank draws its own B rows."""
+    return seed + 1000 * rank
+
+
+def job_rate(tokens_per_rank: int, ms_max: float, world: int) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max / 1000.0)
 
 
 def barrier(world: int):
@@ -248,7 +259,7 @@ def run_ours(args):
     del flat
     if not (rank == 0 and world == 1 and not args.no_cpu_baseline):
         W64 = None
-    tok, tgt = synth.token_rows(wl.seed + 1000 * rank, wl.B, wl.T, wl.vocab, wl.tokens)
+    tok, tgt = synth.token_rows(shard_seed(wl.seed, rank), wl.B, wl.T, wl.vocab, wl.tokens)
     tokens = torch.from_numpy(tok).cuda()
     targets = torch.from_numpy(tgt).cuda()
     grads = torch.empty(model.n_params, dtype=torch.float32, device="cuda")
@@ -291,7 +302,7 @@ def run_ours(args):
         raise RuntimeError(f"device status after the timed steps: {nc.nc_strerror(status)}")
     ms = reduce_max(ms_local, world)
     tokens_per_step = wl.B * wl.T
-    value = world * tokens_per_step / (ms / 1000.0)
+    value = job_rate(tokens_per_step, ms, world)
 
     # ---------------- end to end: host buffers through the public API ----------------
     tok_h = torch.from_numpy(tok).pin_memory()
@@ -318,7 +329,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = reduce_max(e_start.elapsed_time(e_end) / args.steps, world)
-    e2e_value = world * tokens_per_step / (e2e_ms / 1000.0)
+    e2e_value = job_rate(tokens_per_step, e2e_ms, world)
     loss_val = float(loss_h.item())
 
     if rank != 0:
