@@ -1,24 +1,25 @@
-// Causal multi-query attention forward on the 5th-generation tensor cores
-// (energyai.berlin page, "Multi-Query Attention (MQA)": one key/value head
-// shared by the H query heads; scores q.k / sqrt(128), keys j <= i).
+// Causal multi-query attention on the 5th-generation tensor cores, forward
+// and backward (energyai.berlin page, "Multi-Query Attention (MQA)": one
+// key/value head shared by the H query heads; scores q.k / sqrt(128), keys
+// j <= i).
 //
-// CTA = 128 queries of one (row b, head h); keys in tiles of 128.
-//   warp 0      TMA: Q once, then K and V tiles into a 2-stage ring
+// Forward: CTA = 128 queries of one (row b, head h); keys in tiles of 128.
+//   warp 0      TMA: Q once, then K (3-stage ring) and V (2-stage ring) tiles
 //   warp 1      MMA: S_j = Q K_j^T into one of two TMEM score tiles,
-//               O += P_j V_j into a TMEM accumulator
-//   warps 2..5  softmax, one thread per query row: S row out of TMEM, running
-//               max / sum, P_j as bf16 into shared memory (the next MMA's
-//               A operand), O rescaled in TMEM only when the row max grows by
-//               more than 2^8 (the exponent base may lag the true max by up to
-//               8 in the log2 domain, which changes no result: P and the sum
+//               O += P_j V_j into a TMEM accumulator with P_j read from TMEM
+//   warps 2..9  softmax, two warps per query row (64 keys each): S row out of
+//               TMEM, running max / sum, P_j as bf16 pairs back into one of two
+//               TMEM P buffers, O rescaled in TMEM only when the row max grows
+//               by more than 2^8 (the exponent base may lag the true max by up
+//               to 8 in the log2 domain, which changes no result: P and the sum
 //               carry the same factor)
 // S_{j+1} is issued before P_j is ready, so the tensor core works on the next
 // scores while the softmax warps finish the current tile.
 //
 // Operands, all bf16 with 128-byte swizzle: Q, K as K-major (d contiguous)
 // tiles of 2 boxes [64 d x 128 rows]; V as an MN-major B operand (d
-// contiguous) of 4 boxes [64 d x 64 keys]; P as a K-major A operand of 2
-// blocks [64 keys x 128 rows] written by the softmax threads.
+// contiguous) of 4 boxes [64 d x 64 keys].  The backward kernels further down
+// are described where they start.
 #pragma once
 
 #include "tc_common.cuh"
@@ -29,10 +30,8 @@ namespace fatc {
 using namespace tc;
 
 constexpr int kQ = 128, kKV = 128, kD = 128;
-constexpr int kThreads = 192;
 constexpr int kFwdThreads = 320;  // TMA warp, MMA warp, 8 softmax warps
 constexpr int kTileBytes = kQ * kD * 2;      // 32 KB: Q, K, V or P tile
-constexpr int kStageBytes = 2 * kTileBytes;  // K + V
 constexpr int kKStages = 3, kVStages = 2;
 constexpr int kSmem = 1024 + kTileBytes /*Q*/ + (kKStages + kVStages) * kTileBytes + 256 + 3072;
 constexpr int kTmemCols = 512;               // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)

@@ -37,74 +37,10 @@ template <> __device__ __forceinline__ float exp_t<bf16>(float x) { return ex2_f
 template <> __device__ __forceinline__ float exp_t<float>(float x) { return expf(x); }
 
 // ---------------------------------------------------------------------------
-// Register-resident version for bf16 rows of V = 512 threads * 8 * NVEC
-// values (65,536 for NVEC = 16).  tanh(z/15) is kept per element as fp16
-// (|t| <= 1, 11-bit mantissa: finer than the bf16 logit it came from).
-template <int NVEC>
-__global__ void __launch_bounds__(512, 1) ce_fused_bf16_kernel(
-    bf16 *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
-    float *__restrict__ token_loss, int M, int V, float inv_M, int *status) {
-  __shared__ float red[32];
-  __shared__ float s_target;
-  const int row = blockIdx.x;
-  if (row >= M) return;
-  bf16 *zr = z + (size_t)row * ldz;
-  int tgt = targets[row];
-  if (tgt < 0 || tgt >= V) {
-    if (threadIdx.x == 0) set_status(status, kStatusRange);
-    tgt = tgt < 0 ? 0 : V - 1;
-  }
-  __half2 t[NVEC][4];
-  float tmax = -1.f;
-#pragma unroll
-  for (int k = 0; k < NVEC; ++k) {
-    const int v = threadIdx.x + k * 512;
-    uint4 u = *reinterpret_cast<const uint4 *>(zr + v * 8);
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __bfloat1622float2(h[j]);
-      const float a = tanh_fast(f.x * (1.f / kSoftcap)), b = tanh_fast(f.y * (1.f / kSoftcap));
-      t[k][j] = __floats2half2_rn(a, b);
-      const float2 r = __half22float2(t[k][j]);
-      tmax = fmaxf(tmax, fmaxf(r.x, r.y));
-      const int e = v * 8 + 2 * j;
-      if (e == tgt) s_target = kSoftcap * r.x;
-      if (e + 1 == tgt) s_target = kSoftcap * r.y;
-    }
-  }
-  const float smax = kSoftcap * block_max(tmax, red);
-  float sum = 0.f;
-#pragma unroll
-  for (int k = 0; k < NVEC; ++k)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 r = __half22float2(t[k][j]);
-      sum += ex2_fast((kSoftcap * r.x - smax) * kLog2e) + ex2_fast((kSoftcap * r.y - smax) * kLog2e);
-    }
-  sum = block_sum(sum, red);  // contains __syncthreads: s_target is visible after it
-  const float lse = smax + __logf(sum);
-  if (threadIdx.x == 0) token_loss[row] = lse - s_target;
-#pragma unroll
-  for (int k = 0; k < NVEC; ++k) {
-    const int v = threadIdx.x + k * 512;
-    uint4 u;
-    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 r = __half22float2(t[k][j]);
-      const int e = v * 8 + 2 * j;
-      float pa = ex2_fast((kSoftcap * r.x - lse) * kLog2e) - (e == tgt ? 1.f : 0.f);
-      float pb = ex2_fast((kSoftcap * r.y - lse) * kLog2e) - (e + 1 == tgt ? 1.f : 0.f);
-      h[j] = __floats2bfloat162_rn(pa * (1.f - r.x * r.x) * inv_M, pb * (1.f - r.y * r.y) * inv_M);
-    }
-    *reinterpret_cast<uint4 *>(zr + v * 8) = u;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Persistent version of the above (1024 threads, V = 1024 * 8 * NVEC): one CTA
-// per SM walks rows b, b + grid, ...
+// bf16 rows of V = 1024 threads * 8 * NVEC values (65,536 for NVEC = 8),
+// persistent: one CTA per SM walks rows b, b + grid, ...  tanh(z/15) is kept
+// per element as fp16 in registers (|t| <= 1, 11-bit mantissa: finer than the
+// bf16 logit it came from).
 // Each row (V bf16 = 128 KB at V = 65,536) arrives in shared memory by TMA
 // bulk copies; as soon as every thread has its slice in registers the copy of
 // the CTA's next row is issued, so the load of row i+1 and the store of dz for
