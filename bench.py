@@ -40,6 +40,11 @@ def model_flops_per_token(depth: int, C: int, V: int, T: int) -> float:
     return 6.0 * n_mm + 6.0 * T * C * depth
 
 
+def model_flops_per_token_noncausal(depth: int, C: int, V: int, T: int) -> float:
+    """The same count with attention taken dense (every query against all T keys)."""
+    return model_flops_per_token(depth, C, V, T) + 6.0 * T * C * depth
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -370,6 +375,7 @@ def run_ours(args):
 
     D = model.dims
     fpt = model_flops_per_token(wl.depth, D["width"], wl.vocab, wl.T)
+    fpt_nc = model_flops_per_token_noncausal(wl.depth, D["width"], wl.vocab, wl.T)
     model_tflops = value * fpt / 1e12
     launches = sum(s["launches"] for s in stats)
 
@@ -382,6 +388,8 @@ def run_ours(args):
         "mfu": model_tflops / (world * peaks["bf16_tflops"]),
         "mfu_sustained_peak": model_tflops / (world * peaks["bf16_tflops_sustained"]),
         "model_tflops": model_tflops, "model_flops_per_token": fpt,
+        "model_flops_per_token_noncausal": fpt_nc,
+        "mfu_noncausal": value * fpt_nc / 1e12 / (world * peaks["bf16_tflops"]),
         "peaks": {"source": peak_src, "bf16_tflops": peaks["bf16_tflops"],
                   "bf16_tflops_sustained": peaks["bf16_tflops_sustained"], "hbm_gbs": peaks["hbm_gbs"]},
         "roofline": roof,

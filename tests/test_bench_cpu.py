@@ -1,0 +1,39 @@
+"""bench.py's flop accounting, checked on CPU against the step it describes:
+the algorithmic flops of one training step rebuilt from its matrix products
+(forward, input-gradient and weight-gradient GEMMs) plus causal attention
+(forward: Q K^T and P V over the keys j <= i; backward: twice that), and the
+per-configuration values of the scope table."""
+import pytest
+
+import bench
+import oracle
+
+
+def _step_flops_per_token(depth, V, T):
+    D = oracle.dims(depth, V)
+    C, F, H = D["C"], D["F"], D["H"]
+    M = T  # per token: divide everything by the token count M = B*T (B drops out)
+    gemms = [(M, C + 256, C), (M, C, C), (M, F, C), (M, C, F)] * depth + [(M, V, C)]
+    fwd = sum(2.0 * m * n * k for m, n, k in gemms)
+    # causal attention: key j <= i, so T(T+1)/2 pairs per (row, head); two products of d = 128
+    attn_fwd = depth * H * 2 * (2.0 * 128 * T * (T + 1) / 2)
+    return (3 * fwd + 3 * attn_fwd) / M  # backward: dgrad + wgrad per GEMM, 2x the attention forward
+
+
+@pytest.mark.parametrize("name,depth,T,listed", [("d4", 4, 256, 1.195e8), ("d12", 12, 1024, 7.974e8),
+                                                  ("d20", 20, 2048, 2.823e9), ("d24", 24, 2048, 4.511e9),
+                                                  ("d32", 32, 2048, 9.764e9)])
+def test_model_flops_per_token(name, depth, T, listed):
+    C = oracle.dims(depth, 65536)["C"]
+    got = bench.model_flops_per_token(depth, C, 65536, T)
+    # the formula counts T/2 keys per query where the step has (T+1)/2
+    assert got == pytest.approx(_step_flops_per_token(depth, 65536, T), rel=1e-3)
+    assert got == pytest.approx(listed, rel=5e-4)
+    nc = bench.model_flops_per_token_noncausal(depth, C, 65536, T)
+    assert nc - got == pytest.approx(6.0 * T * C * depth)
+
+
+def test_job_rate_and_shard_seed():
+    assert bench.job_rate(32768, 100.0, 1) == pytest.approx(327680.0)
+    assert bench.job_rate(32768, 100.0, 8) == pytest.approx(8 * 327680.0)
+    assert len({bench.shard_seed(2, r) for r in range(8)}) == 8
