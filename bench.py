@@ -45,6 +45,15 @@ def model_flops_per_token_noncausal(depth: int, C: int, V: int, T: int) -> float
     return model_flops_per_token(depth, C, V, T) + 6.0 * T * C * depth
 
 
+def mufu_fraction(ms_per_step: float, tokens: int, vocab: int, num_sms: int, sm_mhz: float,
+                  ops_per_logit: float = 2.0) -> float:
+    """Fraction of the MUFU (special-function) roofline the CE kernel reaches:
+    ops_per_logit operations per logit (tanh, one exponential) against 16 per
+    clock per SM at the clock sampled during the run."""
+    ops_per_s = ops_per_logit * vocab * tokens / (ms_per_step / 1000.0)
+    return ops_per_s / (16.0 * num_sms * sm_mhz * 1e6)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -358,6 +367,13 @@ def run_ours(args):
             k["gbs"] = s["bytes"] / (s["ms"] / 1000.0) / 1e9
             k["hbm_frac"] = k["gbs"] / peaks["hbm_gbs"]
         kernels[s["name"]] = k
+    if "ce_fused" in kernels and clocks and clocks.get("sm_mhz"):
+        try:  # an optional figure: it must never cost the bench line
+            kernels["ce_fused"]["mufu_frac"] = mufu_fraction(
+                kernels["ce_fused"]["ms_per_step"], tokens_per_step, wl.vocab,
+                torch.cuda.get_device_properties(local).multi_processor_count, clocks["sm_mhz"])
+        except Exception as exc:  # noqa: BLE001
+            kernels["ce_fused"]["mufu_frac_error"] = repr(exc)
     if dominant["flops"] > 0:
         achieved = dominant["flops"] / (dominant["ms"] / 1000.0) / 1e12
         peak = peaks["bf16_tflops_sustained"]

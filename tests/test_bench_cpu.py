@@ -37,3 +37,11 @@ def test_job_rate_and_shard_seed():
     assert bench.job_rate(32768, 100.0, 1) == pytest.approx(327680.0)
     assert bench.job_rate(32768, 100.0, 8) == pytest.approx(8 * 327680.0)
     assert len({bench.shard_seed(2, r) for r in range(8)}) == 8
+
+
+def test_mufu_fraction():
+    # two operations per logit for B*T = 32768 tokens of V = 65536 logits at 148 SMs x 1485 MHz:
+    # 4.29e9 operations over 3.52e12 per second = 1.22 ms is the bound
+    bound_ms = 2.0 * 65536 * 32768 / (16 * 148 * 1485e6) * 1e3
+    assert bench.mufu_fraction(bound_ms, 32768, 65536, 148, 1485.0) == pytest.approx(1.0)
+    assert bench.mufu_fraction(2 * bound_ms, 32768, 65536, 148, 1485.0) == pytest.approx(0.5)
