@@ -11,7 +11,8 @@ from ._binding import (NC_BF16, NC_EALIGN, NC_ECUDA, NC_EINVAL, NC_ENOMEM,  # no
                        nc_workspace_bytes, nc_gemm, nc_attention_fwd, nc_attention_bwd,
                        NC_EPI_STORE, NC_EPI_STORE_F32, NC_EPI_ADD, NC_EPI_RELU2, NC_EPI_DRELU2,
                        NC_EPI_SOFTCAP, nc_profile, nc_profile_read,
-                       nc_attention_bwd_noalloc, NC_ATTN_BWD_NOALLOC_MAX_ROWS)
+                       nc_attention_bwd_noalloc, NC_ATTN_BWD_NOALLOC_MAX_ROWS, nc_ops_status,
+                       nc_check_wait_expiry)
 
 
 def __getattr__(name):

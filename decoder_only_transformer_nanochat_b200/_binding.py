@@ -71,6 +71,8 @@ _SIGS = {
                      _I, _I, _I, _P]),
     "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _P]),
     "nc_attention_bwd": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "nc_ops_status": (_I, [_P, _I]),
+    "nc_check_wait_expiry": (_I, [_I, _P]),
 }
 
 NC_EPI_STORE = 0
@@ -161,6 +163,16 @@ def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream) -> int:
 def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream) -> int:
     return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine,
                                            stream)
+
+
+def nc_ops_status(stream, timeout_ms: int) -> int:
+    """Status of the op-level calls (no model handle): read and clear."""
+    return load_library().nc_ops_status(stream, timeout_ms)
+
+
+def nc_check_wait_expiry(wait_us: int, stream) -> int:
+    """Enqueue a wait that runs out after wait_us and records a timeout."""
+    return load_library().nc_check_wait_expiry(wait_us, stream)
 
 
 def nc_profile(handle, enable: int) -> int:

@@ -10,7 +10,6 @@
 // sub + 8*c, c < 16, and dot products are finished with 3 shuffles.
 #pragma once
 
-#include "attn_mma.cuh"
 #include "elementwise.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -245,33 +244,32 @@ inline cudaError_t launch_attn_simt_bwd(const T *qkv, int ld, const T *dO, const
 
 namespace nc {
 
-// engine 0: tensor-core kernels (tcgen05 forward), 1: CUDA cores, 2: warp-level MMA
+// engine 0: the path of the model step -- tcgen05 tensor cores for bf16 (the
+// caller checks fatc::supported / supported_bwd first and reports a
+// misaligned operand; there is no slower fallback), CUDA cores for fp32;
+// engine 1: the CUDA-core kernels for either dtype (a test engine).
 template <typename T>
 inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H,
-                                   int num_sms, int engine, int *status, cudaStream_t st) {
-  (void)num_sms;
-  if (sizeof(T) == 2 && engine == 0 && fatc::supported(qkv, ld, O))
+                                   int engine, int *status, cudaStream_t st) {
+  if (sizeof(T) == 2 && engine == 0) {
+    if (!fatc::supported(qkv, ld, O)) return cudaErrorInvalidValue;
     return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, status, st);
-  if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, O))
-    return fa::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, st);
+  }
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
 }
 
-// D = rowsum(dO * O) is computed inside the tcgen05 dQ kernel; the other
-// engines get it from attn_rowdot_kernel first.  Drow is [B, H, T] scratch.
+// D = rowsum(dO * O) is computed inside the tcgen05 dQ kernel; the CUDA-core
+// engine gets it from attn_rowdot_kernel first.  Drow is [B, H, T] scratch.
 template <typename T>
 inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *O, const T *dO, const float *lse, float *Dr,
-                                   T *dqkv, int B, int T_len, int H, int num_sms, int engine, int *status,
-                                   cudaStream_t st) {
-  (void)num_sms;
-  if (sizeof(T) == 2 && engine == 0 && fatc::supported_bwd(qkv, ld, O, dO, dqkv))
+                                   T *dqkv, int B, int T_len, int H, int engine, int *status, cudaStream_t st) {
+  if (sizeof(T) == 2 && engine == 0) {
+    if (!fatc::supported_bwd(qkv, ld, O, dO, dqkv)) return cudaErrorInvalidValue;
     return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B,
                             T_len, H, status, st);
+  }
   const int M = B * T_len;
   attn_rowdot_kernel<T><<<(unsigned)(((size_t)M * H + 7) / 8), 256, 0, st>>>(dO, O, Dr, M, T_len, H);
-  if (sizeof(T) == 2 && (engine == 0 || engine == 2) && fa::supported(qkv, ld, dO) &&
-      fa::supported(dqkv, ld, dqkv))
-    return fa::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B, T_len, H, st);
   return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);
 }
 

@@ -986,8 +986,12 @@ inline cudaError_t init() {
   return e;
 }
 
+// Operands the TMA tiles can take: 16-byte aligned bases and row strides.
+inline bool aligned(const void *qkv, int64_t ld, const void *O) {
+  return (ld % 8) == 0 && ((uintptr_t)qkv & 15) == 0 && ((uintptr_t)O & 15) == 0;
+}
 inline bool supported(const void *qkv, int64_t ld, const void *O) {
-  return encode_fn() != nullptr && (ld % 8) == 0 && ((uintptr_t)qkv & 15) == 0 && ((uintptr_t)O & 15) == 0;
+  return encode_fn() != nullptr && aligned(qkv, ld, O);
 }
 
 inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int *status,
@@ -1036,8 +1040,11 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   return cudaGetLastError();
 }
 
+inline bool aligned_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const void *dqkv) {
+  return aligned(qkv, ld, dO) && ((uintptr_t)dqkv & 15) == 0 && ((uintptr_t)O & 15) == 0;
+}
 inline bool supported_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const void *dqkv) {
-  return supported(qkv, ld, dO) && ((uintptr_t)dqkv & 15) == 0 && ((uintptr_t)O & 15) == 0;
+  return encode_fn() != nullptr && aligned_bwd(qkv, ld, O, dO, dqkv);
 }
 
 }  // namespace fatc

@@ -445,7 +445,9 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// commit of the pair's MMAs, arriving on the barrier at this offset in every CTA of `mask`
+// commit of the pair's MMAs, arriving on the barrier at this offset in every CTA of `mask`.
+// This is an mbarrier arrive inside the 2-CTA cluster of this GPU, not a
+// load: no TMA or bulk copy in this file uses cluster multicast.
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
@@ -722,14 +724,18 @@ inline cudaError_t tc_init() {
   return e;
 }
 
-template <typename T>
-inline bool tc_gemm_supported(const GemmProblem &p) {
-  if (sizeof(T) != 2) return false;
+// Operands the TMA tiles can take: 16-byte aligned bases and row strides.
+inline bool tc_gemm_aligned(const GemmProblem &p) {
   if (p.M < 1 || p.N < 1 || p.K < 1) return false;
   if ((p.lda % 8) || (p.ldb % 8)) return false;
   if (((uintptr_t)p.A & 15) || ((uintptr_t)p.B & 15) || ((uintptr_t)p.D & 15)) return false;
   if (p.epi == EPI_STORE_F32 ? (p.ldd % 4) : (p.ldd % 8)) return false;
-  return tc::encode_fn() != nullptr;
+  return true;
+}
+
+template <typename T>
+inline bool tc_gemm_supported(const GemmProblem &p) {
+  return sizeof(T) == 2 && tc_gemm_aligned(p) && tc::encode_fn() != nullptr;
 }
 
 inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *status, cudaStream_t st);

@@ -9,6 +9,7 @@
 //                O = causal attention; x += O Wo^T;
 //                xn2 = norm(x); a = relu(xn2 W1^T)^2; x += a W2^T
 //   xf = norm(x); z = xf Wout^T; s = 15 tanh(z/15); loss = mean CE(s, target)
+#include <limits.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -191,7 +192,10 @@ template <typename T>
 int gemm(nc_model *m, const GemmProblem &p, cudaStream_t st) {
   if (p.M <= 0 || p.N <= 0) return NC_OK;
   cudaError_t e;
-  const bool tcp = tc_gemm_supported<T>(p);
+  // bf16 runs on the tensor cores only: operands they cannot take are an
+  // error, not a slower path
+  const bool tcp = sizeof(T) == 2;
+  if (tcp && !tc_gemm_aligned(p)) return NC_EALIGN;
   const long ev = prof_begin(m, st);
   if (tcp) e = launch_gemm_tc(p, m->num_sms, m->status, st);
   else e = launch_gemm_simt<T>(p, st);
@@ -241,8 +245,8 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
            (rope_qknorm_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     NC_RUN(K_ATTN_FWD, attn_flops, 0,
-           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->num_sms, 0,
-                                  m->status, st) != cudaSuccess) return NC_ECUDA);
+           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, 0, m->status, st) !=
+               cudaSuccess) return NC_ECUDA);
     NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, w.x, C, EPI_ADD), st));
     NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
            NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
@@ -310,8 +314,8 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
-           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
-                                  m->num_sms, 0, m->status, st) != cudaSuccess) return NC_ECUDA);
+           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H, 0,
+                                  m->status, st) != cudaSuccess) return NC_ECUDA);
     NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
            (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
@@ -356,34 +360,147 @@ int check_step_args(const nc_model *m, const void *weights, const int32_t *token
 }
 
 
-// Fixed device scratch of nc_attention_bwd_noalloc (rowsum(dO * O)), and its
-// device address per device, looked up once with that device current.
-static __device__ __align__(256) float g_attn_bwd_rowdot[NC_ATTN_BWD_NOALLOC_MAX_ROWS];
-constexpr int kMaxDevices = 64;
-static float *g_attn_bwd_rowdot_addr[kMaxDevices] = {};
-static std::mutex g_attn_bwd_rowdot_mutex;
-
-int noalloc_scratch(float **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NC_ECUDA;
-  std::lock_guard<std::mutex> lock(g_attn_bwd_rowdot_mutex);
-  if (!g_attn_bwd_rowdot_addr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_attn_bwd_rowdot) != cudaSuccess || !ptr) return NC_ECUDA;
-    g_attn_bwd_rowdot_addr[dev] = static_cast<float *>(ptr);
+// Wait at most timeout_ms for the work enqueued so far on `st` (polling),
+// then read and clear a device status word.
+int read_status_word(int *word_dev, cudaStream_t st, int timeout_ms) {
+  cudaEvent_t ev;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return NC_ECUDA;
+  if (cudaEventRecord(ev, st) != cudaSuccess) {
+    cudaEventDestroy(ev);
+    return NC_ECUDA;
   }
-  *out = g_attn_bwd_rowdot_addr[dev];
+  const auto t0 = std::chrono::steady_clock::now();
+  cudaError_t q;
+  while ((q = cudaEventQuery(ev)) == cudaErrorNotReady) {
+    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                        std::chrono::steady_clock::now() - t0).count();
+    if (ms >= timeout_ms) {
+      cudaEventDestroy(ev);
+      return NC_ETIMEOUT;
+    }
+    std::this_thread::sleep_for(std::chrono::microseconds(100));
+  }
+  cudaEventDestroy(ev);
+  if (q != cudaSuccess) return NC_ECUDA;
+  int word = 0;
+  if (cudaMemcpyAsync(&word, word_dev, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(word_dev, 0, sizeof(int), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return NC_ECUDA;
+  if (word & kStatusRange) return NC_ERANGE;
+  if (word & kStatusNonFinite) return NC_ENONFINITE;
+  if (word & kStatusTimeout) return NC_ETIMEOUT;
   return NC_OK;
 }
 
-int op_device_sms(int *num_sms) {
+// File-scope device words of the op-level entry points, which have no model
+// handle: the status word their kernels report to (read by nc_ops_status)
+// and the fixed scratch of nc_attention_bwd_noalloc (rowsum(dO * O)).
+static __device__ int g_ops_status;
+static __device__ __align__(256) float g_attn_bwd_rowdot[NC_ATTN_BWD_NOALLOC_MAX_ROWS];
+
+// In host code those names are host-side stand-ins, not device addresses.
+// Their device addresses belong to the CUDA context (a module is loaded per
+// context), so they are looked up with cudaGetSymbolAddress and cached per
+// context, keyed by the context's unique id: a context created after a
+// cudaDeviceReset gets a new id and a fresh lookup, never a stale address.
+struct SymbolAddrs {
+  unsigned long long ctx_id;
+  int *ops_status;
+  float *rowdot;
+};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+static std::mutex g_sym_mutex;
+static std::vector<SymbolAddrs> g_sym_cache;
+
+int context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_cur || !get_id) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+      return NC_ECUDA;
+    get_cur = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return NC_ECUDA;
+  return get_id(ctx, id) == CUDA_SUCCESS ? NC_OK : NC_ECUDA;
+}
+
+// Addresses of the file-scope device words in the current context; the first
+// call in a context looks them up (and makes the runtime's primary context
+// current if there is none yet).
+int symbol_addrs(SymbolAddrs *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
+  unsigned long long id = 0;
+  if (context_id(&id) != NC_OK) {
+    // no current context yet: a runtime call that needs one creates it
+    void *probe = nullptr;
+    if (cudaGetSymbolAddress(&probe, g_ops_status) != cudaSuccess || context_id(&id) != NC_OK) return NC_ECUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_sym_mutex);
+  for (const SymbolAddrs &e : g_sym_cache)
+    if (e.ctx_id == id) {
+      *out = e;
+      return NC_OK;
+    }
+  SymbolAddrs e;
+  e.ctx_id = id;
+  void *p1 = nullptr, *p2 = nullptr;
+  if (cudaGetSymbolAddress(&p1, g_ops_status) != cudaSuccess || !p1 ||
+      cudaGetSymbolAddress(&p2, g_attn_bwd_rowdot) != cudaSuccess || !p2)
+    return NC_ECUDA;
+  e.ops_status = static_cast<int *>(p1);
+  e.rowdot = static_cast<float *>(p2);
+  g_sym_cache.push_back(e);
+  *out = e;
+  return NC_OK;
+}
+
+// Device set-up shared by the op-level entry points: SM count, kernel
+// attributes, and the status word their kernels report to.
+int op_setup(int *num_sms, int **status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
   if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
-  if (tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess ||
+  if (tc_init() != cudaSuccess || fatc::init() != cudaSuccess ||
       cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            65536 * 2) != cudaSuccess) return NC_ECUDA;
+  SymbolAddrs a;
+  if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
+  *status = a.ops_status;
   return NC_OK;
+}
+
+// The attention ops take the row stride as int64 but the kernels index with
+// 32 bits: strides beyond INT_MAX are a shape error, not a silent truncation.
+inline bool attn_shape_ok(int B, int T, int H, int64_t ld) {
+  return B >= 1 && T >= 1 && H >= 1 && ld >= (int64_t)kHeadDim * (H + 2) && ld <= INT32_MAX &&
+         (int64_t)B * T * ld <= ((int64_t)1 << 40);
+}
+
+// A bounded wait on an mbarrier that nothing completes: it runs out after
+// wait_ns and reports kStatusTimeout, the path every kernel wait takes when
+// its partner never arrives.
+__global__ void wait_expiry_kernel(uint64_t wait_ns, int *status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t a = tc::smem_u32(&bar);
+  tc::mbar_init(a, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const uint64_t t0 = tc::globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    if (tc::mbar_try(a, 0)) return;  // never: nothing arrives on the barrier
+    if ((i & 63) == 0 && tc::globaltimer() - t0 > wait_ns) {
+      set_status(status, kStatusTimeout);
+      return;
+    }
+  }
 }
 
 }  // namespace
@@ -442,7 +559,7 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
-  if (!ok || tc_init() != cudaSuccess || fa::attn_mma_init() != cudaSuccess || fatc::init() != cudaSuccess ||
+  if (!ok || tc_init() != cudaSuccess || fatc::init() != cudaSuccess ||
       cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            65536 * 2) != cudaSuccess) {
     nc_destroy(m);
@@ -493,6 +610,8 @@ int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B, int T
   if (rc != NC_OK) return rc;
   if (!logits) return NC_EINVAL;
   if ((uintptr_t)logits & 15) return NC_EALIGN;
+  // bf16 logit rows leave the tensor-core GEMM by TMA: 16-byte row strides
+  if (m->dtype == NC_BF16 && (m->V % 8)) return NC_EALIGN;
   cudaStream_t st = (cudaStream_t)stream;
   if (m->dtype == NC_F32) return fwd_impl<float>(m, weights, tokens, B, T, workspace, logits, st);
   return fwd_impl<bf16>(m, weights, tokens, B, T, workspace, logits, st);
@@ -500,35 +619,7 @@ int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B, int T
 
 int nc_sync_status(nc_model *m, void *stream, int timeout_ms) {
   if (!m) return NC_EINVAL;
-  cudaStream_t st = (cudaStream_t)stream;
-  cudaEvent_t ev;
-  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return NC_ECUDA;
-  if (cudaEventRecord(ev, st) != cudaSuccess) {
-    cudaEventDestroy(ev);
-    return NC_ECUDA;
-  }
-  const auto t0 = std::chrono::steady_clock::now();
-  cudaError_t q;
-  while ((q = cudaEventQuery(ev)) == cudaErrorNotReady) {
-    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
-                        std::chrono::steady_clock::now() - t0).count();
-    if (ms >= timeout_ms) {
-      cudaEventDestroy(ev);
-      return NC_ETIMEOUT;
-    }
-    std::this_thread::sleep_for(std::chrono::microseconds(100));
-  }
-  cudaEventDestroy(ev);
-  if (q != cudaSuccess) return NC_ECUDA;
-  int word = 0;
-  if (cudaMemcpyAsync(&word, m->status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaMemsetAsync(m->status, 0, sizeof(int), st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return NC_ECUDA;
-  if (word & kStatusRange) return NC_ERANGE;
-  if (word & kStatusNonFinite) return NC_ENONFINITE;
-  if (word & kStatusTimeout) return NC_ETIMEOUT;
-  return NC_OK;
+  return read_status_word(m->status, (cudaStream_t)stream, timeout_ms);
 }
 
 int nc_profile(nc_model *m, int enable) {
@@ -569,33 +660,6 @@ int nc_profile_read(nc_model *m, nc_kernel_stat *out, int max, int *count) {
   return rc;
 }
 
-int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,
-                             const float *lse, void *dqkv, int B, int T, int H, int dtype,
-                             int engine, void *stream) {
-  if (!qkv || !O || !dO || !lse || !dqkv) return NC_EINVAL;
-  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
-  if ((int64_t)B * H * T > NC_ATTN_BWD_NOALLOC_MAX_ROWS) return NC_ENOMEM;
-  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
-  float *Drow = nullptr;
-  int rc = noalloc_scratch(&Drow);
-  if (rc != NC_OK) return rc;
-  int num_sms = 0;
-  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
-  cudaStream_t st = (cudaStream_t)stream;
-  const int M = B * T;
-  cudaError_t e;
-  (void)M;
-  if (dtype == NC_BF16) {
-    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
-                              (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
-  } else {
-    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
-                               (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
-  }
-  if (e == cudaSuccess) e = cudaGetLastError();
-  return e == cudaSuccess ? NC_OK : NC_ECUDA;
-}
-
 const char *nc_strerror(int code) {
   switch (code) {
     case NC_OK: return "ok";
@@ -628,35 +692,50 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
   if (M < 1 || N < 1 || K < 1) return NC_ESHAPE;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
   if (epilogue < NC_EPI_STORE || epilogue > NC_EPI_SOFTCAP || (a_mn | b_mn) & ~1) return NC_EINVAL;
-  int num_sms = 0;
-  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  if (engine < 0 || engine > 2) return NC_EINVAL;
   const GemmProblem p = gp(M, N, K, A, lda, a_mn, B, ldb, b_mn, D, ldd, epilogue);
+  const bool tensor = dtype == NC_BF16 && engine != 1;
+  if (tensor && !tc_gemm_aligned(p)) return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (dtype == NC_BF16) {
-    if ((engine == 0 || engine == 2) && tc_gemm_supported<bf16>(p))
-      e = launch_gemm_tc(p, num_sms, nullptr, st, engine == 0 ? 1 : 0);
-    else e = launch_gemm_simt<bf16>(p, st);
-  } else {
-    e = launch_gemm_simt<float>(p, st);
-  }
+  if (tensor) e = launch_gemm_tc(p, num_sms, status, st, engine == 0 ? 1 : 0);
+  else if (dtype == NC_BF16) e = launch_gemm_simt<bf16>(p, st);
+  else e = launch_gemm_simt<float>(p, st);
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
                      int dtype, int engine, void *stream) {
   if (!qkv || !O || !lse) return NC_EINVAL;
-  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
-  int num_sms = 0;
-  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
+  if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (engine < 0 || engine > 1) return NC_EINVAL;
+  if (dtype == NC_BF16 && engine == 0 && !fatc::aligned(qkv, ld, O)) return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == NC_BF16)
-    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, num_sms, engine, nullptr, st);
-  else if (dtype == NC_F32)
-    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, num_sms, engine, nullptr, st);
+    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, engine, status, st);
   else
-    return NC_EUNSUPPORTED;
+    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, engine, status, st);
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+static int attention_bwd_common(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
+                                float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                                int *status, cudaStream_t st) {
+  cudaError_t e;
+  if (dtype == NC_BF16) {
+    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
+                              (bf16 *)dqkv, B, T, H, engine, status, st);
+  } else {
+    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
+                               (float *)dqkv, B, T, H, engine, status, st);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
@@ -664,24 +743,45 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
                      float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
                      void *stream) {
   if (!qkv || !O || !dO || !lse || !Drow || !dqkv) return NC_EINVAL;
-  if (B < 1 || T < 1 || H < 1 || ld < (int64_t)kHeadDim * (H + 2)) return NC_ESHAPE;
-  int num_sms = 0;
-  if (op_device_sms(&num_sms) != NC_OK) return NC_ECUDA;
-  cudaStream_t st = (cudaStream_t)stream;
-  const int M = B * T;
-  cudaError_t e;
-  (void)M;
-  if (dtype == NC_BF16) {
-    e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
-                              (bf16 *)dqkv, B, T, H, num_sms, engine, nullptr, st);
-  } else if (dtype == NC_F32) {
-    e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
-                               (float *)dqkv, B, T, H, num_sms, engine, nullptr, st);
-  } else {
-    return NC_EUNSUPPORTED;
-  }
-  if (e == cudaSuccess) e = cudaGetLastError();
-  return e == cudaSuccess ? NC_OK : NC_ECUDA;
+  if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (engine < 0 || engine > 1) return NC_EINVAL;
+  if (dtype == NC_BF16 && engine == 0 && !fatc::aligned_bwd(qkv, ld, O, dO, dqkv)) return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
+  return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, status,
+                              (cudaStream_t)stream);
+}
+
+int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,
+                             const float *lse, void *dqkv, int B, int T, int H, int dtype,
+                             int engine, void *stream) {
+  if (!qkv || !O || !dO || !lse || !dqkv) return NC_EINVAL;
+  if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if ((int64_t)B * H * T > NC_ATTN_BWD_NOALLOC_MAX_ROWS) return NC_ENOMEM;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (engine < 0 || engine > 1) return NC_EINVAL;
+  if (dtype == NC_BF16 && engine == 0 && !fatc::aligned_bwd(qkv, ld, O, dO, dqkv)) return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
+  SymbolAddrs a;
+  if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
+  return attention_bwd_common(qkv, ld, O, dO, lse, a.rowdot, dqkv, B, T, H, dtype, engine, status,
+                              (cudaStream_t)stream);
+}
+
+int nc_ops_status(void *stream, int timeout_ms) {
+  SymbolAddrs a;
+  if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
+  return read_status_word(a.ops_status, (cudaStream_t)stream, timeout_ms);
+}
+
+int nc_check_wait_expiry(int wait_us, void *stream) {
+  if (wait_us < 0 || wait_us > 1000000) return NC_EINVAL;
+  SymbolAddrs a;
+  if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
+  wait_expiry_kernel<<<1, 1, 0, (cudaStream_t)stream>>>((uint64_t)wait_us * 1000ull, a.ops_status);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 }  // extern "C"

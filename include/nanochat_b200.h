@@ -120,7 +120,9 @@ int nc_fwd_bwd(nc_model *m, const void *weights, const int32_t *tokens,
                void *stream);
 
 /* Forward only: softcapped logits s = 15 tanh(z/15) of every position.
- *   logits  device [B,T,vocab] in the model dtype (row-major, vocab fastest)
+ *   logits  device [B,T,vocab] in the model dtype (row-major, vocab fastest),
+ *           16-byte aligned; a bf16 model needs vocab % 8 == 0 here (its
+ *           rows are stored by TMA), else NC_EALIGN
  * Other arguments as nc_fwd_bwd. */
 int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B,
            int T, void *workspace, size_t ws_bytes, void *logits, void *stream);

@@ -43,28 +43,34 @@ enum {
  *   B(n,k) = B[n*ldb + k] if b_mn == 0 else B[k*ldb + n]
  *   D[m,n] = D[m*ldd + n]
  * dtype (nc_dtype) is the type of A, B and of D unless NC_EPI_STORE_F32.
- * engine: 0 = the path nc_fwd_bwd takes (tcgen05 tensor cores for bf16
- * operands whose strides are multiples of 8 elements and pointers 16-byte
- * aligned -- pairs of CTAs on 256 x 256 tiles when M >= 256, one CTA per
- * 128 x 256 tile otherwise -- CUDA cores for the rest), 1 = force the
- * CUDA-core kernel, 2 = tcgen05 with one CTA per tile.
- * M, N, K >= 1. */
+ * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores, pairs of
+ * CTAs on 256 x 256 tiles when M >= 256, one CTA per 128 x 256 tile
+ * otherwise; fp32: CUDA cores), 1 = the CUDA-core kernel (a test engine for
+ * either dtype), 2 = tcgen05 with one CTA per tile.  The tensor-core engines
+ * need 16-byte aligned pointers and strides that are multiples of 8 elements
+ * (4 for an fp32 D): anything else returns NC_EALIGN before any work is
+ * enqueued -- there is no silent slower path.
+ * M, N, K >= 1.  Kernel-side problems (a wait that ran out of time) are
+ * reported through nc_ops_status. */
 int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, int b_mn, void *D,
             int64_t ldd, int M, int N, int K, int dtype, int epilogue, int engine, void *stream);
 
 /* Causal multi-query attention forward (energyai.berlin page, "Multi-Query
  * Attention (MQA)": one key/value head shared by the H query heads).
- *   qkv  device [B*T, ld] rows [q (H*128) | k (128) | v (128)], ld >= 128*(H+2)
+ *   qkv  device [B*T, ld] rows [q (H*128) | k (128) | v (128)],
+ *        128*(H+2) <= ld <= INT_MAX, else NC_ESHAPE
  *   O    device [B*T, H*128]: O_h = softmax(q_h k^T / sqrt(128) + causal) v
  *   lse  device fp32 [B, H, T]: log-sum-exp of each score row
- * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores), 1 = the
- * CUDA-core kernel, 2 = the warp-level MMA kernels (bf16; else as 1). */
+ * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores, which
+ * need 16-byte aligned qkv and O and ld % 8 == 0, else NC_EALIGN; fp32: CUDA
+ * cores), 1 = the CUDA-core kernel (a test engine for either dtype). */
 int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
                      int dtype, int engine, void *stream);
 
 /* Its backward.  dO [B*T, H*128] and O as above, lse from the forward.
  *   Drow  device fp32 [B, H, T] scratch, receives rowsum(dO * O)
- *   dqkv  device [B*T, ld]: dq per head; dk, dv summed over the query heads */
+ *   dqkv  device [B*T, ld]: dq per head; dk, dv summed over the query heads
+ * Engines and errors as nc_attention_fwd (dO and dqkv 16-byte aligned too). */
 int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
                      float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
                      void *stream);
@@ -87,19 +93,40 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
  * What it does instead: the scratch is a file-scope device array of
  * NC_ATTN_BWD_NOALLOC_MAX_ROWS floats inside the library, so every GPU that
  * loads the library holds those 4 MiB until the process exits.  The first
- * call on a device looks the array's device address up (cudaGetSymbolAddress,
- * with that device current) and caches it; make that first call before any
- * stream capture.  The call itself allocates nothing.
+ * call in a CUDA context looks the array's device address up
+ * (cudaGetSymbolAddress, with that context current) and caches it under the
+ * context's unique id; make that first call before any stream capture.  A
+ * context created later (after cudaDeviceReset, say) has a new id and gets a
+ * fresh lookup on its first call.  The call itself allocates nothing.
  *
  * Limits and sharing: B*H*T > NC_ATTN_BWD_NOALLOC_MAX_ROWS returns NC_ENOMEM
- * before anything is enqueued.  Every call on a device uses the same array and
- * leaves its contents behind; each call overwrites every entry it reads, so no
- * clearing is needed between calls, but two calls that overlap on the GPU
- * (different streams, or different host threads) race on the array and give
- * wrong results: serialise them. */
+ * before anything is enqueued.  Every call in a context uses the same array
+ * and leaves its contents behind; each call overwrites every entry it reads,
+ * so no clearing is needed between calls, but two calls that overlap on the
+ * GPU (different streams, or different host threads) race on the array and
+ * give wrong results: serialise them.  Kernel-side problems are reported
+ * through nc_ops_status, like the other op-level calls. */
 int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,
                              const float *lse, void *dqkv, int B, int T, int H, int dtype,
                              int engine, void *stream);
+
+/* Status of the op-level calls above (nc_gemm, nc_attention_*, and the
+ * calls below), which have no model handle: waits at most timeout_ms for the
+ * work enqueued so far on `stream` (polling), then reads and clears the
+ * library's op status word of the current CUDA context.  Returns
+ * NC_ETIMEOUT if the stream is still busy or a kernel wait ran out of time
+ * (its output is then not valid), else NC_OK.  The word is one per context,
+ * shared by every stream: read it after the calls whose outcome you need. */
+int nc_ops_status(void *stream, int timeout_ms);
+
+/* Self-check of the wait-expiry path: enqueues one thread that waits on a
+ * barrier nothing completes, gives up after wait_us microseconds
+ * (0 <= wait_us <= 1,000,000, else NC_EINVAL) and records a timeout in the op
+ * status word, exactly as a kernel whose partner never arrives does.  The
+ * next nc_ops_status then returns NC_ETIMEOUT.  No passage of the nanochat
+ * pages corresponds to it; it lets a caller check that expired waits reach
+ * the host without faulting or hanging the GPU. */
+int nc_check_wait_expiry(int wait_us, void *stream);
 
 #ifdef __cplusplus
 }

@@ -76,3 +76,41 @@ def test_init_without_a_b200_fails_cleanly(lib):
         pytest.skip("a GPU is present")
     rc, h = nc.nc_init(4, 65536, 256, nc.NC_F32)
     assert rc in (nc.NC_ECUDA, nc.NC_EUNSUPPORTED) and h is None
+
+
+def test_op_entry_points_reject_bad_arguments_on_the_host(lib):
+    # every check below returns before any device work or CUDA call
+    BF16 = nc.NC_BF16
+    H, B, T = 2, 1, 64
+    ld = 128 * (H + 2)
+    # strides beyond INT_MAX are a shape error, not a silent 32-bit truncation
+    big = (1 << 31) + 8
+    assert nc.nc_attention_fwd(16, big, 16, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE
+    assert nc.nc_attention_bwd(16, big, 16, 16, 16, 16, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE
+    assert nc.nc_attention_bwd_noalloc(16, big, 16, 16, 16, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE
+    assert nc.nc_attention_fwd(16, ld - 8, 16, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE
+    # the tensor-core engines take 16-byte aligned operands only: no slower fallback
+    assert nc.nc_attention_fwd(24, ld, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
+    assert nc.nc_attention_fwd(16, ld + 4, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
+    assert nc.nc_attention_bwd(16, ld, 16, 24, 16, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
+    assert nc.nc_attention_bwd_noalloc(16, ld, 16, 16, 16, 40, B, T, H, BF16, 0, None) == nc.NC_EALIGN
+    # only engines 0 (model path) and 1 (CUDA cores) exist for attention
+    assert nc.nc_attention_fwd(16, ld, 16, 16, B, T, H, BF16, 2, None) == nc.NC_EINVAL
+    assert nc.nc_attention_bwd(16, ld, 16, 16, 16, 16, 16, B, T, H, BF16, 2, None) == nc.NC_EINVAL
+    # GEMM: a bf16 stride that is not a multiple of 8 on a tensor-core engine
+    assert nc.nc_gemm(16, 100, 0, 16, 128, 0, 16, 128, 64, 64, 100, BF16, nc.NC_EPI_STORE, 0,
+                      None) == nc.NC_EALIGN
+    assert nc.nc_gemm(16, 128, 0, 16, 128, 0, 24, 128, 64, 64, 128, BF16, nc.NC_EPI_STORE, 2,
+                      None) == nc.NC_EALIGN
+    assert nc.nc_gemm(16, 128, 0, 16, 128, 0, 16, 128, 64, 64, 128, BF16, nc.NC_EPI_STORE, 3,
+                      None) == nc.NC_EINVAL
+    # the wait-expiry self-check takes 0..1 s only
+    assert nc.nc_check_wait_expiry(-1, None) == nc.NC_EINVAL
+    assert nc.nc_check_wait_expiry(1000001, None) == nc.NC_EINVAL
+
+
+def test_op_status_without_a_gpu_fails_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert nc.nc_ops_status(None, 10) == nc.NC_ECUDA

@@ -158,7 +158,7 @@ ATTN_CASES = [(1, 1, 1), (2, 9, 2), (1, 130, 3), (2, 256, 2), (1, 515, 10)]
 
 @pytest.mark.parametrize("B,T,H", ATTN_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1, 2])
+@pytest.mark.parametrize("engine", [0, 1])
 def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
     import torch
     code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
@@ -186,6 +186,7 @@ def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
     dqkv = torch.zeros(B * T, ld, dtype=qkv_d.dtype, device="cuda")
     assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
                                Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine, st) == 0
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK
     got = dqkv.float().cpu().numpy().astype(np.float64)
     dq_ref = np.empty((B, T, H, 128))
     dk_ref = np.empty((B, T, 128))
@@ -206,3 +207,32 @@ def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
             cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
             assert cos > 0.9995, cos
             assert np.max(np.abs(g - r)) <= 3e-2 * scale
+
+
+def test_expired_wait_reaches_the_host(nc):
+    # a wait that nothing completes runs out after 20 ms and is reported, not hung
+    import torch
+    st = torch.cuda.current_stream().cuda_stream
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK
+    assert nc.nc_check_wait_expiry(20000, st) == nc.NC_OK
+    assert nc.nc_ops_status(st, 60000) == nc.NC_ETIMEOUT
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK  # read once, then cleared
+    # the context is still usable afterwards
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum().item()) == 1024.0
+
+
+def test_misaligned_bf16_operands_are_rejected(nc):
+    import torch
+    st = torch.cuda.current_stream().cuda_stream
+    buf = torch.zeros(1 << 16, dtype=torch.bfloat16, device="cuda")
+    p = buf.data_ptr()
+    H, B, T = 2, 1, 64
+    ld = 128 * (H + 2)
+    assert nc.nc_attention_fwd(p + 2, ld, p, p, B, T, H, nc.NC_BF16, 0, st) == nc.NC_EALIGN
+    assert nc.nc_gemm(p, 100, 0, p, 128, 0, p, 128, 64, 64, 100, nc.NC_BF16, nc.NC_EPI_STORE, 0,
+                      st) == nc.NC_EALIGN
+    # the CUDA-core test engine takes any stride
+    assert nc.nc_gemm(p, 100, 0, p, 128, 0, p + 4096, 128, 64, 64, 100, nc.NC_BF16, nc.NC_EPI_STORE, 1,
+                      st) == nc.NC_OK
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK
