@@ -72,6 +72,7 @@ _SIGS = {
     "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _P]),
     "nc_attention_bwd": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "nc_ops_status": (_I, [_P, _I]),
+    "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
 }
 
@@ -163,6 +164,10 @@ def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream) -> int:
 def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream) -> int:
     return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine,
                                            stream)
+
+
+def nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream) -> int:
+    return load_library().nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream)
 
 
 def nc_ops_status(stream, timeout_ms: int) -> int:

@@ -3,9 +3,18 @@
 //   s = 15 tanh(z / 15)             ("ten modern departures": logit softcap 15,
 //                                     computed in fp32)
 //   loss_i = logsumexp(s_i) - s_i[target_i]
-//   dz = (softmax(s_i) - onehot(target_i)) (1 - (s/15)^2) / M   written over z
-// No fp32 copy of the logits is ever materialised: each row is read once and
-// written once.
+//   dz = (softmax(s_i) - onehot(target_i)) (1 - (s/15)^2) g   written over z
+// with g the gradient scale (1/M for the mean loss).  No fp32 copy of the
+// logits is ever materialised: each row is read once and written once.
+//
+// Precision.  tanh and 1 - tanh^2 are formed to fp32 accuracy from one
+// exponential, E = exp(-2|x|), x = z/15:
+//   u = 1 - |t| = 2E / (1 + E),   t = sign(x)(1 - u),   1 - t^2 = u (2 - u),
+// so 1 - t^2 keeps its relative precision where tanh saturates (a hardware
+// tanh of relative error 2^-11 would leave it none at |z| ~ 45).  The row
+// max comes from the raw logits (tanh is increasing).  The target's term is
+// kept out of the running sum, so 1 - p_target = rest / (rest + e_target)
+// has no cancellation when the target dominates the row.
 #pragma once
 
 #include "common.cuh"
@@ -15,36 +24,75 @@ namespace nc {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-__device__ __forceinline__ float tanh_fast(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ float ex2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// tanh in the precision of the storage type: the hardware approximation
-// (relative error ~2^-11) for bf16 logits, whose storage rounding (2^-9) is
-// larger; the accurate library routine for fp32.
-template <typename T> __device__ __forceinline__ float softcap_tanh(float x);
-template <> __device__ __forceinline__ float softcap_tanh<bf16>(float x) { return tanh_fast(x); }
-template <> __device__ __forceinline__ float softcap_tanh<float>(float x) { return tanhf(x); }
+// t = tanh(z/15) and 1 - t^2 for a bf16 model: E by the MUFU exponential
+// (relative error ~2^-22), 1/(1+E) on the FMA pipe by three Newton steps from
+// the best linear guess on [1, 2] (relative error 1/17, squared by each step).
+__device__ __forceinline__ void softcap_parts_fast(float z, float &t, float &sech2) {
+  const float E = ex2_fast(fabsf(z) * (-2.f * kLog2e / kSoftcap));
+  const float y = 1.f + E;
+  float r = fmaf(-8.f / 17.f, y, 24.f / 17.f);
+  r = fmaf(r, fmaf(-y, r, 1.f), r);
+  r = fmaf(r, fmaf(-y, r, 1.f), r);
+  r = fmaf(r, fmaf(-y, r, 1.f), r);
+  const float u = 2.f * E * r;
+  t = copysignf(1.f - u, z);
+  sech2 = u * (2.f - u);
+}
+
+// Two floats packed into one 32-bit register as fp16 / bf16 (lo in the low half).
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
+  __half2 h;
+  memcpy(&h, &u, 4);
+  return __half22float2(h);
+}
+__device__ __forceinline__ float2 unpack_bf2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// The same for an fp32 model with the library's accurate exponential and a
+// correctly rounded division.
+__device__ __forceinline__ void softcap_parts_precise(float z, float &t, float &sech2) {
+  const float E = expf(fabsf(z) * (-2.f / kSoftcap));
+  const float u = 2.f * E / (1.f + E);
+  t = copysignf(1.f - u, z);
+  sech2 = u * (2.f - u);
+}
+
+template <typename T> __device__ __forceinline__ void softcap_parts(float z, float &t, float &sech2);
+template <> __device__ __forceinline__ void softcap_parts<bf16>(float z, float &t, float &s2) {
+  softcap_parts_fast(z, t, s2);
+}
+template <> __device__ __forceinline__ void softcap_parts<float>(float z, float &t, float &s2) {
+  softcap_parts_precise(z, t, s2);
+}
 template <typename T> __device__ __forceinline__ float exp_t(float x);
 template <> __device__ __forceinline__ float exp_t<bf16>(float x) { return ex2_fast(x * kLog2e); }
 template <> __device__ __forceinline__ float exp_t<float>(float x) { return expf(x); }
 
 // ---------------------------------------------------------------------------
-// bf16 rows of V = 1024 threads * 8 * NVEC values (65,536 for NVEC = 8),
-// persistent: one CTA per SM walks rows b, b + grid, ...  tanh(z/15) is kept
-// per element as fp16 in registers (|t| <= 1, 11-bit mantissa: finer than the
-// bf16 logit it came from).
-// Each row (V bf16 = 128 KB at V = 65,536) arrives in shared memory by TMA
-// bulk copies; as soon as every thread has its slice in registers the copy of
-// the CTA's next row is issued, so the load of row i+1 and the store of dz for
-// row i stream while row i's tanh / exp work runs.
+// bf16 rows of V <= 1024 threads * 8 * NVEC values, V % 8 == 0, persistent:
+// one CTA per SM walks rows b, b + grid, ...  Each row (V bf16 = 128 KB at
+// V = 65,536) arrives in shared memory by TMA bulk copies; as soon as every
+// thread has its slice in registers the copy of the CTA's next row is
+// issued, so the load of row i+1 and the store of dz for row i stream while
+// row i's exponentials run.  Per thread the raw logits, then w = e (1 - t^2)
+// (fp16, w <= 1), are kept packed in registers.
 constexpr int kCeThreads = 1024;
 constexpr int kCeCopy = 32768;  // bytes per bulk copy
 
@@ -68,26 +116,31 @@ __device__ __forceinline__ bool ce_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// One row of `bytes` (a multiple of 16) into shared memory, in copies of at
+// most kCeCopy bytes, completing on `bar`.
 __device__ __forceinline__ void ce_fetch_row(uint32_t dst, const bf16 *src, int bytes, uint32_t bar) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-  for (int o = 0; o < bytes; o += kCeCopy)
+  for (int o = 0; o < bytes; o += kCeCopy) {
+    const int n = bytes - o < kCeCopy ? bytes - o : kCeCopy;
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst + o),
-        "l"(reinterpret_cast<const uint8_t *>(src) + o), "r"(kCeCopy), "r"(bar)
+        "l"(reinterpret_cast<const uint8_t *>(src) + o), "r"(n), "r"(bar)
         : "memory");
+  }
 }
 
 template <int NVEC>
 __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel(
     bf16 *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
-    float *__restrict__ token_loss, int M, int V, float inv_M, int *status) {
+    float *__restrict__ token_loss, int M, int V, float grad_scale, int *status) {
   extern __shared__ __align__(128) uint8_t ce_smem[];
   __shared__ float red[32];
-  __shared__ float s_target;
+  __shared__ float s_target, sech2_target;
   __shared__ __align__(8) uint64_t bar_storage;
   const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&bar_storage));
   const uint32_t buf = static_cast<uint32_t>(__cvta_generic_to_shared(ce_smem));
   const int row_bytes = V * 2;
+  const int n8 = V >> 3;  // 16-byte chunks of a row
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -96,6 +149,7 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
   int row = blockIdx.x;
   if (threadIdx.x == 0 && row < M) ce_fetch_row(buf, z + (size_t)row * ldz, row_bytes, bar);
   uint32_t phase = 0;
+  const float k2 = kSoftcap * kLog2e;
   for (; row < M; row += gridDim.x) {
     const bool ok = ce_wait(bar, phase);
     phase ^= 1;
@@ -109,82 +163,105 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
       tgt = tgt < 0 ? 0 : V - 1;
     }
     if (threadIdx.x == 0) {
-      // the target's softcapped logit, rounded exactly as in the sweep below
-      const float zt = __bfloat162float(reinterpret_cast<const bf16 *>(ce_smem)[tgt]);
-      s_target = kSoftcap * __half2float(__float2half_rn(tanh_fast(zt * (1.f / kSoftcap))));
+      float tt, s2;
+      softcap_parts_fast(__bfloat162float(reinterpret_cast<const bf16 *>(ce_smem)[tgt]), tt, s2);
+      s_target = kSoftcap * tt;
+      sech2_target = s2;
     }
-    __half2 t[NVEC][4];
-    __half2 hmax = __float2half2_rn(-1.f);
+    // raw logits into registers, their max (tanh is increasing)
+    uint32_t pk[NVEC][4];
+    __nv_bfloat162 hmax = __float2bfloat162_rn(-INFINITY);
 #pragma unroll
     for (int k = 0; k < NVEC; ++k) {
-      const uint4 zr = *reinterpret_cast<const uint4 *>(ce_smem + (threadIdx.x + k * kCeThreads) * 16);
-      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&zr);
+      const int c = threadIdx.x + k * kCeThreads;
+      if (c < n8) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(ce_smem + c * 16);
+        pk[k][0] = u.x; pk[k][1] = u.y; pk[k][2] = u.z; pk[k][3] = u.w;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(h[j]);
-        t[k][j] = __floats2half2_rn(tanh_fast(f.x * (1.f / kSoftcap)), tanh_fast(f.y * (1.f / kSoftcap)));
-        hmax = __hmax2(hmax, t[k][j]);
+        for (int j = 0; j < 4; ++j) {
+          __nv_bfloat162 h;
+          memcpy(&h, &pk[k][j], 4);
+          hmax = __hmax2(hmax, h);
+        }
       }
     }
-    const float tmax = fmaxf(__low2float(hmax), __high2float(hmax));
-    __syncthreads();  // the buffer is free: fetch the next row while this one is finished
+    __syncthreads();  // the buffer is free (and s_target visible): fetch the next row
     if (threadIdx.x == 0 && row + (int)gridDim.x < M)
       ce_fetch_row(buf, z + (size_t)(row + gridDim.x) * ldz, row_bytes, bar);
-    const float smax2 = kSoftcap * kLog2e * block_max(tmax, red);
-    // e = exp(s - smax); t is replaced by w = e (1 - t^2), the row's gradient
-    // up to the factor 1 / (sum M), so the write-out needs no second
-    // exponential (two MUFU operations per logit instead of three).  w lies in
-    // [0, 1]; in fp16 it keeps 11 bits where it matters and flushes only
-    // entries far below the bf16 resolution of the row's largest ones.
-    float sum = 0.f;
+    const float zmax = block_max(fmaxf(__low2float(hmax), __high2float(hmax)), red);
+    float tmax, s2max;
+    softcap_parts_fast(zmax, tmax, s2max);
+    const float m2 = k2 * tmax;  // row max of s, log2 domain
+    // e = exp(s - max) summed without the target's term; w = e (1 - t^2)
+    // replaces the logits (the row's gradient up to 1 / sum)
+    float rest = 0.f;
 #pragma unroll
-    for (int k = 0; k < NVEC; ++k)
+    for (int k = 0; k < NVEC; ++k) {
+      const int c = threadIdx.x + k * kCeThreads;
+      if (c < n8) {
+        float e[8], part = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 r = __half22float2(t[k][j]);
-        const float ea = ex2_fast(kSoftcap * kLog2e * r.x - smax2);
-        const float eb = ex2_fast(kSoftcap * kLog2e * r.y - smax2);
-        sum += ea + eb;
-        t[k][j] = __floats2half2_rn(ea * (1.f - r.x * r.x), eb * (1.f - r.y * r.y));
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf2(pk[k][j]);
+          float ta, sa, tb, sb;
+          softcap_parts_fast(f.x, ta, sa);
+          softcap_parts_fast(f.y, tb, sb);
+          e[2 * j] = ex2_fast(fmaf(k2, ta, -m2));
+          e[2 * j + 1] = ex2_fast(fmaf(k2, tb, -m2));
+          part += e[2 * j] + e[2 * j + 1];
+          pk[k][j] = pack_h2(e[2 * j] * sa, e[2 * j + 1] * sb);
+        }
+        if ((unsigned)(tgt - c * 8) < 8u) {  // the target's chunk: its term stays out
+          part = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c * 8 + j != tgt) part += e[j];
+        }
+        rest += part;
       }
-    sum = block_sum(sum, red);  // contains __syncthreads: s_target is visible after it
-    const float lse2 = smax2 + __log2f(sum);  // log-sum-exp in the log2 domain
+    }
+    rest = block_sum(rest, red);  // contains __syncthreads
+    const float e_t = ex2_fast(fmaf(kLog2e, s_target, -m2));
+    const float sum = rest + e_t;
+    const float lse2 = m2 + __log2f(sum);  // log-sum-exp in the log2 domain
     if (threadIdx.x == 0) token_loss[row] = lse2 * kLn2 - s_target;
-    const float scale = inv_M / sum;
+    const float scale = grad_scale / sum;
+    // 1 - p_target = rest / sum: no cancellation when the target dominates
+    const bf16 dz_t = __float2bfloat16_rn(-(rest / sum) * sech2_target * grad_scale);
     bf16 *zrow = z + (size_t)row * ldz;
 #pragma unroll
     for (int k = 0; k < NVEC; ++k) {
-      const int v = threadIdx.x + k * kCeThreads;
-      uint4 u;
-      __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+      const int c = threadIdx.x + k * kCeThreads;
+      if (c < n8) {
+        uint32_t o[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 w = __half22float2(t[k][j]);
-        h[j] = __floats2bfloat162_rn(w.x * scale, w.y * scale);
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_h2(pk[k][j]);
+          o[j] = pack_bf2(f.x * scale, f.y * scale);
+        }
+        if ((unsigned)(tgt - c * 8) < 8u) {
+          const int j = (tgt - c * 8) >> 1;
+          const uint32_t b = __bfloat16_as_ushort(dz_t);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            if (jj == j) o[jj] = (tgt & 1) ? ((o[jj] & 0xffffu) | (b << 16)) : ((o[jj] & 0xffff0000u) | b);
+        }
+        const uint4 u = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(zrow + c * 8) = u;
       }
-      // the one-hot term of the target lives in exactly one thread's vector;
-      // its p and 1 - t^2 come from the target's own softcapped logit
-      if ((unsigned)(tgt - v * 8) < 8u) {
-        const int j = (tgt - v * 8) >> 1;
-        const float rt = s_target * (1.f / kSoftcap);
-        const float pt = ex2_fast(kLog2e * s_target - lse2) - 1.f;
-        const bf16 val = __float2bfloat16_rn(pt * (1.f - rt * rt) * inv_M);
-        if (tgt & 1) h[j].y = val;
-        else h[j].x = val;
-      }
-      *reinterpret_cast<uint4 *>(zrow + v * 8) = u;
     }
     __syncthreads();  // s_target and red are reused by the next row
   }
 }
 
 // ---------------------------------------------------------------------------
-// General version, any V and either dtype: two sweeps over the row (the
-// second is served by L2), online max/sum in the first.
+// General version, any V and either dtype: three sweeps over the row (the
+// second and third are served by L2): the max of the raw logits, the sum of
+// exp(s - max) without the target's term, the write-out.
 template <typename T>
 __global__ void __launch_bounds__(256) ce_fused_generic_kernel(
     T *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
-    float *__restrict__ token_loss, int M, int V, float inv_M, int *status) {
+    float *__restrict__ token_loss, int M, int V, float grad_scale, int *status) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   if (row >= M) return;
@@ -194,27 +271,58 @@ __global__ void __launch_bounds__(256) ce_fused_generic_kernel(
     if (threadIdx.x == 0) set_status(status, kStatusRange);
     tgt = tgt < 0 ? 0 : V - 1;
   }
-  float m = -INFINITY, l = 0.f;
+  float zm = -INFINITY;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) zm = fmaxf(zm, to_f(zr[v]));
+  zm = block_max(zm, red);
+  float tm, s2m, tt, s2t;
+  softcap_parts<T>(zm, tm, s2m);
+  softcap_parts<T>(to_f(zr[tgt]), tt, s2t);
+  const float m = kSoftcap * tm, s_t = kSoftcap * tt;
+  float rest = 0.f;
   for (int v = threadIdx.x; v < V; v += blockDim.x) {
-    const float s = kSoftcap * softcap_tanh<T>(to_f(zr[v]) * (1.f / kSoftcap));
-    if (s > m) {
-      l = l * exp_t<T>(m - s) + 1.f;
-      m = s;
-    } else {
-      l += exp_t<T>(s - m);
-    }
+    float t, s2;
+    softcap_parts<T>(to_f(zr[v]), t, s2);
+    if (v != tgt) rest += exp_t<T>(kSoftcap * t - m);
   }
-  const float gm = block_max(m, red);
-  const float part = (m == -INFINITY) ? 0.f : l * exp_t<T>(m - gm);
-  const float s_t = kSoftcap * softcap_tanh<T>(to_f(zr[tgt]) * (1.f / kSoftcap));
-  const float tot = block_sum(part, red);  // syncs: every read of zr[tgt] precedes the writes
-  const float lse = gm + logf(tot);
+  rest = block_sum(rest, red);  // syncs: every read of zr precedes the writes
+  const float sum = rest + exp_t<T>(s_t - m);
+  const float lse = m + logf(sum);
   if (threadIdx.x == 0) token_loss[row] = lse - s_t;
   for (int v = threadIdx.x; v < V; v += blockDim.x) {
-    const float tt = softcap_tanh<T>(to_f(zr[v]) * (1.f / kSoftcap));
-    const float p = exp_t<T>(kSoftcap * tt - lse) - (v == tgt ? 1.f : 0.f);
-    zr[v] = from_f<T>(p * (1.f - tt * tt) * inv_M);
+    float t, s2;
+    softcap_parts<T>(to_f(zr[v]), t, s2);
+    const float p = v == tgt ? -(rest / sum) : exp_t<T>(kSoftcap * t - lse);
+    zr[v] = from_f<T>(p * s2 * grad_scale);
   }
+}
+
+// Dynamic shared memory of the persistent kernel: one row.
+inline int ce_persistent_smem(int V) { return V * 2; }
+
+// Whether the persistent bf16 kernel takes these rows: V a multiple of 8 up
+// to 65,536, 16-byte aligned rows.
+inline bool ce_persistent_ok(const void *z, int64_t ldz, int V) {
+  return V >= 8 && V <= 65536 && (V % 8) == 0 && (ldz % 8) == 0 && ((uintptr_t)z & 15) == 0;
+}
+
+inline cudaError_t ce_init() {
+  return cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ce_persistent_smem(65536));
+}
+
+// Softcap + CE over M rows of z (dtype T), in place; token losses to
+// token_loss.  The bf16 rows the persistent kernel takes go there.
+template <typename T>
+inline cudaError_t launch_ce(T *z, int64_t ldz, const int32_t *targets, float *token_loss, int M, int V,
+                             float grad_scale, int num_sms, int *status, cudaStream_t st) {
+  if (sizeof(T) == 2 && ce_persistent_ok(z, ldz, V)) {
+    const int grid = M < num_sms ? M : num_sms;
+    ce_fused_bf16_persistent_kernel<8><<<grid, kCeThreads, ce_persistent_smem(V), st>>>(
+        (bf16 *)z, ldz, targets, token_loss, M, V, grad_scale, status);
+  } else {
+    ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(z, ldz, targets, token_loss, M, V, grad_scale, status);
+  }
+  return cudaGetLastError();
 }
 
 // loss = mean of the per-token losses; flags a non-finite result.

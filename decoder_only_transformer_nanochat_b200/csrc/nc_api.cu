@@ -277,16 +277,9 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   NC_TRY(gemm<T>(m, gp(M, V, C, w.xf, C, 0, W.lm_head, C, 0, w.z, w.ldz, EPI_STORE), st));
   float *tl = token_loss ? token_loss : w.tok_loss;
   const float inv_M = 1.f / (float)M;
-  if (sizeof(T) == 2 && V == 65536) {
-    const int grid = M < m->num_sms ? M : m->num_sms;
-    NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
-           (ce_fused_bf16_persistent_kernel<8><<<grid, kCeThreads, V * 2, st>>>(
-               (bf16 *)w.z, w.ldz, targets, tl, M, V, inv_M, m->status)));
-  } else {
-    NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
-           (ce_fused_generic_kernel<T><<<M, 256, 0, st>>>(w.z, w.ldz, targets, tl, M, V, inv_M,
-                                                          m->status)));
-  }
+  NC_RUN(K_CE, 0, M * (2.0 * V * es + 8.0),
+         if (launch_ce<T>(w.z, w.ldz, targets, tl, M, V, inv_M, m->num_sms, m->status, st) != cudaSuccess)
+             return NC_ECUDA);
   NC_RUN(K_LOSS_MEAN, 0, M * 4.0, (loss_mean_kernel<<<1, 1024, 0, st>>>(tl, M, loss, m->status)));
 
   // gradient pointers (fp32, same layout as the weights)
@@ -469,9 +462,7 @@ int op_setup(int *num_sms, int **status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NC_ECUDA;
   if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NC_ECUDA;
-  if (tc_init() != cudaSuccess || fatc::init() != cudaSuccess ||
-      cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           65536 * 2) != cudaSuccess) return NC_ECUDA;
+  if (tc_init() != cudaSuccess || fatc::init() != cudaSuccess || ce_init() != cudaSuccess) return NC_ECUDA;
   SymbolAddrs a;
   if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
   *status = a.ops_status;
@@ -559,9 +550,7 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
-  if (!ok || tc_init() != cudaSuccess || fatc::init() != cudaSuccess ||
-      cudaFuncSetAttribute(ce_fused_bf16_persistent_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           65536 * 2) != cudaSuccess) {
+  if (!ok || tc_init() != cudaSuccess || fatc::init() != cudaSuccess || ce_init() != cudaSuccess) {
     nc_destroy(m);
     return NC_ECUDA;
   }
@@ -768,6 +757,23 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
   if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
   return attention_bwd_common(qkv, ld, O, dO, lse, a.rowdot, dqkv, B, T, H, dtype, engine, status,
                               (cudaStream_t)stream);
+}
+
+int nc_softcap_ce(void *z, int64_t ldz, const int32_t *targets, float *token_loss, int M, int V,
+                  float grad_scale, int dtype, void *stream) {
+  if (!z || !targets || !token_loss) return NC_EINVAL;
+  if (M < 1 || V < 1 || ldz < V) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (((uintptr_t)targets & 3) || ((uintptr_t)token_loss & 3) ||
+      ((uintptr_t)z & (dtype == NC_BF16 ? 1 : 3)))
+    return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = dtype == NC_BF16
+                      ? launch_ce<bf16>((bf16 *)z, ldz, targets, token_loss, M, V, grad_scale, num_sms, status, st)
+                      : launch_ce<float>((float *)z, ldz, targets, token_loss, M, V, grad_scale, num_sms, status, st);
+  return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 int nc_ops_status(void *stream, int timeout_ms) {

@@ -110,6 +110,25 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
                              const float *lse, void *dqkv, int B, int T, int H, int dtype,
                              int engine, void *stream);
 
+/* Logit softcap, log-sum-exp and token cross-entropy, forward and backward
+ * in one pass over each row ("Nanochat: full-stack LLM training in 8,000
+ * lines for $72", section "A Llama-class transformer with ten modern
+ * departures": logits softcapped as 15 tanh(z/15), computed in fp32), in
+ * place:
+ *   z           device [M, ldz] (dtype), row i holds the V logits z_i;
+ *               overwritten by dz_i = (softmax(s_i) - onehot(t_i)) (1 - (s_i/15)^2) g
+ *               with s_i = 15 tanh(z_i / 15); entries past V are untouched
+ *   targets     device int32 [M], ids in [0, V) (others are clamped and
+ *               reported as NC_ERANGE by nc_ops_status)
+ *   token_loss  device fp32 [M]: logsumexp(s_i) - s_i[t_i]
+ *   grad_scale  g (1/M gives the gradient of the mean loss)
+ * tanh and 1 - tanh^2 are formed to fp32 precision for both dtypes.  bf16
+ * rows with V % 8 == 0, V <= 65,536, ldz % 8 == 0 and a 16-byte aligned z
+ * take the persistent kernel the model step uses; other rows a general
+ * kernel.  M, V >= 1, ldz >= V. */
+int nc_softcap_ce(void *z, int64_t ldz, const int32_t *targets, float *token_loss, int M, int V,
+                  float grad_scale, int dtype, void *stream);
+
 /* Status of the op-level calls above (nc_gemm, nc_attention_*, and the
  * calls below), which have no model handle: waits at most timeout_ms for the
  * work enqueued so far on `stream` (polling), then reads and clears the

@@ -39,7 +39,7 @@ import math
 
 import numpy as np
 
-from .model import (HEAD_DIM, _softmax_rows, dims, head_forward_row, head_loss_row,
+from .model import (HEAD_DIM, _softmax_rows, dims, head_backward_row, head_forward_row, head_loss_row,
                     param_layout, rmsnorm, rmsnorm_bwd, rope, rope_bwd, rope_tables)
 
 SHORT_WINDOW = 1024        # p1: short-window layers see 1,024 tokens
@@ -240,10 +240,7 @@ def loss_and_grads(W, tokens, targets, depth, windows=None):
         rows = slice(b * T, (b + 1) * T)
         s = head_forward_row(xf[rows], Wout)
         tl[b], lse = head_loss_row(s, targets[b])
-        ds = np.exp(s - lse[:, None])
-        ds[np.arange(T), targets[b]] -= 1.0
-        ds /= M
-        dz = ds * (1.0 - (s / 15.0) ** 2)
+        dz = head_backward_row(s, lse, targets[b], 1.0 / M)
         dWout += dz.T @ xf[rows]
         dxf[rows] = dz @ Wout
     grads["lm_head"] = dWout

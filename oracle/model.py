@@ -217,6 +217,15 @@ def head_loss_row(s, tgt):
     return lse - s[np.arange(s.shape[0]), tgt], lse
 
 
+def head_backward_row(s, lse, tgt, scale):
+    """d (scale * sum of the rows' losses) / d z for softcapped logits s [T,V]:
+    (softmax(s) - onehot(target)) * (1 - (s/15)^2) * scale, since
+    s = 15 tanh(z/15) has ds/dz = 1 - tanh^2 = 1 - (s/15)^2."""
+    ds = np.exp(s - lse[:, None])
+    ds[np.arange(s.shape[0]), tgt] -= 1.0
+    return ds * (1.0 - (s / SOFTCAP) ** 2) * scale
+
+
 def _embed(W, tokens):
     B, T = tokens.shape
     return W["wte"][tokens.reshape(-1)]
@@ -278,12 +287,8 @@ def loss_and_grads(W, tokens, targets, depth):
         rows = slice(b * T, (b + 1) * T)
         s = head_forward_row(xf[rows], Wout)
         tl[b], lse = head_loss_row(s, targets[b])
-        # d loss / d s = (softmax(s) - onehot(target)) / M
-        ds = np.exp(s - lse[:, None])
-        ds[np.arange(T), targets[b]] -= 1.0
-        ds /= M
-        # s = 15 tanh(z / 15)  =>  ds/dz = 1 - (s / 15)^2
-        dz = ds * (1.0 - (s / SOFTCAP) ** 2)
+        # d loss / d s = (softmax(s) - onehot(target)) / M;  ds/dz = 1 - (s / 15)^2
+        dz = head_backward_row(s, lse, targets[b], 1.0 / M)
         dWout += dz.T @ xf[rows]
         dxf[rows] = dz @ Wout
     grads["lm_head"] = dWout

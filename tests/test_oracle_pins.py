@@ -347,3 +347,36 @@ def test_bf16_rounding_nearest_even():
     got = synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(x))
     np.testing.assert_array_equal(got, [1.0, 1.0, 1 + 2 ** -7, -2.5, 65536.0, float(np.float32(1e-40)) and got[5]])
     assert got[1] == 1.0  # tie goes to even
+
+
+def test_head_backward_row_matches_finite_differences_at_saturation():
+    # d(scale * sum of token losses)/dz by central differences of the loss
+    # itself, on rows whose logits reach deep into tanh saturation (|z| up to
+    # 60), with the target at the row's argmax, at id 0 and at the last id
+    rng = np.random.default_rng(5)
+    V = 37
+    z = rng.normal(0.0, 20.0, size=(4, V))
+    z[1] = rng.uniform(30.0, 60.0, size=V) * rng.choice([-1.0, 1.0], size=V)
+    z[2, 7] = 55.0
+    tgt = np.array([0, V - 1, 7, 3])
+    scale = 0.25
+
+    def loss(zz):
+        s = oracle.head_forward_row(zz, np.eye(V))  # z W^T with W = I
+        return scale * oracle.head_loss_row(s, tgt)[0].sum()
+
+    s = oracle.head_forward_row(z, np.eye(V))
+    _, lse = oracle.head_loss_row(s, tgt)
+    g = oracle.head_backward_row(s, lse, tgt, scale)
+    h = 1e-5
+    fd = np.empty_like(z)
+    for i in range(z.shape[0]):
+        for j in range(V):
+            zp, zm = z.copy(), z.copy()
+            zp[i, j] += h
+            zm[i, j] -= h
+            fd[i, j] = (loss(zp) - loss(zm)) / (2 * h)
+    # central differences of a loss of size ~10 at h = 1e-5: rounding noise ~1e-10
+    np.testing.assert_allclose(g, fd, rtol=1e-6, atol=5e-10)
+    # at saturation the softcap derivative is tiny but not zero
+    assert 0 < np.abs(g[1]).max() < 1e-2
