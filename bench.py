@@ -1,11 +1,17 @@
 #!/usr/bin/env python
 """Training-step throughput of the nanochat decoder (forward + backward: loss
-and every weight gradient) through the C ABI, on the d20 workload:
+and every weight gradient) through the C ABI.  Default workload d20:
 depth 20 (C=1280, 10 query heads of 128 + 1 shared KV head, MLP 5120),
 vocab 65,536, B=16 rows of T=2048 Zipf(1.1) tokens per GPU, bf16 storage with
-fp32 accumulation, random-init weights of that architecture.
+fp32 accumulation, random-init weights of that architecture.  --config picks
+one of the five workloads (d4 fp32, d12, d20, d24, d32).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config d20]
+
+The timed steps run with the library's per-launch accounting off; a second,
+separate pass of the same steps with it on gives the per-kernel times, rates
+and the roofline of the dominant kernel.
 
 N > 1 runs one process per GPU under torch.distributed.run; each rank runs its
 own shard of B rows (data parallel, weak scaling) and the timing is the
@@ -29,7 +35,24 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "train tokens/sec (fwd+bwd) at d20 on 1 B200; MFU vs bf16 dense peak"
-WORKLOAD = "d20"
+DEFAULT_WORKLOAD = "d20"
+
+
+def metric_for(name: str) -> str:
+    return METRIC if name == DEFAULT_WORKLOAD else METRIC.replace("at d20", f"at {name}")
+
+
+def host_cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 # algorithmic flops per token: 6 N_mm + 6 T C L (causal attention), N_mm = every
 # matmul weight including the unembedding (the embedding gather has no flops)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -210,7 +233,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.config]
     lay = oracle.param_layout(wl.depth, wl.vocab)
     _, W64 = synth.make_weights(lay, wl.seed, wl.dtype)
     T_sample = 128
@@ -224,12 +247,13 @@ def run_reference(args):
     value = T_sample / (ms / 1000.0)
     D = oracle.dims(wl.depth, wl.vocab)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": metric_for(wl.name), "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(wl, args.gpus, sample=f"B=1, T={T_sample}"),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one row of {T_sample} Zipf tokens through the full d20 model per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu": host_cpu_model(),
+                         "kind": "oracle",
+                         "sample": f"one row of {T_sample} tokens through the full {wl.name} model per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "model_flops_per_token": model_flops_per_token(wl.depth, D["C"], wl.vocab, T_sample),
     }
@@ -265,11 +289,14 @@ def run_ours(args):
     import decoder_only_transformer_nanochat_b200 as nc
     from decoder_only_transformer_nanochat_b200 import Model
 
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.config]
     model = Model(wl.depth, vocab=wl.vocab, seq=wl.seq, dtype=wl.dtype)
     lay = [(n, r, c) for n, _, r, c in model.layout]
     flat, W64 = synth.make_weights(lay, wl.seed, wl.dtype)
-    weights = torch.from_numpy(flat.view(np.int16)).cuda().view(torch.bfloat16)
+    if wl.dtype == "bf16":
+        weights = torch.from_numpy(flat.view(np.int16)).cuda().view(torch.bfloat16)
+    else:
+        weights = torch.from_numpy(flat).cuda()
     del flat
     if not (rank == 0 and world == 1 and not args.no_cpu_baseline):
         W64 = None
@@ -291,11 +318,11 @@ def run_ours(args):
         raise RuntimeError(f"device status after warm-up: {nc.nc_strerror(rc)}")
     nc.nc_profile_read(model.handle)  # drop warm-up accounting
 
-    # ---------------- device-timed region ----------------
+    # ---------------- device-timed region (no per-launch accounting) ----------------
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     sampler = ClockSampler(gpu_index)
-    nc.nc_profile(model.handle, 1)
+    nc.nc_profile(model.handle, 0)
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
@@ -308,15 +335,26 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
-    nc.nc_profile(model.handle, 0)
     ms_local = t_start.elapsed_time(t_end) / args.steps
-    rc, stats = nc.nc_profile_read(model.handle)
     status = model.sync_status(60000)
     if status != 0:
         raise RuntimeError(f"device status after the timed steps: {nc.nc_strerror(status)}")
+    nc.nc_profile_read(model.handle)  # launch counts of the timed steps: not used
     ms = reduce_max(ms_local, world)
     tokens_per_step = wl.B * wl.T
     value = job_rate(tokens_per_step, ms, world)
+
+    # ---------------- accounting pass: the same steps, every launch between two events ----------------
+    nc.nc_profile(model.handle, 1)
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    nc.nc_profile(model.handle, 0)
+    rc, stats = nc.nc_profile_read(model.handle)
+    status = model.sync_status(60000)
+    if status != 0:
+        raise RuntimeError(f"device status after the accounting steps: {nc.nc_strerror(status)}")
 
     # ---------------- end to end: host buffers through the public API ----------------
     tok_h = torch.from_numpy(tok).pin_memory()
@@ -393,12 +431,12 @@ def run_ours(args):
     fpt = model_flops_per_token(wl.depth, D["width"], wl.vocab, wl.T)
     fpt_nc = model_flops_per_token_noncausal(wl.depth, D["width"], wl.vocab, wl.T)
     model_tflops = value * fpt / 1e12
-    launches = sum(s["launches"] for s in stats)
+    launches = sum(s["launches"] for s in stats)  # the accounting pass ran the same steps
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": metric_for(wl.name), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded Zipf tokens, random-init weights)",
         "config": config_dict(wl, world),
         "mfu": model_tflops / (world * peaks["bf16_tflops"]),
@@ -413,14 +451,16 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(tok.nbytes + tgt.nbytes), "d2h_bytes_per_step": 4},
         "gpu_launches": launches,
+        "kernels_timing": "separate pass of the same steps with per-launch events (the timed steps run without them)",
         "clocks": clocks,
         "loss": loss_val,
     }
     if world == 1 and not args.no_cpu_baseline and W64 is not None:
         T_sample = 128
         tps, dt, cores = cpu_oracle_sample(W64, wl.depth, wl.vocab, T_sample, wl.seed + 7)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"one row of {T_sample} Zipf tokens through the full d20 "
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "cpu": host_cpu_model(),
+                                "kind": "oracle",
+                                "sample": f"one row of {T_sample} tokens through the full {wl.name} "
                                           f"model ({dt:.1f} s)"}
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -436,6 +476,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default=DEFAULT_WORKLOAD, choices=["d4", "d12", "d20", "d24", "d32"])
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -2,10 +2,22 @@
 on seeded inputs and compare it with the fp64 oracle on the same inputs."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 
 import oracle
 import synth
+
+
+def record(kind: str, **fields):
+    """Append one line of measured errors to the file named by NC_PARITY_LOG
+    (if set), for deriving and reviewing tolerances."""
+    path = os.environ.get("NC_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"kind": kind, **fields}) + "\n")
 
 # tolerances of the two precisions
 F32_LOSS_REL = 1e-5          # |dloss| / |loss|
@@ -55,10 +67,19 @@ def cosine(a, b):
     return float(np.sum(a * b) / (na * nb))
 
 
-def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_ref=None):
+def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_ref=None, tag=""):
     """Assert the precision's tolerances; return a per-tensor report."""
     g_gpu = split_grads(g_gpu_flat, lay)
     report = {}
+    fields = {"tag": tag, "dtype": dtype, "dloss": float(loss_gpu - loss_ref)}
+    if tl_gpu is not None:
+        d = np.abs(tl_gpu - tl_ref)
+        fields.update(tl_max=float(d.max()), tl_mean=float(d.mean()),
+                      tl_ref_absmax=float(np.abs(tl_ref).max()))
+    cos = {name: cosine(g_gpu[name], g_ref[name]) for name, _, _ in lay}
+    worst = min(cos, key=cos.get)
+    fields.update(min_cos=cos[worst], min_cos_tensor=worst)
+    record("step", **fields)
     if dtype == "f32":
         assert abs(loss_gpu - loss_ref) <= F32_LOSS_REL * abs(loss_ref), (loss_gpu, loss_ref)
         for name, _, _ in lay:

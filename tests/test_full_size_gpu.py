@@ -9,9 +9,9 @@ oracle where it can follow:
     parameterless norms create (<dWq_h, Wq_h> = <dWk, Wk> = 0,
     <dwte_v, wte_v> = 0), zero rows for tokens that never occur, finiteness;
   * oracle-sized step: loss and every gradient against the oracle on the
-    full d12 workload and on one-row slices of d20 (T=2048), d24 (T=1024)
-    and d32 (T=512), with the bf16 tolerances |dloss| <= 1e-2 and per-tensor
-    cosine >= 0.999.
+    full d12 workload and on one-row slices (B=1 at the workload's T=2048)
+    of d20, d24 and d32, with the bf16 tolerances |dloss| <= 1e-2 and
+    per-tensor cosine >= 0.999.
 """
 import numpy as np
 import pytest
@@ -55,6 +55,8 @@ def test_full_size_step(torch_cuda, name):
     b = wl.B - 1
     _, tl_ref = oracle.forward_loss(W, tok[b:b + 1], tgt[b:b + 1], wl.depth)
     d = np.abs(tl[b] - tl_ref[0])
+    from tests._gpu_helpers import record
+    record("full_size_row", tag=name, tl_max=float(d.max()), tl_mean=float(d.mean()))
     assert d.mean() <= 1e-2 and d.max() <= 0.1, (d.mean(), d.max())
 
     G = split_grads(g, lay)
@@ -75,7 +77,7 @@ def test_full_size_step(torch_cuda, name):
     assert unused.size > 0 and np.all(G["wte"][unused] == 0.0)
 
 
-SLICES = [("d12", 8, 1024), ("d20", 1, 2048), ("d24", 1, 1024), ("d32", 1, 512)]
+SLICES = [("d12", 8, 1024), ("d20", 1, 2048), ("d24", 1, 2048), ("d32", 1, 2048)]
 
 
 @pytest.mark.parametrize("name,B,T", SLICES)
@@ -90,4 +92,4 @@ def test_oracle_sized_step(torch_cuda, name, B, T):
     del model
     assert rc == 0
     loss_ref, tl_ref, g_ref = oracle.loss_and_grads(W, tok, tgt, wl.depth)
-    compare(wl.dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref)
+    compare(wl.dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref, tag=f"{name}-B{B}-T{T}")

@@ -59,7 +59,7 @@ def test_step_matches_oracle(torch_cuda, depth, V, B, T, dtype, seed, dist, hstd
     rc, loss, tl, g = gpu_step(model, flat, tok, tgt, dtype)
     assert rc == 0
     loss_ref, tl_ref, g_ref = oracle.loss_and_grads(W, tok, tgt, depth)
-    compare(dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref)
+    compare(dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref, tag=f"d{depth}-V{V}-B{B}-T{T}-{dtype}")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
