@@ -26,17 +26,20 @@
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "token_sort.cuh"
 
 using namespace nc;
 
 // kernel classes of the per-launch accounting
 enum KernelClass {
   K_GEMM_TC, K_GEMM_SIMT, K_ATTN_FWD, K_ATTN_BWD, K_EMBED, K_RMSNORM, K_ROPE_QKNORM, K_CE,
-  K_LOSS_MEAN, K_RMSNORM_BWD, K_ROWDOT, K_ROPE_QKNORM_BWD, K_EMBED_BWD, K_NUM_CLASSES
+  K_LOSS_MEAN, K_RMSNORM_BWD, K_ROWDOT, K_ROPE_QKNORM_BWD, K_EMBED_BWD, K_TOKEN_SORT, K_SEG_FIXUP,
+  K_NUM_CLASSES
 };
 static const char *kClassName[K_NUM_CLASSES] = {
     "gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd", "embed_norm", "rmsnorm", "rope_qknorm",
-    "ce_fused", "loss_mean", "rmsnorm_bwd", "attn_rowdot", "rope_qknorm_bwd", "embed_bwd"};
+    "ce_fused", "loss_mean", "rmsnorm_bwd", "attn_rowdot", "rope_qknorm_bwd", "embed_bwd",
+    "token_sort", "seg_fixup"};
 
 struct nc_model {
   int depth, C, H, F, V, seq, dtype;
@@ -69,6 +72,9 @@ struct Work {
   T *x, *xf, *z, *dxb, *dO, *dqkv, *dy;
   float *r0, *rf, *tok_loss, *dx, *Drow;
   int64_t ldz;
+  TokenSort sort;                   // positions grouped by token (embedding gradient)
+  float *seg_head, *seg_tail;       // [chunks, C] partial sums of segments cut by chunks
+  int *seg_flags;                   // [chunks]
 };
 
 // Lay the workspace out (base == nullptr only measures it).
@@ -117,6 +123,17 @@ size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
   T *dO = (T *)take(M * C * es);
   T *dqkv = (T *)take(M * ldqkv * es);
   float *Drow = (float *)take(M * H * 4);
+  int32_t *sk0 = (int32_t *)take(M * 4), *sk1 = (int32_t *)take(M * 4);
+  int32_t *sv0 = (int32_t *)take(M * 4), *sv1 = (int32_t *)take(M * 4);
+  int *hist = (int *)take((size_t)256 * sort_tiles((int)M) * 4);
+  const size_t nch = (size_t)seg_chunks((int)M);
+  float *seg_head = (float *)take(nch * C * 4), *seg_tail = (float *)take(nch * C * 4);
+  int *seg_flags = (int *)take(nch * 4);
+  if (w) {
+    w->sort.keys[0] = sk0; w->sort.keys[1] = sk1; w->sort.vals[0] = sv0; w->sort.vals[1] = sv1;
+    w->sort.hist = hist; w->sort.skey = nullptr; w->sort.spos = nullptr;
+    w->seg_head = seg_head; w->seg_tail = seg_tail; w->seg_flags = seg_flags;
+  }
   if (w) {
     w->x = x; w->r0 = r0; w->xf = xf; w->rf = rf; w->z = z; w->ldz = ldz;
     w->tok_loss = tok_loss; w->dx = dx; w->dxb = dxb; w->dy = dy; w->dO = dO;
@@ -319,11 +336,17 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
            NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
                                  w.dy, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
   }
-  // embedding: through the first norm, summed into the selected rows
+  // embedding: through the first norm, summed per token over its positions
+  // in a fixed order (positions sorted by token; no floating-point atomics)
   if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
-  NC_RUN(K_EMBED_BWD, 0, M * (8.0 * C + C * es + 8.0),
-         NC_DISPATCH_NV(C, (embed_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                               w.dx, tokens, W.wte, w.r0, G(0), M, C, V))));
+  NC_RUN(K_TOKEN_SORT, 0, M * 16.0 * sort_passes(V), sort_tokens(tokens, M, V, w.sort, st));
+  const int nch = seg_chunks(M);
+  NC_RUN(K_EMBED_BWD, 0, M * (4.0 * C + C * es + 12.0),
+         NC_DISPATCH_NV(C, (embed_segsum_kernel<T, NV><<<(nch + 7) / 8, 256, 0, st>>>(
+                               w.dx, W.wte, w.r0, w.sort.skey, w.sort.spos, M, C, G(0), w.seg_head, w.seg_tail,
+                               w.seg_flags))));
+  NC_RUN(K_SEG_FIXUP, 0, 0,
+         (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, C, w.seg_head, w.seg_tail, w.seg_flags, nch, G(0))));
   return NC_OK;
 }
 

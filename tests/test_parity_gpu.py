@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import synth
-from tests._gpu_helpers import compare, gpu_step, make_case, to_device
+from tests._gpu_helpers import compare, cosine, gpu_step, make_case, split_grads, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -144,7 +144,45 @@ def test_error_paths(torch_cuda):
     torch.cuda.synchronize()
 
 
-def test_deterministic_loss(torch_cuda):
+def _token_patterns(V, B, T):
+    """Token rows that put segment boundaries where the summation's chunks
+    (16 sorted positions each) make them delicate."""
+    M = B * T
+    same = np.full(M, 5)                                   # one segment over every chunk
+    distinct = np.arange(M) % V                            # runs of one (V >= M) or a few
+    runs16 = (np.arange(M) // 16) % V                      # every run ends on a chunk boundary
+    runs17 = (np.arange(M) // 17) % V                      # runs cross boundaries by one
+    mixed = np.where(np.arange(M) % 3 == 0, 0, (np.arange(M) * 7919) % V)  # one hot token among scattered ones
+    return {"same": same, "distinct": distinct, "runs16": runs16, "runs17": runs17, "mixed": mixed}
+
+
+@pytest.mark.parametrize("pattern", ["same", "distinct", "runs16", "runs17", "mixed"])
+def test_embedding_gradient_segments(torch_cuda, pattern):
+    # fp32 model: the embedding gradient row by row against the oracle, with
+    # the tokens in shuffled order so that positions of a token are far apart
+    depth, V, B, T = 2, 700, 2, 150
+    lay, flat, W, _, tgt = make_case(depth, V, B, T, "f32", 17, "uniform", {"lm_head": 0.5})
+    toks = _token_patterns(V, B, T)[pattern]
+    perm = np.argsort(synth.uniform01(23, 1, B * T))
+    tok = np.ascontiguousarray(toks[perm].reshape(B, T).astype(np.int32))
+    model = _model(depth, V, T, "f32")
+    rc, loss, tl, g = gpu_step(model, flat, tok, tgt, "f32")
+    assert rc == 0
+    loss_ref, tl_ref, g_ref = oracle.loss_and_grads(W, tok, tgt, depth)
+    compare("f32", lay, loss, g, loss_ref, g_ref, tl, tl_ref, tag=f"segments-{pattern}")
+    dwte = g[:V * 128].reshape(V, 128)
+    ref = g_ref["wte"]
+    absent = np.setdiff1d(np.arange(V), tok)
+    assert np.all(dwte[absent] == 0.0)
+    np.testing.assert_allclose(dwte, ref, rtol=0, atol=1e-4 * np.abs(ref).max())
+
+
+def test_deterministic_step(torch_cuda):
+    # Loss, token losses and the embedding and unembedding gradients are
+    # bit-identical run to run (fixed summation orders, no floating-point
+    # atomics).  The weight gradients of the blocks split their reductions
+    # over K across CTAs that add into fp32 in arrival order, so those may
+    # differ in the last bits; they are compared to the gradient tolerance.
     depth, V, B, T = 4, 65536, 2, 128
     lay, flat, W, tok, tgt = make_case(depth, V, B, T, "bf16", 6, "zipf")
     model = _model(depth, V, 128, "bf16")
@@ -152,3 +190,8 @@ def test_deterministic_loss(torch_cuda):
     r2 = gpu_step(model, flat, tok, tgt, "bf16")
     assert r1[1] == r2[1]
     np.testing.assert_array_equal(r1[2], r2[2])
+    g1, g2 = split_grads(r1[3], lay), split_grads(r2[3], lay)
+    np.testing.assert_array_equal(g1["wte"], g2["wte"])
+    np.testing.assert_array_equal(g1["lm_head"], g2["lm_head"])
+    for name, _, _ in lay:
+        assert cosine(g1[name], g2[name]) >= 1 - 1e-6, name
