@@ -36,10 +36,12 @@ if ROOT not in sys.path:
 
 METRIC = "train tokens/sec (fwd+bwd) at d20 on 1 B200; MFU vs bf16 dense peak"
 DEFAULT_WORKLOAD = "d20"
+FULL_BLOCK_WINDOW = 1024  # the short window of the pages' "SSSL" layers
 
 
-def metric_for(name: str) -> str:
-    return METRIC if name == DEFAULT_WORKLOAD else METRIC.replace("at d20", f"at {name}")
+def metric_for(name: str, full_block: bool = False) -> str:
+    m = METRIC if name == DEFAULT_WORKLOAD else METRIC.replace("at d20", f"at {name}")
+    return m.replace(" on 1 B200", " (full reference block) on 1 B200") if full_block else m
 
 
 def host_cpu_model() -> str:
@@ -58,9 +60,14 @@ def host_cpu_model() -> str:
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def model_flops_per_token(depth: int, C: int, V: int, T: int) -> float:
+def model_flops_per_token(depth: int, C: int, V: int, T: int, windows=None) -> float:
+    """windows: per-layer sliding window (0 or None: causal).  A windowed
+    layer's query sees w - w^2/(2T) keys on average (T/2 when causal)."""
     n_mm = depth * (2 * C * C + 2 * 128 * C + 8 * C * C) + V * C
-    return 6.0 * n_mm + 6.0 * T * C * depth
+    if not windows:
+        return 6.0 * n_mm + 6.0 * T * C * depth
+    keys = sum((w - w * w / (2.0 * T)) if (w and w < T) else T / 2.0 for w in windows)
+    return 6.0 * n_mm + 12.0 * C * keys
 
 
 def model_flops_per_token_noncausal(depth: int, C: int, V: int, T: int) -> float:
@@ -261,7 +268,7 @@ def run_reference(args):
     return 0
 
 
-def config_dict(wl, n_gpus, sample=None):
+def config_dict(wl, n_gpus, sample=None, full_block=False):
     d = {
         "workload": (f"{wl.name}: depth {wl.depth}, width {64 * wl.depth}, "
                      f"{64 * wl.depth // 128} query heads x128 + 1 shared KV head, "
@@ -272,6 +279,9 @@ def config_dict(wl, n_gpus, sample=None):
     }
     if sample:
         d["sample"] = sample
+    if full_block:
+        d["block"] = (f"full reference block: SSSL sliding windows of {FULL_BLOCK_WINDOW} tokens (last layer "
+                      "full), gated value embeddings on even layers, resid/x0 scalars (1.0 / 0.1)")
     return d
 
 
@@ -290,9 +300,19 @@ def run_ours(args):
     from decoder_only_transformer_nanochat_b200 import Model
 
     wl = synth.WORKLOADS[args.config]
-    model = Model(wl.depth, vocab=wl.vocab, seq=wl.seq, dtype=wl.dtype)
+    if args.full_block:
+        # the pages' full block: SSSL windows of 1,024, value embeddings, residual scalars
+        model = Model(wl.depth, vocab=wl.vocab, seq=wl.seq, dtype=wl.dtype, window=FULL_BLOCK_WINDOW,
+                      value_embeds=True, resid_scalars=True)
+        n_ve = (wl.depth + 1) // 2
+        values = synth.full_block_values(wl.depth, n_ve)
+    else:
+        model = Model(wl.depth, vocab=wl.vocab, seq=wl.seq, dtype=wl.dtype)
+        values = None
     lay = [(n, r, c) for n, _, r, c in model.layout]
-    flat, W64 = synth.make_weights(lay, wl.seed, wl.dtype)
+    flat, W64 = synth.make_weights(lay, wl.seed, wl.dtype, values=values)
+    if args.full_block:
+        W64 = None  # the CPU baseline times the baseline oracle only
     if wl.dtype == "bf16":
         weights = torch.from_numpy(flat.view(np.int16)).cuda().view(torch.bfloat16)
     else:
@@ -428,17 +448,17 @@ def run_ours(args):
     roof["algorithmic_per_launch"] = (dominant["flops"] or dominant["bytes"]) / dominant["launches"]
 
     D = model.dims
-    fpt = model_flops_per_token(wl.depth, D["width"], wl.vocab, wl.T)
+    fpt = model_flops_per_token(wl.depth, D["width"], wl.vocab, wl.T, model.windows)
     fpt_nc = model_flops_per_token_noncausal(wl.depth, D["width"], wl.vocab, wl.T)
     model_tflops = value * fpt / 1e12
     launches = sum(s["launches"] for s in stats)  # the accounting pass ran the same steps
 
     line = {
-        "metric": metric_for(wl.name), "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": metric_for(wl.name, args.full_block), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded Zipf tokens, random-init weights)",
-        "config": config_dict(wl, world),
+        "config": config_dict(wl, world, full_block=args.full_block),
         "mfu": model_tflops / (world * peaks["bf16_tflops"]),
         "mfu_sustained_peak": model_tflops / (world * peaks["bf16_tflops_sustained"]),
         "model_tflops": model_tflops, "model_flops_per_token": fpt,
@@ -477,6 +497,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", default=DEFAULT_WORKLOAD, choices=["d4", "d12", "d20", "d24", "d32"])
+    ap.add_argument("--full-block", action="store_true",
+                    help="the full reference block (SSSL windows, value embeddings, residual scalars)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -69,8 +69,11 @@ _SIGS = {
     "nc_profile_read": (_I, [_P, ctypes.POINTER(nc_kernel_stat), _I, ctypes.POINTER(_I)]),
     "nc_gemm": (_I, [_P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _I,
                      _I, _I, _I, _P]),
-    "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _P]),
-    "nc_attention_bwd": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "nc_attention_fwd": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "nc_attention_bwd": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "nc_init_ex": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(_P)]),
+    "nc_layer_window": (_I, [_P, _I, ctypes.POINTER(_I)]),
+    "nc_param_count": (_I, [_P, ctypes.POINTER(_I)]),
     "nc_ops_status": (_I, [_P, _I]),
     "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
@@ -106,6 +109,31 @@ def nc_init(depth: int, vocab: int, seq: int, dtype: int):
     h = _P()
     rc = load_library().nc_init(depth, vocab, seq, dtype, ctypes.byref(h))
     return rc, h.value
+
+
+class nc_block_opts(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int), ("value_embeds", ctypes.c_int), ("resid_scalars", ctypes.c_int)]
+
+
+def nc_init_ex(depth: int, vocab: int, seq: int, dtype: int, window: int = 0, value_embeds: bool = False,
+               resid_scalars: bool = False):
+    """Returns (status, handle) of a model with the full block's options."""
+    h = _P()
+    o = nc_block_opts(window, int(value_embeds), int(resid_scalars))
+    rc = load_library().nc_init_ex(depth, vocab, seq, dtype, ctypes.byref(o), ctypes.byref(h))
+    return rc, h.value
+
+
+def nc_layer_window(handle, layer: int):
+    w = _I()
+    rc = load_library().nc_layer_window(handle, layer, ctypes.byref(w))
+    return rc, w.value
+
+
+def nc_param_count(handle):
+    n = _I()
+    rc = load_library().nc_param_count(handle, ctypes.byref(n))
+    return rc, n.value
 
 
 def nc_get_dims(handle):
@@ -157,12 +185,12 @@ def nc_gemm(A, lda, a_mn, B, ldb, b_mn, D, ldd, M, N, K, dtype, epilogue, engine
                                   engine, stream)
 
 
-def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream) -> int:
-    return load_library().nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream)
+def nc_attention_fwd(qkv, ld, O, lse, B, T, H, dtype, engine, stream, window: int = 0) -> int:
+    return load_library().nc_attention_fwd(qkv, ld, O, lse, B, T, H, window, dtype, engine, stream)
 
 
-def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream) -> int:
-    return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine,
+def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, stream, window: int = 0) -> int:
+    return load_library().nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, window, dtype, engine,
                                            stream)
 
 

@@ -8,6 +8,8 @@
 //
 // Each query (or key) row is owned by 8 threads; thread `sub` owns dims
 // sub + 8*c, c < 16, and dot products are finished with 3 shuffles.
+// window > 0 limits query i to keys j with i - j < window (sliding window);
+// window <= 0 is the plain causal mask.
 #pragma once
 
 #include "elementwise.cuh"
@@ -30,7 +32,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(const T *__restrict__ qkv, int ld,
                                                             T *__restrict__ O,
                                                             float *__restrict__ lse, int T_len,
-                                                            int H) {
+                                                            int H, int window) {
   __shared__ float Ks[kSimtKeys][kHeadDim + 1];
   __shared__ float Vs[kSimtKeys][kHeadDim + 1];
   const int b = blockIdx.z, h = blockIdx.y;
@@ -47,8 +49,10 @@ __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(const T *__restrict_
     acc[c] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
+  const int w = window > 0 ? window : T_len;
   const int last = min(T_len - 1, blockIdx.x * kSimtRows + kSimtRows - 1);
-  for (int j0 = 0; j0 <= last; j0 += kSimtKeys) {
+  const int j_first = max(0, (int)blockIdx.x * kSimtRows - w + 1) / kSimtKeys * kSimtKeys;
+  for (int j0 = j_first; j0 <= last; j0 += kSimtKeys) {
     __syncthreads();
     for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
       const int jj = e / kHeadDim, c = e % kHeadDim;
@@ -66,7 +70,7 @@ __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(const T *__restrict_
 #pragma unroll
       for (int c = 0; c < 16; ++c) d = fmaf(q[c], Ks[jj][sub + 8 * c], d);
       d = sub8_sum(d);
-      s[jj] = (j0 + jj <= i) ? d : -INFINITY;
+      s[jj] = (j0 + jj <= i && i - (j0 + jj) < w) ? d : -INFINITY;
       tmax = fmaxf(tmax, s[jj]);
     }
     if (tmax == -INFINITY) continue;  // every key of this tile is in the future
@@ -97,10 +101,11 @@ __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(const T *__restrict_
 template <typename T>
 __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
     const T *__restrict__ qkv, int ld, const T *__restrict__ dO, const float *__restrict__ lse,
-    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H) {
+    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H, int window) {
   __shared__ float Ks[kSimtKeys][kHeadDim + 1];
   __shared__ float Vs[kSimtKeys][kHeadDim + 1];
   const int b = blockIdx.z, h = blockIdx.y;
+  const int w = window > 0 ? window : T_len;
   const int r = threadIdx.x >> 3, sub = threadIdx.x & 7;
   const int i = blockIdx.x * kSimtRows + r;
   const int C = H * kHeadDim;
@@ -117,7 +122,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
   const size_t li = ((size_t)b * H + h) * T_len + (valid ? i : 0);
   const float L = lse[li], Di = Dr[li];
   const int last = min(T_len - 1, blockIdx.x * kSimtRows + kSimtRows - 1);
-  for (int j0 = 0; j0 <= last; j0 += kSimtKeys) {
+  const int j_first = max(0, (int)blockIdx.x * kSimtRows - w + 1) / kSimtKeys * kSimtKeys;
+  for (int j0 = j_first; j0 <= last; j0 += kSimtKeys) {
     __syncthreads();
     for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
       const int jj = e / kHeadDim, c = e % kHeadDim;
@@ -137,7 +143,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
       }
       s = sub8_sum(s);
       dp = sub8_sum(dp);
-      const float p = (j0 + jj <= i) ? expf(s - L) : 0.f;
+      const float p = (j0 + jj <= i && i - (j0 + jj) < w) ? expf(s - L) : 0.f;
       const float ds = p * (dp - Di) * scale;
 #pragma unroll
       for (int c = 0; c < 16; ++c) dq[c] = fmaf(ds, Ks[jj][sub + 8 * c], dq[c]);
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
 template <typename T>
 __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
     const T *__restrict__ qkv, int ld, const T *__restrict__ dO, const float *__restrict__ lse,
-    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H) {
+    const float *__restrict__ Dr, T *__restrict__ dqkv, int T_len, int H, int window) {
   __shared__ float Qs[kSimtKeys][kHeadDim + 1];
   __shared__ float Gs[kSimtKeys][kHeadDim + 1];
   __shared__ float Ls[kSimtKeys], Ds[kSimtKeys];
@@ -174,8 +180,10 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
     dv[c] = 0.f;
   }
   const int first = blockIdx.x * kSimtRows;  // earliest query that sees a key of this block
+  const int w = window > 0 ? window : T_len;
+  const int i_end = min(T_len, first + kSimtRows - 1 + w);  // past the last query that sees one
   for (int h = 0; h < H; ++h) {
-    for (int i0 = (first / kSimtKeys) * kSimtKeys; i0 < T_len; i0 += kSimtKeys) {
+    for (int i0 = (first / kSimtKeys) * kSimtKeys; i0 < i_end; i0 += kSimtKeys) {
       __syncthreads();
       for (int e = threadIdx.x; e < kSimtKeys * kHeadDim; e += blockDim.x) {
         const int ii = e / kHeadDim, c = e % kHeadDim;
@@ -202,7 +210,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
         }
         s = sub8_sum(s) * scale;
         dp = sub8_sum(dp);
-        const bool live = valid && i < T_len && i >= j;
+        const bool live = valid && i < T_len && i >= j && i - j < w;
         const float p = live ? expf(s - Ls[ii]) : 0.f;
         const float ds = p * (dp - Ds[ii]) * scale;
 #pragma unroll
@@ -223,20 +231,20 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
 
 template <typename T>
 inline cudaError_t launch_attn_simt_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len,
-                                        int H, cudaStream_t st) {
+                                        int H, int window, cudaStream_t st) {
   dim3 grid((T_len + kSimtRows - 1) / kSimtRows, H, B);
-  attn_fwd_simt_kernel<T><<<grid, 128, 0, st>>>(qkv, ld, O, lse, T_len, H);
+  attn_fwd_simt_kernel<T><<<grid, 128, 0, st>>>(qkv, ld, O, lse, T_len, H, window);
   return cudaGetLastError();
 }
 
 template <typename T>
 inline cudaError_t launch_attn_simt_bwd(const T *qkv, int ld, const T *dO, const float *lse,
-                                        const float *Dr, T *dqkv, int B, int T_len, int H,
+                                        const float *Dr, T *dqkv, int B, int T_len, int H, int window,
                                         cudaStream_t st) {
   dim3 g1((T_len + kSimtRows - 1) / kSimtRows, H, B);
-  attn_bwd_dq_simt_kernel<T><<<g1, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H);
+  attn_bwd_dq_simt_kernel<T><<<g1, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H, window);
   dim3 g2((T_len + kSimtRows - 1) / kSimtRows, 1, B);
-  attn_bwd_dkdv_simt_kernel<T><<<g2, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H);
+  attn_bwd_dkdv_simt_kernel<T><<<g2, 128, 0, st>>>(qkv, ld, dO, lse, Dr, dqkv, T_len, H, window);
   return cudaGetLastError();
 }
 
@@ -249,28 +257,29 @@ namespace nc {
 // misaligned operand; there is no slower fallback), CUDA cores for fp32;
 // engine 1: the CUDA-core kernels for either dtype (a test engine).
 template <typename T>
-inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H,
+inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H, int window,
                                    int engine, int *status, cudaStream_t st) {
   if (sizeof(T) == 2 && engine == 0) {
     if (!fatc::supported(qkv, ld, O)) return cudaErrorInvalidValue;
-    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, status, st);
+    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, window, status, st);
   }
-  return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, st);
+  return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, window, st);
 }
 
 // D = rowsum(dO * O) is computed inside the tcgen05 dQ kernel; the CUDA-core
 // engine gets it from attn_rowdot_kernel first.  Drow is [B, H, T] scratch.
 template <typename T>
 inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *O, const T *dO, const float *lse, float *Dr,
-                                   T *dqkv, int B, int T_len, int H, int engine, int *status, cudaStream_t st) {
+                                   T *dqkv, int B, int T_len, int H, int window, int engine, int *status,
+                                   cudaStream_t st) {
   if (sizeof(T) == 2 && engine == 0) {
     if (!fatc::supported_bwd(qkv, ld, O, dO, dqkv)) return cudaErrorInvalidValue;
     return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B,
-                            T_len, H, status, st);
+                            T_len, H, window, status, st);
   }
   const int M = B * T_len;
   attn_rowdot_kernel<T><<<(unsigned)(((size_t)M * H + 7) / 8), 256, 0, st>>>(dO, O, Dr, M, T_len, H);
-  return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, st);
+  return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, window, st);
 }
 
 }  // namespace nc

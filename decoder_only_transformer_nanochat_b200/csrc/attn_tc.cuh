@@ -99,10 +99,15 @@ __device__ __forceinline__ uint32_t tile_unit(int r, int u) {
 
 struct FwdParams {
   int T, H, n_qt;
+  int window;   // windowed kernels: query i sees keys j with 0 <= i - j < window
   float *lse;   // [B, H, T]
   int *status;
 };
 
+// kWin: sliding-window variant (compiled separately, so the plain causal
+// kernel is unchanged by it): key tiles start at the window's first tile and
+// keys more than window - 1 before the query are masked.
+template <bool kWin>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
                        const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
@@ -136,7 +141,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int qt = p.n_qt - 1 - (int)blockIdx.x / BH;  // latest query tiles (most keys) first
   const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
   const int q0 = qt * kQ;
-  const int n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV;  // = qt + 1
+  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kKV : 0;   // first key tile any query here sees
+  const int n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV - kt_lo;   // key tiles visited (qt + 1 when causal)
+  const int kbase = kt_lo * kKV;                                  // first key of tile j = kbase + j * kKV
   const int C = p.H * kD;
 
   if (threadIdx.x == 0) {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
         const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
         mbar_expect_tx(k_full(st), kTileBytes);
-        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, j * kKV, b, k_full(st));
+        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b, k_full(st));
         ++issued_k;
         return true;
       };
@@ -185,7 +192,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_expect_tx(v_full(st), kTileBytes);
         for (int hh = 0; hh < 2; ++hh)
           for (int a = 0; a < 2; ++a)
-            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, j * kKV + 64 * hh, b, v_full(st));
+            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, kbase + j * kKV + 64 * hh, b,
+                        v_full(st));
         ++issued_v;
         return true;
       };
@@ -288,11 +296,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < 64; ++i) s[i] = 0.f;
       }
-      const int kv0 = j * kKV + c0;
-      if (kv0 + 64 > q0 || kv0 + 64 > p.T) {
+      const int kv0 = kbase + j * kKV + c0;
+      if (kv0 + 64 > q0 || kv0 + 64 > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window)) {
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-          if (kv0 + i > row || kv0 + i >= p.T) s[i] = -INFINITY;
+          if (kv0 + i > row || kv0 + i >= p.T || (kWin && row - (kv0 + i) >= p.window)) s[i] = -INFINITY;
       }
       float mx = -INFINITY;
 #pragma unroll
@@ -311,6 +319,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         l *= corr;
         m_used = mx;
       }
+      // with a window a row may see no key of its first tile: its base stays
+      // -inf there and its exponentials are taken against 0 (all of them 0)
+      const float mb = (kWin && m_used == -INFINITY) ? 0.f : m_used;
       // P_j in registers first: the exponentials overlap the previous P V
       float sum = 0.f;
       uint32_t pk[32];
@@ -318,8 +329,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int i = 0; i < 64; i += 2) {
         // one exponential in four on the FMA pipe: measured fastest (half makes
         // the loop issue-bound, none leaves it MUFU-bound)
-        const float e0 = ex2(s[i] - m_used);
-        const float e1 = (i & 2) ? ex2_poly(s[i + 1] - m_used) : ex2(s[i + 1] - m_used);
+        const float e0 = ex2(s[i] - mb);
+        const float e1 = (i & 2) ? ex2_poly(s[i + 1] - mb) : ex2(s[i + 1] - mb);
         sum += e0 + e1;
         pk[i / 2] = pack2(e0, e1);
       }
@@ -414,12 +425,14 @@ constexpr int kSoft = 256;
 
 struct BwdParams {
   int T, H, n_tiles, ld;
+  int window;         // windowed kernels: query i sees keys j with 0 <= i - j < window
   const float *lse;   // [B, H, T]
   float *Drow;        // [B, H, T]: rowsum(dO * O), written by the dQ kernel
   const bf16 *O;      // [B*T, H*128]
   int *status;
 };
 
+template <bool kWin>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128 (Q, K, V tiles)
                           const __grid_constant__ CUtensorMap map_do,   // dO [B][T][C], box 64 x 128
@@ -451,7 +464,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int qt = p.n_tiles - 1 - (int)blockIdx.x / BH;
   const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
   const int q0 = qt * kQ;
-  const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK;
+  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kBK : 0;
+  const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK - kt_lo;
+  const int kbase = kt_lo * kBK;
   const int C = p.H * kD;
   // TMEM columns: S at 0, dP at 128 (one buffer, free again as soon as the
   // element-wise warps have loaded it); dQ at 256; dS[2] (bf16 pairs) at 384, 448
@@ -486,11 +501,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait(k_empty(ks), ((j / kDqKStages) & 1) ^ 1, abort_flag, p.status)) break;
         mbar_expect_tx(k_full(ks), kTileBytes);
         for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, j * kBK, b, k_full(ks));
+          tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, kbase + j * kBK, b,
+                      k_full(ks));
         if (!mbar_wait(v_empty(vs), ((j / kDqVStages) & 1) ^ 1, abort_flag, p.status)) break;
         mbar_expect_tx(v_full(vs), kTileBytes);
         for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, j * kBK, b,
+          tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, kbase + j * kBK, b,
                       v_full(vs));
         ++issued;
       }
@@ -602,8 +618,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_empty);
-      const int kv0 = j * kBK + c0;
-      const bool need_mask = kv0 + 64 > q0 || kv0 + 64 > p.T;
+      const int kv0 = kbase + j * kBK + c0;
+      const bool need_mask = kv0 + 64 > q0 || kv0 + 64 > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window);
       uint32_t packed[32];
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
@@ -612,7 +628,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int t = 0; t < 2; ++t) {
           float pr = ex2(__uint_as_float(sv[i + t]) * sc - L);
           const int key = kv0 + i + t;
-          if (need_mask && (key > row || key >= p.T)) pr = 0.f;
+          if (need_mask && (key > row || key >= p.T || (kWin && row - key >= p.window))) pr = 0.f;
           d2[t] = pr * (__uint_as_float(dv[i + t]) - Dv);
         }
         packed[i / 2] = pack2(d2[0], d2[1]);
@@ -678,6 +694,7 @@ static_assert(kQStage % 1024 == 0 && kTileBytes % 1024 == 0,
               "128-byte-swizzled TMA tiles need 1 KB-aligned shared-memory addresses");
 static_assert(kKvSmemTc <= 232448 && kDqSmem <= 232448 && kSmem <= 232448, "shared memory per CTA");
 
+template <bool kWin>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap map_qkv,  // qkv, box 64 x 128 (K, V, Q)
                             const __grid_constant__ CUtensorMap map_do,   // dO, box 64 x 128
@@ -710,7 +727,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int k0 = kt * kQ;
   const int C = p.H * kD;
   const int first = k0 / kBQ2;
-  const int n_q = (p.T + kBQ2 - 1) / kBQ2 - first;
+  const int n_q_all = (p.T + kBQ2 - 1) / kBQ2;
+  // with a window the last query that sees key k0 + 127 is k0 + 127 + window - 1
+  const int last_q = kWin ? min(n_q_all - 1, (k0 + kQ - 1 + p.window - 1) / kBQ2) : n_q_all - 1;
+  const int n_q = last_q - first + 1;
   const int n_it = n_q * p.H;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -875,7 +895,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(s_taken);  // X may take dP^T now
       const float *Ls = reinterpret_cast<const float *>(sQS + st * kQStage + 2 * kTileBytes) + c0;
       const float *Ds = Ls + kBQ2;
-      const bool need_mask = qq0 < key + 1 || qq0 + 64 > p.T;
+      const bool need_mask = qq0 < key + 1 || qq0 + 64 > p.T || (kWin && qq0 + 63 - key >= p.window);
       float pr[64];
       uint32_t pk[32];
 #pragma unroll
@@ -886,7 +906,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int t = 0; t < 4; ++t) {
           const int qi = 4 * i4 + t;
           float v = ex2(__uint_as_float(xv[qi]) * sc - lv[t] * kLog2e);
-          if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T)) v = 0.f;
+          if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T || (kWin && qq0 + qi - key >= p.window))) v = 0.f;
           pr[qi] = v;
         }
         pk[2 * i4] = pack2(pr[4 * i4], pr[4 * i4 + 1]);
@@ -977,14 +997,23 @@ inline bool make_map3(CUtensorMap *map, const void *base, int B, int T, int cols
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline cudaError_t init() {
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+template <bool kWin>
+inline cudaError_t init_variant() {
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
+    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemTc);
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemTc);
   return e;
 }
+inline cudaError_t init() {
+  cudaError_t e = init_variant<false>();
+  return e == cudaSuccess ? init_variant<true>() : e;
+}
+
+// A window that covers every earlier key is the plain causal mask: only a
+// window shorter than the sequence takes the windowed kernels.
+inline bool windowed(int window, int T) { return window > 0 && window < T; }
 
 // Operands the TMA tiles can take: 16-byte aligned bases and row strides.
 inline bool aligned(const void *qkv, int64_t ld, const void *O) {
@@ -994,8 +1023,8 @@ inline bool supported(const void *qkv, int64_t ld, const void *O) {
   return encode_fn() != nullptr && aligned(qkv, ld, O);
 }
 
-inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int *status,
-                              cudaStream_t st) {
+inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int window,
+                              int *status, cudaStream_t st) {
   CUtensorMap mqk, mv, mo;
   const int C = H * kD;
   if (!make_map3(&mqk, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mv, qkv, B, T, (int)ld, ld, 64) ||
@@ -1007,7 +1036,9 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.n_qt = (T + kQ - 1) / kQ;
   p.lse = lse;
   p.status = status;
-  attn_fwd_tc_kernel<<<B * H * p.n_qt, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  p.window = window;
+  if (windowed(window, T)) attn_fwd_tc_kernel<true><<<B * H * p.n_qt, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  else attn_fwd_tc_kernel<false><<<B * H * p.n_qt, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
   return cudaGetLastError();
 }
 
@@ -1018,7 +1049,8 @@ namespace nc {
 namespace fatc {
 
 inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const bf16 *dO, const float *lse,
-                              float *Drow, bf16 *dqkv, int B, int T, int H, int *status, cudaStream_t st) {
+                              float *Drow, bf16 *dqkv, int B, int T, int H, int window, int *status,
+                              cudaStream_t st) {
   CUtensorMap mq128, mdo128, mout;
   const int C = H * kD;
   if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mdo128, dO, B, T, C, C, 128) ||
@@ -1033,10 +1065,14 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   p.O = O;
   p.status = status;
   p.n_tiles = (T + kQ - 1) / kQ;
-  attn_bwd_dq_tc_kernel<<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
+  p.window = window;
+  const bool win = windowed(window, T);
+  if (win) attn_bwd_dq_tc_kernel<true><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
+  else attn_bwd_dq_tc_kernel<false><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc_kernel<<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
+  if (win) attn_bwd_dkdv_tc_kernel<true><<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
+  else attn_bwd_dkdv_tc_kernel<false><<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
   return cudaGetLastError();
 }
 

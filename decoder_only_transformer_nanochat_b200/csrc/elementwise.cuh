@@ -212,13 +212,30 @@ __device__ __forceinline__ float half_warp_sum(float v) {
   return v;
 }
 
+// Value embedding (full reference block): with ve != nullptr the shared v
+// head of the row also gets gate * ve[token] added ("ten modern departures":
+// a gated embedding lookup added to V at alternating layers); v is neither
+// roped nor normed.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_qknorm_kernel(
     T *__restrict__ qkv, int ld, float *__restrict__ rq, float *__restrict__ rk,
-    const float *__restrict__ cos_t, const float *__restrict__ sin_t, int M, int T_len, int H) {
+    const float *__restrict__ cos_t, const float *__restrict__ sin_t, int M, int T_len, int H,
+    const int32_t *__restrict__ tokens = nullptr, const T *__restrict__ ve = nullptr,
+    const T *__restrict__ ve_gate = nullptr, int V = 0) {
   const int tok = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= M) return;
+  if (ve && lane < kHeadDim / 8) {
+    T *vrow = qkv + (size_t)tok * ld + (H + 1) * kHeadDim + lane * 8;
+    const int id = min(max(tokens[tok], 0), V - 1);
+    const float g = to_f(ve_gate[0]);
+    float v[8], e[8];
+    Vec8<T>::load(vrow, v);
+    Vec8<T>::load(ve + (size_t)id * kHeadDim + lane * 8, e);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += g * e[i];
+    Vec8<T>::store(vrow, v);
+  }
   const int pos = tok % T_len;
   const int hw = lane >> 4, j = lane & 15;
   float c[8], s[8];
@@ -301,46 +318,171 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Embedding backward: through the norm after the embedding, then summed into
-// the rows of dwte that the tokens select (repeated tokens add up).
-//   y = wte[tok] r0;  g = r0 (dx - y mean(dx y));  dwte[tok] += g
-// dwte must be zeroed beforehand.
+// Residual scalars of the full reference block ("ten modern departures":
+// resid_lambdas and x0_lambdas mixing each layer's stream with the
+// normalised embedding).  At block entry
+//   x_in = lam_r x + lam_0 x0,   xn = rmsnorm(x_in)
+// x_in is the stream the block's residual adds then go into (written to
+// x_out, a buffer of its own, so x stays for the backward).
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) embed_bwd_kernel(
-    const float *__restrict__ dx, const int32_t *__restrict__ tokens, const T *__restrict__ wte,
-    const float *__restrict__ r0, float *__restrict__ dwte, int M, int C, int V) {
+__global__ void __launch_bounds__(256) mix_rmsnorm_kernel(
+    const T *__restrict__ x, const T *__restrict__ x0, const T *__restrict__ lam_r, const T *__restrict__ lam_0,
+    T *__restrict__ x_out, T *__restrict__ y, float *__restrict__ r_out, int M, int C) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
-  int tok = tokens[row];
-  tok = tok < 0 ? 0 : (tok >= V ? V - 1 : tok);
+  const float a = to_f(lam_r[0]), b = to_f(lam_0[0]);
   const int nv = C >> 3;
-  const float r = r0[row];
   const size_t base = (size_t)row * C;
-  float g[NV][8], yy[NV][8];
-  float dot = 0.f;
+  float v[NV][8];
+  float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (lane + 32 * i);
     if (c < nv) {
-      Vec8<float>::load(dx + base + c * 8, g[i]);
-      Vec8<T>::load(wte + (size_t)tok * C + c * 8, yy[i]);
+      float e[8];
+      Vec8<T>::load(x + base + c * 8, v[i]);
+      Vec8<T>::load(x0 + base + c * 8, e);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        yy[i][j] *= r;
-        dot += g[i][j] * yy[i][j];
+        v[i][j] = a * v[i][j] + b * e[j];
+        ss += v[i][j] * v[i][j];
       }
+      Vec8<T>::store(x_out + base + c * 8, v[i]);
     }
   }
-  dot = warp_sum(dot) / (float)C;
-  float *dst = dwte + (size_t)tok * C;
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)C + kEps);
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (lane + 32 * i);
     if (c < nv) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) atomicAdd(dst + c * 8 + j, r * (g[i][j] - yy[i][j] * dot));
+      for (int j = 0; j < 8; ++j) v[i][j] *= r;
+      Vec8<T>::store(y + base + c * 8, v[i]);
     }
+  }
+  if (lane == 0) r_out[row] = r;
+}
+
+// Backward of the block entry, fused into the norm backward of xn:
+//   dx_in = dx_old + r (dy - y mean(dy y))
+//   dx    = lam_r dx_in          (the stream gradient below the block; fp32 and T)
+//   dx0  (+)= lam_0 dx_in        (first != 0: written, else accumulated)
+//   partial[block] = (sum dx_in x, sum dx_in x0) over the block's rows, in a
+//   fixed order (the scalars' gradients, finished by ordered_sum_rows_kernel)
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_bwd_mix_kernel(
+    const T *__restrict__ dy, const T *__restrict__ y, const float *__restrict__ r, float *__restrict__ dx,
+    T *__restrict__ dx_t, const T *__restrict__ x, const T *__restrict__ x0, const T *__restrict__ lam_r,
+    const T *__restrict__ lam_0, float *__restrict__ dx0, int first, float *__restrict__ part_r,
+    float *__restrict__ part_0, int M, int C) {
+  __shared__ float sh_r[8], sh_0[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  float sum_r = 0.f, sum_0 = 0.f;
+  if (row < M) {
+    const float a = to_f(lam_r[0]), b = to_f(lam_0[0]);
+    const int nv = C >> 3;
+    const size_t base = (size_t)row * C;
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (lane + 32 * i);
+      if (c < nv) {
+        float g[8], yy[8];
+        Vec8<T>::load(dy + base + c * 8, g);
+        Vec8<T>::load(y + base + c * 8, yy);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dot += g[j] * yy[j];
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(dx + base + c * 8));
+      }
+    }
+    dot = warp_sum(dot) / (float)C;
+    const float rr = r[row];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (lane + 32 * i);
+      if (c < nv) {
+        float g[8], yy[8], old[8], xv[8], x0v[8], acc0[8];
+        Vec8<T>::load(dy + base + c * 8, g);
+        Vec8<T>::load(y + base + c * 8, yy);
+        Vec8<float>::load(dx + base + c * 8, old);
+        Vec8<T>::load(x + base + c * 8, xv);
+        Vec8<T>::load(x0 + base + c * 8, x0v);
+        if (!first) Vec8<float>::load(dx0 + base + c * 8, acc0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float din = old[j] + rr * (g[j] - yy[j] * dot);
+          sum_r += din * xv[j];
+          sum_0 += din * x0v[j];
+          g[j] = a * din;
+          acc0[j] = (first ? 0.f : acc0[j]) + b * din;
+        }
+        Vec8<float>::store(dx + base + c * 8, g);
+        Vec8<T>::store(dx_t + base + c * 8, g);
+        Vec8<float>::store(dx0 + base + c * 8, acc0);
+      }
+    }
+    sum_r = warp_sum(sum_r);
+    sum_0 = warp_sum(sum_0);
+  }
+  if (lane == 0) {
+    sh_r[warp] = sum_r;
+    sh_0[warp] = sum_0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f, b = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      a += sh_r[w];
+      b += sh_0[w];
+    }
+    part_r[blockIdx.x] = a;
+    part_0[blockIdx.x] = b;
+  }
+}
+
+// out[row * out_stride] = sum of partial[row * n .. row * n + n) in a fixed order.
+__global__ void __launch_bounds__(256) ordered_sum_rows_kernel(const float *__restrict__ partial, int n,
+                                                               float *__restrict__ out, int out_stride) {
+  __shared__ float sh[32];
+  const float *p = partial + (size_t)blockIdx.x * n;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += p[i];
+  s = block_sum(s, sh);
+  if (threadIdx.x == 0) out[(size_t)blockIdx.x * out_stride] = s;
+}
+
+// Value-embedding gate gradient, first stage: partial[block] = sum over the
+// block's 64 positions of dv_i . ve[tok_i] (dv: v part of dqkv, stride ld), in
+// a fixed order; ordered_sum_kernel adds the partials.
+template <typename T>
+__global__ void __launch_bounds__(256) ve_gate_partial_kernel(const T *__restrict__ dv, int64_t ld,
+                                                              const int32_t *__restrict__ tokens,
+                                                              const T *__restrict__ ve, int V, int M,
+                                                              float *__restrict__ partial) {
+  __shared__ float sh[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc = 0.f;
+  for (int t = 0; t < 8; ++t) {
+    const int i = blockIdx.x * 64 + warp * 8 + t;
+    if (i < M && lane < kHeadDim / 8) {
+      const int id = min(max(tokens[i], 0), V - 1);
+      float a[8], e[8];
+      Vec8<T>::load(dv + (size_t)i * ld + lane * 8, a);
+      Vec8<T>::load(ve + (size_t)id * kHeadDim + lane * 8, e);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc += a[j] * e[j];
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) sh[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += sh[w];
+    partial[blockIdx.x] = s;
   }
 }
 

@@ -34,16 +34,24 @@ using namespace nc;
 enum KernelClass {
   K_GEMM_TC, K_GEMM_SIMT, K_ATTN_FWD, K_ATTN_BWD, K_EMBED, K_RMSNORM, K_ROPE_QKNORM, K_CE,
   K_LOSS_MEAN, K_RMSNORM_BWD, K_ROWDOT, K_ROPE_QKNORM_BWD, K_EMBED_BWD, K_TOKEN_SORT, K_SEG_FIXUP,
-  K_NUM_CLASSES
+  K_VE_BWD, K_NUM_CLASSES
 };
 static const char *kClassName[K_NUM_CLASSES] = {
     "gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd", "embed_norm", "rmsnorm", "rope_qknorm",
     "ce_fused", "loss_mean", "rmsnorm_bwd", "attn_rowdot", "rope_qknorm_bwd", "embed_bwd",
-    "token_sort", "seg_fixup"};
+    "token_sort", "seg_fixup", "block_extras_bwd"};
 
 struct nc_model {
   int depth, C, H, F, V, seq, dtype;
   int64_t n_params;
+  // full reference block (nc_init_ex): short window of the "S" layers (0:
+  // none), value embeddings, residual scalars
+  int window = 0;
+  bool ve = false, scalars = false;
+  std::vector<int> layer_window;  // per layer: keys a query sees (0: plain causal)
+  std::vector<int> ve_param;      // per layer: param index of its value-embedding table, or -1
+  std::vector<int> ve_slot;       // per layer: its entry of ve_gates, or -1
+  int p_resid = -1, p_x0 = -1, p_gates = -1;
   int device;
   int num_sms;
   float *rope_cos;  // [seq, 64] fp32
@@ -75,6 +83,12 @@ struct Work {
   TokenSort sort;                   // positions grouped by token (embedding gradient)
   float *seg_head, *seg_tail;       // [chunks, C] partial sums of segments cut by chunks
   int *seg_flags;                   // [chunks]
+  // residual scalars: the stream entering each block kept ([0] = x0 =
+  // norm(wte[tok])), the gradient reaching x0 through the mixing, and
+  // per-block partial sums of the scalars' gradients [2][L][blocks]
+  std::vector<T *> xs;
+  float *dx0 = nullptr, *scal_part = nullptr;
+  float *ve_part = nullptr;         // value-embedding gate gradient partials [blocks of 64 rows]
 };
 
 // Lay the workspace out (base == nullptr only measures it).
@@ -129,7 +143,21 @@ size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
   const size_t nch = (size_t)seg_chunks((int)M);
   float *seg_head = (float *)take(nch * C * 4), *seg_tail = (float *)take(nch * C * 4);
   int *seg_flags = (int *)take(nch * 4);
+  std::vector<T *> xs;
+  float *dx0 = nullptr, *scal_part = nullptr, *ve_part = nullptr;
+  if (m->scalars) {
+    for (int l = 1; l <= L; ++l) xs.push_back((T *)take(M * C * es));
+    dx0 = (float *)take(M * C * 4);
+    scal_part = (float *)take((size_t)2 * L * ((M + 7) / 8) * 4);
+  }
+  if (m->ve) ve_part = (float *)take(((M + 63) / 64) * 4);
   if (w) {
+    w->xs.clear();
+    if (m->scalars) {
+      w->xs.push_back(x);  // x0: the embedding output is the stream entering block 0
+      for (T *p : xs) w->xs.push_back(p);
+    }
+    w->dx0 = dx0; w->scal_part = scal_part; w->ve_part = ve_part;
     w->sort.keys[0] = sk0; w->sort.keys[1] = sk1; w->sort.vals[0] = sv0; w->sort.vals[1] = sv1;
     w->sort.hist = hist; w->sort.skey = nullptr; w->sort.spos = nullptr;
     w->seg_head = seg_head; w->seg_tail = seg_tail; w->seg_flags = seg_flags;
@@ -147,6 +175,8 @@ template <typename T>
 struct Weights {
   const T *wte, *lm_head;
   std::vector<const T *> wqkv, wo, w1, w2;  // wq, wk, wv are contiguous: [C+256, C]
+  std::vector<const T *> ve;                // per layer: value-embedding table [V, 128] or null
+  const T *resid = nullptr, *x0l = nullptr, *gates = nullptr;  // [L], [L], [n_ve]
 };
 
 template <typename T>
@@ -154,13 +184,17 @@ Weights<T> weight_ptrs(const nc_model *m, const void *weights) {
   const T *base = (const T *)weights;
   Weights<T> w;
   w.wte = base + m->params[0].offset;
-  w.lm_head = base + m->params.back().offset;
   for (int l = 0; l < m->depth; ++l) {
     w.wqkv.push_back(base + m->params[1 + 6 * l].offset);
     w.wo.push_back(base + m->params[1 + 6 * l + 3].offset);
     w.w1.push_back(base + m->params[1 + 6 * l + 4].offset);
     w.w2.push_back(base + m->params[1 + 6 * l + 5].offset);
+    w.ve.push_back(m->ve_param[l] >= 0 ? base + m->params[m->ve_param[l]].offset : nullptr);
   }
+  w.lm_head = base + m->params[1 + 6 * m->depth].offset;
+  if (m->p_resid >= 0) w.resid = base + m->params[m->p_resid].offset;
+  if (m->p_x0 >= 0) w.x0l = base + m->params[m->p_x0].offset;
+  if (m->p_gates >= 0) w.gates = base + m->params[m->p_gates].offset;
   return w;
 }
 
@@ -242,6 +276,13 @@ inline unsigned rows_grid(size_t rows, int rows_per_block) {
     if (rc_ != NC_OK) return rc_; \
   } while (0)
 
+// Keys summed over the queries of one row of T tokens: causal (window 0 or
+// >= T) or sliding window.
+inline double attn_keys(int T, int window) {
+  if (window <= 0 || window >= T) return 0.5 * T * (T + 1.0);
+  return 0.5 * window * (window + 1.0) + (double)(T - window) * window;
+}
+
 // Forward through the blocks and the final norm; leaves xf, rf in the workspace.
 template <typename T>
 int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B, int T_len,
@@ -249,31 +290,42 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
   const int M = B * T_len, C = m->C, H = m->H, F = m->F;
   const int ldqkv = C + 2 * kHeadDim;
   const double es = sizeof(T);
-  const double attn_flops = 2.0 * B * H * (double)kHeadDim * T_len * (T_len + 1.0);
   NC_RUN(K_EMBED, 0, M * (8.0 + 2.0 * C * es),
          NC_DISPATCH_NV(C, (embed_norm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
                                tokens, W.wte, w.x, w.r0, M, C, m->V, m->status))));
+  T *x = w.x;  // the stream the block's residual adds go into
   for (int l = 0; l < m->depth; ++l) {
-    NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
-           NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                                 w.x, w.xn[l], w.r1[l], M, C))));
+    const double attn_flops = 4.0 * B * H * (double)kHeadDim * attn_keys(T_len, m->layer_window[l]);
+    if (m->scalars) {
+      // block entry: x_in = lam_r x + lam_0 x0 into the next stream buffer, xn = norm(x_in)
+      x = w.xs[l + 1];
+      NC_RUN(K_RMSNORM, 0, M * (4.0 + 4.0 * C * es),
+             NC_DISPATCH_NV(C, (mix_rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                   w.xs[l], w.xs[0], W.resid + l, W.x0l + l, x, w.xn[l], w.r1[l], M, C))));
+    } else {
+      NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
+             NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                   x, w.xn[l], w.r1[l], M, C))));
+    }
     NC_TRY(gemm<T>(m, gp(M, ldqkv, C, w.xn[l], C, 0, W.wqkv[l], C, 0, w.qkv[l], ldqkv, EPI_STORE), st));
-    NC_RUN(K_ROPE_QKNORM, 0, M * (2.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
+    const bool ve = W.ve[l] != nullptr;
+    NC_RUN(K_ROPE_QKNORM, 0, M * (2.0 * (C + kHeadDim) * es + 4.0 * (H + 1) + (ve ? 3.0 * kHeadDim * es : 0.0)),
            (rope_qknorm_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
-               w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
+               w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H, tokens, W.ve[l],
+               ve ? W.gates + m->ve_slot[l] : nullptr, m->V)));
     NC_RUN(K_ATTN_FWD, attn_flops, 0,
-           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, 0, m->status, st) !=
-               cudaSuccess) return NC_ECUDA);
-    NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, w.x, C, EPI_ADD), st));
+           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->layer_window[l], 0,
+                                  m->status, st) != cudaSuccess) return NC_ECUDA);
+    NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, x, C, EPI_ADD), st));
     NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
            NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                                 w.x, w.xn2[l], w.r2[l], M, C))));
+                                 x, w.xn2[l], w.r2[l], M, C))));
     NC_TRY(gemm<T>(m, gp(M, F, C, w.xn2[l], C, 0, W.w1[l], C, 0, w.a[l], F, EPI_RELU2), st));
-    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w2[l], F, 0, w.x, C, EPI_ADD), st));
+    NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w2[l], F, 0, x, C, EPI_ADD), st));
   }
   NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
          NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                               w.x, w.xf, w.rf, M, C))));
+                               x, w.xf, w.rf, M, C))));
   return NC_OK;
 }
 
@@ -287,7 +339,6 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   const int M = B * T_len, C = m->C, H = m->H, F = m->F, V = m->V;
   const int ldqkv = C + 2 * kHeadDim;
   const double es = sizeof(T);
-  const double attn_bwd_flops = 4.0 * B * H * (double)kHeadDim * T_len * (T_len + 1.0);
   NC_TRY(forward_body<T>(m, W, tokens, B, T_len, w, st));
 
   // head: z = xf Wout^T, then softcap + CE forward and backward in place
@@ -301,7 +352,7 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
 
   // gradient pointers (fp32, same layout as the weights)
   auto G = [&](int idx) { return grads + m->params[idx].offset; };
-  const int last = (int)m->params.size() - 1;
+  const int last = 1 + 6 * m->depth;  // lm_head
   const double nbwd = M * (8.0 * C + 3.0 * C * es + 4.0);  // dx_old, dx in fp32; dy, y, dx_t in T
   // dWout = dz^T xf ;  dxf = dz Wout
   NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, EPI_STORE_F32), st));
@@ -310,8 +361,15 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
          NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
                                w.dy, w.xf, w.rf, w.dx, w.dxb, M, C, 0))));
 
+  // positions grouped by token: the embedding's and the value embeddings'
+  // table gradients are summed per token in this fixed order
+  NC_RUN(K_TOKEN_SORT, 0, M * 16.0 * sort_passes(V), sort_tokens(tokens, M, V, w.sort, st));
+  const int nch = seg_chunks(M);
+  const unsigned nblk8 = rows_grid(M, 8);
+
   for (int l = m->depth - 1; l >= 0; --l) {
     const int pi = 1 + 6 * l;
+    const double attn_bwd_flops = 8.0 * B * H * (double)kHeadDim * attn_keys(T_len, m->layer_window[l]);
     // MLP: x += a W2^T, a = relu(h)^2, h = xn2 W1^T
     NC_TRY(gemm<T>(m, gp(C, F, M, w.dxb, C, 1, w.a[l], F, 1, G(pi + 5), F, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, F, C, w.dxb, C, 0, W.w2[l], F, 1, w.a[l], F, EPI_DRELU2), st));
@@ -324,27 +382,58 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
-           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H, 0,
-                                  m->status, st) != cudaSuccess) return NC_ECUDA);
+           if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
+                                  m->layer_window[l], 0, m->status, st) != cudaSuccess) return NC_ECUDA);
+    if (W.ve[l]) {
+      // v += g ve[tok]:  dg = sum_i dv_i . ve[tok_i];  dve[v] = g sum_{tok_i = v} dv_i
+      const T *dv = w.dqkv + (size_t)(H + 1) * kHeadDim;
+      const int nb = (M + 63) / 64;
+      float *gv = G(m->ve_param[l]);
+      NC_RUN(K_VE_BWD, 0, M * 2.0 * kHeadDim * es,
+             (ve_gate_partial_kernel<T><<<nb, 256, 0, st>>>(dv, ldqkv, tokens, W.ve[l], V, M, w.ve_part)));
+      NC_RUN(K_VE_BWD, 0, nb * 4.0,
+             (ordered_sum_kernel<<<1, 1024, 0, st>>>(w.ve_part, nb, 1.f, G(m->p_gates) + m->ve_slot[l])));
+      if (cudaMemsetAsync(gv, 0, sizeof(float) * (size_t)V * kHeadDim, st) != cudaSuccess) return NC_ECUDA;
+      ValueEmbedRows<T> src{dv, ldqkv, W.gates + m->ve_slot[l]};
+      NC_RUN(K_VE_BWD, 0, M * (kHeadDim * es + 8.0),
+             (segsum_kernel<ValueEmbedRows<T>, 1><<<(nch + 7) / 8, 256, 0, st>>>(
+                 src, w.sort.skey, w.sort.spos, M, kHeadDim, gv, w.seg_head, w.seg_tail, w.seg_flags)));
+      NC_RUN(K_SEG_FIXUP, 0, 0,
+             (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, kHeadDim, w.seg_head, w.seg_tail, w.seg_flags,
+                                                    nch, gv)));
+    }
     NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
            (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     // [q|k|v] = xn [Wq;Wk;Wv]^T
     NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, EPI_STORE_F32), st));
     NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy, C, EPI_STORE), st));
-    NC_RUN(K_RMSNORM_BWD, 0, nbwd,
-           NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
-                                 w.dy, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
+    if (m->scalars) {
+      // block entry: dx_in = dx + norm bwd;  dx = lam_r dx_in;  dx0 += lam_0 dx_in
+      float *pr = w.scal_part + (size_t)l * nblk8, *p0 = w.scal_part + (size_t)(m->depth + l) * nblk8;
+      NC_RUN(K_RMSNORM_BWD, 0, nbwd + M * (8.0 * C + 2.0 * C * es),
+             NC_DISPATCH_NV(C, (rmsnorm_bwd_mix_kernel<T, NV><<<nblk8, 256, 0, st>>>(
+                                   w.dy, w.xn[l], w.r1[l], w.dx, w.dxb, w.xs[l], w.xs[0], W.resid + l, W.x0l + l,
+                                   w.dx0, l == m->depth - 1, pr, p0, M, C))));
+    } else {
+      NC_RUN(K_RMSNORM_BWD, 0, nbwd,
+             NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                                   w.dy, w.xn[l], w.r1[l], w.dx, w.dxb, M, C, 1))));
+    }
+  }
+  if (m->scalars) {
+    // resid_lambdas and x0_lambdas are adjacent in the layout: 2L sums
+    NC_RUN(K_VE_BWD, 0, 2.0 * m->depth * nblk8 * 4.0,
+           (ordered_sum_rows_kernel<<<2 * m->depth, 256, 0, st>>>(w.scal_part, (int)nblk8, G(m->p_resid), 1)));
   }
   // embedding: through the first norm, summed per token over its positions
   // in a fixed order (positions sorted by token; no floating-point atomics)
+  // (with residual scalars the gradient reaching x0 through the mixing, dx0, adds to dx)
   if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
-  NC_RUN(K_TOKEN_SORT, 0, M * 16.0 * sort_passes(V), sort_tokens(tokens, M, V, w.sort, st));
-  const int nch = seg_chunks(M);
-  NC_RUN(K_EMBED_BWD, 0, M * (4.0 * C + C * es + 12.0),
-         NC_DISPATCH_NV(C, (embed_segsum_kernel<T, NV><<<(nch + 7) / 8, 256, 0, st>>>(
-                               w.dx, W.wte, w.r0, w.sort.skey, w.sort.spos, M, C, G(0), w.seg_head, w.seg_tail,
-                               w.seg_flags))));
+  NC_RUN(K_EMBED_BWD, 0, M * (4.0 * C + C * es + 12.0) + (m->scalars ? M * 4.0 * C : 0.0),
+         NC_DISPATCH_NV(C, (segsum_kernel<EmbedRows<T, NV>, NV><<<(nch + 7) / 8, 256, 0, st>>>(
+                               EmbedRows<T, NV>{w.dx, m->scalars ? w.dx0 : nullptr, W.wte, w.r0, C}, w.sort.skey,
+                               w.sort.spos, M, C, G(0), w.seg_head, w.seg_tail, w.seg_flags))));
   NC_RUN(K_SEG_FIXUP, 0, 0,
          (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, C, w.seg_head, w.seg_tail, w.seg_flags, nch, G(0))));
   return NC_OK;
@@ -522,9 +611,14 @@ __global__ void wait_expiry_kernel(uint64_t wait_ns, int *status) {
 extern "C" {
 
 int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
+  return nc_init_ex(depth, vocab, seq, dtype, nullptr, out);
+}
+
+int nc_init_ex(int depth, int vocab, int seq, int dtype, const nc_block_opts *opts, nc_model **out) {
   if (!out) return NC_EINVAL;
   *out = nullptr;
   if (depth < 1 || vocab < 2 || seq < 1) return NC_EINVAL;
+  if (opts && opts->window < 0) return NC_EINVAL;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
   const int C = kHeadDim * ((64 * depth + kHeadDim - 1) / kHeadDim);
   if (C > 32 * kMaxVecPerLane * 8) return NC_EINVAL;  // widest row the row kernels hold
@@ -557,6 +651,36 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out) {
     snprintf(nm, sizeof(nm), "h%d.w2", l); add(nm, C, 4 * C);
   }
   add("lm_head", vocab, C);
+  // full reference block: the "SSSL" window schedule (last layer always
+  // full), value-embedding tables on layers 0, 2, ..., then the scalars
+  m->window = opts ? opts->window : 0;
+  m->ve = opts && opts->value_embeds;
+  m->scalars = opts && opts->resid_scalars;
+  m->layer_window.assign(depth, 0);
+  m->ve_param.assign(depth, -1);
+  m->ve_slot.assign(depth, -1);
+  for (int l = 0; l < depth; ++l) {
+    const char kind = l == depth - 1 ? 'L' : "SSSL"[l % 4];
+    if (kind == 'S') m->layer_window[l] = m->window;
+  }
+  int n_ve = 0;
+  if (m->ve)
+    for (int l = 0; l < depth; l += 2) {
+      snprintf(nm, sizeof(nm), "ve%d", l);
+      m->ve_param[l] = (int)m->params.size();
+      m->ve_slot[l] = n_ve++;
+      add(nm, vocab, kHeadDim);
+    }
+  if (m->scalars) {
+    m->p_resid = (int)m->params.size();
+    add("resid_lambdas", 1, depth);
+    m->p_x0 = (int)m->params.size();
+    add("x0_lambdas", 1, depth);
+  }
+  if (m->ve) {
+    m->p_gates = (int)m->params.size();
+    add("ve_gates", 1, n_ve);
+  }
   m->n_params = off;
 
   // RoPE table: angle = pos * 10000^(-i/64), built in float64, rounded once.
@@ -586,6 +710,18 @@ int nc_get_dims(const nc_model *m, nc_dims *out) {
   out->depth = m->depth; out->width = m->C; out->n_head = m->H; out->head_dim = kHeadDim;
   out->hidden = m->F; out->vocab = m->V; out->seq = m->seq; out->dtype = m->dtype;
   out->n_params = m->n_params;
+  return NC_OK;
+}
+
+int nc_layer_window(const nc_model *m, int layer, int *window) {
+  if (!m || !window || layer < 0 || layer >= m->depth) return NC_EINVAL;
+  *window = m->layer_window[layer];
+  return NC_OK;
+}
+
+int nc_param_count(const nc_model *m, int *count) {
+  if (!m || !count) return NC_EINVAL;
+  *count = (int)m->params.size();
   return NC_OK;
 }
 
@@ -718,10 +854,11 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
-int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
+int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H, int window,
                      int dtype, int engine, void *stream) {
   if (!qkv || !O || !lse) return NC_EINVAL;
   if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if (window < 0) return NC_EINVAL;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
   if (engine < 0 || engine > 1) return NC_EINVAL;
   if (dtype == NC_BF16 && engine == 0 && !fatc::aligned(qkv, ld, O)) return NC_EALIGN;
@@ -730,38 +867,39 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == NC_BF16)
-    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, engine, status, st);
+    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, window, engine, status, st);
   else
-    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, engine, status, st);
+    e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, window, engine, status, st);
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 static int attention_bwd_common(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
-                                float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                                float *Drow, void *dqkv, int B, int T, int H, int window, int dtype, int engine,
                                 int *status, cudaStream_t st) {
   cudaError_t e;
   if (dtype == NC_BF16) {
     e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
-                              (bf16 *)dqkv, B, T, H, engine, status, st);
+                              (bf16 *)dqkv, B, T, H, window, engine, status, st);
   } else {
     e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
-                               (float *)dqkv, B, T, H, engine, status, st);
+                               (float *)dqkv, B, T, H, window, engine, status, st);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
 int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
-                     float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                     float *Drow, void *dqkv, int B, int T, int H, int window, int dtype, int engine,
                      void *stream) {
   if (!qkv || !O || !dO || !lse || !Drow || !dqkv) return NC_EINVAL;
   if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if (window < 0) return NC_EINVAL;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
   if (engine < 0 || engine > 1) return NC_EINVAL;
   if (dtype == NC_BF16 && engine == 0 && !fatc::aligned_bwd(qkv, ld, O, dO, dqkv)) return NC_EALIGN;
   int num_sms = 0, *status = nullptr;
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
-  return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, status,
+  return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, window, dtype, engine, status,
                               (cudaStream_t)stream);
 }
 
@@ -778,7 +916,7 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   SymbolAddrs a;
   if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
-  return attention_bwd_common(qkv, ld, O, dO, lse, a.rowdot, dqkv, B, T, H, dtype, engine, status,
+  return attention_bwd_common(qkv, ld, O, dO, lse, a.rowdot, dqkv, B, T, H, 0, dtype, engine, status,
                               (cudaStream_t)stream);
 }
 

@@ -193,21 +193,86 @@ __device__ __forceinline__ void seg_store_row(float *dst, const float (&acc)[NV]
   }
 }
 
-// Embedding gradient: for position i with token v,
-//   y = wte[v] r0_i,  g_i = r0_i (dx_i - y mean(dx_i y)),  dwte[v] = sum g_i
-// (the backward of x0 = rmsnorm(wte[tok]); rows of tokens that never occur
-// are left as they are: the caller zeroes the table first).
+// Row sources of the segmented sum: load(row, tok, g, lane) leaves in g
+// (8 values per 16-byte unit, units lane, lane + 32, ...) the row whose sum
+// over a token's positions is that token's gradient row.
+//
+// Embedding: for position i with token v,
+//   y = wte[v] r0_i,  g_i = r0_i (d_i - y mean(d_i y)),  d_i = dx_i (+ dx2_i)
+// the backward of x0 = rmsnorm(wte[tok]) (dx2: a second gradient reaching
+// x0, the residual-scalar mixing; may be null).
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) embed_segsum_kernel(
-    const float *__restrict__ dx, const T *__restrict__ wte, const float *__restrict__ r0,
-    const int32_t *__restrict__ skey, const int32_t *__restrict__ spos, int M, int C,
-    float *__restrict__ dwte, float *__restrict__ head, float *__restrict__ tail, int *__restrict__ flags) {
+struct EmbedRows {
+  const float *dx, *dx2;
+  const T *wte;
+  const float *r0;
+  int C;
+  __device__ __forceinline__ void load(int row, int v, float (&g)[NV][8], int lane) const {
+    const int nv = C >> 3;
+    const float r = r0[row];
+    float y[NV][8], dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = lane + 32 * i;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[i][j] = y[i][j] = 0.f;
+      if (c < nv) {
+        Vec8<float>::load(dx + (size_t)row * C + c * 8, g[i]);
+        if (dx2) {
+          float e[8];
+          Vec8<float>::load(dx2 + (size_t)row * C + c * 8, e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) g[i][j] += e[j];
+        }
+        Vec8<T>::load(wte + (size_t)v * C + c * 8, y[i]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          y[i][j] *= r;
+          dot += g[i][j] * y[i][j];
+        }
+      }
+    }
+    dot = warp_sum(dot) / (float)C;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[i][j] = r * (g[i][j] - y[i][j] * dot);
+  }
+};
+
+// Value embedding: v_i += gate ve[tok_i] in the forward, so the table's
+// gradient row of token v is gate * sum of dv_i over its positions; dv_i is
+// the 128-wide v part of row i of dqkv (stride ld).
+template <typename T>
+struct ValueEmbedRows {
+  const T *dv;
+  int64_t ld;
+  const T *gate;
+  __device__ __forceinline__ void load(int row, int, float (&g)[1][8], int lane) const {
+    const float s = to_f(gate[0]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[0][j] = 0.f;
+    if (lane < kHeadDim / 8) {
+      Vec8<T>::load(dv + (size_t)row * ld + lane * 8, g[0]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[0][j] *= s;
+    }
+  }
+};
+
+// out[v] = sum over token v's positions of src rows (C wide), for every
+// token that occurs; rows of other tokens are left as they are (the caller
+// zeroes the table first).
+template <typename Src, int NV>
+__global__ void __launch_bounds__(256) segsum_kernel(Src src, const int32_t *__restrict__ skey,
+                                                     const int32_t *__restrict__ spos, int M, int C,
+                                                     float *__restrict__ out, float *__restrict__ head,
+                                                     float *__restrict__ tail, int *__restrict__ flags) {
   const int lane = threadIdx.x & 31;
   const int chunk = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int p0 = chunk * kSegChunk;
   if (p0 >= M) return;
   const int p1 = min(M, p0 + kSegChunk);
-  const int nv = C >> 3;
   float acc[NV][8];
 #pragma unroll
   for (int i = 0; i < NV; ++i)
@@ -218,7 +283,7 @@ __global__ void __launch_bounds__(256) embed_segsum_kernel(
     const bool starts = a == 0 || skey[a - 1] != tok;
     const bool ends = b == M || skey[b] != tok;
     if (starts && ends) {
-      seg_store_row<NV>(dwte + (size_t)tok * C, acc, C, lane);
+      seg_store_row<NV>(out + (size_t)tok * C, acc, C, lane);
     } else if (!starts) {  // the chunk's first run, continuing a segment
       seg_store_row<NV>(head + (size_t)chunk * C, acc, C, lane);
       fl |= kSegHead | (ends ? kSegHeadEnds : 0);
@@ -238,29 +303,12 @@ __global__ void __launch_bounds__(256) embed_segsum_kernel(
       run0 = p;
       tok = v;
     }
-    const int row = spos[p];
-    const float r = r0[row];
-    float g[NV][8], y[NV][8], dot = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int c = lane + 32 * i;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) g[i][j] = y[i][j] = 0.f;
-      if (c < nv) {
-        Vec8<float>::load(dx + (size_t)row * C + c * 8, g[i]);
-        Vec8<T>::load(wte + (size_t)v * C + c * 8, y[i]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          y[i][j] *= r;
-          dot += g[i][j] * y[i][j];
-        }
-      }
-    }
-    dot = warp_sum(dot) / (float)C;
+    float g[NV][8];
+    src.load(spos[p], v, g, lane);
 #pragma unroll
     for (int i = 0; i < NV; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] += r * (g[i][j] - y[i][j] * dot);
+      for (int j = 0; j < 8; ++j) acc[i][j] += g[i][j];
   }
   emit(run0, p1);
   if (lane == 0) flags[chunk] = fl;
@@ -296,6 +344,17 @@ __global__ void __launch_bounds__(256) seg_fixup_kernel(const int32_t *__restric
     }
     reinterpret_cast<float4 *>(out + (size_t)tok * C)[q] = a;
   }
+}
+
+// Deterministic sum of n partial values by one CTA: each thread adds a
+// fixed strided subset in order, then a fixed tree; *out = scale * sum.
+__global__ void __launch_bounds__(1024) ordered_sum_kernel(const float *__restrict__ partial, int n, float scale,
+                                                           float *__restrict__ out) {
+  __shared__ float sh[32];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += partial[i];
+  s = block_sum(s, sh);
+  if (threadIdx.x == 0) *out = scale * s;
 }
 
 }  // namespace nc

@@ -11,17 +11,26 @@ class Model:
     """One nanochat decoder of the given depth (one dial: width = depth*64,
     heads = width/128) on the current CUDA device."""
 
-    def __init__(self, depth: int, vocab: int = 65536, seq: int = 2048, dtype: str = "bf16"):
+    def __init__(self, depth: int, vocab: int = 65536, seq: int = 2048, dtype: str = "bf16",
+                 window: int = 0, value_embeds: bool = False, resid_scalars: bool = False):
+        """window / value_embeds / resid_scalars: the full reference block's
+        options (sliding-window "SSSL" layers, gated value embeddings,
+        residual scalars); all off is the baseline decoder."""
         self.dtype_code = B.NC_BF16 if dtype == "bf16" else B.NC_F32
         self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
-        rc, self.handle = B.nc_init(depth, vocab, seq, self.dtype_code)
+        rc, self.handle = B.nc_init_ex(depth, vocab, seq, self.dtype_code, window, value_embeds,
+                                       resid_scalars)
         if rc != B.NC_OK:
-            raise B.NcError(rc, "nc_init")
+            raise B.NcError(rc, "nc_init_ex")
         rc, self.dims = B.nc_get_dims(self.handle)
         if rc != B.NC_OK:
             raise B.NcError(rc, "nc_get_dims")
+        rc, n = B.nc_param_count(self.handle)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_param_count")
+        self.windows = [B.nc_layer_window(self.handle, l)[1] for l in range(depth)]
         self.layout = []
-        for i in range(2 + 6 * depth):
+        for i in range(n):
             rc, p = B.nc_param_layout(self.handle, i)
             if rc != B.NC_OK:
                 raise B.NcError(rc, "nc_param_layout")

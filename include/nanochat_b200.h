@@ -80,7 +80,7 @@ typedef struct {
 } nc_dims;
 
 typedef struct {
-  char name[24];    /* "wte", "h<l>.wq", ..., "lm_head" */
+  char name[24];    /* "wte", "h<l>.wq", ..., "lm_head", then the full block's extras */
   int64_t offset;   /* element offset in the flat weight / gradient buffer */
   int rows, cols;
 } nc_param;
@@ -95,8 +95,44 @@ int nc_init(int depth, int vocab, int seq, int dtype, nc_model **out);
 /* Shapes of the model. */
 int nc_get_dims(const nc_model *m, nc_dims *out);
 
-/* Name, offset and shape of weight tensor `index`, 0 <= index < 2 + 6*depth,
- * in storage order. */
+/* The full reference block's departures from the baseline decoder, all off
+ * by default ("Nanochat: full-stack LLM training in 8,000 lines for $72",
+ * section "A Llama-class transformer with ten modern departures";
+ * "nanochat - full-stack ChatGPT in ~8k lines", section "0. The model"):
+ *   window         > 0: sliding-window attention on the schedule "SSSL" --
+ *                  layer l is "SSSL"[l % 4] and the last layer is "L"; an "S"
+ *                  layer lets query i see keys j with 0 <= i - j < window
+ *                  (the pages: 1,024), an "L" layer the plain causal context
+ *   value_embeds   != 0: a gated value-embedding table [vocab, 128] on
+ *                  layers 0, 2, 4, ...: v += g_l * ve_l[token] before
+ *                  attention, g_l one learnable scalar per such layer (the
+ *                  pages name the gate without its form: this scalar is a
+ *                  reading)
+ *   resid_scalars  != 0: at every block entry the stream becomes
+ *                  resid_lambdas[l] * x + x0_lambdas[l] * x0, x0 the
+ *                  normalised embedding (the pages' initial values: 1.0, 0.1)
+ * The extra tensors follow lm_head in the layout, in this order: ve<l> for
+ * each value-embedding layer, resid_lambdas [1, L], x0_lambdas [1, L],
+ * ve_gates [1, number of value-embedding layers]. */
+typedef struct {
+  int window;
+  int value_embeds;
+  int resid_scalars;
+} nc_block_opts;
+
+/* nc_init with the full reference block's options (opts == NULL: none,
+ * the same model as nc_init).  window < 0 is NC_EINVAL. */
+int nc_init_ex(int depth, int vocab, int seq, int dtype, const nc_block_opts *opts, nc_model **out);
+
+/* Keys a query of layer `layer` sees: the window of an "S" layer, or 0 for
+ * the plain causal mask. */
+int nc_layer_window(const nc_model *m, int layer, int *window);
+
+/* Number of weight tensors: 2 + 6*depth, plus the full block's extras. */
+int nc_param_count(const nc_model *m, int *count);
+
+/* Name, offset and shape of weight tensor `index`, 0 <= index <
+ * nc_param_count(), in storage order. */
 int nc_param_layout(const nc_model *m, int index, nc_param *out);
 
 /* Bytes of device workspace that nc_fwd_bwd / nc_fwd need for B rows of T

@@ -57,22 +57,26 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
 
 /* Causal multi-query attention forward (energyai.berlin page, "Multi-Query
  * Attention (MQA)": one key/value head shared by the H query heads).
- *   qkv  device [B*T, ld] rows [q (H*128) | k (128) | v (128)],
- *        128*(H+2) <= ld <= INT_MAX, else NC_ESHAPE
- *   O    device [B*T, H*128]: O_h = softmax(q_h k^T / sqrt(128) + causal) v
- *   lse  device fp32 [B, H, T]: log-sum-exp of each score row
+ *   qkv     device [B*T, ld] rows [q (H*128) | k (128) | v (128)],
+ *           128*(H+2) <= ld <= INT_MAX, else NC_ESHAPE
+ *   O       device [B*T, H*128]: O_h = softmax(q_h k^T / sqrt(128) + mask) v
+ *   lse     device fp32 [B, H, T]: log-sum-exp of each score row
+ *   window  0: the causal mask (key j <= query i); > 0: a sliding window,
+ *           0 <= i - j < window ("ten modern departures": the short-window
+ *           layers of the SSSL schedule); < 0: NC_EINVAL
  * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores, which
  * need 16-byte aligned qkv and O and ld % 8 == 0, else NC_EALIGN; fp32: CUDA
  * cores), 1 = the CUDA-core kernel (a test engine for either dtype). */
-int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H,
+int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H, int window,
                      int dtype, int engine, void *stream);
 
 /* Its backward.  dO [B*T, H*128] and O as above, lse from the forward.
  *   Drow  device fp32 [B, H, T] scratch, receives rowsum(dO * O)
  *   dqkv  device [B*T, ld]: dq per head; dk, dv summed over the query heads
- * Engines and errors as nc_attention_fwd (dO and dqkv 16-byte aligned too). */
+ * window, engines and errors as nc_attention_fwd (dO and dqkv 16-byte
+ * aligned too). */
 int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
-                     float *Drow, void *dqkv, int B, int T, int H, int dtype, int engine,
+                     float *Drow, void *dqkv, int B, int T, int H, int window, int dtype, int engine,
                      void *stream);
 
 /* Largest B*H*T that nc_attention_bwd_noalloc accepts: the number of fp32
@@ -80,7 +84,7 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
 #define NC_ATTN_BWD_NOALLOC_MAX_ROWS (1 << 20)
 
 /* nc_attention_bwd for callers that cannot allocate device memory: the same
- * computation and arguments minus Drow.  No passage of the nanochat pages
+ * computation (causal mask, window 0) and arguments minus Drow and window.  No passage of the nanochat pages
  * corresponds to this entry point; it exists for the library's users.
  *
  * Who needs it: code that must not call cudaMalloc or any allocating routine

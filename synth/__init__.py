@@ -147,14 +147,17 @@ def init_std(name: str, rows: int, cols: int) -> float:
     return 1.0 / math.sqrt(cols)
 
 
-def make_weights(layout, seed: int, dtype: str, std_override: dict | None = None, want_f64: bool = True):
+def make_weights(layout, seed: int, dtype: str, std_override: dict | None = None, want_f64: bool = True,
+                 values: dict | None = None):
     """Draw every tensor of `layout` (a list of (name, rows, cols)).
 
     Returns (flat, f64) where `flat` is the storage a device buffer receives
     (float32, or uint16 bf16 bits) in layout order, and `f64` maps each name to
     the float64 value of exactly what was stored (empty if not want_f64).
     Work is split into independent (tensor, chunk) jobs run by a thread pool;
-    every element is computed the same way whatever the split.
+    every element is computed the same way whatever the split.  `values`
+    maps a tensor name to fixed values (an array of its shape) stored instead
+    of a draw, rounded like the draws.
     """
     from concurrent.futures import ThreadPoolExecutor
     std_override = std_override or {}
@@ -187,7 +190,31 @@ def make_weights(layout, seed: int, dtype: str, std_override: dict | None = None
 
     with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
         list(ex.map(run, jobs))
+    off = 0
+    for name, rows, cols in layout:
+        n = rows * cols
+        if values and name in values:
+            w32 = np.asarray(values[name], dtype=np.float64).reshape(-1).astype(np.float32)
+            assert w32.size == n, name
+            if dtype == "f32":
+                flat[off:off + n] = w32
+                if want_f64:
+                    f64[name] = w32.astype(np.float64).reshape(rows, cols)
+            else:
+                bits = f32_to_bf16_bits(w32)
+                flat[off:off + n] = bits
+                if want_f64:
+                    f64[name] = bf16_bits_to_f64(bits).reshape(rows, cols)
+        off += n
     return flat, f64
+
+
+def full_block_values(depth: int, n_ve: int, resid: float = 1.0, x0: float = 0.1, gate: float = 1.0) -> dict:
+    """Values of the full block's scalars: the pages' initial resid_lambdas
+    (1.0) and x0_lambdas (0.1); the value-embedding gate has no initial value
+    on the pages (1.0 here)."""
+    return {"resid_lambdas": np.full((1, depth), resid), "x0_lambdas": np.full((1, depth), x0),
+            "ve_gates": np.full((1, n_ve), gate)}
 
 
 # ---------------------------------------------------------------------------

@@ -114,3 +114,11 @@ def test_op_status_without_a_gpu_fails_cleanly(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert nc.nc_ops_status(None, 10) == nc.NC_ECUDA
+
+
+def test_init_ex_rejects_bad_options(lib):
+    # checked on the host before any device call
+    assert nc.nc_init_ex(4, 65536, 2048, nc.NC_BF16, window=-1)[0] == nc.NC_EINVAL
+    assert nc.nc_init_ex(0, 65536, 2048, nc.NC_BF16, window=64)[0] == nc.NC_EINVAL
+    assert nc.nc_layer_window(None, 0)[0] == nc.NC_EINVAL
+    assert nc.nc_param_count(None)[0] == nc.NC_EINVAL

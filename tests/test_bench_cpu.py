@@ -45,3 +45,14 @@ def test_mufu_fraction():
     bound_ms = 2.0 * 65536 * 32768 / (16 * 148 * 1485e6) * 1e3
     assert bench.mufu_fraction(bound_ms, 32768, 65536, 148, 1485.0) == pytest.approx(1.0)
     assert bench.mufu_fraction(2 * bound_ms, 32768, 65536, 148, 1485.0) == pytest.approx(0.5)
+
+
+def test_window_flop_count():
+    import bench
+    # no window, or windows covering T, give the causal count
+    base = bench.model_flops_per_token(20, 1280, 65536, 2048)
+    assert bench.model_flops_per_token(20, 1280, 65536, 2048, [0] * 20) == base
+    assert bench.model_flops_per_token(20, 1280, 65536, 2048, [2048] * 20) == base
+    # a window of w keys: w - w^2/(2T) pairs per query instead of T/2
+    one = bench.model_flops_per_token(1, 1280, 65536, 2048, [1024]) - bench.model_flops_per_token(1, 1280, 65536, 2048, [0])
+    assert abs(one - 12.0 * 1280 * (1024 - 1024 ** 2 / 4096 - 1024)) < 1e-6

@@ -236,3 +236,79 @@ def test_misaligned_bf16_operands_are_rejected(nc):
     assert nc.nc_gemm(p, 100, 0, p, 128, 0, p + 4096, 128, 64, 64, 100, nc.NC_BF16, nc.NC_EPI_STORE, 1,
                       st) == nc.NC_OK
     assert nc.nc_ops_status(st, 60000) == nc.NC_OK
+
+
+WINDOW_CASES = [(1, 515, 3, 1), (1, 515, 3, 64), (2, 256, 2, 129), (1, 300, 10, 200), (1, 1030, 2, 384),
+                (2, 130, 1, 128)]
+
+
+@pytest.mark.parametrize("B,T,H,window", WINDOW_CASES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("engine", [0, 1])
+def test_windowed_attention_fwd_bwd(nc, B, T, H, window, dtype, engine):
+    # sliding window (query i sees keys j with 0 <= i - j < window) against the
+    # full-block oracle's windowed attention
+    import torch
+
+    from oracle import full_block as fb
+    code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
+    qkv, ld, q, k, v = _attn_inputs(B, T, H, 300 + T + H + window, dtype)
+    st = torch.cuda.current_stream().cuda_stream
+    qkv_d = _dev(qkv, dtype)
+    O = torch.zeros(B * T, H * 128, dtype=qkv_d.dtype, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    assert nc.nc_attention_fwd(qkv_d.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, code, engine, st,
+                               window=window) == 0
+    O_ref = np.empty((B, T, H, 128))
+    for b in range(B):
+        O_ref[b], _ = fb.attention(q[b], k[b], v[b], window)
+    got_O = O.float().cpu().numpy().reshape(B, T, H, 128)
+    tolO = 1e-5 if dtype == "f32" else 1.5e-2
+    np.testing.assert_allclose(got_O, O_ref, rtol=0, atol=tolO * np.abs(O_ref).max())
+    if window == 1:
+        # one key: O = v of the query's own position, lse = q.k / sqrt(d)
+        np.testing.assert_allclose(got_O, np.broadcast_to(v[:, :, None, :], got_O.shape), rtol=0,
+                                   atol=tolO * np.abs(v).max())
+    dO = synth.normal(9 + T, 4, B * T * H * 128).reshape(B * T, H * 128)
+    dO = _bf16(dO) if dtype == "bf16" else dO.astype(np.float32).astype(np.float64)
+    dO_d = _dev(dO, dtype)
+    Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    dqkv = torch.zeros(B * T, ld, dtype=qkv_d.dtype, device="cuda")
+    assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
+                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine, st, window=window) == 0
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK
+    got = dqkv.float().cpu().numpy().astype(np.float64)
+    refs = [np.empty((B, T, H, 128)), np.empty((B, T, 128)), np.empty((B, T, 128))]
+    for b in range(B):
+        refs[0][b], refs[1][b], refs[2][b] = fb.attention_bwd(dO.reshape(B, T, H, 128)[b], q[b], k[b], v[b], window)
+    parts = [(got[:, :H * 128], refs[0].reshape(B * T, -1)), (got[:, H * 128:H * 128 + 128], refs[1].reshape(B * T, -1)),
+             (got[:, H * 128 + 128:], refs[2].reshape(B * T, -1))]
+    for i, (g, r) in enumerate(parts):
+        scale = np.abs(r).max()
+        if window == 1 and i < 2:
+            assert np.max(np.abs(g)) <= 1e-6  # one key per query: softmax constant, dq = dk = 0
+            continue
+        if dtype == "f32":
+            np.testing.assert_allclose(g, r, rtol=0, atol=1e-4 * scale)
+        else:
+            cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
+            assert cos > 0.9995, cos
+            assert np.max(np.abs(g - r)) <= 3e-2 * scale
+
+
+def test_window_covering_the_context_is_the_causal_kernel(nc):
+    # window >= T is the plain causal mask: bit-identical to window 0
+    import torch
+    B, T, H = 1, 300, 2
+    qkv, ld, q, k, v = _attn_inputs(B, T, H, 77, "bf16")
+    st = torch.cuda.current_stream().cuda_stream
+    qkv_d = _dev(qkv, "bf16")
+    outs = []
+    for window in (0, T, T + 5):
+        O = torch.zeros(B * T, H * 128, dtype=torch.bfloat16, device="cuda")
+        lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+        assert nc.nc_attention_fwd(qkv_d.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16, 0, st,
+                                   window=window) == 0
+        outs.append((O.view(torch.int16).cpu(), lse.cpu()))
+    for O, lse in outs[1:]:
+        assert torch.equal(O, outs[0][0]) and torch.equal(lse, outs[0][1])
