@@ -26,6 +26,16 @@ BF16_LOSS_ABS = 1e-2         # |dloss|
 BF16_GRAD_COS = 0.999        # per tensor cosine similarity
 
 
+def token_loss_bound(w_out) -> float:
+    """Bound on |per-token loss (bf16 model) - oracle|: a logit z_v = xf . w_v
+    moves by at most u |xf| |w_v| when xf carries a relative error u (one
+    bf16 rounding, u = 2^-8) in the 2-norm, |xf| = sqrt(C) after the final
+    norm; the softcap's slope is at most 1, and a token's loss
+    logsumexp(s) - s_target moves by at most twice the largest logit change."""
+    C = w_out.shape[1]
+    return 2.0 * 2.0 ** -8 * np.sqrt(C) * float(np.linalg.norm(w_out, axis=1).max())
+
+
 def to_device(flat: np.ndarray, dtype: str):
     import torch
     if dtype == "f32":
@@ -67,7 +77,7 @@ def cosine(a, b):
     return float(np.sum(a * b) / (na * nb))
 
 
-def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_ref=None, tag=""):
+def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_ref=None, tag="", tl_bound=None):
     """Assert the precision's tolerances; return a per-tensor report."""
     g_gpu = split_grads(g_gpu_flat, lay)
     report = {}
@@ -97,5 +107,8 @@ def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_r
             report[name] = c
             assert c >= BF16_GRAD_COS, (name, c)
         if tl_gpu is not None:
-            assert np.max(np.abs(tl_gpu - tl_ref)) <= 0.05
+            # tl_bound: token_loss_bound(lm_head); the mean error is far below the worst case
+            d = np.abs(tl_gpu - tl_ref)
+            assert tl_bound is not None
+            assert d.max() <= tl_bound and d.mean() <= tl_bound / 4, (d.max(), d.mean(), tl_bound)
     return report

@@ -19,7 +19,7 @@ import pytest
 import oracle
 import synth
 from oracle import full_block as fb
-from tests._gpu_helpers import compare, gpu_step, split_grads
+from tests._gpu_helpers import compare, gpu_step, split_grads, token_loss_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -84,7 +84,8 @@ def test_full_block_step_matches_oracle(torch_cuda, depth, V, B, T, dtype, seed,
     assert rc == 0
     loss_ref, tl_ref, g_ref = fb.loss_and_grads(W, tok, tgt, depth, windows=windows)
     compare(dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref,
-            tag=f"full-d{depth}-V{V}-B{B}-T{T}-{dtype}-w{window}-ve{int(ve)}-s{int(scalars)}")
+            tag=f"full-d{depth}-V{V}-B{B}-T{T}-{dtype}-w{window}-ve{int(ve)}-s{int(scalars)}",
+            tl_bound=token_loss_bound(W["lm_head"]))
     G = split_grads(g, lay)
     if ve:
         # rows of tokens that never occur get no value-embedding gradient

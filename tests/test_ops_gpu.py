@@ -100,6 +100,10 @@ def test_gemm_bf16(nc, M, N, K, a_mn, b_mn, pad, epi, engine):
     B_dev = _dev(Bs, "bf16")
     rc = nc.nc_gemm(A_dev.data_ptr(), lda, a_mn, B_dev.data_ptr(), ldb, b_mn, D.data_ptr(), ldd,
                     M, N, K, nc.NC_BF16, code, engine, torch.cuda.current_stream().cuda_stream)
+    if engine != 1 and (lda % 8 or ldb % 8 or (ldd % (4 if epi == "STORE_F32" else 8))):
+        # the tensor-core engines take 16-byte row strides only: an error, not a slower path
+        assert rc == nc.NC_EALIGN
+        return
     assert rc == 0
     torch.cuda.synchronize()
     got = D.float().cpu().numpy().astype(np.float64)

@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import synth
-from tests._gpu_helpers import compare, cosine, gpu_step, make_case, split_grads, to_device
+from tests._gpu_helpers import compare, cosine, gpu_step, make_case, split_grads, to_device, token_loss_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +59,8 @@ def test_step_matches_oracle(torch_cuda, depth, V, B, T, dtype, seed, dist, hstd
     rc, loss, tl, g = gpu_step(model, flat, tok, tgt, dtype)
     assert rc == 0
     loss_ref, tl_ref, g_ref = oracle.loss_and_grads(W, tok, tgt, depth)
-    compare(dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref, tag=f"d{depth}-V{V}-B{B}-T{T}-{dtype}")
+    compare(dtype, lay, loss, g, loss_ref, g_ref, tl, tl_ref, tag=f"d{depth}-V{V}-B{B}-T{T}-{dtype}",
+            tl_bound=token_loss_bound(W["lm_head"]))
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
