@@ -274,7 +274,9 @@ def config_dict(wl, n_gpus, sample=None, full_block=False):
                      f"{64 * wl.depth // 128} query heads x128 + 1 shared KV head, "
                      f"MLP {256 * wl.depth}, vocab {wl.vocab}, B={wl.B} x T={wl.T} per GPU, "
                      f"{wl.tokens} tokens, {wl.dtype}"),
-        "global_batch": wl.B * n_gpus, "seq_len": wl.T, "parallelism": f"dp{n_gpus} (independent shards)",
+        "global_batch": wl.B * n_gpus, "seq_len": wl.T,
+        "parallelism": (f"dp{n_gpus}: NCCL all-reduce (mean) of the gradient buckets, overlapped with the backward"
+                        if n_gpus > 1 else "dp1"),
         "l2": "inputs larger than L2 (activations and logits ~20 GB per GPU)",
     }
     if sample:
@@ -328,8 +330,17 @@ def run_ours(args):
     model.workspace(wl.B, wl.T)
     stream = torch.cuda.current_stream()
 
-    def step():
-        model.fwd_bwd(weights, tokens, targets, grads=grads, loss=loss)
+    if world > 1:
+        # data parallel: the ranks' gradients are averaged by NCCL all-reduces of
+        # the gradient buckets, each started as soon as the backward finishes it
+        from decoder_only_transformer_nanochat_b200.dp import DataParallel
+        dpar = DataParallel(model)
+
+        def step():
+            dpar.step(weights, tokens, targets, grads, loss)
+    else:
+        def step():
+            model.fwd_bwd(weights, tokens, targets, grads=grads, loss=loss)
 
     for _ in range(args.warmup):
         step()
@@ -386,7 +397,10 @@ def run_ours(args):
     def e2e_step():
         tok_d.copy_(tok_h, non_blocking=True)
         tgt_d.copy_(tgt_h, non_blocking=True)
-        model.fwd_bwd(weights, tok_d, tgt_d, grads=grads, loss=loss)
+        if world > 1:
+            dpar.step(weights, tok_d, tgt_d, grads, loss)
+        else:
+            model.fwd_bwd(weights, tok_d, tgt_d, grads=grads, loss=loss)
         loss_h.copy_(loss, non_blocking=True)
 
     e2e_step()
@@ -404,6 +418,8 @@ def run_ours(args):
     e2e_value = job_rate(tokens_per_step, e2e_ms, world)
     loss_val = float(loss_h.item())
 
+    if world > 1:
+        dpar.close()
     if rank != 0:
         if world > 1:
             import torch.distributed as dist

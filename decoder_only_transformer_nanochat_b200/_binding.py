@@ -27,6 +27,8 @@ NC_EALIGN = 9
 NC_F32 = 0
 NC_BF16 = 1
 
+NC_ACCUMULATE = 1
+
 
 class NcError(RuntimeError):
     def __init__(self, code: int, where: str = ""):
@@ -74,6 +76,10 @@ _SIGS = {
     "nc_init_ex": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(_P)]),
     "nc_layer_window": (_I, [_P, _I, ctypes.POINTER(_I)]),
     "nc_param_count": (_I, [_P, ctypes.POINTER(_I)]),
+    "nc_fwd_bwd_ex": (_I, [_P, _P, _P, _P, _I, _I, _P, ctypes.c_size_t, _P, _P, _P, _I, _P]),
+    "nc_grad_bucket_count": (_I, [_P, ctypes.POINTER(_I)]),
+    "nc_grad_bucket": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
+    "nc_set_grad_events": (_I, [_P, ctypes.POINTER(_P), _I]),
     "nc_ops_status": (_I, [_P, _I]),
     "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
@@ -158,6 +164,35 @@ def nc_fwd_bwd(handle, weights, tokens, targets, B, T, workspace, ws_bytes, loss
                grads, stream):
     return load_library().nc_fwd_bwd(handle, weights, tokens, targets, B, T, workspace, ws_bytes,
                                      loss, token_loss, grads, stream)
+
+
+def nc_fwd_bwd_ex(handle, weights, tokens, targets, B, T, workspace, ws_bytes, loss, token_loss,
+                  grads, flags, stream):
+    return load_library().nc_fwd_bwd_ex(handle, weights, tokens, targets, B, T, workspace, ws_bytes,
+                                        loss, token_loss, grads, flags, stream)
+
+
+def nc_grad_buckets(handle):
+    """Returns (status, [(offset, count), ...]) in the order the backward finishes them."""
+    lib = load_library()
+    n = _I()
+    rc = lib.nc_grad_bucket_count(handle, ctypes.byref(n))
+    if rc != NC_OK:
+        return rc, []
+    out = []
+    for k in range(n.value):
+        o, c = ctypes.c_int64(), ctypes.c_int64()
+        rc = lib.nc_grad_bucket(handle, k, ctypes.byref(o), ctypes.byref(c))
+        if rc != NC_OK:
+            return rc, []
+        out.append((o.value, c.value))
+    return NC_OK, out
+
+
+def nc_set_grad_events(handle, events) -> int:
+    """events: raw cudaEvent_t handles (ints), one per bucket (or fewer)."""
+    arr = (_P * max(1, len(events)))(*[_P(e) for e in events])
+    return load_library().nc_set_grad_events(handle, arr, len(events))
 
 
 def nc_fwd(handle, weights, tokens, B, T, workspace, ws_bytes, logits, stream):

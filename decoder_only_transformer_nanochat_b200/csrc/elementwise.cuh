@@ -443,15 +443,17 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_mix_kernel(
   }
 }
 
-// out[row * out_stride] = sum of partial[row * n .. row * n + n) in a fixed order.
+// out[row * out_stride] (+)= sum of partial[row * n .. row * n + n) in a fixed order.
 __global__ void __launch_bounds__(256) ordered_sum_rows_kernel(const float *__restrict__ partial, int n,
-                                                               float *__restrict__ out, int out_stride) {
+                                                               float *__restrict__ out, int out_stride,
+                                                               int accumulate) {
   __shared__ float sh[32];
   const float *p = partial + (size_t)blockIdx.x * n;
   float s = 0.f;
   for (int i = threadIdx.x; i < n; i += blockDim.x) s += p[i];
   s = block_sum(s, sh);
-  if (threadIdx.x == 0) out[(size_t)blockIdx.x * out_stride] = s;
+  float *o = out + (size_t)blockIdx.x * out_stride;
+  if (threadIdx.x == 0) *o = s + (accumulate ? *o : 0.f);
 }
 
 // Value-embedding gate gradient, first stage: partial[block] = sum over the

@@ -18,8 +18,12 @@ enum Epilogue : int {
   EPI_RELU2 = 3,      // D = relu(acc)^2              (MLP activation, D in T)
   EPI_DRELU2 = 4,     // D = acc * 2 sqrt(D)          (relu^2 backward: D holds a = relu(h)^2,
                       //                               so relu(h) = sqrt(a); D in T)
-  EPI_SOFTCAP = 5     // D = 15 tanh(acc / 15)        (softcapped logits, D in T)
+  EPI_SOFTCAP = 5,    // D = 15 tanh(acc / 15)        (softcapped logits, D in T)
+  EPI_ACC_F32 = 6     // D = D + acc                  (D in fp32: gradient accumulation)
 };
+
+// Epilogues whose output D is fp32.
+__host__ __device__ inline bool epi_f32(int epi) { return epi == EPI_STORE_F32 || epi == EPI_ACC_F32; }
 
 struct GemmProblem {
   int M, N, K;
@@ -51,6 +55,10 @@ template <typename T>
 __device__ __forceinline__ void epi_apply(int epi, float acc, void *D, size_t idx) {
   if (epi == EPI_STORE_F32) {
     reinterpret_cast<float *>(D)[idx] = acc;
+    return;
+  }
+  if (epi == EPI_ACC_F32) {
+    reinterpret_cast<float *>(D)[idx] += acc;
     return;
   }
   T *d = reinterpret_cast<T *>(D);

@@ -89,7 +89,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params &p, int m, int n, co
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if (p.epi == EPI_STORE_F32) {
+  if (epi_f32(p.epi)) {
     float *d = reinterpret_cast<float *>(p.D) + (size_t)m * p.ldd + n;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int r = quarter * 32 + lane;  // tile row owned by this thread
     const bool leader = warp == 2 && lane == 0;  // issues the epilogue's TMA copies
-    const bool f32_out = p.epi == EPI_STORE_F32;
+    const bool f32_out = epi_f32(p.epi);
     const bool aux = p.epi == EPI_ADD || p.epi == EPI_DRELU2;
     const uint32_t st_addr = smem_u32(staging);
     int acc = 0;
@@ -585,7 +585,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const bool ep_leader = warp == 2 && lane == 0;
-    const bool f32_out = p.epi == EPI_STORE_F32;
+    const bool f32_out = epi_f32(p.epi);
     const bool aux = p.epi == EPI_ADD || p.epi == EPI_DRELU2;
     const uint32_t st_addr = smem_u32(staging);
     int acc = 0;
@@ -729,7 +729,7 @@ inline bool tc_gemm_aligned(const GemmProblem &p) {
   if (p.M < 1 || p.N < 1 || p.K < 1) return false;
   if ((p.lda % 8) || (p.ldb % 8)) return false;
   if (((uintptr_t)p.A & 15) || ((uintptr_t)p.B & 15) || ((uintptr_t)p.D & 15)) return false;
-  if (p.epi == EPI_STORE_F32 ? (p.ldd % 4) : (p.ldd % 8)) return false;
+  if (epi_f32(p.epi) ? (p.ldd % 4) : (p.ldd % 8)) return false;
   return true;
 }
 
@@ -754,14 +754,14 @@ inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status
   else ok = make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 64);
   if (!ok) return cudaErrorInvalidValue;
   CUtensorMap md = ma;  // fp32 outputs are written directly; the map is unused
-  if (g.epi != EPI_STORE_F32 && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
+  if (!epi_f32(g.epi) && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
   Params p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.n_m = (g.M + BM - 1) / BM;
   p.n_n = (g.N + BN - 1) / BN;
   p.kblocks = (g.K + BK - 1) / BK;
   const int tiles = p.n_m * p.n_n;
-  p.splits = g.epi == EPI_STORE_F32 ? choose_splits(tiles, p.kblocks, num_sms) : 1;
+  p.splits = epi_f32(g.epi) ? choose_splits(tiles, p.kblocks, num_sms) : 1;
   {
     // every split must own at least one k-block
     const int per = (p.kblocks + p.splits - 1) / p.splits;
@@ -770,9 +770,10 @@ inline cudaError_t launch_gemm_tc(const GemmProblem &g, int num_sms, int *status
   p.units = tiles * p.splits;
   p.a_mn = g.a_mn; p.b_mn = g.b_mn;
   p.D = g.D; p.ldd = g.ldd; p.epi = g.epi;
-  p.atomic_out = p.splits > 1;
+  // split-K partial sums, and accumulation into an existing D, add with red.global.add
+  p.atomic_out = p.splits > 1 || g.epi == EPI_ACC_F32;
   p.status = status;
-  if (p.atomic_out) {
+  if (p.splits > 1 && g.epi == EPI_STORE_F32) {
     // fp32 partial sums are added into a zeroed output
     cudaError_t e = cudaMemset2DAsync(g.D, (size_t)g.ldd * 4, 0, (size_t)g.N * 4, (size_t)g.M, st);
     if (e != cudaSuccess) return e;
@@ -797,7 +798,7 @@ inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *statu
   else ok = make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 64);
   if (!ok) return cudaErrorInvalidValue;
   CUtensorMap md = ma;
-  if (g.epi != EPI_STORE_F32 && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
+  if (!epi_f32(g.epi) && !make_map(&md, g.D, g.M, g.N, g.ldd, 64, BM)) return cudaErrorInvalidValue;
   Params p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.n_m = (g.M + 255) / 256;
@@ -805,7 +806,7 @@ inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *statu
   p.kblocks = (g.K + BK - 1) / BK;
   const int n_clusters = num_sms / 2;
   const int tiles = p.n_m * p.n_n;
-  p.splits = g.epi == EPI_STORE_F32 ? choose_splits(tiles, p.kblocks, n_clusters) : 1;
+  p.splits = epi_f32(g.epi) ? choose_splits(tiles, p.kblocks, n_clusters) : 1;
   {
     const int per = (p.kblocks + p.splits - 1) / p.splits;
     p.splits = (p.kblocks + per - 1) / per;
@@ -813,9 +814,10 @@ inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *statu
   p.units = tiles * p.splits;
   p.a_mn = g.a_mn; p.b_mn = g.b_mn;
   p.D = g.D; p.ldd = g.ldd; p.epi = g.epi;
-  p.atomic_out = p.splits > 1;
+  // split-K partial sums, and accumulation into an existing D, add with red.global.add
+  p.atomic_out = p.splits > 1 || g.epi == EPI_ACC_F32;
   p.status = status;
-  if (p.atomic_out) {
+  if (p.splits > 1 && g.epi == EPI_STORE_F32) {
     cudaError_t e = cudaMemset2DAsync(g.D, (size_t)g.ldd * 4, 0, (size_t)g.N * 4, (size_t)g.M, st);
     if (e != cudaSuccess) return e;
   }

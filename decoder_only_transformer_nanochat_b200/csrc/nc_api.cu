@@ -52,6 +52,10 @@ struct nc_model {
   std::vector<int> ve_param;      // per layer: param index of its value-embedding table, or -1
   std::vector<int> ve_slot;       // per layer: its entry of ve_gates, or -1
   int p_resid = -1, p_x0 = -1, p_gates = -1;
+  // gradient buckets in the order the backward completes them, and the
+  // caller's events recorded when each one is final (nc_set_grad_events)
+  std::vector<std::pair<int64_t, int64_t>> buckets;  // (offset, count) in elements
+  std::vector<cudaEvent_t> grad_events;
   int device;
   int num_sms;
   float *rope_cos;  // [seq, 64] fp32
@@ -329,10 +333,21 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
   return NC_OK;
 }
 
+// Record the caller's event of gradient bucket k (if set) on the step's stream.
+inline int bucket_done(nc_model *m, int k, cudaStream_t st) {
+  if (k < (int)m->grad_events.size() && m->grad_events[k] &&
+      cudaEventRecord(m->grad_events[k], st) != cudaSuccess)
+    return NC_ECUDA;
+  return NC_OK;
+}
+
 template <typename T>
 int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const int32_t *targets,
                  int B, int T_len, void *workspace, float *loss, float *token_loss, float *grads,
-                 cudaStream_t st) {
+                 int flags, cudaStream_t st) {
+  // accumulate: every gradient is added to grads instead of written over it
+  const int acc = (flags & NC_ACCUMULATE) ? 1 : 0;
+  const int wg = acc ? EPI_ACC_F32 : EPI_STORE_F32;
   Work<T> w;
   carve<T>(m, B, T_len, (char *)workspace, &w);
   const Weights<T> W = weight_ptrs<T>(m, weights);
@@ -355,7 +370,8 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   const int last = 1 + 6 * m->depth;  // lm_head
   const double nbwd = M * (8.0 * C + 3.0 * C * es + 4.0);  // dx_old, dx in fp32; dy, y, dx_t in T
   // dWout = dz^T xf ;  dxf = dz Wout
-  NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, EPI_STORE_F32), st));
+  NC_TRY(gemm<T>(m, gp(V, C, M, w.z, w.ldz, 1, w.xf, C, 1, G(last), C, wg), st));
+  NC_TRY(bucket_done(m, 0, st));
   NC_TRY(gemm<T>(m, gp(M, C, V, w.z, w.ldz, 0, W.lm_head, C, 1, w.dy, C, EPI_STORE), st));
   NC_RUN(K_RMSNORM_BWD, 0, nbwd - M * 4.0 * C,
          NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
@@ -371,15 +387,15 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     const int pi = 1 + 6 * l;
     const double attn_bwd_flops = 8.0 * B * H * (double)kHeadDim * attn_keys(T_len, m->layer_window[l]);
     // MLP: x += a W2^T, a = relu(h)^2, h = xn2 W1^T
-    NC_TRY(gemm<T>(m, gp(C, F, M, w.dxb, C, 1, w.a[l], F, 1, G(pi + 5), F, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(C, F, M, w.dxb, C, 1, w.a[l], F, 1, G(pi + 5), F, wg), st));
     NC_TRY(gemm<T>(m, gp(M, F, C, w.dxb, C, 0, W.w2[l], F, 1, w.a[l], F, EPI_DRELU2), st));
-    NC_TRY(gemm<T>(m, gp(F, C, M, w.a[l], F, 1, w.xn2[l], C, 1, G(pi + 4), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(F, C, M, w.a[l], F, 1, w.xn2[l], C, 1, G(pi + 4), C, wg), st));
     NC_TRY(gemm<T>(m, gp(M, C, F, w.a[l], F, 0, W.w1[l], C, 1, w.dy, C, EPI_STORE), st));
     NC_RUN(K_RMSNORM_BWD, 0, nbwd,
            NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
                                  w.dy, w.xn2[l], w.r2[l], w.dx, w.dxb, M, C, 1))));
     // attention: x += O Wo^T
-    NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, wg), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
            if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
@@ -392,21 +408,22 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
       NC_RUN(K_VE_BWD, 0, M * 2.0 * kHeadDim * es,
              (ve_gate_partial_kernel<T><<<nb, 256, 0, st>>>(dv, ldqkv, tokens, W.ve[l], V, M, w.ve_part)));
       NC_RUN(K_VE_BWD, 0, nb * 4.0,
-             (ordered_sum_kernel<<<1, 1024, 0, st>>>(w.ve_part, nb, 1.f, G(m->p_gates) + m->ve_slot[l])));
-      if (cudaMemsetAsync(gv, 0, sizeof(float) * (size_t)V * kHeadDim, st) != cudaSuccess) return NC_ECUDA;
+             (ordered_sum_kernel<<<1, 1024, 0, st>>>(w.ve_part, nb, 1.f, G(m->p_gates) + m->ve_slot[l], acc)));
+      if (!acc && cudaMemsetAsync(gv, 0, sizeof(float) * (size_t)V * kHeadDim, st) != cudaSuccess) return NC_ECUDA;
       ValueEmbedRows<T> src{dv, ldqkv, W.gates + m->ve_slot[l]};
       NC_RUN(K_VE_BWD, 0, M * (kHeadDim * es + 8.0),
              (segsum_kernel<ValueEmbedRows<T>, 1><<<(nch + 7) / 8, 256, 0, st>>>(
-                 src, w.sort.skey, w.sort.spos, M, kHeadDim, gv, w.seg_head, w.seg_tail, w.seg_flags)));
+                 src, w.sort.skey, w.sort.spos, M, kHeadDim, gv, w.seg_head, w.seg_tail, w.seg_flags, acc)));
       NC_RUN(K_SEG_FIXUP, 0, 0,
              (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, kHeadDim, w.seg_head, w.seg_tail, w.seg_flags,
-                                                    nch, gv)));
+                                                    nch, gv, acc)));
     }
     NC_RUN(K_ROPE_QKNORM_BWD, 0, M * (3.0 * (C + kHeadDim) * es + 4.0 * (H + 1)),
            (rope_qknorm_bwd_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.dqkv, w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H)));
     // [q|k|v] = xn [Wq;Wk;Wv]^T
-    NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, EPI_STORE_F32), st));
+    NC_TRY(gemm<T>(m, gp(ldqkv, C, M, w.dqkv, ldqkv, 1, w.xn[l], C, 1, G(pi), C, wg), st));
+    NC_TRY(bucket_done(m, 1 + (m->depth - 1 - l), st));  // the block's six matrices are final
     NC_TRY(gemm<T>(m, gp(M, C, ldqkv, w.dqkv, ldqkv, 0, W.wqkv[l], C, 1, w.dy, C, EPI_STORE), st));
     if (m->scalars) {
       // block entry: dx_in = dx + norm bwd;  dx = lam_r dx_in;  dx0 += lam_0 dx_in
@@ -424,18 +441,22 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   if (m->scalars) {
     // resid_lambdas and x0_lambdas are adjacent in the layout: 2L sums
     NC_RUN(K_VE_BWD, 0, 2.0 * m->depth * nblk8 * 4.0,
-           (ordered_sum_rows_kernel<<<2 * m->depth, 256, 0, st>>>(w.scal_part, (int)nblk8, G(m->p_resid), 1)));
+           (ordered_sum_rows_kernel<<<2 * m->depth, 256, 0, st>>>(w.scal_part, (int)nblk8, G(m->p_resid), 1,
+                                                                   acc)));
   }
   // embedding: through the first norm, summed per token over its positions
   // in a fixed order (positions sorted by token; no floating-point atomics)
   // (with residual scalars the gradient reaching x0 through the mixing, dx0, adds to dx)
-  if (cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
+  if (!acc && cudaMemsetAsync(G(0), 0, sizeof(float) * (size_t)V * C, st) != cudaSuccess) return NC_ECUDA;
   NC_RUN(K_EMBED_BWD, 0, M * (4.0 * C + C * es + 12.0) + (m->scalars ? M * 4.0 * C : 0.0),
          NC_DISPATCH_NV(C, (segsum_kernel<EmbedRows<T, NV>, NV><<<(nch + 7) / 8, 256, 0, st>>>(
                                EmbedRows<T, NV>{w.dx, m->scalars ? w.dx0 : nullptr, W.wte, w.r0, C}, w.sort.skey,
-                               w.sort.spos, M, C, G(0), w.seg_head, w.seg_tail, w.seg_flags))));
+                               w.sort.spos, M, C, G(0), w.seg_head, w.seg_tail, w.seg_flags, acc))));
   NC_RUN(K_SEG_FIXUP, 0, 0,
-         (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, C, w.seg_head, w.seg_tail, w.seg_flags, nch, G(0))));
+         (seg_fixup_kernel<<<nch, 256, 0, st>>>(w.sort.skey, M, C, w.seg_head, w.seg_tail, w.seg_flags, nch, G(0),
+                                                acc)));
+  NC_TRY(bucket_done(m, m->depth + 1, st));
+  if ((int)m->buckets.size() > m->depth + 2) NC_TRY(bucket_done(m, m->depth + 2, st));  // the extras
   return NC_OK;
 }
 
@@ -682,6 +703,16 @@ int nc_init_ex(int depth, int vocab, int seq, int dtype, const nc_block_opts *op
     add("ve_gates", 1, n_ve);
   }
   m->n_params = off;
+  // gradient buckets, completion order: lm_head, blocks L-1 .. 0, wte, extras
+  const int first_extra = 2 + 6 * depth;
+  m->buckets.push_back({m->params[1 + 6 * depth].offset, (int64_t)vocab * C});
+  for (int l = depth - 1; l >= 0; --l) {
+    const nc_param &a = m->params[1 + 6 * l], &z = m->params[6 + 6 * l];
+    m->buckets.push_back({a.offset, z.offset + (int64_t)z.rows * z.cols - a.offset});
+  }
+  m->buckets.push_back({0, (int64_t)vocab * C});
+  if ((int)m->params.size() > first_extra)
+    m->buckets.push_back({m->params[first_extra].offset, off - m->params[first_extra].offset});
 
   // RoPE table: angle = pos * 10000^(-i/64), built in float64, rounded once.
   std::vector<float> hc((size_t)seq * 64), hs((size_t)seq * 64);
@@ -710,6 +741,26 @@ int nc_get_dims(const nc_model *m, nc_dims *out) {
   out->depth = m->depth; out->width = m->C; out->n_head = m->H; out->head_dim = kHeadDim;
   out->hidden = m->F; out->vocab = m->V; out->seq = m->seq; out->dtype = m->dtype;
   out->n_params = m->n_params;
+  return NC_OK;
+}
+
+int nc_grad_bucket_count(const nc_model *m, int *count) {
+  if (!m || !count) return NC_EINVAL;
+  *count = (int)m->buckets.size();
+  return NC_OK;
+}
+
+int nc_grad_bucket(const nc_model *m, int k, int64_t *offset, int64_t *count) {
+  if (!m || !offset || !count || k < 0 || k >= (int)m->buckets.size()) return NC_EINVAL;
+  *offset = m->buckets[k].first;
+  *count = m->buckets[k].second;
+  return NC_OK;
+}
+
+int nc_set_grad_events(nc_model *m, void *const *events, int n) {
+  if (!m || n < 0 || (n > 0 && !events) || n > (int)m->buckets.size()) return NC_EINVAL;
+  m->grad_events.assign(n, nullptr);
+  for (int i = 0; i < n; ++i) m->grad_events[i] = (cudaEvent_t)events[i];
   return NC_OK;
 }
 
@@ -742,14 +793,22 @@ int nc_workspace_bytes(const nc_model *m, int B, int T, size_t *out) {
 int nc_fwd_bwd(nc_model *m, const void *weights, const int32_t *tokens, const int32_t *targets,
                int B, int T, void *workspace, size_t ws_bytes, float *loss, float *token_loss,
                float *grads, void *stream) {
+  return nc_fwd_bwd_ex(m, weights, tokens, targets, B, T, workspace, ws_bytes, loss, token_loss, grads, 0,
+                       stream);
+}
+
+int nc_fwd_bwd_ex(nc_model *m, const void *weights, const int32_t *tokens, const int32_t *targets,
+                  int B, int T, void *workspace, size_t ws_bytes, float *loss, float *token_loss,
+                  float *grads, int flags, void *stream) {
+  if (flags & ~NC_ACCUMULATE) return NC_EINVAL;
   int rc = check_step_args(m, weights, tokens, B, T, workspace, ws_bytes);
   if (rc != NC_OK) return rc;
   if (!targets || !loss || !grads) return NC_EINVAL;
   if (((uintptr_t)grads & 15) || ((uintptr_t)targets & 3) || ((uintptr_t)loss & 3)) return NC_EALIGN;
   cudaStream_t st = (cudaStream_t)stream;
   if (m->dtype == NC_F32)
-    return fwd_bwd_impl<float>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, st);
-  return fwd_bwd_impl<bf16>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, st);
+    return fwd_bwd_impl<float>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, flags, st);
+  return fwd_bwd_impl<bf16>(m, weights, tokens, targets, B, T, workspace, loss, token_loss, grads, flags, st);
 }
 
 int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B, int T, void *workspace,
@@ -839,7 +898,7 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
   if (!A || !B || !D) return NC_EINVAL;
   if (M < 1 || N < 1 || K < 1) return NC_ESHAPE;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
-  if (epilogue < NC_EPI_STORE || epilogue > NC_EPI_SOFTCAP || (a_mn | b_mn) & ~1) return NC_EINVAL;
+  if (epilogue < NC_EPI_STORE || epilogue > NC_EPI_ACC_F32 || (a_mn | b_mn) & ~1) return NC_EINVAL;
   if (engine < 0 || engine > 2) return NC_EINVAL;
   const GemmProblem p = gp(M, N, K, A, lda, a_mn, B, ldb, b_mn, D, ldd, epilogue);
   const bool tensor = dtype == NC_BF16 && engine != 1;

@@ -182,14 +182,24 @@ inline int sort_tokens(const int32_t *tokens, int M, int V, TokenSort &s, cudaSt
 // here and continues into the next chunk (its sum is in tail[chunk]).
 constexpr int kSegHead = 1, kSegHeadEnds = 2, kSegTail = 4;
 
-// Store the 8*NV-per-lane row sum `acc` (C values) to dst.
+// Store (add != 0: add) the 8*NV-per-lane row sum `acc` (C values) to dst.
 template <int NV>
-__device__ __forceinline__ void seg_store_row(float *dst, const float (&acc)[NV][8], int C, int lane) {
+__device__ __forceinline__ void seg_store_row(float *dst, const float (&acc)[NV][8], int C, int lane, int add = 0) {
   const int nv = C >> 3;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = lane + 32 * i;
-    if (c < nv) Vec8<float>::store(dst + c * 8, acc[i]);
+    if (c < nv) {
+      if (add) {
+        float o[8];
+        Vec8<float>::load(dst + c * 8, o);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] += acc[i][j];
+        Vec8<float>::store(dst + c * 8, o);
+      } else {
+        Vec8<float>::store(dst + c * 8, acc[i]);
+      }
+    }
   }
 }
 
@@ -261,13 +271,15 @@ struct ValueEmbedRows {
 };
 
 // out[v] = sum over token v's positions of src rows (C wide), for every
-// token that occurs; rows of other tokens are left as they are (the caller
-// zeroes the table first).
+// token that occurs (accumulate != 0: added to out[v]); rows of other tokens
+// are left as they are (the caller zeroes the table first when not
+// accumulating).
 template <typename Src, int NV>
 __global__ void __launch_bounds__(256) segsum_kernel(Src src, const int32_t *__restrict__ skey,
                                                      const int32_t *__restrict__ spos, int M, int C,
                                                      float *__restrict__ out, float *__restrict__ head,
-                                                     float *__restrict__ tail, int *__restrict__ flags) {
+                                                     float *__restrict__ tail, int *__restrict__ flags,
+                                                     int accumulate) {
   const int lane = threadIdx.x & 31;
   const int chunk = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int p0 = chunk * kSegChunk;
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__(256) segsum_kernel(Src src, const int32_t *__r
     const bool starts = a == 0 || skey[a - 1] != tok;
     const bool ends = b == M || skey[b] != tok;
     if (starts && ends) {
-      seg_store_row<NV>(out + (size_t)tok * C, acc, C, lane);
+      seg_store_row<NV>(out + (size_t)tok * C, acc, C, lane, accumulate);
     } else if (!starts) {  // the chunk's first run, continuing a segment
       seg_store_row<NV>(head + (size_t)chunk * C, acc, C, lane);
       fl |= kSegHead | (ends ? kSegHeadEnds : 0);
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(256) seg_fixup_kernel(const int32_t *__restric
                                                         const float *__restrict__ head,
                                                         const float *__restrict__ tail,
                                                         const int *__restrict__ flags, int nchunks,
-                                                        float *__restrict__ out) {
+                                                        float *__restrict__ out, int accumulate) {
   const int c = blockIdx.x;
   if (!(flags[c] & kSegTail)) return;
   const int tok = skey[min(M, (c + 1) * kSegChunk) - 1];
@@ -342,19 +354,25 @@ __global__ void __launch_bounds__(256) seg_fixup_kernel(const int32_t *__restric
       const float4 h = reinterpret_cast<const float4 *>(head + (size_t)k * C)[q];
       a.x += h.x; a.y += h.y; a.z += h.z; a.w += h.w;
     }
-    reinterpret_cast<float4 *>(out + (size_t)tok * C)[q] = a;
+    float4 *o = reinterpret_cast<float4 *>(out + (size_t)tok * C) + q;
+    if (accumulate) {
+      const float4 b = *o;
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    *o = a;
   }
 }
 
 // Deterministic sum of n partial values by one CTA: each thread adds a
-// fixed strided subset in order, then a fixed tree; *out = scale * sum.
+// fixed strided subset in order, then a fixed tree; *out = scale * sum
+// (accumulate != 0: *out += scale * sum).
 __global__ void __launch_bounds__(1024) ordered_sum_kernel(const float *__restrict__ partial, int n, float scale,
-                                                           float *__restrict__ out) {
+                                                           float *__restrict__ out, int accumulate) {
   __shared__ float sh[32];
   float s = 0.f;
   for (int i = threadIdx.x; i < n; i += blockDim.x) s += partial[i];
   s = block_sum(s, sh);
-  if (threadIdx.x == 0) *out = scale * s;
+  if (threadIdx.x == 0) *out = scale * s + (accumulate ? *out : 0.f);
 }
 
 }  // namespace nc

@@ -60,20 +60,36 @@ class Model:
 
     def fwd_bwd(self, weights: torch.Tensor, tokens: torch.Tensor, targets: torch.Tensor,
                 grads: torch.Tensor | None = None, loss: torch.Tensor | None = None,
-                token_loss: torch.Tensor | None = None):
+                token_loss: torch.Tensor | None = None, accumulate: bool = False):
+        """Loss and gradients of one step; accumulate=True adds the gradients
+        to `grads` instead of writing over them."""
         Bsz, T = tokens.shape
         ws = self.workspace(Bsz, T)
         if grads is None:
+            if accumulate:
+                raise ValueError("accumulate needs the gradient buffer to add to")
             grads = torch.empty(self.n_params, dtype=torch.float32, device="cuda")
         if loss is None:
             loss = torch.empty(1, dtype=torch.float32, device="cuda")
-        rc = B.nc_fwd_bwd(self.handle, weights.data_ptr(), tokens.data_ptr(), targets.data_ptr(),
-                          Bsz, T, ws.data_ptr(), ws.numel(), loss.data_ptr(),
-                          token_loss.data_ptr() if token_loss is not None else None,
-                          grads.data_ptr(), self._stream())
+        rc = B.nc_fwd_bwd_ex(self.handle, weights.data_ptr(), tokens.data_ptr(), targets.data_ptr(),
+                             Bsz, T, ws.data_ptr(), ws.numel(), loss.data_ptr(),
+                             token_loss.data_ptr() if token_loss is not None else None,
+                             grads.data_ptr(), B.NC_ACCUMULATE if accumulate else 0, self._stream())
         if rc != B.NC_OK:
-            raise B.NcError(rc, "nc_fwd_bwd")
+            raise B.NcError(rc, "nc_fwd_bwd_ex")
         return loss, grads
+
+    def grad_buckets(self):
+        """[(offset, count)] of the gradient buffer, in the order the backward finishes them."""
+        rc, b = B.nc_grad_buckets(self.handle)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_grad_bucket")
+        return b
+
+    def set_grad_events(self, events) -> None:
+        rc = B.nc_set_grad_events(self.handle, events)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_set_grad_events")
 
     def fwd(self, weights: torch.Tensor, tokens: torch.Tensor, logits: torch.Tensor | None = None):
         Bsz, T = tokens.shape

@@ -155,6 +155,35 @@ int nc_fwd_bwd(nc_model *m, const void *weights, const int32_t *tokens,
                size_t ws_bytes, float *loss, float *token_loss, float *grads,
                void *stream);
 
+/* Flags of nc_fwd_bwd_ex. */
+#define NC_ACCUMULATE 1  /* add this step's gradients to grads instead of writing over them */
+
+/* nc_fwd_bwd with flags: NC_ACCUMULATE sums the gradients of several calls
+ * into one buffer (gradient accumulation over micro-batches: scale the sum
+ * yourself, each call's loss being the mean over its own B*T positions).
+ * Unknown flag bits are NC_EINVAL. */
+int nc_fwd_bwd_ex(nc_model *m, const void *weights, const int32_t *tokens,
+                  const int32_t *targets, int B, int T, void *workspace,
+                  size_t ws_bytes, float *loss, float *token_loss, float *grads,
+                  int flags, void *stream);
+
+/* Gradient buckets, for overlapping a reduction of the gradients (the
+ * data-parallel all-reduce, "Nanochat: full-stack LLM training in 8,000
+ * lines for $72", section "A Llama-class transformer with ten modern
+ * departures": DistMuonAdamW / ZeRO-2 over 8 GPUs) with the rest of the
+ * backward.  Bucket k is the contiguous range [offset, offset + count) of
+ * grads, numbered in the order the backward finishes them: 0 lm_head, then
+ * one bucket per block from the last block to the first (its six matrices),
+ * then wte, then (full block) the extras after lm_head in the layout. */
+int nc_grad_bucket_count(const nc_model *m, int *count);
+int nc_grad_bucket(const nc_model *m, int k, int64_t *offset, int64_t *count);
+
+/* Events (cudaEvent_t as void*, owned by the caller, n <= the bucket count,
+ * NULL entries skipped) that every later nc_fwd_bwd(_ex) records on its
+ * stream as soon as bucket k is final; another stream can wait on event k
+ * and reduce bucket k while the backward goes on.  n = 0 turns them off. */
+int nc_set_grad_events(nc_model *m, void *const *events, int n);
+
 /* Forward only: softcapped logits s = 15 tanh(z/15) of every position.
  *   logits  device [B,T,vocab] in the model dtype (row-major, vocab fastest),
  *           16-byte aligned; a bf16 model needs vocab % 8 == 0 here (its

@@ -28,21 +28,24 @@ extern "C" {
  *   NC_EPI_ADD        D = D + acc            (residual add; D in dtype)
  *   NC_EPI_RELU2      D = relu(acc)^2        (relu^2 MLP activation)
  *   NC_EPI_DRELU2     D = acc * 2 sqrt(D)    (its backward: D holds relu(h)^2)
- *   NC_EPI_SOFTCAP    D = 15 tanh(acc / 15)  (logit softcap) */
+ *   NC_EPI_SOFTCAP    D = 15 tanh(acc / 15)  (logit softcap)
+ *   NC_EPI_ACC_F32    D = D + acc            (D fp32: gradient accumulation) */
 enum {
   NC_EPI_STORE = 0,
   NC_EPI_STORE_F32 = 1,
   NC_EPI_ADD = 2,
   NC_EPI_RELU2 = 3,
   NC_EPI_DRELU2 = 4,
-  NC_EPI_SOFTCAP = 5
+  NC_EPI_SOFTCAP = 5,
+  NC_EPI_ACC_F32 = 6
 };
 
 /* D[m,n] = epilogue(sum_k A(m,k) B(n,k)), fp32 accumulation.
  *   A(m,k) = A[m*lda + k] if a_mn == 0 (K-major) else A[k*lda + m] (MN-major)
  *   B(n,k) = B[n*ldb + k] if b_mn == 0 else B[k*ldb + n]
  *   D[m,n] = D[m*ldd + n]
- * dtype (nc_dtype) is the type of A, B and of D unless NC_EPI_STORE_F32.
+ * dtype (nc_dtype) is the type of A, B and of D unless NC_EPI_STORE_F32 or
+ * NC_EPI_ACC_F32.
  * engine: 0 = the path nc_fwd_bwd takes (bf16: tcgen05 tensor cores, pairs of
  * CTAs on 256 x 256 tiles when M >= 256, one CTA per 128 x 256 tile
  * otherwise; fp32: CUDA cores), 1 = the CUDA-core kernel (a test engine for
