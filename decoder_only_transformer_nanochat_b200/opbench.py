@@ -1,33 +1,40 @@
 """Time one kernel of the decoder step in isolation, at the shapes of one
 training step of the d20 workload (M = 16 x 2048 tokens, C = 1280, F = 5120,
 V = 65536, H = 10), through the op-level C entry points.  Used for per-kernel
-timing and for small, single-kernel ncu captures.
+timing and for small, single-kernel ncu captures (--tokens shrinks M, and with
+it every shape that grows with the tokens, so a capture holds a few GB).
 
     python -m decoder_only_transformer_nanochat_b200.opbench --op w1_fwd --iters 5
+    python -m decoder_only_transformer_nanochat_b200.opbench --op ce --tokens 8192
 """
 from __future__ import annotations
 
 import argparse
 import json
 
-M, C, F, V, H = 16 * 2048, 1280, 5120, 65536, 10
-B, T = 16, 2048
+C, F, V, H, T = 1280, 5120, 65536, 10, 2048
 
-# name: (M, N, K, a_mn, b_mn, epilogue)
-GEMMS = {
-    "qkv_fwd": (M, C + 256, C, 0, 0, "STORE"),
-    "o_fwd": (M, C, C, 0, 0, "ADD"),
-    "w1_fwd": (M, F, C, 0, 0, "RELU2"),
-    "w2_fwd": (M, C, F, 0, 0, "ADD"),
-    "head_fwd": (M, V, C, 0, 0, "STORE"),
-    "w2_dgrad": (M, F, C, 0, 1, "DRELU2"),
-    "w1_dgrad": (M, C, F, 0, 1, "STORE_F32"),
-    "w1_wgrad": (F, C, M, 1, 1, "STORE_F32"),
-    "w2_wgrad": (C, F, M, 1, 1, "STORE_F32"),
-    "o_wgrad": (C, C, M, 1, 1, "STORE_F32"),
-    "head_dgrad": (M, C, V, 0, 1, "STORE_F32"),
-    "head_wgrad": (V, C, M, 1, 1, "STORE_F32"),
-}
+
+def gemm_shapes(M: int) -> dict:
+    """name: (M, N, K, a_mn, b_mn, epilogue) of the step's GEMMs for M tokens."""
+    return {
+        "qkv_fwd": (M, C + 256, C, 0, 0, "STORE"),
+        "o_fwd": (M, C, C, 0, 0, "ADD"),
+        "w1_fwd": (M, F, C, 0, 0, "RELU2"),
+        "w2_fwd": (M, C, F, 0, 0, "ADD"),
+        "head_fwd": (M, V, C, 0, 0, "STORE"),
+        "w2_dgrad": (M, F, C, 0, 1, "DRELU2"),
+        "w1_dgrad": (M, C, F, 0, 1, "STORE"),
+        "w1_wgrad": (F, C, M, 1, 1, "STORE_F32"),
+        "w2_wgrad": (C, F, M, 1, 1, "STORE_F32"),
+        "o_wgrad": (C, C, M, 1, 1, "STORE_F32"),
+        "qkv_wgrad": (C + 256, C, M, 1, 1, "STORE_F32"),
+        "head_dgrad": (M, C, V, 0, 1, "STORE"),
+        "head_wgrad": (V, C, M, 1, 1, "STORE_F32"),
+    }
+
+
+GEMMS = gemm_shapes(16 * 2048)
 
 
 def main():
@@ -36,7 +43,9 @@ def main():
     import decoder_only_transformer_nanochat_b200 as nc
     from decoder_only_transformer_nanochat_b200 import build
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm"])
+    ap.add_argument("--op", required=True, choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm", "ce"])
+    ap.add_argument("--tokens", type=int, default=16 * 2048, help="M (a multiple of 2048)")
+    ap.add_argument("--window", type=int, default=0, help="attention: sliding window (0: causal)")
     ap.add_argument("--shape", default=None, help="for --op gemm: M,N,K,a_mn,b_mn,EPILOGUE")
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--engine", type=int, default=0)
@@ -44,14 +53,30 @@ def main():
     build.build()
     g = torch.Generator(device="cuda").manual_seed(0)
     st = torch.cuda.current_stream().cuda_stream
+    shapes = gemm_shapes(args.tokens)
+    B = args.tokens // T
     if args.op == "gemm":
         f = args.shape.split(",")
-        GEMMS["gemm"] = (int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4]), f[5])
-    if args.op in GEMMS:
-        m, n, k, a_mn, b_mn, epi = GEMMS[args.op]
+        shapes["gemm"] = (int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4]), f[5])
+    if args.op == "ce":
+        M = args.tokens
+        z = (torch.randn(M * V, device="cuda", generator=g) * 3.0).to(torch.bfloat16)
+        z0 = z.clone()
+        tgt = torch.randint(0, V, (M,), device="cuda", dtype=torch.int32, generator=g)
+        tl = torch.empty(M, device="cuda", dtype=torch.float32)
+
+        def prep():
+            z.copy_(z0)  # the op works in place: every launch starts from the same logits
+
+        def run():
+            assert nc.nc_softcap_ce(z.data_ptr(), V, tgt.data_ptr(), tl.data_ptr(), M, V, 1.0 / M,
+                                    nc.NC_BF16, st) == 0
+        flops = 0.0
+    elif args.op in shapes:
+        m, n, k, a_mn, b_mn, epi = shapes[args.op]
         A = (torch.randn(m * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
         Bm = (torch.randn(n * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
-        out_f32 = epi == "STORE_F32"
+        out_f32 = epi in ("STORE_F32", "ACC_F32")
         D = torch.rand(m * n, device="cuda", generator=g, dtype=torch.float32)
         if not out_f32:
             D = D.to(torch.bfloat16)
@@ -70,35 +95,45 @@ def main():
         O = torch.empty(B * T * H * 128, device="cuda", dtype=torch.bfloat16)
         lse = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
         rc = nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16,
-                                 args.engine, st)
+                                 args.engine, st, window=args.window)
         assert rc == 0
         dO = (torch.randn(B * T * H * 128, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
         Dr = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
         dqkv = torch.empty(B * T * ld, device="cuda", dtype=torch.bfloat16)
-        causal = 2.0 * B * H * 128 * T * (T + 1.0)
+        w = args.window if 0 < args.window < T else T
+        keys = 0.5 * w * (w + 1.0) + (T - w) * float(w)
+        causal = 4.0 * B * H * 128 * keys
         if args.op == "attn_fwd":
             def run():
                 assert nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H,
-                                           nc.NC_BF16, args.engine, st) == 0
+                                           nc.NC_BF16, args.engine, st, window=args.window) == 0
             flops = causal
         else:
             def run():
                 assert nc.nc_attention_bwd(qkv.data_ptr(), ld, O.data_ptr(), dO.data_ptr(), lse.data_ptr(),
                                            Dr.data_ptr(), dqkv.data_ptr(), B, T, H, nc.NC_BF16, args.engine,
-                                           st) == 0
+                                           st, window=args.window) == 0
             flops = 2.0 * causal
+    prep = locals().get("prep", lambda: None)
+    prep()
     run()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.iters)]
     for i in range(args.iters):
+        prep()
         ev[2 * i].record()
         run()
         ev[2 * i + 1].record()
     torch.cuda.synchronize()
     ms = sorted(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.iters))
     med = ms[len(ms) // 2]
-    print(json.dumps({"op": args.op, "shape": args.shape, "median_ms": med, "min_ms": ms[0],
-                      "tflops": flops / (med / 1000) / 1e12}))
+    out = {"op": args.op, "tokens": args.tokens, "shape": args.shape, "window": args.window, "median_ms": med,
+           "min_ms": ms[0]}
+    if flops:
+        out["tflops"] = flops / (med / 1000) / 1e12
+    if args.op == "ce":
+        out["gbs"] = 2.0 * args.tokens * V * 2 / (med / 1000) / 1e9  # z read once, dz written once
+    print(json.dumps(out))
 
 
 if __name__ == "__main__":
