@@ -22,6 +22,8 @@
 // are described where they start.
 #pragma once
 
+#include <stdio.h>
+
 #include "tc_common.cuh"
 
 namespace nc {
@@ -422,7 +424,7 @@ constexpr int kPairSmem = 1024 + 2 * kTileBytes /*Q0, Q1*/ + (kPairKStages + kPa
 static_assert(kPairSmem <= 232448, "shared memory per CTA");
 
 template <bool kWin>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kPairThreads, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
                          const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
                          const __grid_constant__ CUtensorMap map_o,    // O [B][T][C], box 64 x 128
@@ -586,29 +588,23 @@ __global__ void __maxnreg__(200)
       ok = mbar_wait(s_full(x), j & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      float s[128];
-      {
-        uint32_t (&rr)[128] = *reinterpret_cast<uint32_t(*)[128]>(s);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_nw(s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(rr + 32 * c));
-        tmem_wait_ld();
-      }
       const int kv0 = kbase + j * kKV;
+      const bool edge = kv0 + kKV > q0 || kv0 + kKV > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window);
+      // pass 1: the row max of the raw scores (scale > 0 commutes with max),
+      // 32 columns of TMEM at a time
       float mx = -INFINITY;
-      if (kv0 + kKV > q0 || kv0 + kKV > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window)) {
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(s_col + 32 * c, rr);
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int key = kv0 + i;
-          s[i] = (key > row || key >= p.T || (kWin && row - key >= p.window)) ? -INFINITY : s[i] * sc;
-          mx = fmaxf(mx, s[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          s[i] *= sc;
-          mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 32; ++i) {
+          const int key = kv0 + 32 * c + i;
+          const bool dead = edge && (key > row || key >= p.T || (kWin && row - key >= p.window));
+          mx = dead ? mx : fmaxf(mx, __uint_as_float(rr[i]));
         }
       }
+      mx *= sc;
       // the exponent base moves only when the row max grows by more than 2^8;
       // S_x(j) completing means PV_x(j-1) is done, so O_x can be rescaled now
       if (j == 0 || mx > m_used + kRescaleLog2) {
@@ -628,21 +624,30 @@ __global__ void __maxnreg__(200)
       }
       // with a window a row may see no key of its first tile: base 0 there
       const float mb = (kWin && m_used == -INFINITY) ? 0.f : m_used;
+      // pass 2: P = 2^(s sc - base) chunk by chunk; P's 16 columns of chunk c
+      // go over S columns [16c, 16c + 16), all of them already read
       float sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32], pk[16];
+        tmem_ld32(s_col + 32 * c, rr);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const int k = 64 * c + i;
+        for (int i = 0; i < 32; i += 2) {
+          const int key = kv0 + 32 * c + i;
+          float a = fmaf(__uint_as_float(rr[i]), sc, -mb), b = fmaf(__uint_as_float(rr[i + 1]), sc, -mb);
+          if (edge) {
+            if (key > row || key >= p.T || (kWin && row - key >= p.window)) a = -INFINITY;
+            if (key + 1 > row || key + 1 >= p.T || (kWin && row - key - 1 >= p.window)) b = -INFINITY;
+          }
           // one exponential in four on the FMA pipe, the rest on MUFU
-          const float e0 = ex2(s[k] - mb);
-          const float e1 = (i & 2) ? ex2_poly(s[k + 1] - mb) : ex2(s[k + 1] - mb);
+          const float e0 = ex2(a);
+          const float e1 = (i & 2) ? ex2_poly(b) : ex2(b);
           sum += e0 + e1;
           pk[i / 2] = pack2(e0, e1);
         }
-        tmem_st32(s_col + 32 * c, pk);  // P over the first 64 columns of S_x
+        tmem_st16_nw(s_col + 16 * c, pk);
       }
+      tmem_wait_st();
       l += sum;
       tc_fence_before();
       mbar_arrive(p_full(x));
@@ -1327,9 +1332,19 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.status = status;
   p.window = window;
   const int grid = B * ((H + 1) / 2) * p.n_qt;
-  if (windowed(window, T)) attn_fwd_pair_kernel<true><<<grid, kPairThreads, kPairSmem, st>>>(mqk, mv, mo, p);
+  const bool win = windowed(window, T);
+  if (win) attn_fwd_pair_kernel<true><<<grid, kPairThreads, kPairSmem, st>>>(mqk, mv, mo, p);
   else attn_fwd_pair_kernel<false><<<grid, kPairThreads, kPairSmem, st>>>(mqk, mv, mo, p);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFuncAttributes a;
+    const cudaError_t ea = win ? cudaFuncGetAttributes(&a, attn_fwd_pair_kernel<true>)
+                               : cudaFuncGetAttributes(&a, attn_fwd_pair_kernel<false>);
+    fprintf(stderr, "nanochat_b200: attention forward launch: %s (registers %d, max threads %d, smem %d)\n",
+            cudaGetErrorString(e), ea == cudaSuccess ? a.numRegs : -1, ea == cudaSuccess ? a.maxThreadsPerBlock : -1,
+            kPairSmem);
+  }
+  return e;
 }
 
 }  // namespace fatc
