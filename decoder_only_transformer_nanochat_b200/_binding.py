@@ -80,6 +80,9 @@ _SIGS = {
     "nc_grad_bucket_count": (_I, [_P, ctypes.POINTER(_I)]),
     "nc_grad_bucket": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(_P), _I]),
+    "nc_kv_cache_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_prefill": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]),
+    "nc_decode": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]),
     "nc_ops_status": (_I, [_P, _I]),
     "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
@@ -193,6 +196,22 @@ def nc_set_grad_events(handle, events) -> int:
     """events: raw cudaEvent_t handles (ints), one per bucket (or fewer)."""
     arr = (_P * max(1, len(events)))(*[_P(e) for e in events])
     return load_library().nc_set_grad_events(handle, arr, len(events))
+
+
+def nc_kv_cache_bytes(handle, B: int, T_max: int):
+    n = ctypes.c_size_t()
+    rc = load_library().nc_kv_cache_bytes(handle, B, T_max, ctypes.byref(n))
+    return rc, n.value
+
+
+def nc_prefill(handle, weights, tokens, B, T, cache, T_max, seqlens, workspace, ws_bytes, logits, stream) -> int:
+    return load_library().nc_prefill(handle, weights, tokens, B, T, cache, T_max, seqlens, workspace, ws_bytes,
+                                     logits, stream)
+
+
+def nc_decode(handle, weights, tokens, B, cache, T_max, seqlens, workspace, ws_bytes, logits, stream) -> int:
+    return load_library().nc_decode(handle, weights, tokens, B, cache, T_max, seqlens, workspace, ws_bytes,
+                                    logits, stream)
 
 
 def nc_fwd(handle, weights, tokens, B, T, workspace, ws_bytes, logits, stream):

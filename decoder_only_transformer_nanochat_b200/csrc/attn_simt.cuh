@@ -229,6 +229,74 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(
   }
 }
 
+// Decode attention over the KV cache ("nanochat - full-stack ChatGPT in ~8k
+// lines", section "6. Inference": a KV cache with per-row sequence lengths):
+// one new query per row b at position p_b = pos[b], against the cached keys
+// j <= p_b of that row (window > 0: p_b - j < window).  qkv holds the new
+// token's rows [B, ld] (q heads already roped and normed; its k and v already
+// in the cache).  CTA per (head h, row b), 128 threads: scores into shared
+// memory, their softmax, then thread d sums p_j v_j[d] over the keys (one
+// coalesced 256-byte V row per step).  Bandwidth-bound: the cache of the
+// shared head is read once per query head from L2.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_decode_kernel(const T *__restrict__ qkv, int ld,
+                                                          const T *__restrict__ kc, const T *__restrict__ vc,
+                                                          int64_t cstride, const int32_t *__restrict__ pos,
+                                                          int tmax, int H, int window, T *__restrict__ O) {
+  extern __shared__ float dsm[];
+  __shared__ float red[32];
+  float *q = dsm, *pj = dsm + kHeadDim;
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int p = min(max(pos[b], 0), tmax - 1);
+  const int j0 = window > 0 ? max(0, p - window + 1) : 0;
+  const T *krow0 = kc + (size_t)b * cstride, *vrow0 = vc + (size_t)b * cstride;
+  q[t] = to_f(qkv[(size_t)b * ld + h * kHeadDim + t]) * rsqrtf((float)kHeadDim);
+  __syncthreads();
+  float m = -INFINITY;
+  for (int j = j0 + t; j <= p; j += blockDim.x) {
+    const T *kr = krow0 + (size_t)j * kHeadDim;
+    float d = 0.f;
+#pragma unroll
+    for (int c = 0; c < kHeadDim / 8; ++c) {
+      float k8[8];
+      Vec8<T>::load(kr + 8 * c, k8);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d = fmaf(q[8 * c + i], k8[i], d);
+    }
+    pj[j - j0] = d;
+    m = fmaxf(m, d);
+  }
+  m = block_max(m, red);
+  float l = 0.f;
+  for (int j = j0 + t; j <= p; j += blockDim.x) {
+    const float e = expf(pj[j - j0] - m);
+    pj[j - j0] = e;
+    l += e;
+  }
+  l = block_sum(l, red);  // its barriers also publish every p_j
+  float acc = 0.f;
+  for (int j = j0; j <= p; ++j) acc = fmaf(pj[j - j0], to_f(vrow0[(size_t)j * kHeadDim + t]), acc);
+  O[(size_t)b * H * kHeadDim + h * kHeadDim + t] = from_f<T>(acc / l);
+}
+
+// Shared memory of the decode kernel: the query and one score per cached key.
+inline size_t attn_decode_smem(int tmax) { return (size_t)(kHeadDim + tmax) * sizeof(float); }
+
+template <typename T>
+inline cudaError_t launch_attn_decode(const T *qkv, int ld, const T *kc, const T *vc, int64_t cstride,
+                                      const int32_t *pos, int tmax, int B, int H, int window, T *O,
+                                      cudaStream_t st) {
+  attn_decode_kernel<T><<<dim3(H, B), kHeadDim, attn_decode_smem(tmax), st>>>(qkv, ld, kc, vc, cstride, pos, tmax,
+                                                                               H, window, O);
+  return cudaGetLastError();
+}
+
+// pos[b] += 1 after a decode step; pos[b] = T after a prefill of T tokens.
+__global__ void seqlens_kernel(int32_t *__restrict__ pos, int B, int set_to) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) pos[b] = set_to >= 0 ? set_to : pos[b] + 1;
+}
+
 template <typename T>
 inline cudaError_t launch_attn_simt_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len,
                                         int H, int window, cudaStream_t st) {

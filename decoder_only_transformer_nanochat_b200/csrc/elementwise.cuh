@@ -216,27 +216,49 @@ __device__ __forceinline__ float half_warp_sum(float v) {
 // head of the row also gets gate * ve[token] added ("ten modern departures":
 // a gated embedding lookup added to V at alternating layers); v is neither
 // roped nor normed.
+// KV cache (inference): with kc != nullptr the finished k and v of the row
+// are also written to the cache at [row b, position pos] (stride `cstride`
+// elements between rows b), b = tok / T_len; pos = positions[b] when given
+// (decode: one token per row), else tok % T_len (prefill).
+template <typename T>
+struct KvCacheOut {
+  T *kc = nullptr, *vc = nullptr;
+  int64_t cstride = 0;
+  const int32_t *positions = nullptr;
+  int tmax = 0;        // positions past the cache are clamped and flagged
+  int *status = nullptr;
+};
+
 template <typename T>
 __global__ void __launch_bounds__(256) rope_qknorm_kernel(
     T *__restrict__ qkv, int ld, float *__restrict__ rq, float *__restrict__ rk,
     const float *__restrict__ cos_t, const float *__restrict__ sin_t, int M, int T_len, int H,
     const int32_t *__restrict__ tokens = nullptr, const T *__restrict__ ve = nullptr,
-    const T *__restrict__ ve_gate = nullptr, int V = 0) {
+    const T *__restrict__ ve_gate = nullptr, int V = 0, KvCacheOut<T> cache = KvCacheOut<T>()) {
   const int tok = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= M) return;
-  if (ve && lane < kHeadDim / 8) {
-    T *vrow = qkv + (size_t)tok * ld + (H + 1) * kHeadDim + lane * 8;
-    const int id = min(max(tokens[tok], 0), V - 1);
-    const float g = to_f(ve_gate[0]);
-    float v[8], e[8];
-    Vec8<T>::load(vrow, v);
-    Vec8<T>::load(ve + (size_t)id * kHeadDim + lane * 8, e);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] += g * e[i];
-    Vec8<T>::store(vrow, v);
+  int pos = cache.positions ? cache.positions[tok / T_len] : tok % T_len;
+  if (cache.positions && (pos < 0 || pos >= cache.tmax)) {
+    if (lane == 0) set_status(cache.status, kStatusRange);
+    pos = pos < 0 ? 0 : cache.tmax - 1;
   }
-  const int pos = tok % T_len;
+  T *kc_row = cache.kc ? cache.kc + (size_t)(tok / T_len) * cache.cstride + (size_t)pos * kHeadDim : nullptr;
+  if ((ve || cache.kc) && lane < kHeadDim / 8) {
+    T *vrow = qkv + (size_t)tok * ld + (H + 1) * kHeadDim + lane * 8;
+    float v[8];
+    Vec8<T>::load(vrow, v);
+    if (ve) {
+      const int id = min(max(tokens[tok], 0), V - 1);
+      const float g = to_f(ve_gate[0]);
+      float e[8];
+      Vec8<T>::load(ve + (size_t)id * kHeadDim + lane * 8, e);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += g * e[i];
+      Vec8<T>::store(vrow, v);
+    }
+    if (cache.kc) Vec8<T>::store(cache.vc + (kc_row - cache.kc) + lane * 8, v);
+  }
   const int hw = lane >> 4, j = lane & 15;
   float c[8], s[8];
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
@@ -270,6 +292,7 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(
     for (int i = 0; i < 8; ++i) y[i] *= r;
     if (live) {
       Vec8<T>::store(row + h * kHeadDim + j * 8, y);
+      if (h == H && kc_row) Vec8<T>::store(kc_row + j * 8, y);
       if (j == 0) {
         if (h < H) rq[(size_t)tok * H + h] = r;
         else rk[tok] = r;

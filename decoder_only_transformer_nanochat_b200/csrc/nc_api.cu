@@ -287,10 +287,30 @@ inline double attn_keys(int T, int window) {
   return 0.5 * window * (window + 1.0) + (double)(T - window) * window;
 }
 
+// Inference context of forward_body: the KV cache (per layer K then V, each
+// [B, tmax, 128]) that the RoPE kernel fills, and for a decode step the
+// per-row positions of the new tokens (attention then reads the cache).
+template <typename T>
+struct Infer {
+  T *cache = nullptr;
+  int tmax = 0;
+  const int32_t *positions = nullptr;  // decode only
+  KvCacheOut<T> layer(int l, int B, int *status) const {
+    KvCacheOut<T> o;
+    o.kc = cache + (size_t)l * 2 * B * tmax * kHeadDim;
+    o.vc = o.kc + (size_t)B * tmax * kHeadDim;
+    o.cstride = (int64_t)tmax * kHeadDim;
+    o.positions = positions;
+    o.tmax = tmax;
+    o.status = status;
+    return o;
+  }
+};
+
 // Forward through the blocks and the final norm; leaves xf, rf in the workspace.
 template <typename T>
 int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B, int T_len,
-                 Work<T> &w, cudaStream_t st) {
+                 Work<T> &w, cudaStream_t st, const Infer<T> *inf = nullptr) {
   const int M = B * T_len, C = m->C, H = m->H, F = m->F;
   const int ldqkv = C + 2 * kHeadDim;
   const double es = sizeof(T);
@@ -313,13 +333,21 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
     }
     NC_TRY(gemm<T>(m, gp(M, ldqkv, C, w.xn[l], C, 0, W.wqkv[l], C, 0, w.qkv[l], ldqkv, EPI_STORE), st));
     const bool ve = W.ve[l] != nullptr;
+    const KvCacheOut<T> kvo = inf ? inf->layer(l, B, m->status) : KvCacheOut<T>();
     NC_RUN(K_ROPE_QKNORM, 0, M * (2.0 * (C + kHeadDim) * es + 4.0 * (H + 1) + (ve ? 3.0 * kHeadDim * es : 0.0)),
            (rope_qknorm_kernel<T><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
                w.qkv[l], ldqkv, w.rq[l], w.rk[l], m->rope_cos, m->rope_sin, M, T_len, H, tokens, W.ve[l],
-               ve ? W.gates + m->ve_slot[l] : nullptr, m->V)));
-    NC_RUN(K_ATTN_FWD, attn_flops, 0,
-           if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->layer_window[l], 0,
-                                  m->status, st) != cudaSuccess) return NC_ECUDA);
+               ve ? W.gates + m->ve_slot[l] : nullptr, m->V, kvo)));
+    if (inf && inf->positions) {
+      // decode: the new token's queries against the cached keys of its row
+      NC_RUN(K_ATTN_FWD, 0, 0,
+             if (launch_attn_decode<T>(w.qkv[l], ldqkv, kvo.kc, kvo.vc, kvo.cstride, inf->positions, inf->tmax, B, H,
+                                       m->layer_window[l], w.O[l], st) != cudaSuccess) return NC_ECUDA);
+    } else {
+      NC_RUN(K_ATTN_FWD, attn_flops, 0,
+             if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->layer_window[l], 0,
+                                    m->status, st) != cudaSuccess) return NC_ECUDA);
+    }
     NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, x, C, EPI_ADD), st));
     NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
            NC_DISPATCH_NV(C, (rmsnorm_kernel<T, NV><<<rows_grid(M, 8), 256, 0, st>>>(
@@ -627,6 +655,55 @@ __global__ void wait_expiry_kernel(uint64_t wait_ns, int *status) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Inference with a KV cache
+
+constexpr int kMaxCacheT = 32768;  // longest cache the decode kernel's shared memory holds
+
+template <typename T>
+int prefill_impl(nc_model *m, const void *weights, const int32_t *tokens, int B, int T_len, void *cache, int T_max,
+                 int32_t *seqlens, void *workspace, void *logits, cudaStream_t st) {
+  Work<T> w;
+  carve<T>(m, B, T_len, (char *)workspace, &w);
+  const Weights<T> W = weight_ptrs<T>(m, weights);
+  Infer<T> inf;
+  inf.cache = (T *)cache;
+  inf.tmax = T_max;
+  NC_TRY(forward_body<T>(m, W, tokens, B, T_len, w, st, &inf));
+  seqlens_kernel<<<(B + 255) / 256, 256, 0, st>>>(seqlens, B, T_len);
+  NC_CHECK_LAUNCH();
+  // logits of each row's last position: rows b*T + T-1 of xf (row stride T*C)
+  const int64_t C = m->C;
+  return gemm<T>(m, gp(B, m->V, m->C, w.xf + (T_len - 1) * C, T_len * C, 0, W.lm_head, C, 0, logits, m->V,
+                       EPI_SOFTCAP), st);
+}
+
+template <typename T>
+int decode_impl(nc_model *m, const void *weights, const int32_t *tokens, int B, void *cache, int T_max,
+                int32_t *seqlens, void *workspace, void *logits, cudaStream_t st) {
+  Work<T> w;
+  carve<T>(m, B, 1, (char *)workspace, &w);
+  const Weights<T> W = weight_ptrs<T>(m, weights);
+  Infer<T> inf;
+  inf.cache = (T *)cache;
+  inf.tmax = T_max;
+  inf.positions = seqlens;
+  NC_TRY(forward_body<T>(m, W, tokens, B, 1, w, st, &inf));
+  NC_TRY(gemm<T>(m, gp(B, m->V, m->C, w.xf, m->C, 0, W.lm_head, m->C, 0, logits, m->V, EPI_SOFTCAP), st));
+  seqlens_kernel<<<(B + 255) / 256, 256, 0, st>>>(seqlens, B, -1);
+  NC_CHECK_LAUNCH();
+  return NC_OK;
+}
+
+int check_infer_args(const nc_model *m, void *cache, int T_max, int32_t *seqlens, void *logits, int B) {
+  if (!cache || !seqlens || !logits) return NC_EINVAL;
+  if (T_max < 1 || T_max > m->seq || T_max > kMaxCacheT) return NC_ESHAPE;
+  if (((uintptr_t)cache & 15) || ((uintptr_t)logits & 15) || ((uintptr_t)seqlens & 3)) return NC_EALIGN;
+  if (m->dtype == NC_BF16 && (m->V % 8)) return NC_EALIGN;  // logit rows leave the GEMM by TMA
+  (void)B;
+  return NC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -728,6 +805,11 @@ int nc_init_ex(int depth, int vocab, int seq, int dtype, const nc_block_opts *op
             cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
             cudaMemset(m->status, 0, 256) == cudaSuccess;
+  if (ok)
+    ok = cudaFuncSetAttribute(attn_decode_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)attn_decode_smem(kMaxCacheT)) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)attn_decode_smem(kMaxCacheT)) == cudaSuccess;
   if (!ok || tc_init() != cudaSuccess || fatc::init() != cudaSuccess || ce_init() != cudaSuccess) {
     nc_destroy(m);
     return NC_ECUDA;
@@ -822,6 +904,34 @@ int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B, int T
   cudaStream_t st = (cudaStream_t)stream;
   if (m->dtype == NC_F32) return fwd_impl<float>(m, weights, tokens, B, T, workspace, logits, st);
   return fwd_impl<bf16>(m, weights, tokens, B, T, workspace, logits, st);
+}
+
+int nc_kv_cache_bytes(const nc_model *m, int B, int T_max, size_t *out) {
+  if (!m || !out) return NC_EINVAL;
+  if (B < 1 || T_max < 1 || T_max > m->seq || T_max > kMaxCacheT) return NC_ESHAPE;
+  *out = (size_t)m->depth * 2 * B * T_max * kHeadDim * (m->dtype == NC_F32 ? 4 : 2);
+  return NC_OK;
+}
+
+int nc_prefill(nc_model *m, const void *weights, const int32_t *tokens, int B, int T, void *cache, int T_max,
+               int32_t *seqlens, void *workspace, size_t ws_bytes, void *logits, void *stream) {
+  int rc = check_step_args(m, weights, tokens, B, T, workspace, ws_bytes);
+  if (rc != NC_OK) return rc;
+  if ((rc = check_infer_args(m, cache, T_max, seqlens, logits, B)) != NC_OK) return rc;
+  if (T > T_max) return NC_ESHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->dtype == NC_F32) return prefill_impl<float>(m, weights, tokens, B, T, cache, T_max, seqlens, workspace, logits, st);
+  return prefill_impl<bf16>(m, weights, tokens, B, T, cache, T_max, seqlens, workspace, logits, st);
+}
+
+int nc_decode(nc_model *m, const void *weights, const int32_t *tokens, int B, void *cache, int T_max,
+              int32_t *seqlens, void *workspace, size_t ws_bytes, void *logits, void *stream) {
+  int rc = check_step_args(m, weights, tokens, B, 1, workspace, ws_bytes);
+  if (rc != NC_OK) return rc;
+  if ((rc = check_infer_args(m, cache, T_max, seqlens, logits, B)) != NC_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->dtype == NC_F32) return decode_impl<float>(m, weights, tokens, B, cache, T_max, seqlens, workspace, logits, st);
+  return decode_impl<bf16>(m, weights, tokens, B, cache, T_max, seqlens, workspace, logits, st);
 }
 
 int nc_sync_status(nc_model *m, void *stream, int timeout_ms) {

@@ -102,5 +102,42 @@ class Model:
             raise B.NcError(rc, "nc_fwd")
         return logits
 
+    # ---------------- inference with a KV cache ----------------
+
+    def kv_cache(self, Bsz: int, T_max: int):
+        """A zeroed KV cache for Bsz rows of up to T_max positions, and the
+        per-row sequence lengths (device int32)."""
+        rc, n = B.nc_kv_cache_bytes(self.handle, Bsz, T_max)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_kv_cache_bytes")
+        return (torch.zeros(n, dtype=torch.uint8, device="cuda"),
+                torch.zeros(Bsz, dtype=torch.int32, device="cuda"))
+
+    def prefill(self, weights: torch.Tensor, tokens: torch.Tensor, cache, T_max: int):
+        """Forward over the prompts tokens [B, T]; fills the cache; returns the
+        softcapped logits of each row's last position [B, vocab]."""
+        Bsz, T = tokens.shape
+        kv, seqlens = cache
+        ws = self.workspace(Bsz, T)
+        logits = torch.empty(Bsz, self.dims["vocab"], dtype=self.torch_dtype, device="cuda")
+        rc = B.nc_prefill(self.handle, weights.data_ptr(), tokens.data_ptr(), Bsz, T, kv.data_ptr(), T_max,
+                          seqlens.data_ptr(), ws.data_ptr(), ws.numel(), logits.data_ptr(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_prefill")
+        return logits
+
+    def decode(self, weights: torch.Tensor, tokens: torch.Tensor, cache, T_max: int):
+        """One token per row (tokens [B]) at each row's next position; returns
+        its softcapped logits [B, vocab]."""
+        Bsz = tokens.shape[0]
+        kv, seqlens = cache
+        ws = self.workspace(Bsz, 1)
+        logits = torch.empty(Bsz, self.dims["vocab"], dtype=self.torch_dtype, device="cuda")
+        rc = B.nc_decode(self.handle, weights.data_ptr(), tokens.data_ptr(), Bsz, kv.data_ptr(), T_max,
+                         seqlens.data_ptr(), ws.data_ptr(), ws.numel(), logits.data_ptr(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_decode")
+        return logits
+
     def sync_status(self, timeout_ms: int = 60000) -> int:
         return B.nc_sync_status(self.handle, self._stream(), timeout_ms)

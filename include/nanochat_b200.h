@@ -192,6 +192,36 @@ int nc_set_grad_events(nc_model *m, void *const *events, int n);
 int nc_fwd(nc_model *m, const void *weights, const int32_t *tokens, int B,
            int T, void *workspace, size_t ws_bytes, void *logits, void *stream);
 
+/* Inference with a KV cache ("nanochat - full-stack ChatGPT in ~8k lines",
+ * section "6. Inference": a KV cache with int32 per-row sequence lengths;
+ * energyai.berlin page, "KV caching").  With one shared KV head the cache
+ * holds, per layer, K then V of every position seen, each [B, T_max, 128] in
+ * the model dtype: nc_kv_cache_bytes() bytes of caller-owned device memory
+ * (16-byte aligned).  seqlens: device int32 [B], the number of cached
+ * positions of each row, owned by the caller and kept up to date by the
+ * calls below.  T_max <= seq and T_max <= 32,768 (the decode kernel keeps one
+ * score per cached key in shared memory), else NC_ESHAPE. */
+int nc_kv_cache_bytes(const nc_model *m, int B, int T_max, size_t *out);
+
+/* Runs the forward pass over tokens [B, T] (positions 0..T-1), writes every
+ * layer's K and V into the cache, sets seqlens[b] = T and returns the
+ * softcapped logits of each row's last position: logits device [B, vocab]
+ * (model dtype; bf16 needs vocab % 8 == 0).  workspace as nc_fwd_bwd for
+ * (B, T); T <= T_max. */
+int nc_prefill(nc_model *m, const void *weights, const int32_t *tokens, int B, int T, void *cache,
+               int T_max, int32_t *seqlens, void *workspace, size_t ws_bytes, void *logits,
+               void *stream);
+
+/* One decode step: token b (device int32 [B]) sits at position seqlens[b]
+ * of its row; it attends to the cached positions 0..seqlens[b] (itself
+ * included; the "S" layers of the full block to their last `window`),
+ * its K and V are appended, seqlens[b] is incremented, and the softcapped
+ * logits of the new token are written to logits [B, vocab].  workspace as
+ * nc_fwd_bwd for (B, 1).  A position past T_max - 1 is clamped and reported
+ * as NC_ERANGE by nc_sync_status. */
+int nc_decode(nc_model *m, const void *weights, const int32_t *tokens, int B, void *cache, int T_max,
+              int32_t *seqlens, void *workspace, size_t ws_bytes, void *logits, void *stream);
+
 /* Wait at most timeout_ms for the work enqueued so far on `stream` to finish
  * (polling, never blocking longer), then read and clear the device status
  * word.  Returns NC_ETIMEOUT if the stream is still busy, else the first

@@ -222,6 +222,19 @@ def forward_loss(W, tokens, targets, depth, windows=None):
     return tl.mean(), tl
 
 
+def forward_logits(W, tokens, depth, windows=None):
+    """Softcapped logits s [B,T,V] of every position; windows defaults to SSSL."""
+    windows = window_schedule(depth) if windows is None else windows
+    B, T = tokens.shape
+    xs, _, _, _, _ = _stream(W, tokens, depth, windows)
+    xf, _ = rmsnorm(xs[-1])
+    V = W["lm_head"].shape[0]
+    s = np.empty((B, T, V))
+    for b in range(B):
+        s[b] = head_forward_row(xf[b * T:(b + 1) * T], W["lm_head"])
+    return s
+
+
 def loss_and_grads(W, tokens, targets, depth, windows=None):
     """Loss, per-token losses and the gradient of every weight of
     full_param_layout (float64); windows defaults to the SSSL schedule."""
@@ -260,4 +273,4 @@ def loss_and_grads(W, tokens, targets, depth, windows=None):
 
 __all__ = ["SHORT_WINDOW", "WINDOW_PATTERN", "RESID_LAMBDA_INIT", "X0_LAMBDA_INIT", "window_schedule",
            "ve_layers", "full_param_layout", "init_scalars", "attention", "attention_bwd",
-           "forward_loss", "loss_and_grads", "dims"]
+           "forward_loss", "forward_logits", "loss_and_grads", "dims"]

@@ -170,3 +170,22 @@ def test_finite_differences_every_tensor_full_block():
             w[i, j] = old
             fd = (lp - lm) / (2 * h)
             assert abs(fd - g[name][i, j]) <= 1e-6 * gmax, (name, i, j, fd, g[name][i, j])
+
+
+def test_forward_logits_agree_with_the_loss():
+    # the logits function and the loss function share the forward: the loss
+    # recomputed from the logits (log-sum-exp minus the target's logit) agrees
+    depth = 2
+    lay, W, tok, tgt = _tiny(depth=depth)
+    windows = fb.window_schedule(depth, short=4)
+    s = fb.forward_logits(W, tok, depth, windows=windows)
+    m = s.max(axis=2, keepdims=True)
+    lse = (m + np.log(np.exp(s - m).sum(axis=2, keepdims=True)))[..., 0]
+    tl = lse - np.take_along_axis(s, tgt[..., None], axis=2)[..., 0]
+    loss, tl_ref = fb.forward_loss(W, tok, tgt, depth, windows=windows)
+    np.testing.assert_allclose(tl, tl_ref, rtol=0, atol=1e-12)
+    # causality: logits at position t do not change when later tokens change
+    tok2 = tok.copy()
+    tok2[:, -1] = (tok2[:, -1] + 1) % W["wte"].shape[0]
+    s2 = fb.forward_logits(W, tok2, depth, windows=windows)
+    np.testing.assert_array_equal(s[:, :-1], s2[:, :-1])
