@@ -14,7 +14,8 @@ from ._binding import (NC_BF16, NC_EALIGN, NC_ECUDA, NC_EINVAL, NC_ENOMEM,  # no
                        nc_attention_bwd_noalloc, NC_ATTN_BWD_NOALLOC_MAX_ROWS, nc_ops_status,
                        nc_check_wait_expiry, nc_softcap_ce, nc_init_ex, nc_layer_window,
                        nc_param_count, nc_fwd_bwd_ex, nc_grad_buckets, nc_set_grad_events,
-                       NC_ACCUMULATE, nc_kv_cache_bytes, nc_prefill, nc_decode)
+                       NC_ACCUMULATE, nc_kv_cache_bytes, nc_prefill, nc_decode, nc_optim_state_bytes,
+                       nc_optim_workspace_bytes, nc_optim_init, nc_optim_step)
 
 
 def __getattr__(name):

@@ -81,6 +81,10 @@ _SIGS = {
     "nc_grad_bucket": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(_P), _I]),
     "nc_kv_cache_bytes": (_I, [_P, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_optim_state_bytes": (_I, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_optim_workspace_bytes": (_I, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_optim_init": (_I, [_P, _P, _P, _P]),
+    "nc_optim_step": (_I, [_P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P]),
     "nc_prefill": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]),
     "nc_decode": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, ctypes.c_size_t, _P, _P]),
     "nc_ops_status": (_I, [_P, _I]),
@@ -196,6 +200,35 @@ def nc_set_grad_events(handle, events) -> int:
     """events: raw cudaEvent_t handles (ints), one per bucket (or fewer)."""
     arr = (_P * max(1, len(events)))(*[_P(e) for e in events])
     return load_library().nc_set_grad_events(handle, arr, len(events))
+
+
+class nc_optim_opts(ctypes.Structure):
+    _fields_ = [("lr_matrix", ctypes.c_float), ("lr_embed", ctypes.c_float), ("lr_head", ctypes.c_float),
+                ("lr_scalar", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("muon_momentum", ctypes.c_float), ("ns_steps", ctypes.c_int), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("eps", ctypes.c_float)]
+
+
+def nc_optim_state_bytes(handle):
+    n = ctypes.c_size_t()
+    rc = load_library().nc_optim_state_bytes(handle, ctypes.byref(n))
+    return rc, n.value
+
+
+def nc_optim_workspace_bytes(handle):
+    n = ctypes.c_size_t()
+    rc = load_library().nc_optim_workspace_bytes(handle, ctypes.byref(n))
+    return rc, n.value
+
+
+def nc_optim_init(handle, weights, state, stream) -> int:
+    return load_library().nc_optim_init(handle, weights, state, stream)
+
+
+def nc_optim_step(handle, weights, grads, state, step, opts: dict, workspace, ws_bytes, stream) -> int:
+    o = nc_optim_opts(**opts)
+    return load_library().nc_optim_step(handle, weights, grads, state, step, ctypes.byref(o), workspace,
+                                        ws_bytes, stream)
 
 
 def nc_kv_cache_bytes(handle, B: int, T_max: int):

@@ -14,6 +14,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <chrono>
 #include <mutex>
 #include <thread>
@@ -26,6 +27,7 @@
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "optim.cuh"
 #include "token_sort.cuh"
 
 using namespace nc;
@@ -34,12 +36,12 @@ using namespace nc;
 enum KernelClass {
   K_GEMM_TC, K_GEMM_SIMT, K_ATTN_FWD, K_ATTN_BWD, K_EMBED, K_RMSNORM, K_ROPE_QKNORM, K_CE,
   K_LOSS_MEAN, K_RMSNORM_BWD, K_ROWDOT, K_ROPE_QKNORM_BWD, K_EMBED_BWD, K_TOKEN_SORT, K_SEG_FIXUP,
-  K_VE_BWD, K_NUM_CLASSES
+  K_VE_BWD, K_OPTIM, K_NUM_CLASSES
 };
 static const char *kClassName[K_NUM_CLASSES] = {
     "gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd", "embed_norm", "rmsnorm", "rope_qknorm",
     "ce_fused", "loss_mean", "rmsnorm_bwd", "attn_rowdot", "rope_qknorm_bwd", "embed_bwd",
-    "token_sort", "seg_fixup", "block_extras_bwd"};
+    "token_sort", "seg_fixup", "block_extras_bwd", "optimizer"};
 
 struct nc_model {
   int depth, C, H, F, V, seq, dtype;
@@ -704,6 +706,96 @@ int check_infer_args(const nc_model *m, void *cache, int T_max, int32_t *seqlens
   return NC_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Optimizer step (Muon for the block matrices, AdamW for the rest)
+
+enum ParamGroup { G_MATRIX, G_EMBED, G_HEAD, G_SCALAR };
+
+ParamGroup param_group(const char *name) {
+  if (!strcmp(name, "lm_head")) return G_HEAD;
+  if (!strcmp(name, "wte") || (name[0] == 'v' && name[1] == 'e' && name[2] >= '0' && name[2] <= '9')) return G_EMBED;
+  if (!strcmp(name, "resid_lambdas") || !strcmp(name, "x0_lambdas") || !strcmp(name, "ve_gates")) return G_SCALAR;
+  return G_MATRIX;
+}
+
+// Newton-Schulz scratch: two X buffers of the largest matrix, the Gram matrix
+// of the largest shorter side (fp32) and its coefficient matrix, the norm's
+// partial sums.
+struct OptimWork {
+  char *x0, *x1, *bm;
+  float *gram, *partial;
+};
+
+size_t optim_carve(const nc_model *m, char *base, OptimWork *w) {
+  int64_t big = 0, small = 0;
+  for (const nc_param &p : m->params)
+    if (param_group(p.name) == G_MATRIX) {
+      big = std::max<int64_t>(big, (int64_t)p.rows * p.cols);
+      small = std::max<int64_t>(small, std::min(p.rows, p.cols));
+    }
+  const size_t es = m->dtype == NC_F32 ? 4 : 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char * {
+    char *q = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return q;
+  };
+  char *x0 = take(big * es), *x1 = take(big * es), *bm = take(small * small * es);
+  float *gram = (float *)take(small * small * 4), *partial = (float *)take((kOptBlocks + 1) * 4);
+  if (w) *w = OptimWork{x0, x1, bm, gram, partial};
+  return off;
+}
+
+template <typename T>
+int optim_step_impl(nc_model *m, T *weights, const float *grads, float *state, int step, const nc_optim_opts &o,
+                    void *workspace, cudaStream_t st) {
+  OptimWork ow;
+  optim_carve(m, (char *)workspace, &ow);
+  const int64_t N = m->n_params;
+  float *master = state, *mom = state + N, *vel = state + 2 * N;
+  const float bc1 = 1.f / (1.f - powf(o.beta1, (float)step)), bc2 = 1.f / (1.f - powf(o.beta2, (float)step));
+  const double es = sizeof(T);
+  for (const nc_param &p : m->params) {
+    const int64_t off = p.offset, n = (int64_t)p.rows * p.cols;
+    const ParamGroup grp = param_group(p.name);
+    if (grp != G_MATRIX) {
+      const float lr = grp == G_EMBED ? o.lr_embed : grp == G_HEAD ? o.lr_head : o.lr_scalar;
+      NC_RUN(K_OPTIM, 0, n * (20.0 + es),
+             (adamw_kernel<T><<<ew_grid(n, m->num_sms), 256, 0, st>>>(weights + off, master + off, grads + off,
+                                                                       mom + off, vel + off, n, lr, o.beta1, o.beta2,
+                                                                       o.eps, o.weight_decay, bc1, bc2)));
+      continue;
+    }
+    T *X = (T *)ow.x0, *Y = (T *)ow.x1, *Bm = (T *)ow.bm;
+    NC_RUN(K_OPTIM, 0, n * 12.0,
+           (muon_momentum_kernel<<<kOptBlocks, 256, 0, st>>>(grads + off, mom + off, n, o.muon_momentum,
+                                                             ow.partial)));
+    NC_RUN(K_OPTIM, 0, 0, (ordered_sum_kernel<<<1, 1024, 0, st>>>(ow.partial, kOptBlocks, 1.f,
+                                                                  ow.partial + kOptBlocks, 0)));
+    NC_RUN(K_OPTIM, 0, n * (4.0 + es),
+           (muon_scale_kernel<T><<<ew_grid(n, m->num_sms), 256, 0, st>>>(mom + off, n, ow.partial + kOptBlocks, X)));
+    const int r = p.rows, c = p.cols;
+    for (int k = 0; k < o.ns_steps; ++k) {
+      if (r >= c) {  // X (1.5 I - 0.5 X^T X): the Gram matrix of the columns
+        NC_TRY(gemm<T>(m, gp(c, c, r, X, c, 1, X, c, 1, ow.gram, c, EPI_STORE_F32), st));
+        NC_RUN(K_OPTIM, 0, (double)c * c * (4.0 + es),
+               (ns_coeff_kernel<T><<<ew_grid((int64_t)c * c, m->num_sms), 256, 0, st>>>(ow.gram, c, Bm)));
+        NC_TRY(gemm<T>(m, gp(r, c, c, X, c, 0, Bm, c, 1, Y, c, EPI_STORE), st));
+      } else {       // (1.5 I - 0.5 X X^T) X: the Gram matrix of the rows
+        NC_TRY(gemm<T>(m, gp(r, r, c, X, c, 0, X, c, 0, ow.gram, r, EPI_STORE_F32), st));
+        NC_RUN(K_OPTIM, 0, (double)r * r * (4.0 + es),
+               (ns_coeff_kernel<T><<<ew_grid((int64_t)r * r, m->num_sms), 256, 0, st>>>(ow.gram, r, Bm)));
+        NC_TRY(gemm<T>(m, gp(r, c, r, Bm, r, 0, X, c, 1, Y, c, EPI_STORE), st));
+      }
+      std::swap(X, Y);
+    }
+    NC_RUN(K_OPTIM, 0, n * (8.0 + 2.0 * es),
+           (muon_apply_kernel<T><<<ew_grid(n, m->num_sms), 256, 0, st>>>(master + off, X, weights + off, n,
+                                                                          o.lr_matrix, o.weight_decay)));
+  }
+  return NC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -932,6 +1024,49 @@ int nc_decode(nc_model *m, const void *weights, const int32_t *tokens, int B, vo
   cudaStream_t st = (cudaStream_t)stream;
   if (m->dtype == NC_F32) return decode_impl<float>(m, weights, tokens, B, cache, T_max, seqlens, workspace, logits, st);
   return decode_impl<bf16>(m, weights, tokens, B, cache, T_max, seqlens, workspace, logits, st);
+}
+
+int nc_optim_state_bytes(const nc_model *m, size_t *out) {
+  if (!m || !out) return NC_EINVAL;
+  *out = (size_t)3 * m->n_params * sizeof(float);
+  return NC_OK;
+}
+
+int nc_optim_workspace_bytes(const nc_model *m, size_t *out) {
+  if (!m || !out) return NC_EINVAL;
+  *out = optim_carve(m, nullptr, nullptr);
+  return NC_OK;
+}
+
+int nc_optim_init(nc_model *m, const void *weights, void *state, void *stream) {
+  if (!m || !weights || !state) return NC_EINVAL;
+  if (((uintptr_t)weights & 15) || ((uintptr_t)state & 15)) return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t N = m->n_params;
+  float *master = (float *)state;
+  if (m->dtype == NC_F32)
+    optim_init_kernel<float><<<ew_grid(N, m->num_sms), 256, 0, st>>>((const float *)weights, master, master + N,
+                                                                      master + 2 * N, N);
+  else
+    optim_init_kernel<bf16><<<ew_grid(N, m->num_sms), 256, 0, st>>>((const bf16 *)weights, master, master + N,
+                                                                     master + 2 * N, N);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_optim_step(nc_model *m, void *weights, const float *grads, void *state, int step, const nc_optim_opts *o,
+                  void *workspace, size_t ws_bytes, void *stream) {
+  if (!m || !weights || !grads || !state || !o || !workspace) return NC_EINVAL;
+  if (step < 1 || o->ns_steps < 0 || o->ns_steps > 100 || !(o->beta1 >= 0.f && o->beta1 < 1.f) ||
+      !(o->beta2 >= 0.f && o->beta2 < 1.f) || !(o->eps >= 0.f))
+    return NC_EINVAL;
+  if (ws_bytes < optim_carve(m, nullptr, nullptr)) return NC_ENOMEM;
+  if (((uintptr_t)weights & 15) || ((uintptr_t)grads & 15) || ((uintptr_t)state & 15) ||
+      ((uintptr_t)workspace & (kAlign - 1)))
+    return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m->dtype == NC_F32)
+    return optim_step_impl<float>(m, (float *)weights, grads, (float *)state, step, *o, workspace, st);
+  return optim_step_impl<bf16>(m, (bf16 *)weights, grads, (float *)state, step, *o, workspace, st);
 }
 
 int nc_sync_status(nc_model *m, void *stream, int timeout_ms) {

@@ -102,6 +102,34 @@ class Model:
             raise B.NcError(rc, "nc_fwd")
         return logits
 
+    # ---------------- optimizer ----------------
+
+    def optimizer_state(self, weights: torch.Tensor) -> torch.Tensor:
+        """fp32 state (master copy, moments) initialised from the weights."""
+        rc, n = B.nc_optim_state_bytes(self.handle)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_optim_state_bytes")
+        state = torch.empty(n // 4, dtype=torch.float32, device="cuda")
+        rc = B.nc_optim_init(self.handle, weights.data_ptr(), state.data_ptr(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_optim_init")
+        return state
+
+    def optimizer_step(self, weights: torch.Tensor, grads: torch.Tensor, state: torch.Tensor, step: int,
+                       opts: dict) -> None:
+        """One Muon / AdamW step.  opts: every field of nc_optim_opts (lr_matrix,
+        lr_embed, lr_head, lr_scalar, weight_decay, muon_momentum, ns_steps,
+        beta1, beta2, eps); the pages give no values, so there are no defaults."""
+        rc, n = B.nc_optim_workspace_bytes(self.handle)
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_optim_workspace_bytes")
+        if getattr(self, "_ows", None) is None or self._ows.numel() < n:
+            self._ows = torch.empty(n, dtype=torch.uint8, device="cuda")
+        rc = B.nc_optim_step(self.handle, weights.data_ptr(), grads.data_ptr(), state.data_ptr(), step, opts,
+                             self._ows.data_ptr(), self._ows.numel(), self._stream())
+        if rc != B.NC_OK:
+            raise B.NcError(rc, "nc_optim_step")
+
     # ---------------- inference with a KV cache ----------------
 
     def kv_cache(self, Bsz: int, T_max: int):

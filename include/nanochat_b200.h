@@ -222,6 +222,47 @@ int nc_prefill(nc_model *m, const void *weights, const int32_t *tokens, int B, i
 int nc_decode(nc_model *m, const void *weights, const int32_t *tokens, int B, void *cache, int T_max,
               int32_t *seqlens, void *workspace, size_t ws_bytes, void *logits, void *stream);
 
+/* The optimizer step ("Nanochat: full-stack LLM training in 8,000 lines for
+ * $72", section "A Llama-class transformer with ten modern departures": Muon
+ * for the transformer's matrices, AdamW for the embeddings and scalars;
+ * "nanochat - full-stack ChatGPT in ~8k lines", section "2. Pretrain").
+ * Groups by tensor: "matrix" = wq, wk, wv, wo, w1, w2 of every block (Muon,
+ * each matrix on its own); "embed" = wte and the value-embedding tables,
+ * "head" = lm_head, "scalar" = resid_lambdas, x0_lambdas, ve_gates (AdamW).
+ *   Muon:  buf = mu buf + g;  X = buf / |buf|_F;  ns_steps times
+ *          X = 1.5 X - 0.5 X X^T X (cubic Newton-Schulz towards the polar
+ *          factor of buf; the pages' "Polar Express" coefficients are not on
+ *          them);  w -= lr_matrix (X + weight_decay w)
+ *   AdamW: m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+ *          w -= lr (m / (1-b1^t)) / (sqrt(v / (1-b2^t)) + eps) + lr weight_decay w
+ * The learning-rate and momentum schedules (warm-up, warm-down; Muon's
+ * momentum 0.85 -> 0.97 -> 0.90) are the caller's: pass each step's values. */
+typedef struct {
+  float lr_matrix, lr_embed, lr_head, lr_scalar;
+  float weight_decay;   /* decoupled, every group */
+  float muon_momentum;
+  int ns_steps;         /* Newton-Schulz steps, 0..100 */
+  float beta1, beta2, eps;
+} nc_optim_opts;
+
+/* State: fp32, 3 * n_params: the master copy of the weights, m (AdamW's first
+ * moment or Muon's momentum) and v, each in the weight layout.  16-byte
+ * aligned caller-owned device memory. */
+int nc_optim_state_bytes(const nc_model *m, size_t *out);
+
+/* Device scratch of nc_optim_step (256-byte aligned). */
+int nc_optim_workspace_bytes(const nc_model *m, size_t *out);
+
+/* master = weights (widened to fp32), m = v = 0. */
+int nc_optim_init(nc_model *m, const void *weights, void *state, void *stream);
+
+/* One step t >= 1 with gradients grads (fp32, weight layout): updates the
+ * master copy, the moments, and weights (model dtype, rounded from the
+ * master copy).  NC_EINVAL for t < 1, betas outside [0, 1), eps < 0 or
+ * ns_steps outside 0..100; NC_ENOMEM for a short workspace. */
+int nc_optim_step(nc_model *m, void *weights, const float *grads, void *state, int step,
+                  const nc_optim_opts *opts, void *workspace, size_t ws_bytes, void *stream);
+
 /* Wait at most timeout_ms for the work enqueued so far on `stream` to finish
  * (polling, never blocking longer), then read and clear the device status
  * word.  Returns NC_ETIMEOUT if the stream is still busy, else the first
