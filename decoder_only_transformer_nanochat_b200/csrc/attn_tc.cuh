@@ -406,296 +406,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 // ===========================================================================
-// Forward, two heads per CTA.  MQA shares one K/V head among all query heads,
-// so a CTA takes the same 128 queries of two heads h0, h1: every K and V tile
-// loaded serves both.  TMEM holds one score tile S_x per head (P_x is written
-// back over the first 64 columns of S_x as bf16 pairs) and one accumulator
-// O_x per head:  S0 [0,128)  S1 [128,256)  O0 [256,384)  O1 [384,512).
-// The MMA warp issues, per key tile j,  PV0(j), S0(j+1), PV1(j), S1(j+1):
-// while one head's softmax runs the tensor core works on the other head.
-// Since tcgen05 MMAs of a CTA run in issue order, S_x(j+1) overwrites P_x(j)
-// only after PV_x(j) has read it, and the completion of S_x(j+1) also means
-// PV_x(j) is done, so O_x may be rescaled as soon as S_x(j+1) arrives.
-// Warps: 0 TMA, 1 MMA, 2..5 softmax of h0, 6..9 softmax of h1 (one thread
-// per query row, all 128 keys of a tile).
-constexpr int kPairThreads = 320;
-constexpr int kPairKStages = 2, kPairVStages = 2;
-constexpr int kPairSmem = 1024 + 2 * kTileBytes /*Q0, Q1*/ + (kPairKStages + kPairVStages) * kTileBytes + 256;
-static_assert(kPairSmem <= 232448, "shared memory per CTA");
-
-template <bool kWin>
-__global__ void __launch_bounds__(kPairThreads, 1)
-    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
-                         const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
-                         const __grid_constant__ CUtensorMap map_o,    // O [B][T][C], box 64 x 128
-                         const FwdParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;                                  // Q0, Q1
-  uint8_t *sK = sQ + 2 * kTileBytes;                   // K ring
-  uint8_t *sV = sK + kPairKStages * kTileBytes;        // V ring
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kPairVStages * kTileBytes);
-  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  const uint32_t q_full = smem_u32(bars + 0);
-  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto k_empty = [&](int s) { return smem_u32(bars + 3 + s); };
-  auto v_full = [&](int s) { return smem_u32(bars + 5 + s); };
-  auto v_empty = [&](int s) { return smem_u32(bars + 7 + s); };
-  auto s_full = [&](int x) { return smem_u32(bars + 9 + x); };
-  auto p_full = [&](int x) { return smem_u32(bars + 11 + x); };
-  const uint32_t o_done = smem_u32(bars + 13), drain = smem_u32(bars + 14);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int HP = (p.H + 1) / 2;                      // head pairs
-  const int BHP = gridDim.x / p.n_qt;
-  const int qt = p.n_qt - 1 - (int)blockIdx.x / BHP;  // latest query tiles (most keys) first
-  const int hp = ((int)blockIdx.x % BHP) % HP, b = ((int)blockIdx.x % BHP) / HP;
-  const int h0 = 2 * hp, h1 = min(2 * hp + 1, p.H - 1);  // odd H: the last pair repeats h0, stored once
-  const int q0 = qt * kQ;
-  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kKV : 0;
-  const int n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV - kt_lo;
-  const int kbase = kt_lo * kKV;
-  const int C = p.H * kD;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
-      mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
-      mbar_init(s_full(s), 1);
-      mbar_init(p_full(s), 128);
-    }
-    mbar_init(o_done, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer: Q0, Q1, then K_j, V_j in turn ----------------
-      mbar_expect_tx(q_full, 2 * kTileBytes);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_3d(smem_u32(sQ) + i * 16384, &map_qk, h0 * kD + 64 * i, q0, b, q_full);
-        tma_load_3d(smem_u32(sQ) + kTileBytes + i * 16384, &map_qk, h1 * kD + 64 * i, q0, b, q_full);
-      }
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1, ph = ((j >> 1) & 1) ^ 1;
-        if (!mbar_wait(k_empty(st), ph, abort_flag, p.status)) break;
-        mbar_expect_tx(k_full(st), kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sK) + st * kTileBytes + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b,
-                      k_full(st));
-        if (!mbar_wait(v_empty(st), ph, abort_flag, p.status)) break;
-        mbar_expect_tx(v_full(st), kTileBytes);
-        for (int hh = 0; hh < 2; ++hh)
-          for (int a = 0; a < 2; ++a)
-            tma_load_3d(smem_u32(sV) + st * kTileBytes + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a,
-                        kbase + j * kKV + 64 * hh, b, v_full(st));
-        ++issued;
-      }
-      // no copy of ours may still be landing when the CTA exits
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued - 2); j < issued; ++j) {
-        const uint64_t t1 = globaltimer();
-        while (!mbar_try(k_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
-        while (!mbar_try(v_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t idesc_s = make_idesc(0, 0, kQ, kKV);   // Q K^T: both K-major
-      const uint32_t idesc_o = make_idesc(0, 1, kQ, kD);    // P V: P from TMEM, V MN-major
-      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dKd = smem_desc(smem_u32(sK), 16, 1024);
-      const uint64_t dVd = smem_desc(smem_u32(sV), 8192, 1024);
-      constexpr uint32_t kQ1 = kTileBytes >> 4;
-      auto issue_s = [&](int x, int j) {
-        const uint64_t bK = dKd + (uint64_t)(((j & 1) * kTileBytes) >> 4);
-        const uint64_t aQ = dQd + (x ? kQ1 : 0u);
-#pragma unroll
-        for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t off = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + x * kKV, aQ + off, bK + off, idesc_s, s > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full(x));
-      };
-      auto issue_pv = [&](int x, int j) {
-        const uint64_t bV = dVd + (uint64_t)(((j & 1) * kTileBytes) >> 4);
-#pragma unroll
-        for (int s = 0; s < kKV / 16; ++s) {
-          const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;  // V: MN-major, 16 keys per step
-          tc_mma_ts(tmem + 2 * kKV + x * kD, tmem + x * kKV + 8 * s, bV + b_off, idesc_o,
-                    (j > 0 || s > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full(0), 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        tc_commit(k_empty(0));
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int ph = (j >> 1) & 1;
-        if (!(ok = mbar_wait(v_full(j & 1), ph, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(p_full(0), j & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        const bool more = j + 1 < n_kv;
-        if (more) {
-          if (!(ok = mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        if (!(ok = mbar_wait(p_full(1), j & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        tc_commit(v_empty(j & 1));
-        if (more) {
-          issue_s(1, j + 1);
-          tc_commit(k_empty((j + 1) & 1));
-        }
-      }
-      tc_commit(o_done);
-      tc_commit(drain);
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
-    }
-  } else {
-    // ---------------- softmax warps: thread = query row of head x ----------------
-    const int x = (warp - 2) >> 2;                   // warps 2..5: head h0, 6..9: head h1
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int row = q0 + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_col = lane_base + x * kKV;
-    const float sc = rsqrtf((float)kD) * kLog2e;
-    float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = mbar_wait(s_full(x), j & 1, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const int kv0 = kbase + j * kKV;
-      const bool edge = kv0 + kKV > q0 || kv0 + kKV > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window);
-      // pass 1: the row max of the raw scores (scale > 0 commutes with max),
-      // 32 columns of TMEM at a time
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(s_col + 32 * c, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = kv0 + 32 * c + i;
-          const bool dead = edge && (key > row || key >= p.T || (kWin && row - key >= p.window));
-          mx = dead ? mx : fmaxf(mx, __uint_as_float(rr[i]));
-        }
-      }
-      mx *= sc;
-      // the exponent base moves only when the row max grows by more than 2^8;
-      // S_x(j) completing means PV_x(j-1) is done, so O_x can be rescaled now
-      if (j == 0 || mx > m_used + kRescaleLog2) {
-        if (j > 0) {
-          const float corr = ex2(m_used - mx);
-          l *= corr;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(lane_base + 2 * kKV + x * kD + c * 32, rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * corr);
-            tmem_st32(lane_base + 2 * kKV + x * kD + c * 32, rr);
-          }
-        }
-        m_used = mx;
-      }
-      // with a window a row may see no key of its first tile: base 0 there
-      const float mb = (kWin && m_used == -INFINITY) ? 0.f : m_used;
-      // pass 2: P = 2^(s sc - base) chunk by chunk; P's 16 columns of chunk c
-      // go over S columns [16c, 16c + 16), all of them already read
-      float sum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32], pk[16];
-        tmem_ld32(s_col + 32 * c, rr);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int key = kv0 + 32 * c + i;
-          float a = fmaf(__uint_as_float(rr[i]), sc, -mb), b = fmaf(__uint_as_float(rr[i + 1]), sc, -mb);
-          if (edge) {
-            if (key > row || key >= p.T || (kWin && row - key >= p.window)) a = -INFINITY;
-            if (key + 1 > row || key + 1 >= p.T || (kWin && row - key - 1 >= p.window)) b = -INFINITY;
-          }
-          // one exponential in four on the FMA pipe, the rest on MUFU
-          const float e0 = ex2(a);
-          const float e1 = (i & 2) ? ex2_poly(b) : ex2(b);
-          sum += e0 + e1;
-          pk[i / 2] = pack2(e0, e1);
-        }
-        tmem_st16_nw(s_col + 16 * c, pk);
-      }
-      tmem_wait_st();
-      l += sum;
-      tc_fence_before();
-      mbar_arrive(p_full(x));
-    }
-    // ---------------- epilogue: O_x / l, lse ----------------
-    if (ok) ok = mbar_wait(o_done, 0, abort_flag, p.status);
-    ok = __all_sync(0xffffffffu, ok);
-    const int hx = x ? h1 : h0;
-    const bool store = x == 0 || h1 != h0;
-    uint8_t *sO = sQ + x * kTileBytes;  // Q_x is no longer read
-    if (ok) {
-      tc_fence_after();
-      const float inv = 1.f / l;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + 2 * kKV + x * kD + c * 32, rr);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 w;
-          w.x = pack2(__uint_as_float(rr[8 * u + 0]) * inv, __uint_as_float(rr[8 * u + 1]) * inv);
-          w.y = pack2(__uint_as_float(rr[8 * u + 2]) * inv, __uint_as_float(rr[8 * u + 3]) * inv);
-          w.z = pack2(__uint_as_float(rr[8 * u + 4]) * inv, __uint_as_float(rr[8 * u + 5]) * inv);
-          w.w = pack2(__uint_as_float(rr[8 * u + 6]) * inv, __uint_as_float(rr[8 * u + 7]) * inv);
-          *reinterpret_cast<uint4 *>(sO + tile_unit(r, c * 4 + u)) = w;
-        }
-      }
-      if (store && row < p.T) p.lse[((int64_t)b * p.H + hx) * p.T + row] = (m_used + __log2f(l)) * (1.f / kLog2e);
-    }
-    fence_proxy_async();
-    // the four warps of this head meet (named barrier 2 + x), then one stores
-    asm volatile("bar.sync %0, 128;" ::"r"(2 + x) : "memory");
-    if (ok && store && (warp & 3) == 2 && lane == 0) {
-      for (int i = 0; i < 2; ++i) tma_store_3d(&map_o, smem_u32(sO) + i * 16384, hx * kD + 64 * i, q0, b);
-      bulk_commit();
-      bulk_wait0();
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// ===========================================================================
 // Backward.  With P = exp(S - lse) recomputed from the saved log-sum-exp and
 // D = rowsum(dO * O):  dS = P (dO V^T - D),  dQ = dS K / sqrt(d),
 // dK = dS^T Q / sqrt(d) and dV = P^T dO, the last two summed over every query
@@ -1589,8 +1299,7 @@ inline bool make_map3(CUtensorMap *map, const void *base, int B, int T, int cols
 template <bool kWin>
 inline cudaError_t init_variant() {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attn_fwd_pair_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
   if (e == cudaSuccess)
@@ -1630,19 +1339,12 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.lse = lse;
   p.status = status;
   p.window = window;
-  const int grid = B * ((H + 1) / 2) * p.n_qt;
+  const int grid = B * H * p.n_qt;
   const bool win = windowed(window, T);
-  if (win) attn_fwd_pair_kernel<true><<<grid, kPairThreads, kPairSmem, st>>>(mqk, mv, mo, p);
-  else attn_fwd_pair_kernel<false><<<grid, kPairThreads, kPairSmem, st>>>(mqk, mv, mo, p);
+  if (win) attn_fwd_tc_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  else attn_fwd_tc_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
   const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    cudaFuncAttributes a;
-    const cudaError_t ea = win ? cudaFuncGetAttributes(&a, attn_fwd_pair_kernel<true>)
-                               : cudaFuncGetAttributes(&a, attn_fwd_pair_kernel<false>);
-    fprintf(stderr, "nanochat_b200: attention forward launch: %s (registers %d, max threads %d, smem %d)\n",
-            cudaGetErrorString(e), ea == cudaSuccess ? a.numRegs : -1, ea == cudaSuccess ? a.maxThreadsPerBlock : -1,
-            kPairSmem);
-  }
+  if (e != cudaSuccess) fprintf(stderr, "nanochat_b200: attention forward launch: %s\n", cudaGetErrorString(e));
   return e;
 }
 

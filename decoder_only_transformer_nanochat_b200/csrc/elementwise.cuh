@@ -263,21 +263,14 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(
   float c[8], s[8];
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
   T *row = qkv + (size_t)tok * ld;
-  // the next head pair is loaded before the current one is worked on, so a
-  // warp always has a load in flight
-  float x[8];
-  if (hw < H + 1) Vec8<T>::load(row + hw * kHeadDim + j * 8, x);
-  else
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = 0.f;
   for (int h0 = 0; h0 < H + 1; h0 += 2) {
     const int h = h0 + hw;
     const bool live = h < H + 1;  // uniform per half-warp
-    float xn[8];
-    if (h + 2 < H + 1) Vec8<T>::load(row + (h + 2) * kHeadDim + j * 8, xn);
+    float x[8];
+    if (live) Vec8<T>::load(row + h * kHeadDim + j * 8, x);
     else
 #pragma unroll
-      for (int i = 0; i < 8; ++i) xn[i] = 0.f;
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
     float y[8], ss = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -298,8 +291,6 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(
         else rk[tok] = r;
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = xn[i];
   }
 }
 
@@ -320,25 +311,16 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
   T *drow = dqkv + (size_t)tok * ld;
   const T *yrow = qkv + (size_t)tok * ld;
-  // the next head pair is loaded before the current one is worked on
-  float dy[8], y[8];
-  if (hw < H + 1) {
-    Vec8<T>::load(drow + hw * kHeadDim + j * 8, dy);
-    Vec8<T>::load(yrow + hw * kHeadDim + j * 8, y);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { dy[i] = 0.f; y[i] = 0.f; }
-  }
   for (int h0 = 0; h0 < H + 1; h0 += 2) {
     const int h = h0 + hw;
     const bool live = h < H + 1;
-    float dyn[8], yn[8];
-    if (h + 2 < H + 1) {
-      Vec8<T>::load(drow + (h + 2) * kHeadDim + j * 8, dyn);
-      Vec8<T>::load(yrow + (h + 2) * kHeadDim + j * 8, yn);
+    float dy[8], y[8];
+    if (live) {
+      Vec8<T>::load(drow + h * kHeadDim + j * 8, dy);
+      Vec8<T>::load(yrow + h * kHeadDim + j * 8, y);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { dyn[i] = 0.f; yn[i] = 0.f; }
+      for (int i = 0; i < 8; ++i) { dy[i] = 0.f; y[i] = 0.f; }
     }
     const float r = live ? (h < H ? rq[(size_t)tok * H + h] : rk[tok]) : 0.f;
     float dot = 0.f;
@@ -355,11 +337,6 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
       out[i] = j < 8 ? g[i] * c[i] + partner * s[i] : g[i] * c[i] - partner * s[i];
     }
     if (live) Vec8<T>::store(drow + h * kHeadDim + j * 8, out);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      dy[i] = dyn[i];
-      y[i] = yn[i];
-    }
   }
 }
 

@@ -90,12 +90,16 @@ def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_r
     worst = min(cos, key=cos.get)
     fields.update(min_cos=cos[worst], min_cos_tensor=worst)
     record("step", **fields)
+    # a tensor whose exact gradient vanishes (a one-key window: a softmax over
+    # one key has no gradient with respect to its score) is compared against
+    # the largest gradient: its computed values are rounding noise of that size
+    gmax = max(float(np.max(np.abs(g_ref[name]))) for name, _, _ in lay)
     if dtype == "f32":
         assert abs(loss_gpu - loss_ref) <= F32_LOSS_REL * abs(loss_ref), (loss_gpu, loss_ref)
         for name, _, _ in lay:
             ref = g_ref[name]
             err = np.max(np.abs(g_gpu[name] - ref))
-            scale = np.max(np.abs(ref))
+            scale = max(float(np.max(np.abs(ref))), 1e-6 * gmax)
             report[name] = err / scale if scale > 0 else err
             assert err <= F32_GRAD_MAXABS * scale, (name, err, scale)
         if tl_gpu is not None:
@@ -103,6 +107,9 @@ def compare(dtype, lay, loss_gpu, g_gpu_flat, loss_ref, g_ref, tl_gpu=None, tl_r
     else:
         assert abs(loss_gpu - loss_ref) <= BF16_LOSS_ABS, (loss_gpu, loss_ref)
         for name, _, _ in lay:
+            if np.max(np.abs(g_ref[name])) <= 1e-6 * gmax:
+                assert np.max(np.abs(g_gpu[name])) <= 1e-3 * gmax, name  # a vanishing gradient
+                continue
             c = cosine(g_gpu[name], g_ref[name])
             report[name] = c
             assert c >= BF16_GRAD_COS, (name, c)
