@@ -327,39 +327,58 @@ __global__ void __launch_bounds__(256) segsum_kernel(Src src, const int32_t *__r
 }
 
 // A segment that starts in chunk c and continues: tail[c] + head[c+1] + ...
-// up to the chunk whose head run ends it, added in chunk order.
+// up to the chunk whose head run ends it.  The 8 warps of the CTA each add
+// every 8th head partial (warp w: chunks c+1+w, c+9+w, ... in order), then
+// the partials meet in a fixed order (tail, warp 0, ..., warp 7): the same
+// sum on every run, with a chain 8 times shorter than one warp's.
+constexpr int kFixCols = 256;  // float4 columns per pass
 __global__ void __launch_bounds__(256) seg_fixup_kernel(const int32_t *__restrict__ skey, int M, int C,
                                                         const float *__restrict__ head,
                                                         const float *__restrict__ tail,
                                                         const int *__restrict__ flags, int nchunks,
                                                         float *__restrict__ out, int accumulate) {
+  __shared__ float4 part[8][kFixCols];
   const int c = blockIdx.x;
   if (!(flags[c] & kSegTail)) return;
   const int tok = skey[min(M, (c + 1) * kSegChunk) - 1];
   int last = c + 1;
   while (last < nchunks - 1 && !(flags[last] & kSegHeadEnds)) ++last;
-  for (int q = threadIdx.x; q < C / 4; q += blockDim.x) {
-    float4 a = reinterpret_cast<const float4 *>(tail + (size_t)c * C)[q];
-    int k = c + 1;
-    for (; k + 4 <= last + 1; k += 4) {
-      float4 h[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C4 = C / 4;
+  for (int q0 = 0; q0 < C4; q0 += kFixCols) {
+    float4 acc[kFixCols / 32];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) h[u] = reinterpret_cast<const float4 *>(head + (size_t)(k + u) * C)[q];
+    for (int i = 0; i < kFixCols / 32; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = c + 1 + warp; k <= last; k += 8) {
+      const float4 *hk = reinterpret_cast<const float4 *>(head + (size_t)k * C) + q0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a.x += h[u].x; a.y += h[u].y; a.z += h[u].z; a.w += h[u].w;
+      for (int i = 0; i < kFixCols / 32; ++i) {
+        const int q = lane + 32 * i;
+        if (q0 + q < C4) {
+          const float4 h = hk[q];
+          acc[i].x += h.x; acc[i].y += h.y; acc[i].z += h.z; acc[i].w += h.w;
+        }
       }
     }
-    for (; k <= last; ++k) {
-      const float4 h = reinterpret_cast<const float4 *>(head + (size_t)k * C)[q];
-      a.x += h.x; a.y += h.y; a.z += h.z; a.w += h.w;
+#pragma unroll
+    for (int i = 0; i < kFixCols / 32; ++i) part[warp][lane + 32 * i] = acc[i];
+    __syncthreads();
+    const int q = q0 + (int)threadIdx.x;
+    if (threadIdx.x < kFixCols && q < C4) {
+      float4 a = reinterpret_cast<const float4 *>(tail + (size_t)c * C)[q];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float4 h = part[w][threadIdx.x];
+        a.x += h.x; a.y += h.y; a.z += h.z; a.w += h.w;
+      }
+      float4 *o = reinterpret_cast<float4 *>(out + (size_t)tok * C) + q;
+      if (accumulate) {
+        const float4 bb = *o;
+        a.x += bb.x; a.y += bb.y; a.z += bb.z; a.w += bb.w;
+      }
+      *o = a;
     }
-    float4 *o = reinterpret_cast<float4 *>(out + (size_t)tok * C) + q;
-    if (accumulate) {
-      const float4 b = *o;
-      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-    }
-    *o = a;
+    __syncthreads();
   }
 }
 
