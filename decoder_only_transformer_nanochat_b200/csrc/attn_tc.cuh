@@ -679,303 +679,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-// ---------------- dQ, two heads per CTA ----------------
-// CTA = the same 128 queries of two heads h0, h1 of row b (MQA: each K, V tile
-// loaded serves both).  TMEM per head x: X_x (S_x, then dP_x of the same tile;
-// dS_x as bf16 pairs over its first 64 columns, the A operand of dQ) and the
-// accumulator dQ_x:  X0 [0,128)  X1 [128,256)  dQ0 [256,384)  dQ1 [384,512).
-// MMA order per key tile: S0, S1, dP0, dP1, dQ0, (S0 of the next tile), dQ1,
-// (S1 of the next tile), ... -- one head's element-wise work overlaps the
-// other head's MMAs.  In-order MMA execution keeps every reuse of X_x safe:
-// dP_x(j) is issued after the element-wise warps read S_x(j), S_x(j+1) after
-// dQ_x(j) (which reads dS_x(j) from X_x).  Shared memory: Q and dO of both
-// heads (128 KB), K in two stages, V in one (it is read by dP only).
-constexpr int kDqpThreads = 320;
-constexpr int kDqpSmem = 1024 + 4 * kTileBytes + 3 * kTileBytes + 256;
-static_assert(kDqpSmem <= 232448, "shared memory per CTA");
-
-template <bool kWin>
-__global__ void __launch_bounds__(kDqpThreads, 1)
-    attn_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128
-                            const __grid_constant__ CUtensorMap map_do,   // dO [B][T][C], box 64 x 128
-                            const __grid_constant__ CUtensorMap map_dq,   // dqkv, box 64 x 128
-                            const BwdParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;                      // Q0, Q1
-  uint8_t *sG = sQ + 2 * kTileBytes;       // dO0, dO1
-  uint8_t *sK = sG + 2 * kTileBytes;       // K ring (2 stages)
-  uint8_t *sV = sK + 2 * kTileBytes;       // V (1 stage)
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kTileBytes);
-  // q_full, k_full[2], k_empty[2], v_full, v_empty, s_full[2], x_free[2], dp_full[2], ds_full[2], fin, drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  const uint32_t q_full = smem_u32(bars + 0);
-  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto k_empty = [&](int s) { return smem_u32(bars + 3 + s); };
-  const uint32_t v_full = smem_u32(bars + 5), v_empty = smem_u32(bars + 6);
-  auto s_full = [&](int x) { return smem_u32(bars + 7 + x); };
-  auto x_free = [&](int x) { return smem_u32(bars + 9 + x); };
-  auto dp_full = [&](int x) { return smem_u32(bars + 11 + x); };
-  auto ds_full = [&](int x) { return smem_u32(bars + 13 + x); };
-  const uint32_t fin = smem_u32(bars + 15), drain = smem_u32(bars + 16);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int HP = (p.H + 1) / 2;
-  const int BHP = gridDim.x / p.n_tiles;
-  const int qt = p.n_tiles - 1 - (int)blockIdx.x / BHP;  // latest query tiles (most keys) first
-  const int hp = ((int)blockIdx.x % BHP) % HP, b = ((int)blockIdx.x % BHP) / HP;
-  const int h0 = 2 * hp, h1 = min(2 * hp + 1, p.H - 1);   // odd H: the last pair repeats h0, stored once
-  const int q0 = qt * kQ;
-  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kBK : 0;
-  const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK - kt_lo;
-  const int kbase = kt_lo * kBK;
-  const int C = p.H * kD;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
-      mbar_init(s_full(s), 1);
-      mbar_init(x_free(s), 128);
-      mbar_init(dp_full(s), 1);
-      mbar_init(ds_full(s), 128);
-    }
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
-    mbar_init(fin, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer: Q and dO of both heads, then K_j, V_j ----------------
-      mbar_expect_tx(q_full, 4 * kTileBytes);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_3d(smem_u32(sQ) + i * 16384, &map_q, h0 * kD + 64 * i, q0, b, q_full);
-        tma_load_3d(smem_u32(sQ) + kTileBytes + i * 16384, &map_q, h1 * kD + 64 * i, q0, b, q_full);
-        tma_load_3d(smem_u32(sG) + i * 16384, &map_do, h0 * kD + 64 * i, q0, b, q_full);
-        tma_load_3d(smem_u32(sG) + kTileBytes + i * 16384, &map_do, h1 * kD + 64 * i, q0, b, q_full);
-      }
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j & 1;
-        if (!mbar_wait(k_empty(ks), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-        mbar_expect_tx(k_full(ks), kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, kbase + j * kBK, b,
-                      k_full(ks));
-        ++issued_k;
-        if (!mbar_wait(v_empty, (j & 1) ^ 1, abort_flag, p.status)) break;
-        mbar_expect_tx(v_full, kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sV) + i * 16384, &map_q, C + kD + 64 * i, kbase + j * kBK, b, v_full);
-        ++issued_v;
-      }
-      // let the loads in flight land before the CTA can exit
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued_k - 2); j < issued_k; ++j) {
-        const uint64_t t1 = globaltimer();
-        while (!mbar_try(k_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
-      }
-      if (issued_v > 0) {
-        const uint64_t t1 = globaltimer();
-        while (!mbar_try(v_full, (issued_v - 1) & 1) && globaltimer() - t1 < kWaitNs) {}
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t idesc_s = make_idesc(0, 0, kQ, kBK);   // Q K^T, dO V^T: both K-major
-      const uint32_t idesc_q = make_idesc(0, 1, kQ, kD);    // dS K: dS from TMEM, K MN-major
-      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dGd = smem_desc(smem_u32(sG), 16, 1024);
-      const uint64_t dKs = smem_desc(smem_u32(sK), 16, 1024);      // K-major view of K stage 0
-      const uint64_t dKm = smem_desc(smem_u32(sK), 16384, 1024);   // MN-major view of K stage 0
-      const uint64_t dVs = smem_desc(smem_u32(sV), 16, 1024);
-      constexpr uint32_t kT1 = kTileBytes >> 4;  // head 1's tile after head 0's
-      auto issue_s = [&](int x, int j) {
-        const uint64_t k = dKs + (uint64_t)(((j & 1) * kTileBytes) >> 4);
-#pragma unroll
-        for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + x * kBK, dQd + (x ? kT1 : 0u) + o, k + o, idesc_s, s > 0);
-        }
-        tc_commit(s_full(x));
-      };
-      auto issue_dp = [&](int x) {
-#pragma unroll
-        for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + x * kBK, dGd + (x ? kT1 : 0u) + o, dVs + o, idesc_s, s > 0);
-        }
-        tc_commit(dp_full(x));
-      };
-      auto issue_dq = [&](int x, int j) {
-        const uint64_t k = dKm + (uint64_t)(((j & 1) * kTileBytes) >> 4);
-#pragma unroll
-        for (int s = 0; s < kBK / 16; ++s)
-          tc_mma_ts(tmem + 2 * kBK + x * kD, tmem + x * kBK + 8 * s, k + ((s * 2048) >> 4), idesc_q,
-                    (j > 0 || s > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full(0), 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const uint32_t par = j & 1;
-        if (!(ok = mbar_wait(v_full, par, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(x_free(0), par, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_dp(0);
-        if (!(ok = mbar_wait(x_free(1), par, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_dp(1);
-        tc_commit(v_empty);  // V_j is read by the two dP only
-        const bool more = j + 1 < n_kv;
-        if (!(ok = mbar_wait(ds_full(0), par, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_dq(0, j);
-        if (more) {
-          if (!(ok = mbar_wait(k_full((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        if (!(ok = mbar_wait(ds_full(1), par, abort_flag, p.status))) break;
-        tc_fence_after();
-        issue_dq(1, j);
-        tc_commit(k_empty(j & 1));  // K_j is done after both dQ
-        if (more) issue_s(1, j + 1);
-      }
-      tc_commit(fin);
-      tc_commit(drain);
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
-    }
-  } else {
-    // ---------------- element-wise warps: thread = query row of head x ----------------
-    const int x = (warp - 2) >> 2;
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int row = q0 + r;
-    const int hx = x ? h1 : h0;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t x_col = lane_base + x * kBK;
-    const float sc = rsqrtf((float)kD) * kLog2e;
-    const int rr_ = min(row, p.T - 1);
-    const float L = p.lse[((int64_t)b * p.H + hx) * p.T + rr_] * kLog2e;
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-    // D = rowsum(dO * O) for this row: dO from the staged tile, O from global
-    float Dv = 0.f;
-    if (ok && row < p.T) {
-      const bf16 *orow = p.O + ((int64_t)b * p.T + row) * C + hx * kD;
-      const uint8_t *grow = sG + x * kTileBytes;
-#pragma unroll 4
-      for (int u = 0; u < 16; ++u) {
-        float o8[8], g8[8];
-        Vec8<bf16>::load(orow + 8 * u, o8);
-        Vec8<bf16>::load(reinterpret_cast<const bf16 *>(grow + tile_unit(r, u)), g8);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) Dv += o8[i] * g8[i];
-      }
-      if (x == 0 || h1 != h0) p.Drow[((int64_t)b * p.H + hx) * p.T + row] = Dv;
-    }
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const uint32_t par = j & 1;
-      ok = mbar_wait(s_full(x), par, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const int kv0 = kbase + j * kBK;
-      const bool edge = kv0 + kBK > q0 || kv0 + kBK > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window);
-      // P = 2^(s sc - L) for the 128 keys, kept as bf16 pairs
-      uint32_t pp[64];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(x_col + 32 * c, v);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int key = kv0 + 32 * c + i;
-          float a = ex2(fmaf(__uint_as_float(v[i]), sc, -L)), bb = ex2(fmaf(__uint_as_float(v[i + 1]), sc, -L));
-          if (edge) {
-            if (key > row || key >= p.T || (kWin && row - key >= p.window)) a = 0.f;
-            if (key + 1 > row || key + 1 >= p.T || (kWin && row - key - 1 >= p.window)) bb = 0.f;
-          }
-          pp[16 * c + i / 2] = pack2(a, bb);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(x_free(x));  // X_x may take dP_x now
-      ok = mbar_wait(dp_full(x), par, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      // dS = P (dP - D), chunk by chunk, written over X columns already read
-      // (unrolled: pp is indexed by constants and stays in registers)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32], ds[16];
-        tmem_ld32(x_col + 32 * c, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162 *>(&pp[16 * c + i]);
-          const float2 pf = __bfloat1622float2(pr);
-          ds[i] = pack2(pf.x * (__uint_as_float(v[2 * i]) - Dv), pf.y * (__uint_as_float(v[2 * i + 1]) - Dv));
-        }
-        tmem_st16_nw(x_col + 16 * c, ds);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(ds_full(x));
-    }
-    if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
-    ok = __all_sync(0xffffffffu, ok);
-    const bool store = x == 0 || h1 != h0;
-    uint8_t *sO = sQ + x * kTileBytes;  // Q_x is no longer read
-    if (ok) {
-      tc_fence_after();
-      const float scale = rsqrtf((float)kD);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + 2 * kBK + x * kD + c * 32, rr);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 w;
-          w.x = pack2(__uint_as_float(rr[8 * u + 0]) * scale, __uint_as_float(rr[8 * u + 1]) * scale);
-          w.y = pack2(__uint_as_float(rr[8 * u + 2]) * scale, __uint_as_float(rr[8 * u + 3]) * scale);
-          w.z = pack2(__uint_as_float(rr[8 * u + 4]) * scale, __uint_as_float(rr[8 * u + 5]) * scale);
-          w.w = pack2(__uint_as_float(rr[8 * u + 6]) * scale, __uint_as_float(rr[8 * u + 7]) * scale);
-          *reinterpret_cast<uint4 *>(sO + tile_unit(r, c * 4 + u)) = w;
-        }
-      }
-    }
-    fence_proxy_async();
-    asm volatile("bar.sync %0, 128;" ::"r"(2 + x) : "memory");
-    if (ok && store && (warp & 3) == 2 && lane == 0) {
-      for (int i = 0; i < 2; ++i) tma_store_3d(&map_dq, smem_u32(sO) + i * 16384, hx * kD + 64 * i, q0, b);
-      bulk_commit();
-      bulk_wait0();
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
 // ---------------- dK, dV: CTA = 128 keys of row b; loop over heads x 128-query tiles ----------------
 // 128-query tiles keep every MMA at N = 128.  TMEM holds one 128-column
 // score buffer X that takes S^T and then dP^T of a tile in turn, P^T and dS^T
@@ -1302,8 +1005,7 @@ inline cudaError_t init_variant() {
 
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attn_bwd_dq_pair_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqpSmem);
+
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemTc);
   return e;
@@ -1373,9 +1075,8 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   p.n_tiles = (T + kQ - 1) / kQ;
   p.window = window;
   const bool win = windowed(window, T);
-  const int grid_dq = B * ((H + 1) / 2) * p.n_tiles;
-  if (win) attn_bwd_dq_pair_kernel<true><<<grid_dq, kDqpThreads, kDqpSmem, st>>>(mq128, mdo128, mout, p);
-  else attn_bwd_dq_pair_kernel<false><<<grid_dq, kDqpThreads, kDqpSmem, st>>>(mq128, mdo128, mout, p);
+  if (win) attn_bwd_dq_tc_kernel<true><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
+  else attn_bwd_dq_tc_kernel<false><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     fprintf(stderr, "nanochat_b200: attention dQ launch: %s\n", cudaGetErrorString(e));

@@ -290,7 +290,9 @@ def test_windowed_attention_fwd_bwd(nc, B, T, H, window, dtype, engine):
     for i, (g, r) in enumerate(parts):
         scale = np.abs(r).max()
         if window == 1 and i < 2:
-            assert np.max(np.abs(g)) <= 1e-6  # one key per query: softmax constant, dq = dk = 0
+            # one key per query: the softmax is constant, dq = dk = 0 up to the
+            # rounding of dP - D (a few ulps of dv's size)
+            assert np.max(np.abs(g)) <= 1e-5 * np.abs(parts[2][1]).max()
             continue
         if dtype == "f32":
             np.testing.assert_allclose(g, r, rtol=0, atol=1e-4 * scale)
