@@ -410,6 +410,7 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
   // positions grouped by token: the embedding's and the value embeddings'
   // table gradients are summed per token in this fixed order
   NC_RUN(K_TOKEN_SORT, 0, M * 16.0 * sort_passes(V), sort_tokens(tokens, M, V, w.sort, st));
+  m->launches[K_TOKEN_SORT] += 3 * sort_passes(V) - 1;  // one accounting entry, three launches per pass
   const int nch = seg_chunks(M);
   const unsigned nblk8 = rows_grid(M, 8);
 
