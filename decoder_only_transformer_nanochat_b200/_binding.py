@@ -90,6 +90,10 @@ _SIGS = {
     "nc_ops_status": (_I, [_P, _I]),
     "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
+    "nc_rmsnorm": (_I, [_P, _P, _P, _I, _I, _I, _P]),
+    "nc_rmsnorm_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "nc_rope_qknorm": (_I, [_P, _P, ctypes.c_int64, _P, _P, _I, _I, _P]),
+    "nc_rope_qknorm_bwd": (_I, [_P, _P, _P, ctypes.c_int64, _P, _P, _I, _I, _P]),
 }
 
 NC_EPI_STORE = 0
@@ -283,6 +287,22 @@ def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, st
 
 def nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream) -> int:
     return load_library().nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream)
+
+
+def nc_rmsnorm(x, y, r, M, C, dtype, stream) -> int:
+    return load_library().nc_rmsnorm(x, y, r, M, C, dtype, stream)
+
+
+def nc_rmsnorm_bwd(dy, y, r, dx, dx_t, M, C, accumulate, dtype, stream) -> int:
+    return load_library().nc_rmsnorm_bwd(dy, y, r, dx, dx_t, M, C, accumulate, dtype, stream)
+
+
+def nc_rope_qknorm(handle, qkv, ld, rq, rk, B, T, stream) -> int:
+    return load_library().nc_rope_qknorm(handle, qkv, ld, rq, rk, B, T, stream)
+
+
+def nc_rope_qknorm_bwd(handle, dqkv, qkv, ld, rq, rk, B, T, stream) -> int:
+    return load_library().nc_rope_qknorm_bwd(handle, dqkv, qkv, ld, rq, rk, B, T, stream)
 
 
 def nc_ops_status(stream, timeout_ms: int) -> int:

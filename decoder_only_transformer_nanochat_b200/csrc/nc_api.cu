@@ -1242,6 +1242,83 @@ int nc_softcap_ce(void *z, int64_t ldz, const int32_t *targets, float *token_los
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
 }
 
+static bool rows_ok(int M, int C, const void *a, const void *b, const void *c) {
+  return M >= 1 && C >= 8 && C % 8 == 0 && C <= 32 * kMaxVecPerLane * 8 &&
+         !(((uintptr_t)a | (uintptr_t)b | (uintptr_t)c) & 15);
+}
+
+int nc_rmsnorm(const void *x, void *y, float *r, int M, int C, int dtype, void *stream) {
+  if (!x || !y || !r) return NC_EINVAL;
+  if (M < 1 || C < 8 || C % 8 || C > 32 * kMaxVecPerLane * 8) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (!rows_ok(M, C, x, y, nullptr) || ((uintptr_t)r & 3)) return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == NC_BF16)
+    NC_DISPATCH_NV(C, (rmsnorm_kernel<bf16, NV><<<rows_grid(M, 8), 256, 0, st>>>((const bf16 *)x, (bf16 *)y, r,
+                                                                                 M, C)));
+  else
+    NC_DISPATCH_NV(C, (rmsnorm_kernel<float, NV><<<rows_grid(M, 8), 256, 0, st>>>((const float *)x, (float *)y,
+                                                                                  r, M, C)));
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_rmsnorm_bwd(const void *dy, const void *y, const float *r, float *dx, void *dx_t, int M, int C,
+                   int accumulate, int dtype, void *stream) {
+  if (!dy || !y || !r || !dx || !dx_t) return NC_EINVAL;
+  if (M < 1 || C < 8 || C % 8 || C > 32 * kMaxVecPerLane * 8) return NC_ESHAPE;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (!rows_ok(M, C, dy, y, dx) || ((uintptr_t)dx_t & 15) || ((uintptr_t)r & 3)) return NC_EALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int acc = accumulate ? 1 : 0;
+  if (dtype == NC_BF16)
+    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<bf16, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                          (const bf16 *)dy, (const bf16 *)y, r, dx, (bf16 *)dx_t, M, C, acc)));
+  else
+    NC_DISPATCH_NV(C, (rmsnorm_bwd_kernel<float, NV><<<rows_grid(M, 8), 256, 0, st>>>(
+                          (const float *)dy, (const float *)y, r, dx, (float *)dx_t, M, C, acc)));
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+static int rope_args_ok(const nc_model *m, const void *a, const void *b, int64_t ld, int B, int T) {
+  if (B < 1 || T < 1 || T > m->seq || ld < (int64_t)kHeadDim * (m->H + 2) || ld > INT32_MAX ||
+      (int64_t)B * T * ld > ((int64_t)1 << 40))
+    return NC_ESHAPE;
+  const int es = m->dtype == NC_BF16 ? 2 : 4;
+  if ((((uintptr_t)a | (uintptr_t)b) & 15) || (ld * es) % 16) return NC_EALIGN;
+  return NC_OK;
+}
+
+int nc_rope_qknorm(const nc_model *m, void *qkv, int64_t ld, float *rq, float *rk, int B, int T, void *stream) {
+  if (!m || !qkv || !rq || !rk) return NC_EINVAL;
+  const int rc = rope_args_ok(m, qkv, nullptr, ld, B, T);
+  if (rc != NC_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int M = B * T;
+  if (m->dtype == NC_BF16)
+    rope_qknorm_kernel<bf16><<<rows_grid((size_t)M, 8), 256, 0, st>>>((bf16 *)qkv, (int)ld, rq, rk, m->rope_cos,
+                                                                      m->rope_sin, M, T, m->H);
+  else
+    rope_qknorm_kernel<float><<<rows_grid((size_t)M, 8), 256, 0, st>>>((float *)qkv, (int)ld, rq, rk, m->rope_cos,
+                                                                       m->rope_sin, M, T, m->H);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_rope_qknorm_bwd(const nc_model *m, void *dqkv, const void *qkv, int64_t ld, const float *rq,
+                       const float *rk, int B, int T, void *stream) {
+  if (!m || !dqkv || !qkv || !rq || !rk) return NC_EINVAL;
+  const int rc = rope_args_ok(m, dqkv, qkv, ld, B, T);
+  if (rc != NC_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int M = B * T;
+  if (m->dtype == NC_BF16)
+    rope_qknorm_bwd_kernel<bf16><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
+        (bf16 *)dqkv, (const bf16 *)qkv, (int)ld, rq, rk, m->rope_cos, m->rope_sin, M, T, m->H);
+  else
+    rope_qknorm_bwd_kernel<float><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
+        (float *)dqkv, (const float *)qkv, (int)ld, rq, rk, m->rope_cos, m->rope_sin, M, T, m->H);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
 int nc_ops_status(void *stream, int timeout_ms) {
   SymbolAddrs a;
   if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;

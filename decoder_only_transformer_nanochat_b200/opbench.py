@@ -6,6 +6,7 @@ it every shape that grows with the tokens, so a capture holds a few GB).
 
     python -m decoder_only_transformer_nanochat_b200.opbench --op w1_fwd --iters 5
     python -m decoder_only_transformer_nanochat_b200.opbench --op ce --tokens 8192
+    python -m decoder_only_transformer_nanochat_b200.opbench --op rmsnorm --tokens 65536
 """
 from __future__ import annotations
 
@@ -35,6 +36,7 @@ def gemm_shapes(M: int) -> dict:
 
 
 GEMMS = gemm_shapes(16 * 2048)
+ROW_OPS = ["rmsnorm", "rmsnorm_bwd", "rope", "rope_bwd"]
 
 
 def main():
@@ -43,7 +45,8 @@ def main():
     import decoder_only_transformer_nanochat_b200 as nc
     from decoder_only_transformer_nanochat_b200 import build
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm", "ce"])
+    ap.add_argument("--op", required=True,
+                    choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm", "ce"] + ROW_OPS)
     ap.add_argument("--tokens", type=int, default=16 * 2048, help="M (a multiple of 2048)")
     ap.add_argument("--window", type=int, default=0, help="attention: sliding window (0: causal)")
     ap.add_argument("--shape", default=None, help="for --op gemm: M,N,K,a_mn,b_mn,EPILOGUE")
@@ -93,6 +96,57 @@ def main():
                             nc.NC_BF16, code, args.engine, st)
             assert rc == 0, rc
         flops = 2.0 * m * n * k
+    elif args.op in ("rmsnorm", "rmsnorm_bwd"):
+        M = args.tokens
+        x = torch.randn(M * C, device="cuda", generator=g).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        r = torch.empty(M, device="cuda", dtype=torch.float32)
+        assert nc.nc_rmsnorm(x.data_ptr(), y.data_ptr(), r.data_ptr(), M, C, nc.NC_BF16, st) == 0
+        if args.op == "rmsnorm":
+            def run():
+                assert nc.nc_rmsnorm(x.data_ptr(), y.data_ptr(), r.data_ptr(), M, C, nc.NC_BF16, st) == 0
+            nbytes = M * (2.0 * C * 2 + 4)
+        else:
+            dy = torch.randn(M * C, device="cuda", generator=g).to(torch.bfloat16)
+            dx = torch.zeros(M * C, device="cuda", dtype=torch.float32)
+            dx_t = torch.empty_like(x)
+
+            def run():  # accumulating into the residual-stream gradient, as the step does
+                assert nc.nc_rmsnorm_bwd(dy.data_ptr(), y.data_ptr(), r.data_ptr(), dx.data_ptr(),
+                                         dx_t.data_ptr(), M, C, 1, nc.NC_BF16, st) == 0
+            nbytes = M * (C * (2.0 + 2.0 + 4.0 + 4.0 + 2.0) + 4)
+        flops = 0.0
+    elif args.op in ("rope", "rope_bwd"):
+        from decoder_only_transformer_nanochat_b200 import Model
+        model = Model(depth=20, vocab=V, seq=T, dtype="bf16")
+        ld = 128 * (H + 2)
+        qkv = (torch.randn(B * T * ld, device="cuda", generator=g) * 0.09).to(torch.bfloat16)
+        rq = torch.empty(B * T * H, device="cuda", dtype=torch.float32)
+        rk = torch.empty(B * T, device="cuda", dtype=torch.float32)
+        assert nc.nc_rope_qknorm(model.handle, qkv.data_ptr(), ld, rq.data_ptr(), rk.data_ptr(), B, T, st) == 0
+        per_head = 128 * 2.0
+        if args.op == "rope":
+            qkv0 = qkv.clone()
+
+            def prep():
+                qkv.copy_(qkv0)  # in place: every launch starts from the projections
+
+            def run():
+                assert nc.nc_rope_qknorm(model.handle, qkv.data_ptr(), ld, rq.data_ptr(), rk.data_ptr(), B, T,
+                                         st) == 0
+            nbytes = B * T * (H + 1) * (2 * per_head + 4)
+        else:
+            d0 = (torch.randn(B * T * ld, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+            dqkv = d0.clone()
+
+            def prep():
+                dqkv.copy_(d0)
+
+            def run():
+                assert nc.nc_rope_qknorm_bwd(model.handle, dqkv.data_ptr(), qkv.data_ptr(), ld, rq.data_ptr(),
+                                             rk.data_ptr(), B, T, st) == 0
+            nbytes = B * T * (H + 1) * (3 * per_head + 4)
+        flops = 0.0
     else:
         ld = 128 * (H + 2)
         qkv = (torch.randn(B * T * ld, device="cuda", generator=g) * 0.09).to(torch.bfloat16)
@@ -136,6 +190,8 @@ def main():
         out["tflops"] = flops / (med / 1000) / 1e12
     if args.op == "ce":
         out["gbs"] = 2.0 * args.tokens * V * 2 / (med / 1000) / 1e9  # z read once, dz written once
+    if args.op in ROW_OPS:
+        out["gbs"] = nbytes / (med / 1000) / 1e9  # every operand read once, every output written once
     print(json.dumps(out))
 
 

@@ -136,6 +136,39 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
 int nc_softcap_ce(void *z, int64_t ldz, const int32_t *targets, float *token_loss, int M, int V,
                   float grad_scale, int dtype, void *stream);
 
+/* Parameterless RMSNorm of M rows of C ("A Llama-class transformer with ten
+ * modern departures": RMSNorm without learnable parameters):
+ *   r[m] = 1 / sqrt(mean_c x[m,c]^2 + eps),  y[m,c] = x[m,c] r[m],  eps = 2^-23
+ * x, y: [M, C] row-major in dtype (y may equal x); r: [M] fp32.  The kernel
+ * the model's norms run.  8 <= C <= 4096 with C % 8 == 0 (else NC_ESHAPE);
+ * x, y 16-byte aligned and r 4-byte aligned (else NC_EALIGN). */
+int nc_rmsnorm(const void *x, void *y, float *r, int M, int C, int dtype, void *stream);
+
+/* Its backward, with the residual-stream gradient it feeds:
+ *   g[m,c] = r[m] (dy[m,c] - y[m,c] mean_c(dy[m,:] y[m,:]))
+ *   dx = g (accumulate == 0) or dx + g (accumulate != 0), dx fp32 [M, C];
+ *   dx_t = the new dx in dtype (the next GEMM's operand).
+ * y, r: the outputs of nc_rmsnorm.  Shapes and alignment as nc_rmsnorm (dx,
+ * dx_t 16-byte aligned). */
+int nc_rmsnorm_bwd(const void *dy, const void *y, const float *r, float *dx, void *dx_t, int M, int C,
+                   int accumulate, int dtype, void *stream);
+
+/* RoPE (theta 10,000, dims i and i+64 of each head rotated by the angle
+ * pos * 10000^(-i/64), pos = row index mod T) then QK-norm (parameterless
+ * RMSNorm over each head's 128 dims), in place on the m->H query heads and the
+ * shared key head of the fused rows qkv [B*T, ld] = [q | k | v] ("ten modern
+ * departures": rotary embeddings, QK normalisation after them).  rq [B*T, H]
+ * and rk [B*T] receive the heads' reciprocal rms.  The model's RoPE tables
+ * are used, so T <= the model's seq (else NC_ESHAPE); ld >= 128 (H + 2)
+ * elements; qkv 16-byte aligned with 16-byte rows (else NC_EALIGN). */
+int nc_rope_qknorm(const nc_model *m, void *qkv, int64_t ld, float *rq, float *rk, int B, int T, void *stream);
+
+/* Backward of nc_rope_qknorm, in place on the q and k parts of dqkv [B*T, ld]
+ * (the v part is left as it is): qkv, rq, rk are nc_rope_qknorm's outputs.
+ *   g = r (dy - y mean(dy y)) per head, then the rotation by -angle. */
+int nc_rope_qknorm_bwd(const nc_model *m, void *dqkv, const void *qkv, int64_t ld, const float *rq,
+                       const float *rk, int B, int T, void *stream);
+
 /* Status of the op-level calls above (nc_gemm, nc_attention_*, and the
  * calls below), which have no model handle: waits at most timeout_ms for the
  * work enqueued so far on `stream` (polling), then reads and clears the
