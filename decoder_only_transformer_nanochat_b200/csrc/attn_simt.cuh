@@ -327,9 +327,10 @@ namespace nc {
 template <typename T>
 inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H, int window,
                                    int engine, int *status, cudaStream_t st) {
-  if (sizeof(T) == 2 && engine == 0) {
+  if (sizeof(T) == 2 && (engine == 0 || engine == 2)) {
     if (!fatc::supported(qkv, ld, O)) return cudaErrorInvalidValue;
-    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, window, status, st);
+    const bool pp = (engine == 0) == fatc::kFwdPingPongDefault;
+    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, window, pp, status, st);
   }
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, window, st);
 }

@@ -405,6 +405,311 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
+// ---------------- forward, ping-pong: two softmax warpgroups on alternating key tiles ----------------
+// Same CTA (128 queries of one (row b, head h)), TMA warp and operand layouts
+// as above; what changes is how the element-wise work is split:
+//   warps 2..5  softmax of the even key tiles, warps 6..9 of the odd ones;
+//               thread = query row, the whole 128-key tile of its row in
+//               registers, its own running max and sum (no exchange between
+//               threads, no block-wide barrier inside the key loop)
+//   warp 1      MMA: S_j = Q K_j^T into TMEM buffer j & 1, P_j written back
+//               over S_j as bf16 pairs, O_{j&1} += P_j V_j; tensor-core order
+//               S_0, S_1, PV_0, S_2, PV_1, S_3 ... (MMAs issued by one thread
+//               run in order, so S_{j+2} overwrites P_j only after PV_j read it)
+// TMEM: S/P_0 [0,128), S/P_1 [128,256), O_0 [256,384), O_1 [384,512).
+// The two partial outputs are merged once at the end:
+//   m = max(m_0, m_1),  a_g = 2^(m_g - m),
+//   O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1),  lse = m + log2(a_0 l_0 + a_1 l_1)
+// (log2 domain), the online-softmax merge of two disjoint key sets.  The
+// commit that signals S_j covers every earlier MMA, so a group that rescales
+// its O on a grown max finds its previous P V already complete.
+constexpr int kPpOCol = 256;  // O_g at kPpOCol + 128 g
+// engine 0 runs this kernel when true, the one above when false (engine 2 the other)
+constexpr bool kFwdPingPongDefault = false;
+
+template <bool kWin>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
+                       const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
+                       const __grid_constant__ CUtensorMap map_o,    // O [B][T][C], box 64 x 128
+                       const FwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;
+  uint8_t *sK = sQ + kTileBytes;
+  uint8_t *sV = sK + kKStages * kTileBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kVStages * kTileBytes);
+  // bars: q_full, k_full[3], k_empty[3], s_full[2], p_full[2], o_done[2],
+  //       v_full[2], v_empty[2], drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *sML = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [group][m, l][128]
+  const uint32_t q_full = smem_u32(bars + 0);
+  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
+  auto k_empty = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
+  auto p_full = [&](int s) { return smem_u32(bars + 9 + s); };
+  auto o_done = [&](int s) { return smem_u32(bars + 11 + s); };
+  auto v_full = [&](int s) { return smem_u32(bars + 13 + s); };
+  auto v_empty = [&](int s) { return smem_u32(bars + 15 + s); };
+  const uint32_t drain = smem_u32(bars + 17);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = gridDim.x / p.n_qt;
+  const int qt = p.n_qt - 1 - (int)blockIdx.x / BH;  // latest query tiles (most keys) first
+  const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
+  const int q0 = qt * kQ;
+  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kKV : 0;
+  const int n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV - kt_lo;
+  const int kbase = kt_lo * kKV;
+  const int C = p.H * kD;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), 128);  // one warpgroup
+      mbar_init(o_done(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (as in the kernel above) ----------------
+      mbar_expect_tx(q_full, kTileBytes);
+      for (int i = 0; i < 2; ++i) tma_load_3d(smem_u32(sQ) + i * 16384, &map_qk, h * kD + 64 * i, q0, b, q_full);
+      int issued_k = 0, issued_v = 0;
+      auto load_k = [&](int j) -> bool {
+        const int st = j % kKStages;
+        if (!mbar_wait(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
+        const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
+        mbar_expect_tx(k_full(st), kTileBytes);
+        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b, k_full(st));
+        ++issued_k;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(v_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
+        mbar_expect_tx(v_full(st), kTileBytes);
+        for (int hh = 0; hh < 2; ++hh)
+          for (int a = 0; a < 2; ++a)
+            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, kbase + j * kKV + 64 * hh, b,
+                        v_full(st));
+        ++issued_v;
+        return true;
+      };
+      bool okp = load_k(0) && (n_kv < 2 || load_k(1));
+      for (int j = 0; j < n_kv && okp; ++j) {
+        if (j + 2 < n_kv && !load_k(j + 2)) break;
+        if (!load_v(j)) break;
+      }
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
+      for (int j = max(0, issued_k - kKStages); j < issued_k; ++j) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(k_full(j % kKStages), (j / kKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+      for (int j = max(0, issued_v - 2); j < issued_v; ++j) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(v_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc_s = make_idesc(0, 0, kQ, kKV);
+      const uint32_t idesc_o = make_idesc(0, 1, kQ, kD);
+      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dKd = smem_desc(smem_u32(sK), 16, 1024);
+      const uint64_t dVd = smem_desc(smem_u32(sV), 8192, 1024);
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      auto issue_s = [&](int j) -> bool {
+        const int ks = j % kKStages;
+        if (!mbar_wait(k_full(ks), (j / kKStages) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint64_t bK = dKd + (uint64_t)((ks * kTileBytes) >> 4);
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+          const uint32_t off = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+          tc_mma(tmem + (j & 1) * kKV, dQd + off, bK + off, idesc_s, s > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full(j & 1));
+        tc_commit(k_empty(ks));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && n_kv > 1) ok = issue_s(1);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int bb = j & 1;
+        if (!(ok = mbar_wait(p_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(v_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint64_t bV = dVd + (uint64_t)((bb * kTileBytes) >> 4);
+        const uint32_t a_p = tmem + bb * kKV;  // P_j over the first 64 columns of S_j
+#pragma unroll
+        for (int s = 0; s < kKV / 16; ++s) {
+          const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;
+          tc_mma_ts(tmem + kPpOCol + bb * kD, a_p + 8 * s, bV + b_off, idesc_o, (j >= 2 || s > 0) ? 1u : 0u);
+        }
+        tc_commit(o_done(bb));
+        tc_commit(v_empty(bb));
+        if (j + 2 < n_kv) ok = issue_s(j + 2);
+      }
+      tc_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ---------------- softmax warpgroups: group g takes key tiles j = g, g + 2, ... ----------------
+    const int grp = (warp - 2) >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int row = q0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t t_s = lane_base + grp * kKV;           // S_j, then P_j
+    const uint32_t t_o = lane_base + kPpOCol + grp * kD;  // this group's O
+    const float sc = rsqrtf((float)kD) * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = grp; j < n_kv; j += 2) {
+      ok = mbar_wait(s_full(grp), (j >> 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      float s[kKV];
+      {
+        uint32_t u[kKV];
+#pragma unroll
+        for (int c = 0; c < kKV / 32; ++c) tmem_ld32_nw(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < kKV; ++i) s[i] = __uint_as_float(u[i]);  // raw scores: the scale goes into the exponent
+      }
+      const int kv0 = kbase + j * kKV;
+      if (kv0 + kKV - 1 > q0 || kv0 + kKV > p.T || (kWin && kv0 <= q0 + kQ - 1 - p.window)) {
+#pragma unroll
+        for (int i = 0; i < kKV; ++i)
+          if (kv0 + i > row || kv0 + i >= p.T || (kWin && row - (kv0 + i) >= p.window)) s[i] = -INFINITY;
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < kKV; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sc;
+      // the exponent base moves only when the max grows by more than 2^8
+      const bool first = j == grp;
+      const bool grow = first || mx > m_used + kRescaleLog2;
+      const float corr = (!first && grow) ? ex2(m_used - mx) : 1.f;
+      if (grow) {
+        l *= corr;
+        m_used = mx;
+      }
+      // a row that has seen no key yet (windows only) keeps its base at -inf
+      // and takes its exponentials against 0 (all of them 0)
+      const float nmb = m_used == -INFINITY ? 0.f : -m_used;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kKV / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int k = 32 * c + i;
+          // one exponential in four on the FMA pipe
+          const float e0 = ex2(fmaf(s[k], sc, nmb));
+          const float e1 = (i & 2) ? ex2_poly(fmaf(s[k + 1], sc, nmb)) : ex2(fmaf(s[k + 1], sc, nmb));
+          sum4[(i >> 1) & 3] += e0 + e1;
+          pk[i / 2] = pack2(e0, e1);
+        }
+        tmem_st16_nw(t_s + 16 * c, pk);  // keys [32c, 32c + 32) as 16 columns of bf16 pairs
+      }
+      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (!first && __any_sync(0xffffffffu, grow)) {
+        // the max grew: bring this group's O to the new base before P_j V_j
+        // adds to it (its previous P V is complete: see the kernel's header)
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(t_o + 32 * c, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * corr);
+          tmem_st32(t_o + 32 * c, rr);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(grp));
+    }
+    // ---------------- merge of the two groups, O / l, lse ----------------
+    const int last = n_kv - 1 - ((n_kv - 1 - grp) & 1);  // this group's last tile (-1: none)
+    if (ok && last >= 0) ok = mbar_wait(o_done(grp), (last >> 1) & 1, abort_flag, p.status);
+    ok = __all_sync(0xffffffffu, ok);
+    sML[(grp * 2 + 0) * kQ + r] = m_used;
+    sML[(grp * 2 + 1) * kQ + r] = l;
+    ok = epi_vote_all256(ok);  // also the barrier that publishes sML
+    const int n1 = n_kv / 2;   // tiles of group 1 (group 0 has at least one)
+    if (ok) {
+      tc_fence_after();
+      const float m0 = sML[r], l0 = sML[kQ + r];
+      const float m1 = sML[2 * kQ + r], l1 = sML[3 * kQ + r];
+      const float mm = fmaxf(m0, m1);
+      const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+      const float a1 = (n1 == 0 || m1 == -INFINITY) ? 0.f : ex2(m1 - mm);
+      const float lt = a0 * l0 + a1 * l1;
+      const float inv = 1.f / lt;
+      const float f0 = a0 * inv, f1 = a1 * inv;
+      // group g writes O's columns [64g, 64g + 64)
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const int col = 64 * grp + 32 * c;
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nw(lane_base + kPpOCol + col, r0);
+        if (n1 > 0) tmem_ld32_nw(lane_base + kPpOCol + kD + col, r1);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          o[i] = n1 > 0 ? __uint_as_float(r0[i]) * f0 + __uint_as_float(r1[i]) * f1 : __uint_as_float(r0[i]) * f0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack2(o[8 * u + 0], o[8 * u + 1]);
+          w.y = pack2(o[8 * u + 2], o[8 * u + 3]);
+          w.z = pack2(o[8 * u + 4], o[8 * u + 5]);
+          w.w = pack2(o[8 * u + 6], o[8 * u + 7]);
+          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, 8 * grp + 4 * c + u)) = w;  // Q is no longer read
+        }
+      }
+      if (grp == 0 && row < p.T) p.lse[((int64_t)b * p.H + h) * p.T + row] = (mm + __log2f(lt)) * (1.f / kLog2e);
+    }
+    fence_proxy_async();
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (ok && warp == 2 && lane == 0) {
+      for (int i = 0; i < 2; ++i) tma_store_3d(&map_o, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
+      bulk_commit();
+      bulk_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ===========================================================================
 // Backward.  With P = exp(S - lse) recomputed from the saved log-sum-exp and
 // D = rowsum(dO * O):  dS = P (dO V^T - D),  dQ = dS K / sqrt(d),
@@ -1002,6 +1307,8 @@ inline bool make_map3(CUtensorMap *map, const void *base, int B, int T, int cols
 template <bool kWin>
 inline cudaError_t init_variant() {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_fwd_pp_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
 
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
@@ -1027,8 +1334,9 @@ inline bool supported(const void *qkv, int64_t ld, const void *O) {
   return encode_fn() != nullptr && aligned(qkv, ld, O);
 }
 
+// pingpong: the kernel with two softmax warpgroups on alternating key tiles
 inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int window,
-                              int *status, cudaStream_t st) {
+                              bool pingpong, int *status, cudaStream_t st) {
   CUtensorMap mqk, mv, mo;
   const int C = H * kD;
   if (!make_map3(&mqk, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mv, qkv, B, T, (int)ld, ld, 64) ||
@@ -1043,8 +1351,13 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.window = window;
   const int grid = B * H * p.n_qt;
   const bool win = windowed(window, T);
-  if (win) attn_fwd_tc_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
-  else attn_fwd_tc_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  if (pingpong) {
+    if (win) attn_fwd_pp_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+    else attn_fwd_pp_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  } else {
+    if (win) attn_fwd_tc_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+    else attn_fwd_tc_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) fprintf(stderr, "nanochat_b200: attention forward launch: %s\n", cudaGetErrorString(e));
   return e;

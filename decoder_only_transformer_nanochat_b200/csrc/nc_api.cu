@@ -1165,8 +1165,8 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
   if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
   if (window < 0) return NC_EINVAL;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
-  if (engine < 0 || engine > 1) return NC_EINVAL;
-  if (dtype == NC_BF16 && engine == 0 && !fatc::aligned(qkv, ld, O)) return NC_EALIGN;
+  if (engine < 0 || engine > 2) return NC_EINVAL;
+  if (dtype == NC_BF16 && engine != 1 && !fatc::aligned(qkv, ld, O)) return NC_EALIGN;
   int num_sms = 0, *status = nullptr;
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;

@@ -162,8 +162,9 @@ ATTN_CASES = [(1, 1, 1), (2, 9, 2), (1, 130, 3), (2, 256, 2), (1, 515, 10)]
 
 @pytest.mark.parametrize("B,T,H", ATTN_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 2])
 def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
+    # engine 2: the other tcgen05 forward kernel; its O and lse then feed the backward
     import torch
     code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
     qkv, ld, q, k, v = _attn_inputs(B, T, H, 100 + T + H, dtype)
@@ -189,7 +190,7 @@ def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
     Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
     dqkv = torch.zeros(B * T, ld, dtype=qkv_d.dtype, device="cuda")
     assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
-                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine, st) == 0
+                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine % 2, st) == 0
     assert nc.nc_ops_status(st, 60000) == nc.NC_OK
     got = dqkv.float().cpu().numpy().astype(np.float64)
     dq_ref = np.empty((B, T, H, 128))
@@ -248,7 +249,7 @@ WINDOW_CASES = [(1, 515, 3, 1), (1, 515, 3, 64), (2, 256, 2, 129), (1, 300, 10, 
 
 @pytest.mark.parametrize("B,T,H,window", WINDOW_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 2])
 def test_windowed_attention_fwd_bwd(nc, B, T, H, window, dtype, engine):
     # sliding window (query i sees keys j with 0 <= i - j < window) against the
     # full-block oracle's windowed attention
@@ -279,7 +280,8 @@ def test_windowed_attention_fwd_bwd(nc, B, T, H, window, dtype, engine):
     Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
     dqkv = torch.zeros(B * T, ld, dtype=qkv_d.dtype, device="cuda")
     assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
-                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine, st, window=window) == 0
+                               Drow.data_ptr(), dqkv.data_ptr(), B, T, H, code, engine % 2, st,
+                               window=window) == 0
     assert nc.nc_ops_status(st, 60000) == nc.NC_OK
     got = dqkv.float().cpu().numpy().astype(np.float64)
     refs = [np.empty((B, T, H, 128)), np.empty((B, T, 128)), np.empty((B, T, 128))]
