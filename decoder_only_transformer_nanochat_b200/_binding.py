@@ -90,6 +90,9 @@ _SIGS = {
     "nc_ops_status": (_I, [_P, _I]),
     "nc_softcap_ce": (_I, [_P, ctypes.c_int64, _P, _P, _I, _I, ctypes.c_float, _I, _P]),
     "nc_check_wait_expiry": (_I, [_I, _P]),
+    "nc_attention_bwd_scratch_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "nc_attention_bwd_ex": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _I, _I, _I, _I,
+                                 _I, _I, _P]),
     "nc_rmsnorm": (_I, [_P, _P, _P, _I, _I, _I, _P]),
     "nc_rmsnorm_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "nc_rope_qknorm": (_I, [_P, _P, ctypes.c_int64, _P, _P, _I, _I, _P]),
@@ -287,6 +290,18 @@ def nc_attention_bwd(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, dtype, engine, st
 
 def nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream) -> int:
     return load_library().nc_softcap_ce(z, ldz, targets, token_loss, M, V, grad_scale, dtype, stream)
+
+
+def nc_attention_bwd_scratch_bytes(B, T, H, window: int = 0):
+    n = ctypes.c_size_t(0)
+    rc = load_library().nc_attention_bwd_scratch_bytes(B, T, H, window, ctypes.byref(n))
+    return rc, n.value
+
+
+def nc_attention_bwd_ex(qkv, ld, O, dO, lse, Drow, scratch, scratch_bytes, dqkv, B, T, H, dtype, engine, stream,
+                        window: int = 0) -> int:
+    return load_library().nc_attention_bwd_ex(qkv, ld, O, dO, lse, Drow, scratch, scratch_bytes, dqkv, B, T, H,
+                                              window, dtype, engine, stream)
 
 
 def nc_rmsnorm(x, y, r, M, C, dtype, stream) -> int:

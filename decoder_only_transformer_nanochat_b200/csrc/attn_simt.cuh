@@ -337,14 +337,17 @@ inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B
 
 // D = rowsum(dO * O) is computed inside the tcgen05 dQ kernel; the CUDA-core
 // engine gets it from attn_rowdot_kernel first.  Drow is [B, H, T] scratch.
+// part: scratch that lets the tcgen05 dK/dV kernel cut large key tiles into
+// pieces (fatc::dkdv_scratch_bytes; nullptr: no cut).
 template <typename T>
 inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *O, const T *dO, const float *lse, float *Dr,
                                    T *dqkv, int B, int T_len, int H, int window, int engine, int *status,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, float *part = nullptr, size_t part_bytes = 0,
+                                   int num_sms = 148) {
   if (sizeof(T) == 2 && engine == 0) {
     if (!fatc::supported_bwd(qkv, ld, O, dO, dqkv)) return cudaErrorInvalidValue;
-    return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, (bf16 *)dqkv, B,
-                            T_len, H, window, status, st);
+    return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, part, part_bytes,
+                            (bf16 *)dqkv, B, T_len, H, window, num_sms, status, st);
   }
   const int M = B * T_len;
   attn_rowdot_kernel<T><<<(unsigned)(((size_t)M * H + 7) / 8), 256, 0, st>>>(dO, O, Dr, M, T_len, H);

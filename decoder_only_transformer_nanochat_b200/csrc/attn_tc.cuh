@@ -737,7 +737,22 @@ struct BwdParams {
   float *Drow;        // [B, H, T]: rowsum(dO * O), written by the dQ kernel
   const bf16 *O;      // [B*T, H*128]
   int *status;
+  // dK/dV schedule: key tile kt's (head, query tile) iterations are cut into
+  // ceil(n_it / chunk) pieces, one CTA each (chunk = 0: one piece); a tile cut
+  // into several pieces leaves fp32 partial sums in `part` that
+  // attn_bwd_dkdv_reduce_kernel adds in piece order
+  int B, chunk;
+  float *part;        // [grid][128][256]: dK | dV rows of a piece, unscaled
 };
+
+// Iterations (head x 128-query tile) of key tile kt in the dK/dV kernel.
+__host__ __device__ inline int dkdv_iters(int kt, int n_tiles, int H, int window, bool win) {
+  const int last_q = win ? min(n_tiles - 1, (kt * 128 + 127 + window - 1) / 128) : n_tiles - 1;
+  return (last_q - kt + 1) * H;
+}
+__host__ __device__ inline int dkdv_pieces(int n_it, int chunk) {
+  return chunk > 0 ? (n_it + chunk - 1) / chunk : 1;
+}
 
 template <bool kWin>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -1028,17 +1043,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t fin = smem_u32(bars + kB + 8), drain = smem_u32(bars + kB + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Bn = gridDim.x / p.n_tiles;
-  const int kt = (int)blockIdx.x / Bn;  // key tile 0 has the most work: launched first
-  const int b = (int)blockIdx.x % Bn;
+  // CTA -> (key tile, piece, row b): pieces of key tile 0 (the most work) first
+  const int b = (int)blockIdx.x % p.B;
+  int kt = 0, piece = (int)blockIdx.x / p.B, n_it = 0, n_pieces = 1;
+  for (;; ++kt) {
+    n_it = dkdv_iters(kt, p.n_tiles, p.H, p.window, kWin);
+    n_pieces = dkdv_pieces(n_it, p.chunk);
+    if (piece < n_pieces || kt == p.n_tiles - 1) break;
+    piece -= n_pieces;
+  }
+  const int it0 = (int)((int64_t)piece * n_it / n_pieces), it1 = (int)((int64_t)(piece + 1) * n_it / n_pieces);
+  const int my_n = it1 - it0;  // this CTA's iterations it0 .. it1 - 1
   const int k0 = kt * kQ;
   const int C = p.H * kD;
   const int first = k0 / kBQ2;
-  const int n_q_all = (p.T + kBQ2 - 1) / kBQ2;
-  // with a window the last query that sees key k0 + 127 is k0 + 127 + window - 1
-  const int last_q = kWin ? min(n_q_all - 1, (k0 + kQ - 1 + p.window - 1) / kBQ2) : n_q_all - 1;
-  const int n_q = last_q - first + 1;
-  const int n_it = n_q * p.H;
+  const int n_q = n_it / p.H;  // iteration it: head it / n_q, query tile first + it % n_q
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < kKvStages; ++s) {
@@ -1075,9 +1094,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
-      const int st = it % kKvStages;
-      const bool okw = mbar_wait(q_empty(st), ((it / kKvStages) & 1) ^ 1, abort_flag, p.status);
+    for (int j = 0; j < my_n; ++j) {
+      const int it = it0 + j, st = j % kKvStages;
+      const bool okw = mbar_wait(q_empty(st), ((j / kKvStages) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, okw)) break;
       const int hh = it / n_q, qq0 = (first + it % n_q) * kBQ2;
       uint8_t *stage = sQS + st * kQStage;
@@ -1142,7 +1161,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         x_mma(dKd, dQs);
         tc_commit(s_full);
       }
-      for (int j = 0; j < n_it && ok; ++j) {
+      for (int j = 0; j < my_n && ok; ++j) {
         const int st = j % kKvStages;
         const uint64_t qs = dQs + (uint64_t)((st * kQStage) >> 4), qm = dQm + (uint64_t)((st * kQStage) >> 4);
         const uint32_t par = j & 1;
@@ -1157,7 +1176,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         g_mma(kDvCol, kPtCol, qm + kGo, j == 0);
         tc_commit(p_empty);
         // S^T_{j+1} = K Q_{j+1}^T once dP^T_j has left X
-        if (j + 1 < n_it) {
+        if (j + 1 < my_n) {
           const int st1 = (j + 1) % kKvStages;
           if (!(ok = mbar_wait(dp_taken, par, abort_flag, p.status))) break;
           if (!(ok = mbar_wait(q_full(st1), ((j + 1) / kKvStages) & 1, abort_flag, p.status))) break;
@@ -1186,12 +1205,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sc = rsqrtf((float)kD) * kLog2e;
     const int c0 = g * 64;  // this thread's 64 queries of the 128-query tile
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int st = it % kKvStages;
-      const uint32_t par = it & 1;
-      const int qq0 = (first + it % n_q) * kBQ2 + c0;
+    for (int j = 0; j < my_n; ++j) {
+      const int st = j % kKvStages;
+      const uint32_t par = j & 1;
+      const int qq0 = (first + (it0 + j) % n_q) * kBQ2 + c0;
       ok = mbar_wait(s_full, par, abort_flag, p.status) &&
-           mbar_wait(ld_full(st), (it / kKvStages) & 1, abort_flag, p.status);
+           mbar_wait(ld_full(st), (j / kKvStages) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t xv[64];
@@ -1251,7 +1270,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    const bool split = n_pieces > 1;
+    // a piece of a split key tile: its fp32 rows (dK | dV, unscaled) go to the
+    // idle Q/dO stages, 16-byte unit u of row r at unit (u ^ (r & 7)), then out
+    // to its partial-sum slot with coalesced stores
+    float *stg = reinterpret_cast<float *>(sQS);
+    if (ok && split) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_base + (g == 0 ? kDkCol : kDvCol) + c * 32, rr);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int u = 32 * g + 8 * c + q;
+          *reinterpret_cast<float4 *>(stg + r * 256 + ((u ^ (r & 7)) << 2)) =
+              make_float4(__uint_as_float(rr[4 * q]), __uint_as_float(rr[4 * q + 1]), __uint_as_float(rr[4 * q + 2]),
+                          __uint_as_float(rr[4 * q + 3]));
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       // warpgroup 0 drains dK (scaled) into the K tile, warpgroup 1 dV into the V tile
       uint8_t *dst = g == 0 ? sK : sV;
@@ -1273,7 +1311,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     fence_proxy_async();
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (ok && warp == 2 && lane == 0) {
+    if (ok && split) {
+      float4 *dst = reinterpret_cast<float4 *>(p.part + (size_t)blockIdx.x * kQ * 2 * kD);
+      for (int q = (int)threadIdx.x - 64; q < kQ * 64; q += kSoft) {
+        const int row = q >> 6, u = q & 63;
+        dst[q] = *reinterpret_cast<const float4 *>(stg + row * 256 + ((u ^ (row & 7)) << 2));
+      }
+    } else if (ok && warp == 2 && lane == 0) {
       for (int i = 0; i < 2; ++i) {
         tma_store_3d(&map_out, smem_u32(sK) + i * 16384, C + 64 * i, k0, b);
         tma_store_3d(&map_out, smem_u32(sV) + i * 16384, C + kD + 64 * i, k0, b);
@@ -1288,6 +1332,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dK, dV of the key tiles cut into pieces: the pieces' partial sums added in
+// piece order (a fixed order: the result does not depend on which piece
+// finished first), dK scaled by 1/sqrt(128), both written to dqkv in bf16.
+// Block = (key tile, row b); tiles left whole were written by their CTA.
+__global__ void __launch_bounds__(256) attn_bwd_dkdv_reduce_kernel(const BwdParams p, bool win, bf16 *dqkv) {
+  const int kt = (int)blockIdx.x / p.B, b = (int)blockIdx.x % p.B;
+  int prefix = 0;
+  for (int t = 0; t < kt; ++t) prefix += dkdv_pieces(dkdv_iters(t, p.n_tiles, p.H, p.window, win), p.chunk);
+  const int np = dkdv_pieces(dkdv_iters(kt, p.n_tiles, p.H, p.window, win), p.chunk);
+  if (np == 1) return;
+  const float f = rsqrtf((float)kD);
+  const int C = p.H * kD;
+  for (int q = threadIdx.x; q < kQ * 64; q += blockDim.x) {
+    const int row = q >> 6, u = q & 63;  // 4 columns of dK (u < 32) or dV
+    const int key = kt * kQ + row;
+    if (key >= p.T) break;  // rows are visited in order: the rest are past T too
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < np; ++c) {
+      const float4 v = reinterpret_cast<const float4 *>(p.part + ((size_t)(prefix + c) * p.B + b) * kQ * 2 * kD)[q];
+      a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    }
+    if (u < 32) { a.x *= f; a.y *= f; a.z *= f; a.w *= f; }
+    uint2 o;
+    o.x = pack2(a.x, a.y);
+    o.y = pack2(a.z, a.w);
+    *reinterpret_cast<uint2 *>(dqkv + ((size_t)b * p.T + key) * p.ld + C + 4 * u) = o;
   }
 }
 
@@ -1369,9 +1442,44 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
 namespace nc {
 namespace fatc {
 
+// Piece size of the dK/dV schedule: about half of one SM's share of the
+// iterations, at least 4; 0 (no cut) when no key tile has more than that.
+inline int dkdv_chunk(int B, int T, int H, int window, int num_sms) {
+  const int n_tiles = (T + kQ - 1) / kQ;
+  const bool win = windowed(window, T);
+  int64_t total = 0;
+  int most = 0;
+  for (int kt = 0; kt < n_tiles; ++kt) {
+    const int n = dkdv_iters(kt, n_tiles, H, window, win);
+    total += n;
+    most = max(most, n);
+  }
+  total *= B;
+  const int64_t share = (total + 2 * (int64_t)num_sms - 1) / (2 * (int64_t)num_sms);
+  const int chunk = (int)(share > 4 ? share : 4);
+  return most > chunk ? chunk : 0;
+}
+
+// CTAs of the dK/dV kernel for a piece size.
+inline int dkdv_grid(int B, int T, int H, int window, int chunk) {
+  const int n_tiles = (T + kQ - 1) / kQ;
+  const bool win = windowed(window, T);
+  int pieces = 0;
+  for (int kt = 0; kt < n_tiles; ++kt) pieces += dkdv_pieces(dkdv_iters(kt, n_tiles, H, window, win), chunk);
+  return pieces * B;
+}
+
+// Bytes of partial sums the cut schedule needs (0 when nothing is cut).
+inline size_t dkdv_scratch_bytes(int B, int T, int H, int window, int num_sms) {
+  const int chunk = dkdv_chunk(B, T, H, window, num_sms);
+  return chunk ? (size_t)dkdv_grid(B, T, H, window, chunk) * kQ * 2 * kD * sizeof(float) : 0;
+}
+
+// part: scratch for the cut dK/dV schedule (part_bytes >= dkdv_scratch_bytes);
+// nullptr: every key tile in one CTA.
 inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const bf16 *dO, const float *lse,
-                              float *Drow, bf16 *dqkv, int B, int T, int H, int window, int *status,
-                              cudaStream_t st) {
+                              float *Drow, float *part, size_t part_bytes, bf16 *dqkv, int B, int T, int H,
+                              int window, int num_sms, int *status, cudaStream_t st) {
   CUtensorMap mq128, mdo128, mout;
   const int C = H * kD;
   if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mdo128, dO, B, T, C, C, 128) ||
@@ -1387,6 +1495,14 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   p.status = status;
   p.n_tiles = (T + kQ - 1) / kQ;
   p.window = window;
+  p.B = B;
+  p.chunk = 0;
+  p.part = nullptr;
+  if (part && part_bytes >= dkdv_scratch_bytes(B, T, H, window, num_sms)) {
+    p.chunk = dkdv_chunk(B, T, H, window, num_sms);
+    p.part = part;
+  }
+  const int grid_kv = dkdv_grid(B, T, H, window, p.chunk);
   const bool win = windowed(window, T);
   if (win) attn_bwd_dq_tc_kernel<true><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   else attn_bwd_dq_tc_kernel<false><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
@@ -1395,8 +1511,9 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
     fprintf(stderr, "nanochat_b200: attention dQ launch: %s\n", cudaGetErrorString(e));
     return e;
   }
-  if (win) attn_bwd_dkdv_tc_kernel<true><<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
-  else attn_bwd_dkdv_tc_kernel<false><<<B * p.n_tiles, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
+  if (win) attn_bwd_dkdv_tc_kernel<true><<<grid_kv, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
+  else attn_bwd_dkdv_tc_kernel<false><<<grid_kv, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
+  if (p.chunk) attn_bwd_dkdv_reduce_kernel<<<B * p.n_tiles, 256, 0, st>>>(p, win, dqkv);
   return cudaGetLastError();
 }
 

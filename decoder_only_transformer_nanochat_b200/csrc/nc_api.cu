@@ -85,6 +85,8 @@ struct Work {
   std::vector<float *> r1, rq, rk, lse, r2;
   T *x, *xf, *z, *dxb, *dO, *dqkv, *dy;
   float *r0, *rf, *tok_loss, *dx, *Drow;
+  float *attn_part = nullptr;  // partial dK/dV sums of key tiles cut into pieces
+  size_t attn_part_bytes = 0;
   int64_t ldz;
   TokenSort sort;                   // positions grouped by token (embedding gradient)
   float *seg_head, *seg_tail;       // [chunks, C] partial sums of segments cut by chunks
@@ -143,6 +145,11 @@ size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
   T *dO = (T *)take(M * C * es);
   T *dqkv = (T *)take(M * ldqkv * es);
   float *Drow = (float *)take(M * H * 4);
+  size_t part_bytes = 0;
+  if (sizeof(T) == 2)
+    for (int l = 0; l < L; ++l)
+      part_bytes = std::max(part_bytes, fatc::dkdv_scratch_bytes(B, T_len, H, m->layer_window[l], m->num_sms));
+  float *attn_part = part_bytes ? (float *)take(part_bytes) : nullptr;
   int32_t *sk0 = (int32_t *)take(M * 4), *sk1 = (int32_t *)take(M * 4);
   int32_t *sv0 = (int32_t *)take(M * 4), *sv1 = (int32_t *)take(M * 4);
   int *hist = (int *)take((size_t)256 * sort_tiles((int)M) * 4);
@@ -172,6 +179,7 @@ size_t carve(const nc_model *m, int B, int T_len, char *base, Work<T> *w) {
     w->x = x; w->r0 = r0; w->xf = xf; w->rf = rf; w->z = z; w->ldz = ldz;
     w->tok_loss = tok_loss; w->dx = dx; w->dxb = dxb; w->dy = dy; w->dO = dO;
     w->dqkv = dqkv; w->Drow = Drow;
+    w->attn_part = attn_part; w->attn_part_bytes = part_bytes;
   }
   return off;
 }
@@ -430,7 +438,8 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
            if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
-                                  m->layer_window[l], 0, m->status, st) != cudaSuccess) return NC_ECUDA);
+                                  m->layer_window[l], 0, m->status, st, w.attn_part, w.attn_part_bytes,
+                                  m->num_sms) != cudaSuccess) return NC_ECUDA);
     if (W.ve[l]) {
       // v += g ve[tok]:  dg = sum_i dv_i . ve[tok_i];  dve[v] = g sum_{tok_i = v} dv_i
       const T *dv = w.dqkv + (size_t)(H + 1) * kHeadDim;
@@ -1180,11 +1189,13 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
 
 static int attention_bwd_common(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
                                 float *Drow, void *dqkv, int B, int T, int H, int window, int dtype, int engine,
-                                int *status, cudaStream_t st) {
+                                int *status, cudaStream_t st, void *scratch = nullptr, size_t scratch_bytes = 0,
+                                int num_sms = 148) {
   cudaError_t e;
   if (dtype == NC_BF16) {
     e = launch_attn_bwd<bf16>((const bf16 *)qkv, (int)ld, (const bf16 *)O, (const bf16 *)dO, lse, Drow,
-                              (bf16 *)dqkv, B, T, H, window, engine, status, st);
+                              (bf16 *)dqkv, B, T, H, window, engine, status, st, (float *)scratch, scratch_bytes,
+                              num_sms);
   } else {
     e = launch_attn_bwd<float>((const float *)qkv, (int)ld, (const float *)O, (const float *)dO, lse, Drow,
                                (float *)dqkv, B, T, H, window, engine, status, st);
@@ -1206,6 +1217,34 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, window, dtype, engine, status,
                               (cudaStream_t)stream);
+}
+
+int nc_attention_bwd_scratch_bytes(int B, int T, int H, int window, size_t *out) {
+  if (!out) return NC_EINVAL;
+  if (B < 1 || T < 1 || H < 1) return NC_ESHAPE;
+  if (window < 0) return NC_EINVAL;
+  int dev = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return NC_ECUDA;
+  *out = fatc::dkdv_scratch_bytes(B, T, H, window, num_sms);
+  return NC_OK;
+}
+
+int nc_attention_bwd_ex(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
+                        float *Drow, void *scratch, size_t scratch_bytes, void *dqkv, int B, int T, int H,
+                        int window, int dtype, int engine, void *stream) {
+  if (!qkv || !O || !dO || !lse || !Drow || !dqkv) return NC_EINVAL;
+  if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
+  if (window < 0) return NC_EINVAL;
+  if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
+  if (engine < 0 || engine > 1) return NC_EINVAL;
+  if (dtype == NC_BF16 && engine == 0 && !fatc::aligned_bwd(qkv, ld, O, dO, dqkv)) return NC_EALIGN;
+  if (scratch && ((uintptr_t)scratch & 15)) return NC_EALIGN;
+  int num_sms = 0, *status = nullptr;
+  if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
+  return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, window, dtype, engine, status,
+                              (cudaStream_t)stream, scratch, scratch ? scratch_bytes : 0, num_sms);
 }
 
 int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const void *dO,

@@ -48,6 +48,7 @@ def main():
     ap.add_argument("--op", required=True,
                     choices=sorted(GEMMS) + ["attn_fwd", "attn_bwd", "gemm", "ce"] + ROW_OPS)
     ap.add_argument("--tokens", type=int, default=16 * 2048, help="M (a multiple of 2048)")
+    ap.add_argument("--heads", type=int, default=H, help="attention: query heads (d20: 10)")
     ap.add_argument("--window", type=int, default=0, help="attention: sliding window (0: causal)")
     ap.add_argument("--shape", default=None, help="for --op gemm: M,N,K,a_mn,b_mn,EPILOGUE")
     ap.add_argument("--iters", type=int, default=5)
@@ -148,29 +149,35 @@ def main():
             nbytes = B * T * (H + 1) * (3 * per_head + 4)
         flops = 0.0
     else:
-        ld = 128 * (H + 2)
+        Ha = args.heads
+        ld = 128 * (Ha + 2)
         qkv = (torch.randn(B * T * ld, device="cuda", generator=g) * 0.09).to(torch.bfloat16)
-        O = torch.empty(B * T * H * 128, device="cuda", dtype=torch.bfloat16)
-        lse = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
-        rc = nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16,
+        O = torch.empty(B * T * Ha * 128, device="cuda", dtype=torch.bfloat16)
+        lse = torch.empty(B * Ha * T, device="cuda", dtype=torch.float32)
+        rc = nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, Ha, nc.NC_BF16,
                                  args.engine, st, window=args.window)
         assert rc == 0
-        dO = (torch.randn(B * T * H * 128, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
-        Dr = torch.empty(B * H * T, device="cuda", dtype=torch.float32)
+        dO = (torch.randn(B * T * Ha * 128, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+        Dr = torch.empty(B * Ha * T, device="cuda", dtype=torch.float32)
         dqkv = torch.empty(B * T * ld, device="cuda", dtype=torch.bfloat16)
         w = args.window if 0 < args.window < T else T
         keys = 0.5 * w * (w + 1.0) + (T - w) * float(w)
-        causal = 4.0 * B * H * 128 * keys
+        causal = 4.0 * B * Ha * 128 * keys
         if args.op == "attn_fwd":
             def run():
-                assert nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H,
+                assert nc.nc_attention_fwd(qkv.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, Ha,
                                            nc.NC_BF16, args.engine, st, window=args.window) == 0
             flops = causal
         else:
+            # with the dK/dV scratch, as the model's step runs it
+            rc, nbytes = nc.nc_attention_bwd_scratch_bytes(B, T, Ha, args.window)
+            assert rc == 0
+            scratch = torch.empty(max(nbytes, 16) // 4, device="cuda", dtype=torch.float32)
+
             def run():
-                assert nc.nc_attention_bwd(qkv.data_ptr(), ld, O.data_ptr(), dO.data_ptr(), lse.data_ptr(),
-                                           Dr.data_ptr(), dqkv.data_ptr(), B, T, H, nc.NC_BF16, args.engine,
-                                           st, window=args.window) == 0
+                assert nc.nc_attention_bwd_ex(qkv.data_ptr(), ld, O.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                                              Dr.data_ptr(), scratch.data_ptr(), nbytes, dqkv.data_ptr(), B, T, Ha,
+                                              nc.NC_BF16, args.engine, st, window=args.window) == 0
             flops = 2.0 * causal
     prep()
     run()

@@ -80,11 +80,30 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
 /* Its backward.  dO [B*T, H*128] and O as above, lse from the forward.
  *   Drow  device fp32 [B, H, T] scratch, receives rowsum(dO * O)
  *   dqkv  device [B*T, ld]: dq per head; dk, dv summed over the query heads
- * window, engines and errors as nc_attention_fwd (dO and dqkv 16-byte
- * aligned too). */
+ * window and errors as nc_attention_fwd (dO and dqkv 16-byte aligned too);
+ * engine 0 or 1 (else NC_EINVAL). */
 int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
                      float *Drow, void *dqkv, int B, int T, int H, int window, int dtype, int engine,
                      void *stream);
+
+/* Scratch with which nc_attention_bwd_ex cuts the dK/dV work of the key tiles
+ * with the most (head, query-tile) pairs into pieces that spread over every
+ * SM of the current device: *out = the bytes needed (0 when no tile needs
+ * cutting at this shape).  The tcgen05 dK/dV kernel otherwise gives each
+ * 128-key tile of each row one CTA, which leaves SMs idle when B * T / 128
+ * is small against the SM count or the earliest key tiles (which every later
+ * query sees) carry most of the work. */
+int nc_attention_bwd_scratch_bytes(int B, int T, int H, int window, size_t *out);
+
+/* nc_attention_bwd with that scratch (device, 16-byte aligned, scratch_bytes
+ * long).  With scratch_bytes >= nc_attention_bwd_scratch_bytes each cut key
+ * tile's pieces leave fp32 partial sums there that a second kernel adds in
+ * piece order: deterministic, and equal to the uncut result up to the order
+ * of the fp32 sums.  scratch == NULL or smaller: no cut (nc_attention_bwd).
+ * Only the bf16 tcgen05 engine cuts; the scratch is not read afterwards. */
+int nc_attention_bwd_ex(const void *qkv, int64_t ld, const void *O, const void *dO, const float *lse,
+                        float *Drow, void *scratch, size_t scratch_bytes, void *dqkv, int B, int T, int H,
+                        int window, int dtype, int engine, void *stream);
 
 /* Largest B*H*T that nc_attention_bwd_noalloc accepts: the number of fp32
  * entries of its fixed device scratch (4 MiB). */

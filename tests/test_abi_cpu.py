@@ -94,9 +94,17 @@ def test_op_entry_points_reject_bad_arguments_on_the_host(lib):
     assert nc.nc_attention_fwd(16, ld + 4, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
     assert nc.nc_attention_bwd(16, ld, 16, 24, 16, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
     assert nc.nc_attention_bwd_noalloc(16, ld, 16, 16, 16, 40, B, T, H, BF16, 0, None) == nc.NC_EALIGN
-    # only engines 0 (model path) and 1 (CUDA cores) exist for attention
+    # attention forward engines: 0 (model path), 1 (CUDA cores), 2 (the other
+    # tcgen05 kernel); backward engines: 0 and 1
     assert nc.nc_attention_fwd(16, ld, 16, 16, B, T, H, BF16, 3, None) == nc.NC_EINVAL
     assert nc.nc_attention_bwd(16, ld, 16, 16, 16, 16, 16, B, T, H, BF16, 2, None) == nc.NC_EINVAL
+    # the backward with dK/dV scratch: same argument checks, and a misaligned scratch
+    assert nc.nc_attention_bwd_ex(16, big, 16, 16, 16, 16, 16, 1 << 20, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE
+    assert nc.nc_attention_bwd_ex(16, ld, 16, 16, 16, 16, 16, 1 << 20, 16, B, T, H, BF16, 2, None) == nc.NC_EINVAL
+    assert nc.nc_attention_bwd_ex(16, ld, 16, 16, 16, 16, 20, 1 << 20, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
+    assert nc.nc_attention_bwd_ex(0, ld, 16, 16, 16, 16, 16, 1 << 20, 16, B, T, H, BF16, 0, None) == nc.NC_EINVAL
+    assert nc.nc_attention_bwd_scratch_bytes(0, T, H, 0)[0] == nc.NC_ESHAPE
+    assert nc.nc_attention_bwd_scratch_bytes(B, T, H, -1)[0] == nc.NC_EINVAL
     # GEMM: a bf16 stride that is not a multiple of 8 on a tensor-core engine
     assert nc.nc_gemm(16, 100, 0, 16, 128, 0, 16, 128, 64, 64, 100, BF16, nc.NC_EPI_STORE, 0,
                       None) == nc.NC_EALIGN

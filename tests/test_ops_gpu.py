@@ -320,3 +320,57 @@ def test_window_covering_the_context_is_the_causal_kernel(nc):
         outs.append((O.view(torch.int16).cpu(), lse.cpu()))
     for O, lse in outs[1:]:
         assert torch.equal(O, outs[0][0]) and torch.equal(lse, outs[0][1])
+
+
+CUT_CASES = [(1, 130, 3, 0), (1, 515, 10, 0), (1, 515, 3, 64), (1, 1030, 2, 384), (1, 300, 10, 200),
+             (3, 1024, 4, 0)]
+
+
+@pytest.mark.parametrize("B,T,H,window", CUT_CASES)
+def test_attention_bwd_with_cut_key_tiles(nc, B, T, H, window):
+    # nc_attention_bwd_ex with its scratch cuts the dK/dV work of the larger key
+    # tiles into pieces whose fp32 partial sums a second kernel adds in piece
+    # order: against the oracle, against the uncut call (dq bit-identical: the
+    # same dQ kernel), and bit-identical from one call to the next
+    import torch
+
+    from oracle import full_block as fb
+    qkv, ld, q, k, v = _attn_inputs(B, T, H, 500 + T + H + window, "bf16")
+    st = torch.cuda.current_stream().cuda_stream
+    qkv_d = _dev(qkv, "bf16")
+    O = torch.zeros(B * T, H * 128, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    assert nc.nc_attention_fwd(qkv_d.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16, 0, st,
+                               window=window) == 0
+    dO = _bf16(synth.normal(11 + T, 4, B * T * H * 128).reshape(B * T, H * 128))
+    dO_d = _dev(dO, "bf16")
+    rc, nbytes = nc.nc_attention_bwd_scratch_bytes(B, T, H, window)
+    assert rc == nc.NC_OK and nbytes > 0, "these shapes are cut"
+    scratch = torch.full((nbytes // 4,), float("nan"), dtype=torch.float32, device="cuda")
+    Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    runs = []
+    for _ in range(2):
+        dqkv = torch.zeros(B * T, ld, dtype=torch.bfloat16, device="cuda")
+        assert nc.nc_attention_bwd_ex(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
+                                      Drow.data_ptr(), scratch.data_ptr(), nbytes, dqkv.data_ptr(), B, T, H,
+                                      nc.NC_BF16, 0, st, window=window) == 0
+        runs.append(dqkv)
+    whole = torch.zeros(B * T, ld, dtype=torch.bfloat16, device="cuda")
+    assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
+                               Drow.data_ptr(), whole.data_ptr(), B, T, H, nc.NC_BF16, 0, st, window=window) == 0
+    assert nc.nc_ops_status(st, 60000) == nc.NC_OK
+    assert torch.equal(runs[0].view(torch.int16), runs[1].view(torch.int16)), "cut schedule is deterministic"
+    assert torch.equal(runs[0][:, :H * 128].view(torch.int16), whole[:, :H * 128].view(torch.int16))
+    got = runs[0].float().cpu().numpy().astype(np.float64)
+    uncut = whole.float().cpu().numpy().astype(np.float64)
+    # the cut changes only the order of fp32 sums before one bf16 rounding
+    kv = slice(H * 128, ld)
+    assert np.max(np.abs(got[:, kv] - uncut[:, kv])) <= 2.0 ** -7 * np.abs(uncut[:, kv]).max()
+    refs = [np.empty((B, T, 128)), np.empty((B, T, 128))]
+    for b in range(B):
+        _, refs[0][b], refs[1][b] = fb.attention_bwd(dO.reshape(B, T, H, 128)[b], q[b], k[b], v[b], window)
+    for g, r in ((got[:, H * 128:H * 128 + 128], refs[0].reshape(B * T, -1)),
+                 (got[:, H * 128 + 128:], refs[1].reshape(B * T, -1))):
+        cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
+        assert cos > 0.9995, cos
+        assert np.max(np.abs(g - r)) <= 3e-2 * np.abs(r).max()
