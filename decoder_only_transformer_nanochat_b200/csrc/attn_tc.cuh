@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 // its O on a grown max finds its previous P V already complete.
 constexpr int kPpOCol = 256;  // O_g at kPpOCol + 128 g
 // engine 0 runs this kernel when true, the one above when false (engine 2 the other)
-constexpr bool kFwdPingPongDefault = false;
+constexpr bool kFwdPingPongDefault = true;
 
 template <bool kWin>
 __global__ void __launch_bounds__(kFwdThreads, 1)
