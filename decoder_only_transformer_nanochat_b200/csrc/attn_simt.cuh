@@ -343,12 +343,13 @@ template <typename T>
 inline cudaError_t launch_attn_bwd(const T *qkv, int ld, const T *O, const T *dO, const float *lse, float *Dr,
                                    T *dqkv, int B, int T_len, int H, int window, int engine, int *status,
                                    cudaStream_t st, float *part = nullptr, size_t part_bytes = 0,
-                                   int num_sms = 148) {
+                                   int num_sms = 148, int *launched = nullptr) {
   if (sizeof(T) == 2 && engine == 0) {
     if (!fatc::supported_bwd(qkv, ld, O, dO, dqkv)) return cudaErrorInvalidValue;
     return fatc::launch_bwd((const bf16 *)qkv, ld, (const bf16 *)O, (const bf16 *)dO, lse, Dr, part, part_bytes,
-                            (bf16 *)dqkv, B, T_len, H, window, num_sms, status, st);
+                            (bf16 *)dqkv, B, T_len, H, window, num_sms, status, st, launched);
   }
+  if (launched) *launched = 3;
   const int M = B * T_len;
   attn_rowdot_kernel<T><<<(unsigned)(((size_t)M * H + 7) / 8), 256, 0, st>>>(dO, O, Dr, M, T_len, H);
   return launch_attn_simt_bwd<T>(qkv, ld, dO, lse, Dr, dqkv, B, T_len, H, window, st);

@@ -1479,7 +1479,7 @@ inline size_t dkdv_scratch_bytes(int B, int T, int H, int window, int num_sms) {
 // nullptr: every key tile in one CTA.
 inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const bf16 *dO, const float *lse,
                               float *Drow, float *part, size_t part_bytes, bf16 *dqkv, int B, int T, int H,
-                              int window, int num_sms, int *status, cudaStream_t st) {
+                              int window, int num_sms, int *status, cudaStream_t st, int *launched = nullptr) {
   CUtensorMap mq128, mdo128, mout;
   const int C = H * kD;
   if (!make_map3(&mq128, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mdo128, dO, B, T, C, C, 128) ||
@@ -1514,6 +1514,7 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   if (win) attn_bwd_dkdv_tc_kernel<true><<<grid_kv, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
   else attn_bwd_dkdv_tc_kernel<false><<<grid_kv, kBwdThreads, kKvSmemTc, st>>>(mq128, mdo128, mout, p);
   if (p.chunk) attn_bwd_dkdv_reduce_kernel<<<B * p.n_tiles, 256, 0, st>>>(p, win, dqkv);
+  if (launched) *launched = p.chunk ? 3 : 2;
   return cudaGetLastError();
 }
 

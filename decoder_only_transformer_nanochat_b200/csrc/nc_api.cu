@@ -436,10 +436,12 @@ int fwd_bwd_impl(nc_model *m, const void *weights, const int32_t *tokens, const 
     // attention: x += O Wo^T
     NC_TRY(gemm<T>(m, gp(C, C, M, w.dxb, C, 1, w.O[l], C, 1, G(pi + 3), C, wg), st));
     NC_TRY(gemm<T>(m, gp(M, C, C, w.dxb, C, 0, W.wo[l], C, 1, w.dO, C, EPI_STORE), st));
+    int attn_launched = 1;
     NC_RUN(K_ATTN_BWD, attn_bwd_flops, 0,
            if (launch_attn_bwd<T>(w.qkv[l], ldqkv, w.O[l], w.dO, w.lse[l], w.Drow, w.dqkv, B, T_len, H,
                                   m->layer_window[l], 0, m->status, st, w.attn_part, w.attn_part_bytes,
-                                  m->num_sms) != cudaSuccess) return NC_ECUDA);
+                                  m->num_sms, &attn_launched) != cudaSuccess) return NC_ECUDA);
+    m->launches[K_ATTN_BWD] += attn_launched - 1;  // one accounting entry, two or three kernels
     if (W.ve[l]) {
       // v += g ve[tok]:  dg = sum_i dv_i . ve[tok_i];  dve[v] = g sum_{tok_i = v} dv_i
       const T *dv = w.dqkv + (size_t)(H + 1) * kHeadDim;

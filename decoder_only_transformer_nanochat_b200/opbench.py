@@ -29,6 +29,8 @@ def gemm_shapes(M: int) -> dict:
         "w1_wgrad": (F, C, M, 1, 1, "STORE_F32"),
         "w2_wgrad": (C, F, M, 1, 1, "STORE_F32"),
         "o_wgrad": (C, C, M, 1, 1, "STORE_F32"),
+        "o_dgrad": (M, C, C, 0, 1, "STORE"),
+        "qkv_dgrad": (M, C, C + 256, 0, 1, "STORE"),
         "qkv_wgrad": (C + 256, C, M, 1, 1, "STORE_F32"),
         "head_dgrad": (M, C, V, 0, 1, "STORE"),
         "head_wgrad": (V, C, M, 1, 1, "STORE_F32"),
@@ -82,12 +84,11 @@ def main():
         flops = 0.0
     elif args.op in shapes:
         m, n, k, a_mn, b_mn, epi = shapes[args.op]
-        A = (torch.randn(m * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
-        Bm = (torch.randn(n * k, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+        # drawn in their storage types: the logit-sized operands stay near 4 GB on the device
+        A = torch.randn(m * k, device="cuda", generator=g, dtype=torch.bfloat16).mul_(0.05)
+        Bm = torch.randn(n * k, device="cuda", generator=g, dtype=torch.bfloat16).mul_(0.05)
         out_f32 = epi in ("STORE_F32", "ACC_F32")
-        D = torch.rand(m * n, device="cuda", generator=g, dtype=torch.float32)
-        if not out_f32:
-            D = D.to(torch.bfloat16)
+        D = torch.rand(m * n, device="cuda", generator=g, dtype=torch.float32 if out_f32 else torch.bfloat16)
         lda = m if a_mn else k
         ldb = n if b_mn else k
         code = getattr(nc, "NC_EPI_" + epi)
