@@ -62,6 +62,26 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
+// The same for a pair of exponents in f32x2 form (bit-identical to two
+// ex2_poly calls): with t = x + 1.5 * 2^23, (t's bits << 23) is n << 23
+// modulo 2^32, since 0x4B400000 << 23 vanishes there.
+__device__ __forceinline__ void ex2_poly2(uint64_t x, float &e0, float &e1) {
+  float x0, x1;
+  f2split(x, x0, x1);
+  const uint64_t xc = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = add2(xc, f2(12582912.f, 12582912.f));
+  const uint64_t u = add2(t, f2(-12582912.f, -12582912.f));
+  const uint64_t f = fma2(u, f2(-1.f, -1.f), xc);
+  uint64_t q = fma2(f, f2(0.05500858f, 0.05500858f), f2(0.24221037f, 0.24221037f));
+  q = fma2(f, q, f2(0.69328290f, 0.69328290f));
+  q = fma2(f, q, f2(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2split(q, p0, p1);
+  f2split(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // MMA with the A operand read from TMEM (K-major, bf16 pairs per column)
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -606,8 +626,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < kKV; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sc;
+      for (int i = 0; i < kKV; i += 2) mx4[(i >> 1) & 3] = max3(mx4[(i >> 1) & 3], s[i], s[i + 1]);
+      const float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sc;
       // the exponent base moves only when the max grows by more than 2^8
       const bool first = j == grp;
       const bool grow = first || mx > m_used + kRescaleLog2;
@@ -619,22 +639,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // a row that has seen no key yet (windows only) keeps its base at -inf
       // and takes its exponentials against 0 (all of them 0)
       const float nmb = m_used == -INFINITY ? 0.f : -m_used;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // exponents s sc - m two at a time (f32x2), then one pair in four on the
+      // FMA pipe and the rest on MUFU; the row sum in two f32x2 accumulators
+      const uint64_t sc2 = f2(sc, sc), nmb2 = f2(nmb, nmb);
+      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < kKV / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const int k = 32 * c + i;
-          // one exponential in four on the FMA pipe
-          const float e0 = ex2(fmaf(s[k], sc, nmb));
-          const float e1 = (i & 2) ? ex2_poly(fmaf(s[k + 1], sc, nmb)) : ex2(fmaf(s[k + 1], sc, nmb));
-          sum4[(i >> 1) & 3] += e0 + e1;
+          const uint64_t x = fma2(f2(s[k], s[k + 1]), sc2, nmb2);
+          float e0, e1;
+          if ((i & 6) == 6) {
+            ex2_poly2(x, e0, e1);
+          } else {
+            float x0, x1;
+            f2split(x, x0, x1);
+            e0 = ex2(x0);
+            e1 = ex2(x1);
+          }
+          sum2[(i >> 1) & 1] = add2(sum2[(i >> 1) & 1], f2(e0, e1));
           pk[i / 2] = pack2(e0, e1);
         }
         tmem_st16_nw(t_s + 16 * c, pk);  // keys [32c, 32c + 32) as 16 columns of bf16 pairs
       }
-      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      {
+        float a0, a1, b0, b1;
+        f2split(sum2[0], a0, a1);
+        f2split(sum2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       if (!first && __any_sync(0xffffffffu, grow)) {
         // the max grew: bring this group's O to the new base before P_j V_j
         // adds to it (its previous P V is complete: see the kernel's header)
@@ -948,7 +983,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float d2[2];
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          float pr = ex2(__uint_as_float(sv[i + t]) * sc - L);
+          float pr = ex2(fmaf(__uint_as_float(sv[i + t]), sc, -L));
           const int key = kv0 + i + t;
           if (need_mask && (key > row || key >= p.T || (kWin && row - key >= p.window))) pr = 0.f;
           d2[t] = pr * (__uint_as_float(dv[i + t]) - Dv);
@@ -1222,21 +1257,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float *Ls = reinterpret_cast<const float *>(sQS + st * kQStage + 2 * kTileBytes) + c0;
       const float *Ds = Ls + kBQ2;
       const bool need_mask = qq0 < key + 1 || qq0 + 64 > p.T || (kWin && qq0 + 63 - key >= p.window);
+      // P^T = 2^(s sc - lse log2 e), two queries at a time (f32x2)
+      const uint64_t sc2 = f2(sc, sc), nl2e = f2(-kLog2e, -kLog2e);
       float pr[64];
       uint32_t pk[32];
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
         const float4 l4 = reinterpret_cast<const float4 *>(Ls)[i4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int qi = 4 * i4 + t;
-          float v = ex2(__uint_as_float(xv[qi]) * sc - lv[t] * kLog2e);
-          if (need_mask && (qq0 + qi < key || qq0 + qi >= p.T || (kWin && qq0 + qi - key >= p.window))) v = 0.f;
-          pr[qi] = v;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int qi = 4 * i4 + 2 * h2;
+          const uint64_t nl = mul2(h2 ? f2(l4.z, l4.w) : f2(l4.x, l4.y), nl2e);
+          float x0, x1;
+          f2split(fma2(f2(__uint_as_float(xv[qi]), __uint_as_float(xv[qi + 1])), sc2, nl), x0, x1);
+          float v0 = ex2(x0), v1 = ex2(x1);
+          if (need_mask) {
+            if (qq0 + qi < key || qq0 + qi >= p.T || (kWin && qq0 + qi - key >= p.window)) v0 = 0.f;
+            if (qq0 + qi + 1 < key || qq0 + qi + 1 >= p.T || (kWin && qq0 + qi + 1 - key >= p.window)) v1 = 0.f;
+          }
+          pr[qi] = v0;
+          pr[qi + 1] = v1;
+          pk[qi / 2] = pack2(v0, v1);
         }
-        pk[2 * i4] = pack2(pr[4 * i4], pr[4 * i4 + 1]);
-        pk[2 * i4 + 1] = pack2(pr[4 * i4 + 2], pr[4 * i4 + 3]);
       }
       // P^T once dV += P^T_{it-1} dO has read the previous one
       ok = mbar_wait(p_empty, par ^ 1, abort_flag, p.status);
@@ -1252,15 +1294,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(dp_taken);  // X may take the next S^T now
+      // dS^T = P^T (dP^T - D), two queries at a time (f32x2)
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
         const float4 d4 = reinterpret_cast<const float4 *>(Ds)[i4];
-        const float dd4[4] = {d4.x, d4.y, d4.z, d4.w};
-        float ds[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) ds[t] = pr[4 * i4 + t] * (__uint_as_float(xv[4 * i4 + t]) - dd4[t]);
-        pk[2 * i4] = pack2(ds[0], ds[1]);
-        pk[2 * i4 + 1] = pack2(ds[2], ds[3]);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int qi = 4 * i4 + 2 * h2;
+          const uint64_t t = add2(f2(__uint_as_float(xv[qi]), __uint_as_float(xv[qi + 1])),
+                                  h2 ? f2(-d4.z, -d4.w) : f2(-d4.x, -d4.y));
+          float d0, d1;
+          f2split(mul2(f2(pr[qi], pr[qi + 1]), t), d0, d1);
+          pk[qi / 2] = pack2(d0, d1);
+        }
       }
       ok = mbar_wait(ds_empty, par ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -1442,8 +1488,11 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
 namespace nc {
 namespace fatc {
 
-// Piece size of the dK/dV schedule: about half of one SM's share of the
-// iterations, at least 4; 0 (no cut) when no key tile has more than that.
+// Piece size of the dK/dV schedule.  0 (no cut) while the heaviest key tile
+// carries at most 1.25 SM shares of the iterations: whole tiles, heaviest
+// first, then pack the SMs within a few percent (d20: 160 against 147), and
+// every piece costs a prologue, a K/V load and a partial-sum round trip.
+// Otherwise pieces of two thirds of a share (at least 4 iterations).
 inline int dkdv_chunk(int B, int T, int H, int window, int num_sms) {
   const int n_tiles = (T + kQ - 1) / kQ;
   const bool win = windowed(window, T);
@@ -1455,8 +1504,10 @@ inline int dkdv_chunk(int B, int T, int H, int window, int num_sms) {
     most = max(most, n);
   }
   total *= B;
-  const int64_t share = (total + 2 * (int64_t)num_sms - 1) / (2 * (int64_t)num_sms);
-  const int chunk = (int)(share > 4 ? share : 4);
+  const int64_t share = (total + num_sms - 1) / num_sms;
+  if (4 * (int64_t)most <= 5 * share) return 0;
+  const int64_t piece = (2 * total + 3 * (int64_t)num_sms - 1) / (3 * (int64_t)num_sms);
+  const int chunk = (int)(piece > 4 ? piece : 4);
   return most > chunk ? chunk : 0;
 }
 

@@ -368,7 +368,8 @@ def test_attention_bwd_with_cut_key_tiles(nc, B, T, H, window):
     assert np.max(np.abs(got[:, kv] - uncut[:, kv])) <= 2.0 ** -7 * np.abs(uncut[:, kv]).max()
     refs = [np.empty((B, T, 128)), np.empty((B, T, 128))]
     for b in range(B):
-        _, refs[0][b], refs[1][b] = fb.attention_bwd(dO.reshape(B, T, H, 128)[b], q[b], k[b], v[b], window)
+        # (window None: the full-block oracle's plain causal mask)
+        _, refs[0][b], refs[1][b] = fb.attention_bwd(dO.reshape(B, T, H, 128)[b], q[b], k[b], v[b], window or None)
     for g, r in ((got[:, H * 128:H * 128 + 128], refs[0].reshape(B * T, -1)),
                  (got[:, H * 128 + 128:], refs[1].reshape(B * T, -1))):
         cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
