@@ -326,11 +326,12 @@ namespace nc {
 // engine 1: the CUDA-core kernels for either dtype (a test engine).
 template <typename T>
 inline cudaError_t launch_attn_fwd(const T *qkv, int ld, T *O, float *lse, int B, int T_len, int H, int window,
-                                   int engine, int *status, cudaStream_t st) {
-  if (sizeof(T) == 2 && (engine == 0 || engine == 2)) {
+                                   int engine, int *status, cudaStream_t st, int num_sms = 148) {
+  if (sizeof(T) == 2 && (engine == 0 || engine == 2 || engine == 3)) {
     if (!fatc::supported(qkv, ld, O)) return cudaErrorInvalidValue;
-    const bool pp = (engine == 0) == fatc::kFwdPingPongDefault;
-    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, window, pp, status, st);
+    const bool pp = engine == 3 || (engine == 0) == fatc::kFwdPingPongDefault;
+    return fatc::launch_fwd((const bf16 *)qkv, ld, (bf16 *)O, lse, B, T_len, H, window, pp,
+                            engine == 3 ? 0 : num_sms, status, st);
   }
   return launch_attn_simt_fwd<T>(qkv, ld, O, lse, B, T_len, H, window, st);
 }

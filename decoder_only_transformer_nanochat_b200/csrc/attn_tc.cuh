@@ -120,7 +120,7 @@ __device__ __forceinline__ uint32_t tile_unit(int r, int u) {
 }
 
 struct FwdParams {
-  int T, H, n_qt;
+  int T, H, n_qt, B;
   int window;   // windowed kernels: query i sees keys j with 0 <= i - j < window
   float *lse;   // [B, H, T]
   int *status;
@@ -426,16 +426,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 // ---------------- forward, ping-pong: two softmax warpgroups on alternating key tiles ----------------
-// Same CTA (128 queries of one (row b, head h)), TMA warp and operand layouts
-// as above; what changes is how the element-wise work is split:
-//   warps 2..5  softmax of the even key tiles, warps 6..9 of the odd ones;
-//               thread = query row, the whole 128-key tile of its row in
-//               registers, its own running max and sum (no exchange between
-//               threads, no block-wide barrier inside the key loop)
+// Work item = 128 queries of one (row b, head h); operand layouts as above.
+//   warp 0      TMA: Q of each item (two buffers: the next item's Q lands
+//               while the current one runs), K and V rings of two tiles
 //   warp 1      MMA: S_j = Q K_j^T into TMEM buffer j & 1, P_j written back
 //               over S_j as bf16 pairs, O_{j&1} += P_j V_j; tensor-core order
 //               S_0, S_1, PV_0, S_2, PV_1, S_3 ... (MMAs issued by one thread
 //               run in order, so S_{j+2} overwrites P_j only after PV_j read it)
+//   warps 4..7  softmax of the even key tiles, warps 8..11 of the odd ones;
+//               thread = query row, the whole 128-key tile of its row in
+//               registers, its own running max and sum (no exchange between
+//               threads, no block-wide barrier inside the key loop)
 // TMEM: S/P_0 [0,128), S/P_1 [128,256), O_0 [256,384), O_1 [384,512).
 // The two partial outputs are merged once at the end:
 //   m = max(m_0, m_1),  a_g = 2^(m_g - m),
@@ -443,60 +444,81 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 // (log2 domain), the online-softmax merge of two disjoint key sets.  The
 // commit that signals S_j covers every earlier MMA, so a group that rescales
 // its O on a grown max finds its previous P V already complete.
+// Persistent: CTA c takes items c, c + grid, c + 2 grid, ... (items ordered
+// latest query tiles first, the most keys), so the next item's Q load and
+// first score MMAs overlap the current item's merge and store; with grid =
+// the item count every CTA takes one item.  Barrier phases count uses across
+// items: a group's tiles for s_full, p_full and o_done, the K and V loads for
+// their rings, the items for the Q buffers and o_free (the merge has read O).
 constexpr int kPpOCol = 256;  // O_g at kPpOCol + 128 g
+constexpr int kPpStages = 2;  // K and V ring depth (with two Q buffers: six tiles of 32 KB)
+// Three warpgroups: warp 0 TMA, warp 1 MMA (warps 2, 3 idle), warps 4..7 and
+// 8..11 the two softmax groups.  The first warpgroup gives registers to the
+// other two (setmaxnreg): 128 x 56 + 256 x 224 = 64,512, all of the 384 x 168
+// the CTA is launched with, so every increase can be met.
+constexpr int kPpThreads = 384;
+constexpr int kPpRegsLow = 56, kPpRegsHigh = 224;
+static_assert(128 * kPpRegsLow + 256 * kPpRegsHigh <= kPpThreads * 168, "register split within the launch");
 // engine 0 runs this kernel when true, the one above when false (engine 2 the other)
 constexpr bool kFwdPingPongDefault = true;
 
 template <bool kWin>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kPpThreads, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap map_qk,   // qkv [B][T][ld], box 64 x 128
                        const __grid_constant__ CUtensorMap map_v,    // qkv, box 64 x 64
                        const __grid_constant__ CUtensorMap map_o,    // O [B][T][C], box 64 x 128
                        const FwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;
-  uint8_t *sK = sQ + kTileBytes;
-  uint8_t *sV = sK + kKStages * kTileBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kVStages * kTileBytes);
-  // bars: q_full, k_full[3], k_empty[3], s_full[2], p_full[2], o_done[2],
-  //       v_full[2], v_empty[2], drain
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  uint8_t *sQ = smem;                              // two Q buffers; an item's output is staged in its own
+  uint8_t *sK = sQ + 2 * kTileBytes;
+  uint8_t *sV = sK + kPpStages * kTileBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kPpStages * kTileBytes);
+  // bars: q_full[2], q_empty[2], k_full[2], k_empty[2], v_full[2], v_empty[2],
+  //       s_full[2], p_full[2], o_done[2], o_free, drain
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *sML = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [group][m, l][128]
-  const uint32_t q_full = smem_u32(bars + 0);
-  auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto k_empty = [&](int s) { return smem_u32(bars + 4 + s); };
-  auto s_full = [&](int s) { return smem_u32(bars + 7 + s); };
-  auto p_full = [&](int s) { return smem_u32(bars + 9 + s); };
-  auto o_done = [&](int s) { return smem_u32(bars + 11 + s); };
-  auto v_full = [&](int s) { return smem_u32(bars + 13 + s); };
-  auto v_empty = [&](int s) { return smem_u32(bars + 15 + s); };
-  const uint32_t drain = smem_u32(bars + 17);
+  auto q_full = [&](int s) { return smem_u32(bars + 0 + s); };
+  auto q_empty = [&](int s) { return smem_u32(bars + 2 + s); };
+  auto k_full = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto k_empty = [&](int s) { return smem_u32(bars + 6 + s); };
+  auto v_full = [&](int s) { return smem_u32(bars + 8 + s); };
+  auto v_empty = [&](int s) { return smem_u32(bars + 10 + s); };
+  auto s_full = [&](int s) { return smem_u32(bars + 12 + s); };
+  auto p_full = [&](int s) { return smem_u32(bars + 14 + s); };
+  auto o_done = [&](int s) { return smem_u32(bars + 16 + s); };
+  const uint32_t o_free = smem_u32(bars + 18);
+  const uint32_t drain = smem_u32(bars + 19);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = gridDim.x / p.n_qt;
-  const int qt = p.n_qt - 1 - (int)blockIdx.x / BH;  // latest query tiles (most keys) first
-  const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
-  const int q0 = qt * kQ;
-  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kKV : 0;
-  const int n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV - kt_lo;
-  const int kbase = kt_lo * kKV;
+  const int BH = p.B * p.H;
+  const int n_items = BH * p.n_qt;
   const int C = p.H * kD;
+  // item -> (q0, b, h, first key tile, key tiles)
+  auto item_of = [&](int it, int &q0, int &b, int &h, int &kbase, int &n_kv) {
+    const int qt = p.n_qt - 1 - it / BH;  // latest query tiles (most keys) first
+    h = (it % BH) % p.H;
+    b = (it % BH) / p.H;
+    q0 = qt * kQ;
+    const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kKV : 0;
+    n_kv = (min(q0 + kQ, p.T) + kKV - 1) / kKV - kt_lo;
+    kbase = kt_lo * kKV;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
       mbar_init(s_full(s), 1);
       mbar_init(p_full(s), 128);  // one warpgroup
       mbar_init(o_done(s), 1);
-      mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
     }
+    mbar_init(o_free, 256);  // both warpgroups, after the merge has read O
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -507,47 +529,59 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPpRegsLow));
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer (as in the kernel above) ----------------
-      mbar_expect_tx(q_full, kTileBytes);
-      for (int i = 0; i < 2; ++i) tma_load_3d(smem_u32(sQ) + i * 16384, &map_qk, h * kD + 64 * i, q0, b, q_full);
-      int issued_k = 0, issued_v = 0;
-      auto load_k = [&](int j) -> bool {
-        const int st = j % kKStages;
-        if (!mbar_wait(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
-        const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
-        mbar_expect_tx(k_full(st), kTileBytes);
-        for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b, k_full(st));
-        ++issued_k;
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(v_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
-        const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
-        mbar_expect_tx(v_full(st), kTileBytes);
-        for (int hh = 0; hh < 2; ++hh)
-          for (int a = 0; a < 2; ++a)
-            tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, kbase + j * kKV + 64 * hh, b,
-                        v_full(st));
-        ++issued_v;
-        return true;
-      };
-      bool okp = load_k(0) && (n_kv < 2 || load_k(1));
-      for (int j = 0; j < n_kv && okp; ++j) {
-        if (j + 2 < n_kv && !load_k(j + 2)) break;
-        if (!load_v(j)) break;
+      // ---------------- TMA producer ----------------
+      int kc = 0, vc = 0, li = 0;  // K and V tiles and items requested so far
+      bool okp = true;
+      for (int it = blockIdx.x; it < n_items && okp; it += gridDim.x, ++li) {
+        int q0, b, h, kbase, n_kv;
+        item_of(it, q0, b, h, kbase, n_kv);
+        const int qb = li & 1;
+        if (!(okp = mbar_wait(q_empty(qb), ((li >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_expect_tx(q_full(qb), kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          tma_load_3d(smem_u32(sQ) + qb * kTileBytes + i * 16384, &map_qk, h * kD + 64 * i, q0, b, q_full(qb));
+        auto load_k = [&](int j) -> bool {
+          const int st = kc % kPpStages;
+          if (!mbar_wait(k_empty(st), ((kc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
+          const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
+          mbar_expect_tx(k_full(st), kTileBytes);
+          for (int i = 0; i < 2; ++i)
+            tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b, k_full(st));
+          ++kc;
+          return true;
+        };
+        auto load_v = [&](int j) -> bool {
+          const int st = vc % kPpStages;
+          if (!mbar_wait(v_empty(st), ((vc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
+          const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
+          mbar_expect_tx(v_full(st), kTileBytes);
+          for (int hh = 0; hh < 2; ++hh)
+            for (int a = 0; a < 2; ++a)
+              tma_load_3d(v_dst + hh * 16384 + a * 8192, &map_v, C + kD + 64 * a, kbase + j * kKV + 64 * hh, b,
+                          v_full(st));
+          ++vc;
+          return true;
+        };
+        // V_j is requested before K_{j+2}, whose slot frees only when S_j is done
+        okp = load_k(0) && (n_kv < 2 || load_k(1));
+        for (int j = 0; j < n_kv && okp; ++j) okp = load_v(j) && (j + 2 >= n_kv || load_k(j + 2));
       }
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued_k - kKStages); j < issued_k; ++j) {
+      // no copy of ours may still be landing when the CTA exits
+      for (int i = max(0, li - 2); i < li; ++i) {
         const uint64_t t1 = globaltimer();
-        while (!mbar_try(k_full(j % kKStages), (j / kKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(q_full(i & 1), (i >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
-      for (int j = max(0, issued_v - 2); j < issued_v; ++j) {
+      for (int c = max(0, kc - kPpStages); c < kc; ++c) {
         const uint64_t t1 = globaltimer();
-        while (!mbar_try(v_full(j & 1), (j >> 1) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(k_full(c % kPpStages), (c / kPpStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+      for (int c = max(0, vc - kPpStages); c < vc; ++c) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(v_full(c % kPpStages), (c / kPpStages) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
     }
   } else if (warp == 1) {
@@ -555,58 +589,82 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = make_idesc(0, 0, kQ, kKV);
       const uint32_t idesc_o = make_idesc(0, 1, kQ, kD);
-      const uint64_t dQd = smem_desc(smem_u32(sQ), 16, 1024), dKd = smem_desc(smem_u32(sK), 16, 1024);
+      const uint64_t dQ0 = smem_desc(smem_u32(sQ), 16, 1024), dKd = smem_desc(smem_u32(sK), 16, 1024);
       const uint64_t dVd = smem_desc(smem_u32(sV), 8192, 1024);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-      auto issue_s = [&](int j) -> bool {
-        const int ks = j % kKStages;
-        if (!mbar_wait(k_full(ks), (j / kKStages) & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint64_t bK = dKd + (uint64_t)((ks * kTileBytes) >> 4);
+      int kc = 0, vc = 0, li = 0;
+      int pc[2] = {0, 0};  // P tiles taken per score buffer
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++li) {
+        int q0, b, h, kbase, n_kv;
+        item_of(it, q0, b, h, kbase, n_kv);
+        const int qb = li & 1;
+        if (!(ok = mbar_wait(q_full(qb), (li >> 1) & 1, abort_flag, p.status))) break;
+        const uint64_t dQd = dQ0 + (uint64_t)((qb * kTileBytes) >> 4);
+        auto issue_s = [&](int j) -> bool {
+          const int ks = kc % kPpStages;
+          if (!mbar_wait(k_full(ks), (kc / kPpStages) & 1, abort_flag, p.status)) return false;
+          tc_fence_after();
+          const uint64_t bK = dKd + (uint64_t)((ks * kTileBytes) >> 4);
 #pragma unroll
-        for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t off = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + (j & 1) * kKV, dQd + off, bK + off, idesc_s, s > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full(j & 1));
-        tc_commit(k_empty(ks));
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && n_kv > 1) ok = issue_s(1);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int bb = j & 1;
-        if (!(ok = mbar_wait(p_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(v_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        const uint64_t bV = dVd + (uint64_t)((bb * kTileBytes) >> 4);
-        const uint32_t a_p = tmem + bb * kKV;  // P_j over the first 64 columns of S_j
+          for (int s = 0; s < kD / 16; ++s) {
+            const uint32_t off = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+            tc_mma(tmem + (j & 1) * kKV, dQd + off, bK + off, idesc_s, s > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full(j & 1));
+          tc_commit(k_empty(ks));
+          ++kc;
+          return true;
+        };
+        ok = issue_s(0) && (n_kv < 2 || issue_s(1));
+        // the previous item's merge must have read O before P_0 V_0 overwrites it
+        if (ok && li > 0) ok = mbar_wait(o_free, (li - 1) & 1, abort_flag, p.status);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int bb = j & 1;
+          if (!(ok = mbar_wait(p_full(bb), pc[bb] & 1, abort_flag, p.status))) break;
+          ++pc[bb];
+          const int vs = vc % kPpStages;
+          if (!(ok = mbar_wait(v_full(vs), (vc / kPpStages) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint64_t bV = dVd + (uint64_t)((vs * kTileBytes) >> 4);
+          const uint32_t a_p = tmem + bb * kKV;  // P_j over the first 64 columns of S_j
 #pragma unroll
-        for (int s = 0; s < kKV / 16; ++s) {
-          const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;
-          tc_mma_ts(tmem + kPpOCol + bb * kD, a_p + 8 * s, bV + b_off, idesc_o, (j >= 2 || s > 0) ? 1u : 0u);
+          for (int s = 0; s < kKV / 16; ++s) {
+            const uint32_t b_off = ((s >> 2) * 16384 + (s & 3) * 2048) >> 4;
+            tc_mma_ts(tmem + kPpOCol + bb * kD, a_p + 8 * s, bV + b_off, idesc_o, (j >= 2 || s > 0) ? 1u : 0u);
+          }
+          tc_commit(o_done(bb));
+          tc_commit(v_empty(vs));
+          ++vc;
+          if (j + 2 < n_kv) ok = issue_s(j + 2);
         }
-        tc_commit(o_done(bb));
-        tc_commit(v_empty(bb));
-        if (j + 2 < n_kv) ok = issue_s(j + 2);
       }
       tc_commit(drain);
       const uint64_t t0 = globaltimer();
       while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPpRegsHigh));
     // ---------------- softmax warpgroups: group g takes key tiles j = g, g + 2, ... ----------------
-    const int grp = (warp - 2) >> 2, quarter = warp & 3;
+    const int grp = (warp - 4) >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int row = q0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t t_s = lane_base + grp * kKV;           // S_j, then P_j
     const uint32_t t_o = lane_base + kPpOCol + grp * kD;  // this group's O
     const float sc = rsqrtf((float)kD) * kLog2e;
-    float m_used = -INFINITY, l = 0.f;
+    int scnt = 0;  // this group's tiles so far, over all items (phase of s_full, p_full, o_done)
+    int li = 0;
     bool ok = true;
-    for (int j = grp; j < n_kv; j += 2) {
-      ok = mbar_wait(s_full(grp), (j >> 1) & 1, abort_flag, p.status);
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
+    int q0, b, h, kbase, n_kv;
+    item_of(it, q0, b, h, kbase, n_kv);
+    const int row = q0 + r;
+    const int qb = li & 1;
+    uint8_t *sQb = sQ + qb * kTileBytes;  // this item's Q, then its output tile
+    float m_used = -INFINITY, l = 0.f;
+    int mine = 0;
+    for (int j = grp; j < n_kv && ok; j += 2) {
+      ok = mbar_wait(s_full(grp), scnt & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float s[kKV];
@@ -685,10 +743,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full(grp));
+      ++scnt;
+      ++mine;
     }
     // ---------------- merge of the two groups, O / l, lse ----------------
-    const int last = n_kv - 1 - ((n_kv - 1 - grp) & 1);  // this group's last tile (-1: none)
-    if (ok && last >= 0) ok = mbar_wait(o_done(grp), (last >> 1) & 1, abort_flag, p.status);
+    if (ok && mine > 0) ok = mbar_wait(o_done(grp), (scnt - 1) & 1, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
     sML[(grp * 2 + 0) * kQ + r] = m_used;
     sML[(grp * 2 + 1) * kQ + r] = l;
@@ -723,18 +782,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           w.y = pack2(o[8 * u + 2], o[8 * u + 3]);
           w.z = pack2(o[8 * u + 4], o[8 * u + 5]);
           w.w = pack2(o[8 * u + 6], o[8 * u + 7]);
-          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, 8 * grp + 4 * c + u)) = w;  // Q is no longer read
+          *reinterpret_cast<uint4 *>(sQb + tile_unit(r, 8 * grp + 4 * c + u)) = w;  // Q is no longer read
         }
       }
       if (grp == 0 && row < p.T) p.lse[((int64_t)b * p.H + h) * p.T + row] = (mm + __log2f(lt)) * (1.f / kLog2e);
     }
+    tc_fence_before();
+    mbar_arrive(o_free);  // O_0, O_1 may take the next item's P V now
     fence_proxy_async();
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (ok && warp == 2 && lane == 0) {
-      for (int i = 0; i < 2; ++i) tma_store_3d(&map_o, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
+    if (ok && warp == 4 && lane == 0) {
+      for (int i = 0; i < 2; ++i) tma_store_3d(&map_o, smem_u32(sQb) + i * 16384, h * kD + 64 * i, q0, b);
       bulk_commit();
-      bulk_wait0();
+      bulk_wait_read0();
+      mbar_arrive(q_empty(qb));  // the buffer may take a later item's Q
     }
+    if (!ok) break;
+    }
+    if (warp == 4 && lane == 0) bulk_wait0();  // every store complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -744,6 +809,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
 }
+
 
 // ===========================================================================
 // Backward.  With P = exp(S - lse) recomputed from the saved log-sum-exp and
@@ -1453,9 +1519,10 @@ inline bool supported(const void *qkv, int64_t ld, const void *O) {
   return encode_fn() != nullptr && aligned(qkv, ld, O);
 }
 
-// pingpong: the kernel with two softmax warpgroups on alternating key tiles
+// pingpong: the kernel with two softmax warpgroups on alternating key tiles,
+// persistent over grid = min(items, num_sms) CTAs (num_sms = 0: one CTA per item)
 inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int window,
-                              bool pingpong, int *status, cudaStream_t st) {
+                              bool pingpong, int num_sms, int *status, cudaStream_t st) {
   CUtensorMap mqk, mv, mo;
   const int C = H * kD;
   if (!make_map3(&mqk, qkv, B, T, (int)ld, ld, 128) || !make_map3(&mv, qkv, B, T, (int)ld, ld, 64) ||
@@ -1468,11 +1535,13 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   p.lse = lse;
   p.status = status;
   p.window = window;
+  p.B = B;
   const int grid = B * H * p.n_qt;
   const bool win = windowed(window, T);
   if (pingpong) {
-    if (win) attn_fwd_pp_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
-    else attn_fwd_pp_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
+    const int g = num_sms > 0 && num_sms < grid ? num_sms : grid;
+    if (win) attn_fwd_pp_kernel<true><<<g, kPpThreads, kSmem, st>>>(mqk, mv, mo, p);
+    else attn_fwd_pp_kernel<false><<<g, kPpThreads, kSmem, st>>>(mqk, mv, mo, p);
   } else {
     if (win) attn_fwd_tc_kernel<true><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);
     else attn_fwd_tc_kernel<false><<<grid, kFwdThreads, kSmem, st>>>(mqk, mv, mo, p);

@@ -356,7 +356,7 @@ int forward_body(nc_model *m, const Weights<T> &W, const int32_t *tokens, int B,
     } else {
       NC_RUN(K_ATTN_FWD, attn_flops, 0,
              if (launch_attn_fwd<T>(w.qkv[l], ldqkv, w.O[l], w.lse[l], B, T_len, H, m->layer_window[l], 0,
-                                    m->status, st) != cudaSuccess) return NC_ECUDA);
+                                    m->status, st, m->num_sms) != cudaSuccess) return NC_ECUDA);
     }
     NC_TRY(gemm<T>(m, gp(M, C, C, w.O[l], C, 0, W.wo[l], C, 0, x, C, EPI_ADD), st));
     NC_RUN(K_RMSNORM, 0, M * (4.0 + 2.0 * C * es),
@@ -1176,14 +1176,15 @@ int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, in
   if (!attn_shape_ok(B, T, H, ld)) return NC_ESHAPE;
   if (window < 0) return NC_EINVAL;
   if (dtype != NC_F32 && dtype != NC_BF16) return NC_EUNSUPPORTED;
-  if (engine < 0 || engine > 2) return NC_EINVAL;
+  if (engine < 0 || engine > 3) return NC_EINVAL;
   if (dtype == NC_BF16 && engine != 1 && !fatc::aligned(qkv, ld, O)) return NC_EALIGN;
   int num_sms = 0, *status = nullptr;
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (dtype == NC_BF16)
-    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, window, engine, status, st);
+    e = launch_attn_fwd<bf16>((const bf16 *)qkv, (int)ld, (bf16 *)O, lse, B, T, H, window, engine, status, st,
+                              num_sms);
   else
     e = launch_attn_fwd<float>((const float *)qkv, (int)ld, (float *)O, lse, B, T, H, window, engine, status, st);
   return e == cudaSuccess ? NC_OK : NC_ECUDA;
