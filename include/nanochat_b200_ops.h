@@ -72,8 +72,9 @@ int nc_gemm(const void *A, int64_t lda, int a_mn, const void *B, int64_t ldb, in
  * cores), 1 = the CUDA-core kernel (a test engine for either dtype), 2 = the
  * other tcgen05 forward kernel (bf16 only; the two differ in how the softmax
  * work is split between warps: one pair of warps per query row on every key
- * tile, or one thread per row with two warpgroups on alternating key tiles).
- * Engine 2 with fp32 runs the CUDA-core kernel. */
+ * tile, or one thread per row with two warpgroups on alternating key tiles),
+ * 3 = the model's kernel with one CTA per 128-query tile instead of one
+ * persistent CTA per SM.  Engines 2 and 3 with fp32 run the CUDA-core kernel. */
 int nc_attention_fwd(const void *qkv, int64_t ld, void *O, float *lse, int B, int T, int H, int window,
                      int dtype, int engine, void *stream);
 

@@ -94,9 +94,9 @@ def test_op_entry_points_reject_bad_arguments_on_the_host(lib):
     assert nc.nc_attention_fwd(16, ld + 4, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
     assert nc.nc_attention_bwd(16, ld, 16, 24, 16, 16, 16, B, T, H, BF16, 0, None) == nc.NC_EALIGN
     assert nc.nc_attention_bwd_noalloc(16, ld, 16, 16, 16, 40, B, T, H, BF16, 0, None) == nc.NC_EALIGN
-    # attention forward engines: 0 (model path), 1 (CUDA cores), 2 (the other
+    # attention forward engines: 0 (model path), 1 (CUDA cores), 2 and 3 (the other
     # tcgen05 kernel); backward engines: 0 and 1
-    assert nc.nc_attention_fwd(16, ld, 16, 16, B, T, H, BF16, 3, None) == nc.NC_EINVAL
+    assert nc.nc_attention_fwd(16, ld, 16, 16, B, T, H, BF16, 4, None) == nc.NC_EINVAL
     assert nc.nc_attention_bwd(16, ld, 16, 16, 16, 16, 16, B, T, H, BF16, 2, None) == nc.NC_EINVAL
     # the backward with dK/dV scratch: same argument checks, and a misaligned scratch
     assert nc.nc_attention_bwd_ex(16, big, 16, 16, 16, 16, 16, 1 << 20, 16, B, T, H, BF16, 0, None) == nc.NC_ESHAPE

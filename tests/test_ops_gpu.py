@@ -162,9 +162,10 @@ ATTN_CASES = [(1, 1, 1), (2, 9, 2), (1, 130, 3), (2, 256, 2), (1, 515, 10)]
 
 @pytest.mark.parametrize("B,T,H", ATTN_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1, 2])
+@pytest.mark.parametrize("engine", [0, 1, 2, 3])
 def test_attention_fwd_bwd(nc, B, T, H, dtype, engine):
-    # engine 2: the other tcgen05 forward kernel; its O and lse then feed the backward
+    # engines 2 and 3: the other tcgen05 forward kernel, and the model's kernel
+    # with one CTA per query tile; their O and lse then feed the backward
     import torch
     code = nc.NC_BF16 if dtype == "bf16" else nc.NC_F32
     qkv, ld, q, k, v = _attn_inputs(B, T, H, 100 + T + H, dtype)
@@ -249,7 +250,7 @@ WINDOW_CASES = [(1, 515, 3, 1), (1, 515, 3, 64), (2, 256, 2, 129), (1, 300, 10, 
 
 @pytest.mark.parametrize("B,T,H,window", WINDOW_CASES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("engine", [0, 1, 2])
+@pytest.mark.parametrize("engine", [0, 1, 2, 3])
 def test_windowed_attention_fwd_bwd(nc, B, T, H, window, dtype, engine):
     # sliding window (query i sees keys j with 0 <= i - j < window) against the
     # full-block oracle's windowed attention
