@@ -63,6 +63,32 @@ __device__ __forceinline__ void set_status(int *status, int bit) {
 }
 
 // Element-wise helpers to load/store 8 contiguous values of T as floats.
+// Four consecutive elements (8 bytes of bf16, 16 of fp32) to and from fp32.
+template <typename T> struct Vec4;
+template <> struct Vec4<bf16> {
+  static __device__ __forceinline__ void load(const bf16 *p, float *f) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+  }
+  static __device__ __forceinline__ void store(bf16 *p, const float *f) {
+    uint2 u;
+    *reinterpret_cast<__nv_bfloat162 *>(&u.x) = __floats2bfloat162_rn(f[0], f[1]);
+    *reinterpret_cast<__nv_bfloat162 *>(&u.y) = __floats2bfloat162_rn(f[2], f[3]);
+    *reinterpret_cast<uint2 *>(p) = u;
+  }
+};
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ void load(const float *p, float *f) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  }
+  static __device__ __forceinline__ void store(float *p, const float *f) {
+    *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+};
+
 template <typename T> struct Vec8;
 template <> struct Vec8<bf16> {
   static __device__ __forceinline__ void load(const bf16 *p, float *f) {

@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
 //   y_i = x_i cos - x_{i+64} sin,  y_{i+64} = x_i sin + x_{i+64} cos,
 // angle = pos * theta^(-i/64), pos = token index within its row of T.
 // QK-norm after RoPE: per-head parameterless RMSNorm over the 128 dims.
-// One warp per (token, head); lane l owns dims {2l, 2l+1} and {64+2l, 65+2l}.
 template <typename T> struct Pair2;
 template <> struct Pair2<bf16> {
   static __device__ __forceinline__ float2 load(const bf16 *p) {
@@ -190,20 +189,18 @@ template <> struct Pair2<float> {
 };
 
 // One warp per token: the q heads and the k head of a token are H+1
-// contiguous 128-wide rows; each half-warp holds one head, 8 values per lane
-// (lane j of the half-warp: dims 8j..8j+7), so a warp covers two heads per
-// step with 16-byte accesses.  The RoPE partner of dim i < 64 is dim i + 64,
-// held by lane j + 8 of the same half-warp (one shuffle); the head's sum of
-// squares is a 16-lane reduction.
+// contiguous 128-wide rows; each half-warp holds one head, so a warp covers
+// two heads per step.  Lane j of the half-warp holds both members of its four
+// RoPE pairs, dims 4j..4j+3 and 64+4j..64+4j+3 (two 8-byte loads for bf16), so
+// the rotation needs no data from other lanes; the head's sum of squares is a
+// 16-lane reduction.
 template <typename T>
 __device__ __forceinline__ void rope_pair_tables(const float *cos_t, const float *sin_t, int pos, int j,
-                                                 float (&c)[8], float (&s)[8]) {
-  const int i0 = (j & 7) * 8;  // dims i0..i0+7 of the first half share their angles with i0+64..
-  const float4 *cp = reinterpret_cast<const float4 *>(cos_t + pos * 64 + i0);
-  const float4 *sp = reinterpret_cast<const float4 *>(sin_t + pos * 64 + i0);
-  const float4 c0 = cp[0], c1 = cp[1], s0 = sp[0], s1 = sp[1];
-  c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w; c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
-  s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w; s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+                                                 float (&c)[4], float (&s)[4]) {
+  const float4 c4 = *reinterpret_cast<const float4 *>(cos_t + pos * 64 + 4 * j);
+  const float4 s4 = *reinterpret_cast<const float4 *>(sin_t + pos * 64 + 4 * j);
+  c[0] = c4.x; c[1] = c4.y; c[2] = c4.z; c[3] = c4.w;
+  s[0] = s4.x; s[1] = s4.y; s[2] = s4.z; s[3] = s4.w;
 }
 
 __device__ __forceinline__ float half_warp_sum(float v) {
@@ -260,32 +257,39 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(
     if (cache.kc) Vec8<T>::store(cache.vc + (kc_row - cache.kc) + lane * 8, v);
   }
   const int hw = lane >> 4, j = lane & 15;
-  float c[8], s[8];
+  float c[4], s[4];
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
   T *row = qkv + (size_t)tok * ld;
   for (int h0 = 0; h0 < H + 1; h0 += 2) {
     const int h = h0 + hw;
     const bool live = h < H + 1;  // uniform per half-warp
-    float x[8];
-    if (live) Vec8<T>::load(row + h * kHeadDim + j * 8, x);
-    else
+    float a[4], b[4];             // dims 4j.. and 64 + 4j..
+    if (live) {
+      Vec4<T>::load(row + h * kHeadDim + 4 * j, a);
+      Vec4<T>::load(row + h * kHeadDim + 64 + 4 * j, b);
+    } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
-    float y[8], ss = 0.f;
+      for (int i = 0; i < 4; ++i) { a[i] = 0.f; b[i] = 0.f; }
+    }
+    float ya[4], yb[4], ss = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float partner = __shfl_xor_sync(0xffffffffu, x[i], 8);
-      // first half: y_i = x_i cos - x_{i+64} sin ; second half: y_{i+64} = x_i sin + x_{i+64} cos
-      y[i] = j < 8 ? x[i] * c[i] - partner * s[i] : partner * s[i] + x[i] * c[i];
-      ss += y[i] * y[i];
+    for (int i = 0; i < 4; ++i) {
+      // y_i = x_i cos - x_{i+64} sin ;  y_{i+64} = x_i sin + x_{i+64} cos
+      ya[i] = a[i] * c[i] - b[i] * s[i];
+      yb[i] = a[i] * s[i] + b[i] * c[i];
+      ss += ya[i] * ya[i] + yb[i] * yb[i];
     }
     ss = half_warp_sum(ss);
     const float r = rsqrtf(ss / (float)kHeadDim + kEps);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] *= r;
+    for (int i = 0; i < 4; ++i) { ya[i] *= r; yb[i] *= r; }
     if (live) {
-      Vec8<T>::store(row + h * kHeadDim + j * 8, y);
-      if (h == H && kc_row) Vec8<T>::store(kc_row + j * 8, y);
+      Vec4<T>::store(row + h * kHeadDim + 4 * j, ya);
+      Vec4<T>::store(row + h * kHeadDim + 64 + 4 * j, yb);
+      if (h == H && kc_row) {
+        Vec4<T>::store(kc_row + 4 * j, ya);
+        Vec4<T>::store(kc_row + 64 + 4 * j, yb);
+      }
       if (j == 0) {
         if (h < H) rq[(size_t)tok * H + h] = r;
         else rk[tok] = r;
@@ -307,36 +311,40 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(
   if (tok >= M) return;
   const int pos = tok % T_len;
   const int hw = lane >> 4, j = lane & 15;
-  float c[8], s[8];
+  float c[4], s[4];
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
   T *drow = dqkv + (size_t)tok * ld;
   const T *yrow = qkv + (size_t)tok * ld;
   for (int h0 = 0; h0 < H + 1; h0 += 2) {
     const int h = h0 + hw;
     const bool live = h < H + 1;
-    float dy[8], y[8];
+    float da[4], db[4], ya[4], yb[4];  // dims 4j.. and 64 + 4j..
     if (live) {
-      Vec8<T>::load(drow + h * kHeadDim + j * 8, dy);
-      Vec8<T>::load(yrow + h * kHeadDim + j * 8, y);
+      Vec4<T>::load(drow + h * kHeadDim + 4 * j, da);
+      Vec4<T>::load(drow + h * kHeadDim + 64 + 4 * j, db);
+      Vec4<T>::load(yrow + h * kHeadDim + 4 * j, ya);
+      Vec4<T>::load(yrow + h * kHeadDim + 64 + 4 * j, yb);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { dy[i] = 0.f; y[i] = 0.f; }
+      for (int i = 0; i < 4; ++i) { da[i] = 0.f; db[i] = 0.f; ya[i] = 0.f; yb[i] = 0.f; }
     }
     const float r = live ? (h < H ? rq[(size_t)tok * H + h] : rk[tok]) : 0.f;
     float dot = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dot += dy[i] * y[i];
+    for (int i = 0; i < 4; ++i) dot += da[i] * ya[i] + db[i] * yb[i];
     dot = half_warp_sum(dot) / (float)kHeadDim;
-    float g[8], out[8];
+    float oa[4], ob[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] = r * (dy[i] - y[i] * dot);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float partner = __shfl_xor_sync(0xffffffffu, g[i], 8);
-      // first half: g_i cos + g_{i+64} sin ; second half: -g_i sin + g_{i+64} cos
-      out[i] = j < 8 ? g[i] * c[i] + partner * s[i] : g[i] * c[i] - partner * s[i];
+    for (int i = 0; i < 4; ++i) {
+      const float ga = r * (da[i] - ya[i] * dot), gb = r * (db[i] - yb[i] * dot);
+      // dx_i = g_i cos + g_{i+64} sin ;  dx_{i+64} = -g_i sin + g_{i+64} cos
+      oa[i] = ga * c[i] + gb * s[i];
+      ob[i] = gb * c[i] - ga * s[i];
     }
-    if (live) Vec8<T>::store(drow + h * kHeadDim + j * 8, out);
+    if (live) {
+      Vec4<T>::store(drow + h * kHeadDim + 4 * j, oa);
+      Vec4<T>::store(drow + h * kHeadDim + 64 + 4 * j, ob);
+    }
   }
 }
 
