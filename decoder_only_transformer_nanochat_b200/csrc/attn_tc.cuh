@@ -855,6 +855,15 @@ __host__ __device__ inline int dkdv_pieces(int n_it, int chunk) {
   return chunk > 0 ? (n_it + chunk - 1) / chunk : 1;
 }
 
+// Persistent: CTA c takes the work items c, c + grid, ... (item = 128 queries
+// of one (b, h), latest query tiles first); grid = the item count gives one
+// item per CTA.  Q and dO have one buffer each: the next item's tiles are
+// requested as soon as the last score MMAs of the current one are done
+// (qg_free), so they land while its last dS, dQ MMA and store finish.  The
+// output tile is staged in the V ring slot of the item's last key tile, whose
+// release (v_empty) then waits for the store to have read it; the next item's
+// first dQ MMA waits until the store's TMEM read is done (dq_free).  Barrier
+// phases count uses over all items of the CTA.
 template <bool kWin>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q,    // qkv, box 64 x 128 (Q, K, V tiles)
@@ -867,10 +876,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *sK = sG + kTileBytes;                 // K ring
   uint8_t *sV = sK + kDqKStages * kTileBytes;    // V ring
   uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kDqVStages * kTileBytes);
-  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_empty, ds_full[2], ds_empty[2], fin, drain
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_empty, ds_full[2], ds_empty[2], fin,
+  // drain, qg_free, dq_free
   constexpr int kB = 1 + 2 * kDqKStages + 2 * kDqVStages;
-  static_assert((kB + 8) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 8);
+  static_assert((kB + 10) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 10);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t q_full = smem_u32(bars);
   auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
@@ -881,16 +891,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto ds_full = [&](int s) { return smem_u32(bars + kB + 2 + s); };
   auto ds_empty = [&](int s) { return smem_u32(bars + kB + 4 + s); };
   const uint32_t fin = smem_u32(bars + kB + 6), drain = smem_u32(bars + kB + 7);
+  const uint32_t qg_free = smem_u32(bars + kB + 8), dq_free = smem_u32(bars + kB + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = gridDim.x / p.n_tiles;
-  const int qt = p.n_tiles - 1 - (int)blockIdx.x / BH;
-  const int h = ((int)blockIdx.x % BH) % p.H, b = ((int)blockIdx.x % BH) / p.H;
-  const int q0 = qt * kQ;
-  const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kBK : 0;
-  const int n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK - kt_lo;
-  const int kbase = kt_lo * kBK;
+  const int BH = p.B * p.H;
+  const int n_items = BH * p.n_tiles;
   const int C = p.H * kD;
+  auto item_of = [&](int it, int &q0, int &b, int &h, int &kbase, int &n_kv) {
+    const int qt = p.n_tiles - 1 - it / BH;
+    h = (it % BH) % p.H;
+    b = (it % BH) / p.H;
+    q0 = qt * kQ;
+    const int kt_lo = kWin ? max(0, q0 - p.window + 1) / kBK : 0;
+    n_kv = (min(q0 + kQ, p.T) + kBK - 1) / kBK - kt_lo;
+    kbase = kt_lo * kBK;
+  };
   // TMEM columns: S at 0, dP at 128 (one buffer, free again as soon as the
   // element-wise warps have loaded it); dQ at 256; dS[2] (bf16 pairs) at 384, 448
   if (threadIdx.x == 0) {
@@ -902,6 +917,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < 2; ++s) { mbar_init(ds_full(s), kSoft); mbar_init(ds_empty(s), 1); }
     mbar_init(fin, 1);
     mbar_init(drain, 1);
+    mbar_init(qg_free, 1);
+    mbar_init(dq_free, kSoft);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -913,33 +930,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(q_full, 2 * kTileBytes);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_3d(smem_u32(sQ) + i * 16384, &map_q, h * kD + 64 * i, q0, b, q_full);
-        tma_load_3d(smem_u32(sG) + i * 16384, &map_do, h * kD + 64 * i, q0, b, q_full);
-      }
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j % kDqKStages, vs = j % kDqVStages;
-        if (!mbar_wait(k_empty(ks), ((j / kDqKStages) & 1) ^ 1, abort_flag, p.status)) break;
-        mbar_expect_tx(k_full(ks), kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, kbase + j * kBK, b,
-                      k_full(ks));
-        if (!mbar_wait(v_empty(vs), ((j / kDqVStages) & 1) ^ 1, abort_flag, p.status)) break;
-        mbar_expect_tx(v_full(vs), kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, kbase + j * kBK, b,
-                      v_full(vs));
-        ++issued;
+      int kc = 0, vc = 0, li = 0, nq = 0;  // K, V tiles, items, Q/dO pairs requested so far
+      bool okp = true;
+      for (int it = blockIdx.x; it < n_items && okp; it += gridDim.x, ++li) {
+        int q0, b, h, kbase, n_kv;
+        item_of(it, q0, b, h, kbase, n_kv);
+        // Q and dO take the next item once the previous item's last score MMAs are done
+        if (li > 0 && !(okp = mbar_wait(qg_free, (li - 1) & 1, abort_flag, p.status))) break;
+        mbar_expect_tx(q_full, 2 * kTileBytes);
+        for (int i = 0; i < 2; ++i) {
+          tma_load_3d(smem_u32(sQ) + i * 16384, &map_q, h * kD + 64 * i, q0, b, q_full);
+          tma_load_3d(smem_u32(sG) + i * 16384, &map_do, h * kD + 64 * i, q0, b, q_full);
+        }
+        ++nq;
+        for (int j = 0; j < n_kv; ++j) {
+          const int ks = kc % kDqKStages, vs = vc % kDqVStages;
+          if (!(okp = mbar_wait(k_empty(ks), ((kc / kDqKStages) & 1) ^ 1, abort_flag, p.status))) break;
+          mbar_expect_tx(k_full(ks), kTileBytes);
+          for (int i = 0; i < 2; ++i)
+            tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, kbase + j * kBK, b,
+                        k_full(ks));
+          ++kc;
+          if (!(okp = mbar_wait(v_empty(vs), ((vc / kDqVStages) & 1) ^ 1, abort_flag, p.status))) break;
+          mbar_expect_tx(v_full(vs), kTileBytes);
+          for (int i = 0; i < 2; ++i)
+            tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, kbase + j * kBK, b,
+                        v_full(vs));
+          ++vc;
+        }
       }
       // let the loads in flight land before the CTA can exit
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try(q_full, 0) && globaltimer() - t0 < kWaitNs) {}
-      for (int j = max(0, issued - kDqVStages); j < issued; ++j) {
+      if (nq > 0) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(q_full, (nq - 1) & 1) && globaltimer() - t0 < kWaitNs) {}
+      }
+      for (int c = max(0, kc - kDqKStages); c < kc; ++c) {
         const uint64_t t1 = globaltimer();
-        while (!mbar_try(k_full(j % kDqKStages), (j / kDqKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
-        while (!mbar_try(v_full(j % kDqVStages), (j / kDqVStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+        while (!mbar_try(k_full(c % kDqKStages), (c / kDqKStages) & 1) && globaltimer() - t1 < kWaitNs) {}
+      }
+      for (int c = max(0, vc - kDqVStages); c < vc; ++c) {
+        const uint64_t t1 = globaltimer();
+        while (!mbar_try(v_full(c % kDqVStages), (c / kDqVStages) & 1) && globaltimer() - t1 < kWaitNs) {}
       }
     }
   } else if (warp == 1) {
@@ -955,41 +986,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dKs = smem_desc(smem_u32(sK), 16, 1024);      // K-major view of K stage 0
       const uint64_t dKm = smem_desc(smem_u32(sK), 16384, 1024);   // MN-major view of K stage 0
       const uint64_t dVs = smem_desc(smem_u32(sV), 16, 1024);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-      auto issue_sdp = [&](int j) -> bool {
-        const int ks = j % kDqKStages, vs = j % kDqVStages;
-        if (!mbar_wait(k_full(ks), (j / kDqKStages) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(v_full(vs), (j / kDqVStages) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint64_t k = dKs + (uint64_t)((ks * kTileBytes) >> 4), v = dVs + (uint64_t)((vs * kTileBytes) >> 4);
+      int kc = 0, vc = 0, sc = 0, li = 0;  // K, V tiles, score tiles and items taken so far
+      int dsc[2] = {0, 0};                // dS tiles per TMEM buffer
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++li) {
+        int q0, b, h, kbase, n_kv;
+        item_of(it, q0, b, h, kbase, n_kv);
+        if (!(ok = mbar_wait(q_full, li & 1, abort_flag, p.status))) break;
+        const int kc0 = kc;  // this item's first K tile
+        auto issue_sdp = [&](int j) -> bool {
+          const int ks = kc % kDqKStages, vs = vc % kDqVStages;
+          if (!mbar_wait(k_full(ks), (kc / kDqKStages) & 1, abort_flag, p.status)) return false;
+          if (!mbar_wait(v_full(vs), (vc / kDqVStages) & 1, abort_flag, p.status)) return false;
+          if (!mbar_wait(s_empty, (sc & 1) ^ 1, abort_flag, p.status)) return false;
+          tc_fence_after();
+          const uint64_t k = dKs + (uint64_t)((ks * kTileBytes) >> 4), v = dVs + (uint64_t)((vs * kTileBytes) >> 4);
 #pragma unroll
-        for (int s = 0; s < kD / 16; ++s) {
-          const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
-          tc_mma(tmem + 0, dQd + o, k + o, idesc_s, s > 0);
-          tc_mma(tmem + 128, dGd + o, v + o, idesc_s, s > 0);
+          for (int s = 0; s < kD / 16; ++s) {
+            const uint32_t o = ((s >> 2) * 16384 + (s & 3) * 32) >> 4;
+            tc_mma(tmem + 0, dQd + o, k + o, idesc_s, s > 0);
+            tc_mma(tmem + 128, dGd + o, v + o, idesc_s, s > 0);
+          }
+          tc_commit(s_full);
+          if (j + 1 < n_kv) tc_commit(v_empty(vs));  // V is read by dP only; the last slot stages the output
+          else tc_commit(qg_free);                    // Q and dO are read by no later MMA of this item
+          ++kc;
+          ++vc;
+          ++sc;
+          return true;
+        };
+        // Fixed order S_{j+1}, then dQ += dS_j K_j: the scores of the next tile
+        // are on the tensor core while the element-wise warps turn S_j into dS_j.
+        ok = issue_sdp(0);
+        // the previous item's dQ must have left TMEM before this item's first dQ MMA
+        if (ok && li > 0) ok = mbar_wait(dq_free, (li - 1) & 1, abort_flag, p.status);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          if (j + 1 < n_kv && !(ok = issue_sdp(j + 1))) break;
+          const int bb = j & 1, ks = (kc0 + j) % kDqKStages;
+          if (!(ok = mbar_wait(ds_full(bb), dsc[bb] & 1, abort_flag, p.status))) break;
+          ++dsc[bb];
+          tc_fence_after();
+          const uint64_t k = dKm + (uint64_t)((ks * kTileBytes) >> 4);
+#pragma unroll
+          for (int s = 0; s < kBK / 16; ++s)
+            tc_mma_ts(tmem + 256, tmem + kDsCol + bb * 64 + 8 * s, k + ((s * 2048) >> 4), idesc_q,
+                      (j > 0 || s > 0) ? 1u : 0u);
+          tc_commit(ds_empty(bb));
+          tc_commit(k_empty(ks));
         }
-        tc_commit(s_full);
-        tc_commit(v_empty(vs));  // V is read by dP only
-        return true;
-      };
-      // Fixed order S_{j+1}, then dQ += dS_j K_j: the scores of the next tile
-      // are on the tensor core while the element-wise warps turn S_j into dS_j.
-      if (ok) ok = issue_sdp(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !(ok = issue_sdp(j + 1))) break;
-        const int bb = j & 1, ks = j % kDqKStages;
-        if (!(ok = mbar_wait(ds_full(bb), (j >> 1) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
-        const uint64_t k = dKm + (uint64_t)((ks * kTileBytes) >> 4);
-#pragma unroll
-        for (int s = 0; s < kBK / 16; ++s)
-          tc_mma_ts(tmem + 256, tmem + kDsCol + bb * 64 + 8 * s, k + ((s * 2048) >> 4), idesc_q,
-                    (j > 0 || s > 0) ? 1u : 0u);
-        tc_commit(ds_empty(bb));
-        tc_commit(k_empty(ks));
+        if (ok) tc_commit(fin);
       }
-      tc_commit(fin);
       tc_commit(drain);
       const uint64_t t0 = globaltimer();
       while (!mbar_try(drain, 0) && globaltimer() - t0 < kWaitNs) {}
@@ -998,16 +1044,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ---------------- element-wise warps: thread = query row, half g of the keys ----------------
     const int quarter = warp & 3, g = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
-    const int row = q0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = rsqrtf((float)kD) * kLog2e;
+    const int c0 = g * 64;  // this thread's 64 keys of the 128-key tile
+    float *sDpart = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [2][128]
+    int tc = 0, vcount = 0, li = 0;  // score tiles, V tiles and items so far
+    int dsc[2] = {0, 0};
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
+    int q0, b, h, kbase, n_kv;
+    item_of(it, q0, b, h, kbase, n_kv);
+    const int row = q0 + r;
     const int rr_ = min(row, p.T - 1);
     const float L = p.lse[((int64_t)b * p.H + h) * p.T + rr_] * kLog2e;
-    const int c0 = g * 64;  // this thread's 64 keys of the 128-key tile
     // D = rowsum(dO * O) for this row: dO from the shared tile, O from global;
     // warpgroup g sums dims [64g, 64g + 64) and the halves meet in shared memory
-    float *sDpart = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [2][128]
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+    if (ok) ok = mbar_wait(q_full, li & 1, abort_flag, p.status);
     {
       float part = 0.f;
       if (row < p.T) {
@@ -1026,10 +1078,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     asm volatile("bar.sync 1, 256;" ::: "memory");
     const float Dv = sDpart[r] + sDpart[kQ + r];
     if (g == 0 && row < p.T) p.Drow[((int64_t)b * p.H + h) * p.T + row] = Dv;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_kv && ok; ++j) {
       const int bb = j & 1;
-      ok = mbar_wait(s_full, j & 1, abort_flag, p.status);
+      ok = mbar_wait(s_full, tc & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      ++tc;
       tc_fence_after();
       // all 64 S and dP values of this row half at once, so the buffer is
       // free for the next tile's MMAs before any arithmetic here
@@ -1056,15 +1109,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         packed[i / 2] = pack2(d2[0], d2[1]);
       }
-      // dS_j into TMEM buffer bb once dQ += dS_{j-2} K_{j-2} has read it
-      ok = mbar_wait(ds_empty(bb), ((j >> 1) & 1) ^ 1, abort_flag, p.status);
+      // dS_j into TMEM buffer bb once the dQ MMA two tiles back has read it
+      ok = mbar_wait(ds_empty(bb), (dsc[bb] & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      ++dsc[bb];
       tmem_st32(lane_base + kDsCol + bb * 64 + 32 * g, packed);
       tc_fence_before();
       mbar_arrive(ds_full(bb));
     }
-    if (ok) ok = mbar_wait(fin, 0, abort_flag, p.status);
-    ok = __all_sync(0xffffffffu, ok);
+    vcount += n_kv;
+    const int vslot = (vcount - 1) % kDqVStages;  // the item's last V tile: its slot stages the output
+    uint8_t *stg = sV + vslot * kTileBytes;
+    if (ok) ok = mbar_wait(fin, li & 1, abort_flag, p.status);
+    ok = epi_vote_all256(ok);
     if (ok) {
       tc_fence_after();
       const float scale = rsqrtf((float)kD);
@@ -1079,17 +1136,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           w.y = pack2(__uint_as_float(rr[8 * u + 2]) * scale, __uint_as_float(rr[8 * u + 3]) * scale);
           w.z = pack2(__uint_as_float(rr[8 * u + 4]) * scale, __uint_as_float(rr[8 * u + 5]) * scale);
           w.w = pack2(__uint_as_float(rr[8 * u + 6]) * scale, __uint_as_float(rr[8 * u + 7]) * scale);
-          *reinterpret_cast<uint4 *>(sQ + tile_unit(r, c * 4 + u)) = w;  // Q is no longer read
+          *reinterpret_cast<uint4 *>(stg + tile_unit(r, c * 4 + u)) = w;  // V of this slot is no longer read
         }
       }
     }
+    tc_fence_before();
+    mbar_arrive(dq_free);  // the dQ accumulator may take the next item's MMAs
     fence_proxy_async();
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok && warp == 2 && lane == 0) {
-      for (int i = 0; i < 2; ++i) tma_store_3d(&map_dq, smem_u32(sQ) + i * 16384, h * kD + 64 * i, q0, b);
+      for (int i = 0; i < 2; ++i) tma_store_3d(&map_dq, smem_u32(stg) + i * 16384, h * kD + 64 * i, q0, b);
       bulk_commit();
-      bulk_wait0();
+      bulk_wait_read0();
+      mbar_arrive(v_empty(vslot));  // the slot may take a later V tile
     }
+    if (!ok) break;
+    }
+    if (warp == 2 && lane == 0) bulk_wait0();  // every store complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -1624,8 +1687,11 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   }
   const int grid_kv = dkdv_grid(B, T, H, window, p.chunk);
   const bool win = windowed(window, T);
-  if (win) attn_bwd_dq_tc_kernel<true><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
-  else attn_bwd_dq_tc_kernel<false><<<B * H * p.n_tiles, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
+  // dQ: persistent, one CTA per SM over the B * H * n_tiles query tiles
+  const int dq_items = B * H * p.n_tiles;
+  const int grid_dq = num_sms > 0 && num_sms < dq_items ? num_sms : dq_items;
+  if (win) attn_bwd_dq_tc_kernel<true><<<grid_dq, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
+  else attn_bwd_dq_tc_kernel<false><<<grid_dq, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     fprintf(stderr, "nanochat_b200: attention dQ launch: %s\n", cudaGetErrorString(e));
