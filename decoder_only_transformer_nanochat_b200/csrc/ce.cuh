@@ -45,6 +45,29 @@ __device__ __forceinline__ void softcap_parts_fast(float z, float &t, float &sec
   sech2 = u * (2.f - u);
 }
 
+// The same for two logits at once, the FMA-pipe steps in packed f32x2 form
+// (each lane rounds exactly as the scalar form above, so the results are
+// bit-identical to two softcap_parts_fast calls).
+__device__ __forceinline__ void softcap_parts_fast2(float za, float zb, float &ta, float &tb, float &sa,
+                                                    float &sb) {
+  constexpr float c = -2.f * kLog2e / kSoftcap;
+  const uint64_t E = f2(ex2_fast(fabsf(za) * c), ex2_fast(fabsf(zb) * c));
+  const uint64_t one = f2(1.f, 1.f), m1 = f2(-1.f, -1.f);
+  const uint64_t y = add2(one, E);
+  const uint64_t ny = fma2(E, m1, m1);  // -(1 + E), exactly
+  uint64_t r = fma2(f2(-8.f / 17.f, -8.f / 17.f), y, f2(24.f / 17.f, 24.f / 17.f));
+  r = fma2(r, fma2(ny, r, one), r);
+  r = fma2(r, fma2(ny, r, one), r);
+  r = fma2(r, fma2(ny, r, one), r);
+  const uint64_t two = f2(2.f, 2.f);
+  const uint64_t u = mul2(mul2(two, E), r);
+  float va, vb;
+  f2split(fma2(u, m1, one), va, vb);  // 1 - u
+  ta = copysignf(va, za);
+  tb = copysignf(vb, zb);
+  f2split(mul2(u, fma2(u, m1, two)), sa, sb);  // u (2 - u)
+}
+
 // Two floats packed into one 32-bit register as fp16 / bf16 (lo in the low half).
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   uint32_t d;
@@ -200,16 +223,26 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
       const int c = threadIdx.x + k * kCeThreads;
       if (c < n8) {
         float e[8], part = 0.f;
+        uint64_t part2 = f2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = unpack_bf2(pk[k][j]);
           float ta, sa, tb, sb;
-          softcap_parts_fast(f.x, ta, sa);
-          softcap_parts_fast(f.y, tb, sb);
-          e[2 * j] = ex2_fast(fmaf(k2, ta, -m2));
-          e[2 * j + 1] = ex2_fast(fmaf(k2, tb, -m2));
-          part += e[2 * j] + e[2 * j + 1];
-          pk[k][j] = pack_h2(e[2 * j] * sa, e[2 * j + 1] * sb);
+          softcap_parts_fast2(f.x, f.y, ta, tb, sa, sb);
+          float xa, xb;
+          f2split(fma2(f2(k2, k2), f2(ta, tb), f2(-m2, -m2)), xa, xb);
+          e[2 * j] = ex2_fast(xa);
+          e[2 * j + 1] = ex2_fast(xb);
+          const uint64_t ee = f2(e[2 * j], e[2 * j + 1]);
+          part2 = add2(part2, ee);
+          float wa, wb;
+          f2split(mul2(ee, f2(sa, sb)), wa, wb);
+          pk[k][j] = pack_h2(wa, wb);
+        }
+        {
+          float pa, pb;
+          f2split(part2, pa, pb);
+          part = pa + pb;
         }
         if ((unsigned)(tgt - c * 8) < 8u) {  // the target's chunk: its term stays out
           part = 0.f;
@@ -234,10 +267,13 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
       const int c = threadIdx.x + k * kCeThreads;
       if (c < n8) {
         uint32_t o[4];
+        const uint64_t scale2 = f2(scale, scale);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = unpack_h2(pk[k][j]);
-          o[j] = pack_bf2(f.x * scale, f.y * scale);
+          float oa, ob;
+          f2split(mul2(f2(f.x, f.y), scale2), oa, ob);
+          o[j] = pack_bf2(oa, ob);
         }
         if ((unsigned)(tgt - c * 8) < 8u) {
           const int j = (tgt - c * 8) >> 1;
