@@ -122,26 +122,6 @@ template <> struct Vec4<float> {
   }
 };
 
-// The same four elements kept in their storage form between a load and its
-// use, so a warp can issue several loads before the first conversion.
-template <typename T> struct Raw4;
-template <> struct Raw4<bf16> {
-  using type = uint2;
-  static __device__ __forceinline__ type load(const bf16 *p) { return *reinterpret_cast<const uint2 *>(p); }
-  static __device__ __forceinline__ void to_f(type u, float *f) {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-  }
-  static __device__ __forceinline__ type zero() { return make_uint2(0u, 0u); }
-};
-template <> struct Raw4<float> {
-  using type = float4;
-  static __device__ __forceinline__ type load(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-  static __device__ __forceinline__ void to_f(type u, float *f) { f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w; }
-  static __device__ __forceinline__ type zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-};
-
 template <typename T> struct Vec8;
 template <> struct Vec8<bf16> {
   static __device__ __forceinline__ void load(const bf16 *p, float *f) {

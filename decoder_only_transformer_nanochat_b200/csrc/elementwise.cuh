@@ -260,54 +260,39 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(
   float c[4], s[4];
   rope_pair_tables<T>(cos_t, sin_t, pos, j, c, s);
   T *row = qkv + (size_t)tok * ld;
-  // heads two at a time (one per half-warp), four steps' loads issued before
-  // the first step's arithmetic: the stores write the same rows in place, so
-  // the loads could not otherwise move ahead of them
-  constexpr int kAhead = 4;
-  for (int h00 = 0; h00 < H + 1; h00 += 2 * kAhead) {
-    typename Raw4<T>::type ra[kAhead], rb[kAhead];  // dims 4j.. and 64 + 4j.. of each step's head
+  for (int h0 = 0; h0 < H + 1; h0 += 2) {
+    const int h = h0 + hw;
+    const bool live = h < H + 1;  // uniform per half-warp
+    float a[4], b[4];             // dims 4j.. and 64 + 4j..
+    if (live) {
+      Vec4<T>::load(row + h * kHeadDim + 4 * j, a);
+      Vec4<T>::load(row + h * kHeadDim + 64 + 4 * j, b);
+    } else {
 #pragma unroll
-    for (int t = 0; t < kAhead; ++t) {
-      const int h = h00 + 2 * t + hw;
-      if (h < H + 1) {
-        ra[t] = Raw4<T>::load(row + h * kHeadDim + 4 * j);
-        rb[t] = Raw4<T>::load(row + h * kHeadDim + 64 + 4 * j);
-      } else {
-        ra[t] = Raw4<T>::zero();
-        rb[t] = Raw4<T>::zero();
-      }
+      for (int i = 0; i < 4; ++i) { a[i] = 0.f; b[i] = 0.f; }
     }
+    float ya[4], yb[4], ss = 0.f;
 #pragma unroll
-    for (int t = 0; t < kAhead; ++t) {
-      const int h = h00 + 2 * t + hw;
-      if (h00 + 2 * t >= H + 1) break;  // uniform: no head left for either half-warp
-      const bool live = h < H + 1;      // uniform per half-warp
-      float a[4], b[4];
-      Raw4<T>::to_f(ra[t], a);
-      Raw4<T>::to_f(rb[t], b);
-      float ya[4], yb[4], ss = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      // y_i = x_i cos - x_{i+64} sin ;  y_{i+64} = x_i sin + x_{i+64} cos
+      ya[i] = a[i] * c[i] - b[i] * s[i];
+      yb[i] = a[i] * s[i] + b[i] * c[i];
+      ss += ya[i] * ya[i] + yb[i] * yb[i];
+    }
+    ss = half_warp_sum(ss);
+    const float r = rsqrtf(ss / (float)kHeadDim + kEps);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        // y_i = x_i cos - x_{i+64} sin ;  y_{i+64} = x_i sin + x_{i+64} cos
-        ya[i] = a[i] * c[i] - b[i] * s[i];
-        yb[i] = a[i] * s[i] + b[i] * c[i];
-        ss += ya[i] * ya[i] + yb[i] * yb[i];
+    for (int i = 0; i < 4; ++i) { ya[i] *= r; yb[i] *= r; }
+    if (live) {
+      Vec4<T>::store(row + h * kHeadDim + 4 * j, ya);
+      Vec4<T>::store(row + h * kHeadDim + 64 + 4 * j, yb);
+      if (h == H && kc_row) {
+        Vec4<T>::store(kc_row + 4 * j, ya);
+        Vec4<T>::store(kc_row + 64 + 4 * j, yb);
       }
-      ss = half_warp_sum(ss);
-      const float r = rsqrtf(ss / (float)kHeadDim + kEps);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { ya[i] *= r; yb[i] *= r; }
-      if (live) {
-        Vec4<T>::store(row + h * kHeadDim + 4 * j, ya);
-        Vec4<T>::store(row + h * kHeadDim + 64 + 4 * j, yb);
-        if (h == H && kc_row) {
-          Vec4<T>::store(kc_row + 4 * j, ya);
-          Vec4<T>::store(kc_row + 64 + 4 * j, yb);
-        }
-        if (j == 0) {
-          if (h < H) rq[(size_t)tok * H + h] = r;
-          else rk[tok] = r;
-        }
+      if (j == 0) {
+        if (h < H) rq[(size_t)tok * H + h] = r;
+        else rk[tok] = r;
       }
     }
   }
