@@ -16,7 +16,8 @@ from ._binding import (NC_BF16, NC_EALIGN, NC_ECUDA, NC_EINVAL, NC_ENOMEM,  # no
                        nc_param_count, nc_fwd_bwd_ex, nc_grad_buckets, nc_set_grad_events,
                        NC_ACCUMULATE, nc_kv_cache_bytes, nc_prefill, nc_decode, nc_optim_state_bytes,
                        nc_optim_workspace_bytes, nc_optim_init, nc_optim_step, nc_rmsnorm, nc_rmsnorm_bwd,
-                       nc_rope_qknorm, nc_rope_qknorm_bwd, nc_attention_bwd_scratch_bytes, nc_attention_bwd_ex)
+                       nc_rope_qknorm, nc_rope_qknorm_bwd, nc_attention_bwd_scratch_bytes, nc_attention_bwd_ex,
+                       nc_set_attention_ctas)
 
 
 def __getattr__(name):

@@ -93,6 +93,7 @@ _SIGS = {
     "nc_attention_bwd_scratch_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "nc_attention_bwd_ex": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _I, _I, _I, _I,
                                  _I, _I, _P]),
+    "nc_set_attention_ctas": (_I, [_I]),
     "nc_rmsnorm": (_I, [_P, _P, _P, _I, _I, _I, _P]),
     "nc_rmsnorm_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "nc_rope_qknorm": (_I, [_P, _P, ctypes.c_int64, _P, _P, _I, _I, _P]),
@@ -302,6 +303,11 @@ def nc_attention_bwd_ex(qkv, ld, O, dO, lse, Drow, scratch, scratch_bytes, dqkv,
                         window: int = 0) -> int:
     return load_library().nc_attention_bwd_ex(qkv, ld, O, dO, lse, Drow, scratch, scratch_bytes, dqkv, B, T, H,
                                               window, dtype, engine, stream)
+
+
+def nc_set_attention_ctas(ctas: int) -> int:
+    """Cap on the CTAs of the persistent attention kernels (0: one per SM)."""
+    return load_library().nc_set_attention_ctas(ctas)
 
 
 def nc_rmsnorm(x, y, r, M, C, dtype, stream) -> int:

@@ -24,6 +24,8 @@
 
 #include <stdio.h>
 
+#include <atomic>
+
 #include "tc_common.cuh"
 
 namespace nc {
@@ -859,7 +861,9 @@ __host__ __device__ inline int dkdv_pieces(int n_it, int chunk) {
 // of one (b, h), latest query tiles first); grid = the item count gives one
 // item per CTA.  Q and dO have one buffer each: the next item's tiles are
 // requested as soon as the last score MMAs of the current one are done
-// (qg_free), so they land while its last dS, dQ MMA and store finish.  The
+// (qg_free) and its D has been read out of the dO tile (d_done: an item with
+// one key tile can finish its MMAs before that), so they land while its last
+// dS, dQ MMA and store finish.  The
 // output tile is staged in the V ring slot of the item's last key tile, whose
 // release (v_empty) then waits for the store to have read it; the next item's
 // first dQ MMA waits until the store's TMEM read is done (dq_free).  Barrier
@@ -877,10 +881,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *sV = sK + kDqKStages * kTileBytes;    // V ring
   uint64_t *bars = reinterpret_cast<uint64_t *>(sV + kDqVStages * kTileBytes);
   // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_empty, ds_full[2], ds_empty[2], fin,
-  // drain, qg_free, dq_free
+  // drain, qg_free, dq_free, d_done
   constexpr int kB = 1 + 2 * kDqKStages + 2 * kDqVStages;
-  static_assert((kB + 10) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 10);
+  static_assert((kB + 11) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB + 11);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t q_full = smem_u32(bars);
   auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
@@ -892,6 +896,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto ds_empty = [&](int s) { return smem_u32(bars + kB + 4 + s); };
   const uint32_t fin = smem_u32(bars + kB + 6), drain = smem_u32(bars + kB + 7);
   const uint32_t qg_free = smem_u32(bars + kB + 8), dq_free = smem_u32(bars + kB + 9);
+  const uint32_t d_done = smem_u32(bars + kB + 10);  // the item's D has been read out of the dO tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
@@ -919,6 +924,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(drain, 1);
     mbar_init(qg_free, 1);
     mbar_init(dq_free, kSoft);
+    mbar_init(d_done, kSoft);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -935,8 +941,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int it = blockIdx.x; it < n_items && okp; it += gridDim.x, ++li) {
         int q0, b, h, kbase, n_kv;
         item_of(it, q0, b, h, kbase, n_kv);
-        // Q and dO take the next item once the previous item's last score MMAs are done
-        if (li > 0 && !(okp = mbar_wait(qg_free, (li - 1) & 1, abort_flag, p.status))) break;
+        // Q and dO take the next item once the previous item's last score MMAs
+        // are done and its D has been formed from the dO tile (with one key
+        // tile the MMAs can finish first)
+        if (li > 0 && !(okp = mbar_wait(qg_free, (li - 1) & 1, abort_flag, p.status) &&
+                              mbar_wait(d_done, (li - 1) & 1, abort_flag, p.status)))
+          break;
         mbar_expect_tx(q_full, 2 * kTileBytes);
         for (int i = 0; i < 2; ++i) {
           tma_load_3d(smem_u32(sQ) + i * 16384, &map_q, h * kD + 64 * i, q0, b, q_full);
@@ -1076,6 +1086,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       sDpart[g * kQ + r] = part;
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
+    mbar_arrive(d_done);  // every thread has read its part of the dO tile
     const float Dv = sDpart[r] + sDpart[kQ + r];
     if (g == 0 && row < p.T) p.Drow[((int64_t)b * p.H + h) * p.T + row] = Dv;
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -1582,8 +1593,19 @@ inline bool supported(const void *qkv, int64_t ld, const void *O) {
   return encode_fn() != nullptr && aligned(qkv, ld, O);
 }
 
+// Process-wide cap on the CTAs of the persistent attention kernels (0: one
+// per SM): fewer CTAs leave SMs to other streams and give each CTA more items.
+inline std::atomic<int> &persistent_cap() {
+  static std::atomic<int> cap{0};
+  return cap;
+}
+inline int persistent_ctas(int num_sms) {
+  const int c = persistent_cap().load();
+  return c > 0 && c < num_sms ? c : num_sms;
+}
+
 // pingpong: the kernel with two softmax warpgroups on alternating key tiles,
-// persistent over grid = min(items, num_sms) CTAs (num_sms = 0: one CTA per item)
+// persistent over grid = min(items, CTAs) CTAs (num_sms = 0: one CTA per item)
 inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, int B, int T, int H, int window,
                               bool pingpong, int num_sms, int *status, cudaStream_t st) {
   CUtensorMap mqk, mv, mo;
@@ -1602,7 +1624,8 @@ inline cudaError_t launch_fwd(const bf16 *qkv, int64_t ld, bf16 *O, float *lse, 
   const int grid = B * H * p.n_qt;
   const bool win = windowed(window, T);
   if (pingpong) {
-    const int g = num_sms > 0 && num_sms < grid ? num_sms : grid;
+    const int ctas = num_sms > 0 ? persistent_ctas(num_sms) : 0;
+    const int g = ctas > 0 && ctas < grid ? ctas : grid;
     if (win) attn_fwd_pp_kernel<true><<<g, kPpThreads, kSmem, st>>>(mqk, mv, mo, p);
     else attn_fwd_pp_kernel<false><<<g, kPpThreads, kSmem, st>>>(mqk, mv, mo, p);
   } else {
@@ -1689,7 +1712,8 @@ inline cudaError_t launch_bwd(const bf16 *qkv, int64_t ld, const bf16 *O, const 
   const bool win = windowed(window, T);
   // dQ: persistent, one CTA per SM over the B * H * n_tiles query tiles
   const int dq_items = B * H * p.n_tiles;
-  const int grid_dq = num_sms > 0 && num_sms < dq_items ? num_sms : dq_items;
+  const int dq_ctas = persistent_ctas(num_sms);
+  const int grid_dq = dq_ctas > 0 && dq_ctas < dq_items ? dq_ctas : dq_items;
   if (win) attn_bwd_dq_tc_kernel<true><<<grid_dq, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   else attn_bwd_dq_tc_kernel<false><<<grid_dq, kBwdThreads, kDqSmem, st>>>(mq128, mdo128, mout, p);
   cudaError_t e = cudaGetLastError();

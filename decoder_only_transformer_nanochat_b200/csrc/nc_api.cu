@@ -1219,7 +1219,7 @@ int nc_attention_bwd(const void *qkv, int64_t ld, const void *O, const void *dO,
   int num_sms = 0, *status = nullptr;
   if (op_setup(&num_sms, &status) != NC_OK) return NC_ECUDA;
   return attention_bwd_common(qkv, ld, O, dO, lse, Drow, dqkv, B, T, H, window, dtype, engine, status,
-                              (cudaStream_t)stream);
+                              (cudaStream_t)stream, nullptr, 0, num_sms);
 }
 
 int nc_attention_bwd_scratch_bytes(int B, int T, int H, int window, size_t *out) {
@@ -1264,7 +1264,7 @@ int nc_attention_bwd_noalloc(const void *qkv, int64_t ld, const void *O, const v
   SymbolAddrs a;
   if (symbol_addrs(&a) != NC_OK) return NC_ECUDA;
   return attention_bwd_common(qkv, ld, O, dO, lse, a.rowdot, dqkv, B, T, H, 0, dtype, engine, status,
-                              (cudaStream_t)stream);
+                              (cudaStream_t)stream, nullptr, 0, num_sms);
 }
 
 int nc_softcap_ce(void *z, int64_t ldz, const int32_t *targets, float *token_loss, int M, int V,
@@ -1359,6 +1359,12 @@ int nc_rope_qknorm_bwd(const nc_model *m, void *dqkv, const void *qkv, int64_t l
     rope_qknorm_bwd_kernel<float><<<rows_grid((size_t)M, 8), 256, 0, st>>>(
         (float *)dqkv, (const float *)qkv, (int)ld, rq, rk, m->rope_cos, m->rope_sin, M, T, m->H);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ECUDA;
+}
+
+int nc_set_attention_ctas(int ctas) {
+  if (ctas < 0) return NC_EINVAL;
+  fatc::persistent_cap().store(ctas);
+  return NC_OK;
 }
 
 int nc_ops_status(void *stream, int timeout_ms) {

@@ -193,6 +193,13 @@ int nc_rope_qknorm(const nc_model *m, void *qkv, int64_t ld, float *rq, float *r
 int nc_rope_qknorm_bwd(const nc_model *m, void *dqkv, const void *qkv, int64_t ld, const float *rq,
                        const float *rk, int B, int T, void *stream);
 
+/* Cap on the CTAs of the persistent attention kernels (the forward and the
+ * dQ kernel of the backward, in nc_fwd_bwd and the op-level calls): 0 (the
+ * default) = one CTA per SM; n > 0 = at most n CTAs, each then taking more
+ * 128-query tiles (fewer CTAs leave SMs to other streams, e.g. gradient
+ * all-reduces).  Process-wide, for launches that follow; < 0: NC_EINVAL. */
+int nc_set_attention_ctas(int ctas);
+
 /* Status of the op-level calls above (nc_gemm, nc_attention_*, and the
  * calls below), which have no model handle: waits at most timeout_ms for the
  * work enqueued so far on `stream` (polling), then reads and clears the

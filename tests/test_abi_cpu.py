@@ -105,6 +105,7 @@ def test_op_entry_points_reject_bad_arguments_on_the_host(lib):
     assert nc.nc_attention_bwd_ex(0, ld, 16, 16, 16, 16, 16, 1 << 20, 16, B, T, H, BF16, 0, None) == nc.NC_EINVAL
     assert nc.nc_attention_bwd_scratch_bytes(0, T, H, 0)[0] == nc.NC_ESHAPE
     assert nc.nc_attention_bwd_scratch_bytes(B, T, H, -1)[0] == nc.NC_EINVAL
+    assert nc.nc_set_attention_ctas(-1) == nc.NC_EINVAL
     # GEMM: a bf16 stride that is not a multiple of 8 on a tensor-core engine
     assert nc.nc_gemm(16, 100, 0, 16, 128, 0, 16, 128, 64, 64, 100, BF16, nc.NC_EPI_STORE, 0,
                       None) == nc.NC_EALIGN

@@ -376,3 +376,51 @@ def test_attention_bwd_with_cut_key_tiles(nc, B, T, H, window):
         cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
         assert cos > 0.9995, cos
         assert np.max(np.abs(g - r)) <= 3e-2 * np.abs(r).max()
+
+
+PERSIST_CASES = [(1, 515, 3, 0), (2, 300, 2, 0), (1, 515, 3, 64), (1, 1030, 2, 384), (2, 512, 2, 1)]
+
+
+@pytest.mark.parametrize("B,T,H,window", PERSIST_CASES)
+def test_persistent_attention_with_few_ctas(nc, B, T, H, window):
+    # the persistent forward and dQ kernels with their CTA count capped at 3,
+    # so every CTA walks several query tiles (one-key-tile tiles among them):
+    # bit-identical to one CTA per SM (each tile's arithmetic is the same),
+    # and against the oracle through the earlier tests' tolerances
+    import torch
+
+    from oracle import full_block as fb
+    qkv, ld, q, k, v = _attn_inputs(B, T, H, 700 + T + H + window, "bf16")
+    st = torch.cuda.current_stream().cuda_stream
+    qkv_d = _dev(qkv, "bf16")
+    dO = _bf16(synth.normal(13 + T, 4, B * T * H * 128).reshape(B * T, H * 128))
+    dO_d = _dev(dO, "bf16")
+    outs = []
+    try:
+        for cap in (0, 3, 0):
+            assert nc.nc_set_attention_ctas(cap) == nc.NC_OK
+            O = torch.zeros(B * T, H * 128, dtype=torch.bfloat16, device="cuda")
+            lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+            assert nc.nc_attention_fwd(qkv_d.data_ptr(), ld, O.data_ptr(), lse.data_ptr(), B, T, H, nc.NC_BF16, 0,
+                                       st, window=window) == 0
+            Drow = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+            dqkv = torch.zeros(B * T, ld, dtype=torch.bfloat16, device="cuda")
+            assert nc.nc_attention_bwd(qkv_d.data_ptr(), ld, O.data_ptr(), dO_d.data_ptr(), lse.data_ptr(),
+                                       Drow.data_ptr(), dqkv.data_ptr(), B, T, H, nc.NC_BF16, 0, st,
+                                       window=window) == 0
+            assert nc.nc_ops_status(st, 60000) == nc.NC_OK
+            outs.append((O.view(torch.int16).cpu(), lse.cpu(), dqkv.view(torch.int16).cpu(), Drow.cpu()))
+    finally:
+        nc.nc_set_attention_ctas(0)
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b), "capped CTAs change no bit"
+    got = outs[1][2].view(torch.bfloat16).float().numpy().astype(np.float64)
+    dq_ref = np.empty((B, T, H, 128))
+    for bb in range(B):
+        dq_ref[bb], _, _ = fb.attention_bwd(dO.reshape(B, T, H, 128)[bb], q[bb], k[bb], v[bb], window or None)
+    g, r = got[:, :H * 128], dq_ref.reshape(B * T, -1)
+    if window == 1:
+        assert np.max(np.abs(g)) <= 1e-5 * np.abs(v).max()
+    else:
+        cos = np.sum(g * r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300)
+        assert cos > 0.9995, cos
