@@ -190,6 +190,10 @@ def main():
         run()
         ev[2 * i + 1].record()
     torch.cuda.synchronize()
+    # a kernel wait that ran out of time makes the timing meaningless: fail loudly
+    rc = nc.nc_ops_status(st, 60000)
+    if rc != 0:
+        raise SystemExit(f"device status after the timed launches: {nc.nc_strerror(rc)}")
     ms = sorted(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.iters))
     med = ms[len(ms) // 2]
     out = {"op": args.op, "tokens": args.tokens, "shape": args.shape, "window": args.window, "median_ms": med,
