@@ -1408,9 +1408,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int h2 = 0; h2 < 2; ++h2) {
           const int qi = 4 * i4 + 2 * h2;
           const uint64_t nl = mul2(h2 ? f2(l4.z, l4.w) : f2(l4.x, l4.y), nl2e);
-          float x0, x1;
-          f2split(fma2(f2(__uint_as_float(xv[qi]), __uint_as_float(xv[qi + 1])), sc2, nl), x0, x1);
-          float v0 = ex2(x0), v1 = ex2(x1);
+          const uint64_t x = fma2(f2(__uint_as_float(xv[qi]), __uint_as_float(xv[qi + 1])), sc2, nl);
+          float v0, v1;
+          if (h2 && (i4 & 1)) {
+            ex2_poly2(x, v0, v1);  // one pair in four on the FMA pipe: MUFU bounds this loop
+          } else {
+            float x0, x1;
+            f2split(x, x0, x1);
+            v0 = ex2(x0);
+            v1 = ex2(x1);
+          }
           if (need_mask) {
             if (qq0 + qi < key || qq0 + qi >= p.T || (kWin && qq0 + qi - key >= p.window)) v0 = 0.f;
             if (qq0 + qi + 1 < key || qq0 + qi + 1 >= p.T || (kWin && qq0 + qi + 1 - key >= p.window)) v1 = 0.f;
