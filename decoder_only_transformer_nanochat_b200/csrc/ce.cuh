@@ -125,13 +125,13 @@ __device__ __forceinline__ bool ce_wait(uint32_t bar, uint32_t parity) {
   for (uint32_t i = 0;; ++i) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(1u << 20)  // sleep in hardware until the row lands (<= ~1 ms)
         : "memory");
     if (ok) return true;
-    if ((i & 255) == 255) {
+    if ((i & 15) == 15) {
       uint64_t t;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
       if (t - t0 > 4000000000ull) return false;

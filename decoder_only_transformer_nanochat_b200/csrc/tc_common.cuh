@@ -42,14 +42,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Suspend-time hint of the blocking barrier waits (ns): a waiting thread
+// sleeps in hardware until the phase completes or this much time passes, so
+// the TMA and MMA threads' waits do not take issue slots from the warps that
+// share their scheduler (the element-wise and epilogue warps).
+constexpr uint32_t kWaitHintNs = 1u << 20;
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kWaitHintNs)
       : "memory");
   return ok != 0;
 }
@@ -73,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 255) == 0) {
+    if ((i & 15) == 0) {  // each try may have slept up to kWaitHintNs
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitNs) {
         *abort_flag = 1;
