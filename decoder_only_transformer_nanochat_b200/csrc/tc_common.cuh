@@ -46,16 +46,29 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // sleeps in hardware until the phase completes or this much time passes, so
 // the TMA and MMA threads' waits do not take issue slots from the warps that
 // share their scheduler (the element-wise and epilogue warps).
-constexpr uint32_t kWaitHintNs = 1u << 20;
+#ifndef NC_WAIT_HINT_NS
+#define NC_WAIT_HINT_NS (1u << 20)
+#endif
+constexpr uint32_t kWaitHintNs = NC_WAIT_HINT_NS;  // 0: the hardware's default time limit
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(kWaitHintNs)
-      : "memory");
+  if (kWaitHintNs > 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(kWaitHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 // Non-blocking test of a phase (try_wait may suspend the thread for a while
