@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         const Unit x = unit_of(p, u);
         for (int kb = x.kb0; kb < x.kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait<true>(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
           mbar_expect_tx(full_bar(stage), STAGE_BYTES);
@@ -269,11 +269,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         const Unit x = unit_of(p, u);
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = x.kb0; kb < x.kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait<true>(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Unit x = unit_of(p, u);
       // every lane waits; the vote over all epilogue threads keeps their
       // branches (and named barriers) uniform and re-converges each warp
-      ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      ok = epi_vote_all(mbar_wait<true>(tfull_bar(acc), acc_phase, abort_flag, p.status));
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
           if (aux) {
-            ok = epi_vote_all(mbar_wait(aux_bar, aux_phase, abort_flag, p.status));
+            ok = epi_vote_all(mbar_wait<true>(aux_bar, aux_phase, abort_flag, p.status));
             aux_phase ^= 1;
             if (!ok) break;
           } else {
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int m_row = x.m_blk * 256 + (int)rank * BM;
         const int n_row = x.n_blk * BN2 + (int)rank * BH2;
         for (int kb = x.kb0; kb < x.kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait<true>(empty_bar(stage), phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
           const uint32_t sb = sa + A_BYTES;
           if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES2);
@@ -557,11 +557,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int u = cluster; u < p.units && ok; u += n_clusters) {
         const Unit x = unit_of2(p, u);
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait<true>(tempty_bar(acc), acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN2;
         for (int kb = x.kb0; kb < x.kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait<true>(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
           const uint32_t sb = sa + A_BYTES;
@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     for (int u = cluster; u < p.units && ok; u += n_clusters) {
       const Unit x = unit_of2(p, u);
-      ok = epi_vote_all(mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      ok = epi_vote_all(mbar_wait<true>(tfull_bar(acc), acc_phase, abort_flag, p.status));
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
           if (aux) {
-            ok = epi_vote_all(mbar_wait(aux_bar, aux_phase, abort_flag, p.status));
+            ok = epi_vote_all(mbar_wait<true>(aux_bar, aux_phase, abort_flag, p.status));
             aux_phase ^= 1;
             if (!ok) break;
           } else {

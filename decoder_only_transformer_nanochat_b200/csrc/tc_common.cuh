@@ -42,17 +42,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// Suspend-time hint of the blocking barrier waits (ns): a waiting thread
-// sleeps in hardware until the phase completes or this much time passes, so
-// the TMA and MMA threads' waits do not take issue slots from the warps that
-// share their scheduler (the element-wise and epilogue warps).
-#ifndef NC_WAIT_HINT_NS
-#define NC_WAIT_HINT_NS (1u << 20)
-#endif
-constexpr uint32_t kWaitHintNs = NC_WAIT_HINT_NS;  // 0: the hardware's default time limit
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+// Two forms of the blocking barrier test.  Spinning (the hardware's default
+// time limit) reacts fastest; sleeping (a suspend-time hint) lets a waiting
+// thread leave the issue slots of its scheduler to the warps that share it.
+// Measured on the B200 at d20 shapes: the GEMMs, whose TMA and MMA threads
+// share schedulers with the epilogue warps, run 2-3 % faster with sleeping
+// waits; the attention kernels, whose MMA thread must react at once to the
+// element-wise warps' hand-offs, run 3 % slower.  So the GEMM sleeps and the
+// attention spins.
+constexpr uint32_t kWaitHintNs = 1u << 20;
+template <bool kSleep>
+__device__ __forceinline__ bool mbar_try_t(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  if (kWaitHintNs > 0) {
+  if constexpr (kSleep) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -71,6 +73,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   }
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) { return mbar_try_t<false>(bar, parity); }
 // Non-blocking test of a phase (try_wait may suspend the thread for a while
 // before it gives up, which stalls a loop that polls several barriers).
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
@@ -85,13 +88,14 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait; false if this CTA is aborting (flag set here or elsewhere).
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int *status) {
-  if (mbar_try(bar, parity)) return true;
+  if (mbar_try_t<kSleep>(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 15) == 0) {  // each try may have slept up to kWaitHintNs
+    if (mbar_try_t<kSleep>(bar, parity)) return true;
+    if ((i & (kSleep ? 15 : 255)) == 0) {  // a sleeping try may take up to kWaitHintNs
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitNs) {
         *abort_flag = 1;
