@@ -34,13 +34,6 @@ namespace fatc {
 using namespace tc;
 
 constexpr int kQ = 128, kKV = 128, kD = 128;
-// The TMA producers' waits (a ring slot or a Q/dO buffer coming free) are not
-// on the critical path and sleep in hardware, leaving issue slots to the
-// element-wise warps on their scheduler; the MMA and element-wise waits spin.
-#ifndef NC_ATTN_PRODUCER_SLEEP
-#define NC_ATTN_PRODUCER_SLEEP 1
-#endif
-constexpr bool kProducerSleep = NC_ATTN_PRODUCER_SLEEP != 0;
 constexpr int kFwdThreads = 320;  // TMA warp, MMA warp, 8 softmax warps
 constexpr int kTileBytes = kQ * kD * 2;      // 32 KB: Q, K, V or P tile
 constexpr int kKStages = 3, kVStages = 2;
@@ -209,7 +202,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int issued_k = 0, issued_v = 0;
       auto load_k = [&](int j) -> bool {
         const int st = j % kKStages;
-        if (!mbar_wait<kProducerSleep>(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(k_empty(st), ((j / kKStages) & 1) ^ 1, abort_flag, p.status)) return false;
         const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
         mbar_expect_tx(k_full(st), kTileBytes);
         for (int i = 0; i < 2; ++i) tma_load_3d(k_dst + i * 16384, &map_qk, C + 64 * i, kbase + j * kKV, b, k_full(st));
@@ -218,7 +211,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       auto load_v = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait<kProducerSleep>(v_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(v_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
         const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
         mbar_expect_tx(v_full(st), kTileBytes);
         for (int hh = 0; hh < 2; ++hh)
@@ -549,13 +542,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         int q0, b, h, kbase, n_kv;
         item_of(it, q0, b, h, kbase, n_kv);
         const int qb = li & 1;
-        if (!(okp = mbar_wait<kProducerSleep>(q_empty(qb), ((li >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        if (!(okp = mbar_wait(q_empty(qb), ((li >> 1) & 1) ^ 1, abort_flag, p.status))) break;
         mbar_expect_tx(q_full(qb), kTileBytes);
         for (int i = 0; i < 2; ++i)
           tma_load_3d(smem_u32(sQ) + qb * kTileBytes + i * 16384, &map_qk, h * kD + 64 * i, q0, b, q_full(qb));
         auto load_k = [&](int j) -> bool {
           const int st = kc % kPpStages;
-          if (!mbar_wait<kProducerSleep>(k_empty(st), ((kc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
+          if (!mbar_wait(k_empty(st), ((kc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
           const uint32_t k_dst = smem_u32(sK) + st * kTileBytes;
           mbar_expect_tx(k_full(st), kTileBytes);
           for (int i = 0; i < 2; ++i)
@@ -565,7 +558,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         };
         auto load_v = [&](int j) -> bool {
           const int st = vc % kPpStages;
-          if (!mbar_wait<kProducerSleep>(v_empty(st), ((vc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
+          if (!mbar_wait(v_empty(st), ((vc / kPpStages) & 1) ^ 1, abort_flag, p.status)) return false;
           const uint32_t v_dst = smem_u32(sV) + st * kTileBytes;
           mbar_expect_tx(v_full(st), kTileBytes);
           for (int hh = 0; hh < 2; ++hh)
@@ -951,8 +944,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // Q and dO take the next item once the previous item's last score MMAs
         // are done and its D has been formed from the dO tile (with one key
         // tile the MMAs can finish first)
-        if (li > 0 && !(okp = mbar_wait<kProducerSleep>(qg_free, (li - 1) & 1, abort_flag, p.status) &&
-                              mbar_wait<kProducerSleep>(d_done, (li - 1) & 1, abort_flag, p.status)))
+        if (li > 0 && !(okp = mbar_wait(qg_free, (li - 1) & 1, abort_flag, p.status) &&
+                              mbar_wait(d_done, (li - 1) & 1, abort_flag, p.status)))
           break;
         mbar_expect_tx(q_full, 2 * kTileBytes);
         for (int i = 0; i < 2; ++i) {
@@ -962,13 +955,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++nq;
         for (int j = 0; j < n_kv; ++j) {
           const int ks = kc % kDqKStages, vs = vc % kDqVStages;
-          if (!(okp = mbar_wait<kProducerSleep>(k_empty(ks), ((kc / kDqKStages) & 1) ^ 1, abort_flag, p.status))) break;
+          if (!(okp = mbar_wait(k_empty(ks), ((kc / kDqKStages) & 1) ^ 1, abort_flag, p.status))) break;
           mbar_expect_tx(k_full(ks), kTileBytes);
           for (int i = 0; i < 2; ++i)
             tma_load_3d(smem_u32(sK) + ks * kTileBytes + i * 16384, &map_q, C + 64 * i, kbase + j * kBK, b,
                         k_full(ks));
           ++kc;
-          if (!(okp = mbar_wait<kProducerSleep>(v_empty(vs), ((vc / kDqVStages) & 1) ^ 1, abort_flag, p.status))) break;
+          if (!(okp = mbar_wait(v_empty(vs), ((vc / kDqVStages) & 1) ^ 1, abort_flag, p.status))) break;
           mbar_expect_tx(v_full(vs), kTileBytes);
           for (int i = 0; i < 2; ++i)
             tma_load_3d(smem_u32(sV) + vs * kTileBytes + i * 16384, &map_q, C + kD + 64 * i, kbase + j * kBK, b,
@@ -1278,7 +1271,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int issued = 0;
     for (int j = 0; j < my_n; ++j) {
       const int it = it0 + j, st = j % kKvStages;
-      const bool okw = mbar_wait<kProducerSleep>(q_empty(st), ((j / kKvStages) & 1) ^ 1, abort_flag, p.status);
+      const bool okw = mbar_wait(q_empty(st), ((j / kKvStages) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, okw)) break;
       const int hh = it / n_q, qq0 = (first + it % n_q) * kBQ2;
       uint8_t *stage = sQS + st * kQStage;
