@@ -115,7 +115,11 @@ template <> __device__ __forceinline__ float exp_t<float>(float x) { return expf
 // thread has its slice in registers the copy of the CTA's next row is
 // issued, so the load of row i+1 and the store of dz for row i stream while
 // row i's exponentials run.  Per thread the raw logits, then w = e (1 - t^2)
-// (fp16, w <= 1), are kept packed in registers.
+// (fp16, w <= 1), are kept packed in registers.  A row takes two block-wide
+// barriers: one publishes the warps' maxima (and frees the buffer), one their
+// sums.  The small shared values alternate between two slots by row parity,
+// so a warp that has stored its part of row i goes on to row i+1 without
+// waiting for the others; the next row's target id is read a row ahead.
 constexpr int kCeThreads = 1024;
 constexpr int kCeCopy = 32768;  // bytes per bulk copy
 
@@ -157,13 +161,16 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
     bf16 *__restrict__ z, int64_t ldz, const int32_t *__restrict__ targets,
     float *__restrict__ token_loss, int M, int V, float grad_scale, int *status) {
   extern __shared__ __align__(128) uint8_t ce_smem[];
-  __shared__ float red[32];
-  __shared__ float s_target, sech2_target;
+  constexpr int kWarps = kCeThreads / 32;
+  static_assert(kWarps == 32, "one warp reads every warp's partial, one per lane");
+  __shared__ float red_max[2][kWarps], red_sum[2][kWarps];
+  __shared__ float s_target[2], sech2_target[2];
   __shared__ __align__(8) uint64_t bar_storage;
   const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&bar_storage));
   const uint32_t buf = static_cast<uint32_t>(__cvta_generic_to_shared(ce_smem));
   const int row_bytes = V * 2;
   const int n8 = V >> 3;  // 16-byte chunks of a row
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -173,14 +180,12 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
   if (threadIdx.x == 0 && row < M) ce_fetch_row(buf, z + (size_t)row * ldz, row_bytes, bar);
   uint32_t phase = 0;
   const float k2 = kSoftcap * kLog2e;
-  for (; row < M; row += gridDim.x) {
+  int tgt_next = row < M ? targets[row] : 0;
+  for (int par = 0; row < M; row += gridDim.x, par ^= 1) {
+    int tgt = tgt_next;
+    if (row + (int)gridDim.x < M) tgt_next = targets[row + gridDim.x];  // used by the next row
     const bool ok = ce_wait(bar, phase);
     phase ^= 1;
-    if (!__syncthreads_and(ok)) {
-      if (threadIdx.x == 0) set_status(status, kStatusTimeout);
-      break;
-    }
-    int tgt = targets[row];
     if (tgt < 0 || tgt >= V) {
       if (threadIdx.x == 0) set_status(status, kStatusRange);
       tgt = tgt < 0 ? 0 : V - 1;
@@ -188,8 +193,8 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
     if (threadIdx.x == 0) {
       float tt, s2;
       softcap_parts_fast(__bfloat162float(reinterpret_cast<const bf16 *>(ce_smem)[tgt]), tt, s2);
-      s_target = kSoftcap * tt;
-      sech2_target = s2;
+      s_target[par] = kSoftcap * tt;
+      sech2_target[par] = s2;
     }
     // raw logits into registers, their max (tanh is increasing)
     uint32_t pk[NVEC][4];
@@ -208,10 +213,20 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
         }
       }
     }
-    __syncthreads();  // the buffer is free (and s_target visible): fetch the next row
+    {
+      const float wm = warp_max(fmaxf(__low2float(hmax), __high2float(hmax)));
+      if (lane == 0) red_max[par][wid] = wm;
+    }
+    // every slice is in registers (the buffer may take the next row), the
+    // warps' maxima and the target's terms are visible, and all threads agree
+    // that the row arrived
+    if (!__syncthreads_and(ok)) {
+      if (threadIdx.x == 0) set_status(status, kStatusTimeout);
+      break;
+    }
     if (threadIdx.x == 0 && row + (int)gridDim.x < M)
       ce_fetch_row(buf, z + (size_t)(row + gridDim.x) * ldz, row_bytes, bar);
-    const float zmax = block_max(fmaxf(__low2float(hmax), __high2float(hmax)), red);
+    const float zmax = warp_max(red_max[par][lane]);
     float tmax, s2max;
     softcap_parts_fast(zmax, tmax, s2max);
     const float m2 = k2 * tmax;  // row max of s, log2 domain
@@ -253,14 +268,20 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
         rest += part;
       }
     }
-    rest = block_sum(rest, red);  // contains __syncthreads
-    const float e_t = ex2_fast(fmaf(kLog2e, s_target, -m2));
+    {
+      const float ws = warp_sum(rest);
+      if (lane == 0) red_sum[par][wid] = ws;
+    }
+    __syncthreads();
+    rest = warp_sum(red_sum[par][lane]);
+    const float s_t = s_target[par];
+    const float e_t = ex2_fast(fmaf(kLog2e, s_t, -m2));
     const float sum = rest + e_t;
     const float lse2 = m2 + __log2f(sum);  // log-sum-exp in the log2 domain
-    if (threadIdx.x == 0) token_loss[row] = lse2 * kLn2 - s_target;
+    if (threadIdx.x == 0) token_loss[row] = lse2 * kLn2 - s_t;
     const float scale = grad_scale / sum;
     // 1 - p_target = rest / sum: no cancellation when the target dominates
-    const bf16 dz_t = __float2bfloat16_rn(-(rest / sum) * sech2_target * grad_scale);
+    const bf16 dz_t = __float2bfloat16_rn(-(rest / sum) * sech2_target[par] * grad_scale);
     bf16 *zrow = z + (size_t)row * ldz;
 #pragma unroll
     for (int k = 0; k < NVEC; ++k) {
@@ -286,7 +307,8 @@ __global__ void __launch_bounds__(kCeThreads, 1) ce_fused_bf16_persistent_kernel
         *reinterpret_cast<uint4 *>(zrow + c * 8) = u;
       }
     }
-    __syncthreads();  // s_target and red are reused by the next row
+    // no barrier here: the next row writes the other parity's slots, and this
+    // row's slots are rewritten only after both of the next row's barriers
   }
 }
 

@@ -101,6 +101,7 @@ CASES = [
     # V, M, dtype, row padding: the model path (persistent), then the general kernel
     (65536, 12, "bf16", 64),
     (65536, 10, "bf16", 0),
+    (65536, 451, "bf16", 0),    # 3 x 148 + 7 rows: every CTA of the persistent kernel walks 3-4 rows
     (1000, 12, "bf16", 8),      # V % 8 == 0, small: persistent kernel with idle threads
     (1003, 12, "bf16", 5),      # ragged: the general kernel
     (65536, 12, "f32", 64),
