@@ -467,8 +467,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *staging = smem + STAGES2 * STAGE_BYTES2;
   uint64_t *bars = reinterpret_cast<uint64_t *>(staging + STAGING_BYTES);
-  // bars: full[S], empty[S], tfull[2], tempty[2], drain, aux
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES2 + 6);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, aux[2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES2 + 7);
+  static_assert((2 * STAGES2 + 7) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -479,7 +480,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * STAGES2 + a); };
   auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * STAGES2 + 2 + a); };
   const uint32_t drain_bar = smem_u32(bars + 2 * STAGES2 + 4);
-  const uint32_t aux_bar = smem_u32(bars + 2 * STAGES2 + 5);
+  auto aux_bar = [&](int b) { return smem_u32(bars + 2 * STAGES2 + 5 + b); };
+  // An epilogue that reads its output tile first (residual add, relu^2
+  // backward) runs the ring with one stage fewer and takes that stage's 32 KB
+  // as a second staging tile: the input of the next half tile loads into one
+  // while the current half is computed and stored from the other.
+  const bool aux_pipe = (p.epi == EPI_ADD || p.epi == EPI_DRELU2) && !epi_f32(p.epi);
+  const int nst = aux_pipe ? STAGES2 - 1 : STAGES2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES2; ++s) {
@@ -491,7 +498,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty_bar(a), 256);  // both CTAs' epilogue threads
     }
     mbar_init(drain_bar, 1);
-    mbar_init(aux_bar, 1);
+    mbar_init(aux_bar(0), 1);
+    mbar_init(aux_bar(1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -537,7 +545,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < BH2 / 64; ++i) tma_load_2d_pair(sb + i * 8192, &map_b, n_row + 64 * i, k0, fb);
           }
           ++issued;
-          if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+          if (++stage == nst) { stage = 0; phase ^= 1; }
         }
       }
       // our copies complete on the leader's barriers; every one of them is
@@ -570,7 +578,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_mma_pair(d_tmem, smem_desc(sa + kk * a_kstep, a_lbo, 1024), smem_desc(sb + kk * b_kstep, b_lbo, 1024),
                         idesc, (kb > x.kb0 || kk > 0) ? 1u : 0u);
           tc_commit_pair(empty_bar(stage), 0x3);
-          if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+          if (++stage == nst) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar(acc), 0x3);
@@ -586,16 +594,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = quarter * 32 + lane;
     const bool ep_leader = warp == 2 && lane == 0;
     const bool f32_out = epi_f32(p.epi);
-    const bool aux = p.epi == EPI_ADD || p.epi == EPI_DRELU2;
-    const uint32_t st_addr = smem_u32(staging);
+    const bool aux = aux_pipe;
+    // staging tile 0 is the one after the ring; tile 1 (aux epilogues only)
+    // is the ring's last stage, which their ring does not use
+    auto stg_tile = [&](int b) { return b ? smem + (STAGES2 - 1) * STAGE_BYTES2 : staging; };
     int acc = 0;
-    uint32_t acc_phase = 0, aux_phase = 0;
+    uint32_t acc_phase = 0;
+    uint32_t aux_phases = 0;    // bit b: the phase of aux_bar(b)
+    int halves = 0;             // half tiles this CTA has taken (their staging tile alternates)
+    uint32_t aux_inflight = 0;  // ep_leader, bit b: a load into tile b not yet waited for
     bool ok = true;
     auto release_tmem = [&](int a) {
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(a));
       else mbar_arrive_remote(tempty_bar(a), 0);
     };
+    // ep_leader: this CTA's rows of half `hh` of unit `uu`, read from D into staging tile `b`
+    auto load_aux = [&](int uu, int hh, int b) {
+      const Unit y = unit_of2(p, uu);
+      const int ym0 = y.m_blk * 256 + (int)rank * BM;
+      const int yn = y.n_blk * BN2 + hh * 128;
+      const bool yb1 = yn + 64 < p.N;
+      const uint32_t dst = smem_u32(stg_tile(b));
+      mbar_expect_tx(aux_bar(b), yb1 ? 2 * BM * 128 : BM * 128);
+      tma_load_2d(dst, &map_d, yn, ym0, aux_bar(b));
+      if (yb1) tma_load_2d(dst + BM * 128, &map_d, yn + 64, ym0, aux_bar(b));
+      aux_inflight |= 1u << b;
+    };
+    if (aux && ep_leader && cluster < p.units) load_aux(cluster, 0, 0);
     for (int u = cluster; u < p.units && ok; u += n_clusters) {
       const Unit x = unit_of2(p, u);
       ok = epi_vote_all(mbar_wait<true>(tfull_bar(acc), acc_phase, abort_flag, p.status));
@@ -620,19 +646,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int half = 0; half < 2; ++half) {
           const int n_half = x.n_blk * BN2 + half * 128;
           const bool box1 = n_half + 64 < p.N;
-          if (ep_leader) {
-            bulk_wait_read0();
-            if (aux) {
-              mbar_expect_tx(aux_bar, box1 ? 2 * BM * 128 : BM * 128);
-              tma_load_2d(st_addr, &map_d, n_half, m0, aux_bar);
-              if (box1) tma_load_2d(st_addr + BM * 128, &map_d, n_half + 64, m0, aux_bar);
-            }
-          }
+          const bool last_half = half == 1 || n_half + 128 >= p.N;
+          const int b = aux ? (halves & 1) : 0;
+          uint8_t *const stg = stg_tile(b);
+          const uint32_t st_addr = smem_u32(stg);
           if (aux) {
-            ok = epi_vote_all(mbar_wait<true>(aux_bar, aux_phase, abort_flag, p.status));
-            aux_phase ^= 1;
+            if (ep_leader) {
+              // the next half tile's input goes to the other staging tile as
+              // soon as the store that last read it (the previous half's) is done
+              const int nu = last_half ? u + n_clusters : u, nh = last_half ? 0 : 1;
+              if (nu < p.units) {
+                bulk_wait_read0();
+                load_aux(nu, nh, b ^ 1);
+              }
+            }
+            ok = epi_vote_all(mbar_wait<true>(aux_bar(b), (aux_phases >> b) & 1u, abort_flag, p.status));
             if (!ok) break;
+            aux_phases ^= 1u << b;
+            aux_inflight &= ~(1u << b);
+            ++halves;
           } else {
+            if (ep_leader) bulk_wait_read0();  // the previous stores have read the staging tile
             epi_bar();
           }
           __syncwarp();
@@ -640,9 +674,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < 4; ++c) {
             uint32_t rr[32];
             tmem_ld32(t_row + half * 128 + c * 32, rr);
-            epilogue_stage(p.epi, staging, r, c, rr);
+            epilogue_stage(p.epi, stg, r, c, rr);
           }
-          if (half == 1 || n_half + 128 >= p.N) release_tmem(acc);
+          if (last_half) release_tmem(acc);
           fence_proxy_async();
           epi_bar();
           if (ep_leader) {
@@ -656,7 +690,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
-    if (ep_leader) bulk_wait0();
+    if (ep_leader) {
+      bulk_wait0();
+      // only after an abort: loads issued for halves that were never taken
+      // land before the CTA's shared memory goes away (bounded)
+      for (int b = 0; b < 2; ++b) {
+        if (!((aux_inflight >> b) & 1u)) continue;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(aux_bar(b), (aux_phases >> b) & 1u) && globaltimer() - t0 < kWaitNs) {}
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();

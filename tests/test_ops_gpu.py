@@ -62,6 +62,10 @@ GEMM_CASES = [
     (256, 256, 8192, 1, 1, 0),     # few tiles, long K: split-K path for fp32 output
     (520, 392, 136, 0, 1, 8),      # M not a multiple of 256: the second CTA of a pair is partly empty
     (1280, 5120, 256, 1, 1, 0),    # weight-gradient shape with a full second CTA
+    # several tiles per CTA pair whose N tiles alternate two half tiles and one
+    # (the epilogue's staging tiles alternate by half tile across tiles)
+    (20480, 320, 128, 0, 0, 0),
+    (20480, 392, 64, 0, 1, 8),     # ... and a last half tile of 8 columns
 ]
 
 
