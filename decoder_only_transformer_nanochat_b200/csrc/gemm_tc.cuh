@@ -399,6 +399,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // leader's "tmem empty" barrier.
 constexpr int BN2 = 256, BH2 = 128;                  // tile N, B rows per CTA
 constexpr int STAGES2 = 6;
+// Eight epilogue warps (2..9): two per TMEM lane quarter (warp % 4), each
+// taking one of the two column groups of every half tile, so an epilogue
+// that reads its output tile first keeps pace with the main loop.
+constexpr int EPI_WARPS2 = 8;
+constexpr int NUM_THREADS2 = 64 + 32 * EPI_WARPS2;
 constexpr int STAGE_BYTES2 = A_BYTES + BH2 * BK * 2;  // 32 KB
 constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + 256;
 static_assert(SMEM_BYTES2 <= 232448, "shared memory per CTA");
@@ -455,12 +460,27 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
       : "memory");
 }
 
+// barrier, and barrier with an AND vote, among the 256 epilogue threads of the two-CTA kernel
+__device__ __forceinline__ void epi_bar2() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool epi_vote_all2(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
+}
+
 __device__ __forceinline__ Unit unit_of2(const Params &p, int u) {
   // p.n_m counts 256-row blocks here
   return unit_of(p, u);
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS2, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_d, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -495,7 +515,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 256);  // both CTAs' epilogue threads
+      mbar_init(tempty_bar(a), 2 * 32 * EPI_WARPS2);  // both CTAs' epilogue threads
     }
     mbar_init(drain_bar, 1);
     mbar_init(aux_bar(0), 1);
@@ -589,8 +609,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < kWaitNs) {}
     }
   } else {
-    // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+    // ---------------- epilogue warps 2..9 (both CTAs) ----------------
     const int quarter = warp & 3;
+    const int cg = (warp - 2) >> 2;  // column group: chunks [2 cg, 2 cg + 2) of each half tile
     const int r = quarter * 32 + lane;
     const bool ep_leader = warp == 2 && lane == 0;
     const bool f32_out = epi_f32(p.epi);
@@ -624,7 +645,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (aux && ep_leader && cluster < p.units) load_aux(cluster, 0, 0);
     for (int u = cluster; u < p.units && ok; u += n_clusters) {
       const Unit x = unit_of2(p, u);
-      ok = epi_vote_all(mbar_wait<true>(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      ok = epi_vote_all2(mbar_wait<true>(tfull_bar(acc), acc_phase, abort_flag, p.status));
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -633,7 +654,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (f32_out) {
         const int m = m0 + r;
 #pragma unroll 1
-        for (int c = 0; c < BN2 / 32; ++c) {
+        for (int c = 4 * cg; c < 4 * cg + 4; ++c) {
           const int n = x.n_blk * BN2 + c * 32;
           if (n >= p.N) break;  // warp-uniform
           uint32_t rr[32];
@@ -660,25 +681,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 load_aux(nu, nh, b ^ 1);
               }
             }
-            ok = epi_vote_all(mbar_wait<true>(aux_bar(b), (aux_phases >> b) & 1u, abort_flag, p.status));
+            ok = epi_vote_all2(mbar_wait<true>(aux_bar(b), (aux_phases >> b) & 1u, abort_flag, p.status));
             if (!ok) break;
             aux_phases ^= 1u << b;
             aux_inflight &= ~(1u << b);
             ++halves;
           } else {
             if (ep_leader) bulk_wait_read0();  // the previous stores have read the staging tile
-            epi_bar();
+            epi_bar2();
           }
           __syncwarp();
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 2 * cg; c < 2 * cg + 2; ++c) {
             uint32_t rr[32];
             tmem_ld32(t_row + half * 128 + c * 32, rr);
             epilogue_stage(p.epi, stg, r, c, rr);
           }
           if (last_half) release_tmem(acc);
           fence_proxy_async();
-          epi_bar();
+          epi_bar2();
           if (ep_leader) {
             tma_store_2d(&map_d, st_addr, n_half, m0);
             if (box1) tma_store_2d(&map_d, st_addr + BM * 128, n_half + 64, m0);
@@ -867,7 +888,7 @@ inline cudaError_t launch_gemm_tc2(const GemmProblem &g, int num_sms, int *statu
   const int clusters = p.units < n_clusters ? p.units : n_clusters;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(NUM_THREADS2);
   cfg.dynamicSmemBytes = SMEM_BYTES2;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
