@@ -392,8 +392,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // (its A slice and its half of the accumulator) and loads half of B
 // (tile columns [128r, 128r+128)); the leader (r = 0) issues every MMA, which
 // reads A and B from both CTAs' shared memory.  Per SM a k-block moves 32 KB
-// instead of 48 KB for the same flops, so six stages fit and L2 traffic for
-// the B operand halves.  Both CTAs' TMA loads complete on the leader's "full"
+// instead of 48 KB for the same flops, so six stages fit (five, plus a second
+// staging tile, for the epilogues that read their output tile first) and L2
+// traffic for the B operand halves.  Both CTAs' TMA loads complete on the leader's "full"
 // barrier; the leader's commits arrive on both CTAs' "empty" and "tmem full"
 // barriers; both CTAs' epilogue threads release the accumulator on the
 // leader's "tmem empty" barrier.
