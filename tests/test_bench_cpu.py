@@ -56,3 +56,23 @@ def test_window_flop_count():
     # a window of w keys: w - w^2/(2T) pairs per query instead of T/2
     one = bench.model_flops_per_token(1, 1280, 65536, 2048, [1024]) - bench.model_flops_per_token(1, 1280, 65536, 2048, [0])
     assert abs(one - 12.0 * 1280 * (1024 - 1024 ** 2 / 4096 - 1024)) < 1e-6
+
+
+def test_traffic_is_reported_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
+    # roofline.traffic comes from a committed ncu summary, and only while the
+    # kernel source still hashes to the one recorded there
+    import hashlib
+    src = tmp_path / "k.cuh"
+    src.write_text("// kernel v1\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    (prof / "k_traffic.txt").write_text(
+        f"source_file: k.cuh\nsource_sha256: {sha}\ntraffic_bytes_per_launch: 1234.5\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("k") == 1234.5
+    src.write_text("// kernel v2\n")  # the kernel changed after the capture
+    assert bench.traffic_record("k") is None
+    assert bench.traffic_record("other") is None  # no summary at all
+    (prof / "k_traffic.txt").write_text("traffic_bytes_per_launch: 1.0\n")  # no source recorded
+    assert bench.traffic_record("k") is None
